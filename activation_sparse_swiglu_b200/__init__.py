@@ -1,0 +1,230 @@
+"""B200-native Prox two-stage sparse SwiGLU FFN decode step.
+
+Python binding over the C ABI of libprox.so (include/prox.h).  PyTorch is used
+only for device memory and CUDA streams; every step of the computation runs
+in the library's sm_100a kernels.
+
+    import activation_sparse_swiglu_b200 as prox
+    tau = prox.calibrate_thresholds(x_cal, s1=0.5)
+    layer = prox.Layer(w_gate, w_up, w_down, tau=tau, k=4301)
+    y = layer.forward(x)          # x: fp32 [B, d_model] on the GPU
+"""
+
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from ._lib import (DEVERR_MASK_INDEX, DEVERR_WAIT_TIMEOUT, LayerInfo, ProxError, check,
+                   last_error, lib)
+
+__all__ = ["Layer", "pack_proxy", "calibrate_thresholds", "rmsnorm", "copy", "version",
+           "ProxError", "DEVERR_MASK_INDEX", "DEVERR_WAIT_TIMEOUT", "last_error", "lib"]
+
+GROUP = 128
+
+
+def version() -> str:
+    return lib.prox_version().decode()
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _ptr(t: torch.Tensor | None) -> ctypes.c_void_p:
+    if t is None:
+        return ctypes.c_void_p(0)
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _dev(t: torch.Tensor, dtype: torch.dtype, name: str) -> torch.Tensor:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def pack_proxy(w: torch.Tensor, group: int = GROUP, stream=None):
+    """INT4 proxy of a bf16 [d_model, d_ff] weight: (codes uint8 [d, d_ff/2],
+    scales fp16 [d/group, d_ff])."""
+    _dev(w, torch.bfloat16, "w")
+    d, f = w.shape
+    codes = torch.empty((d, f // 2), dtype=torch.uint8, device=w.device)
+    scales = torch.empty((d // group, f), dtype=torch.float16, device=w.device)
+    check(lib.prox_pack_proxy(_ptr(w), d, f, group, _ptr(codes), _ptr(scales), _stream(stream)))
+    return codes, scales
+
+
+def calibrate_thresholds(x_cal: torch.Tensor, s1: float, stream=None) -> float:
+    """Exact s1-quantile of |x_cal| (fp32 [n_tok, d_model] on the GPU)."""
+    _dev(x_cal, torch.float32, "x_cal")
+    n, d = x_cal.shape
+    tau = ctypes.c_float(0.0)
+    check(lib.prox_calibrate_thresholds(_ptr(x_cal), n, d, float(s1), ctypes.byref(tau),
+                                        _stream(stream)))
+    return float(tau.value)
+
+
+def rmsnorm(y: torch.Tensor, eps: float = 1e-6, out: torch.Tensor | None = None, stream=None):
+    _dev(y, torch.float32, "y")
+    y2 = y.reshape(-1, y.shape[-1])
+    if out is None:
+        out = torch.empty_like(y)
+    check(lib.prox_rmsnorm(_ptr(y2), _ptr(out), y2.shape[0], y2.shape[1], float(eps),
+                           _stream(stream)))
+    return out
+
+
+def copy(src: torch.Tensor, dst: torch.Tensor, stream=None) -> None:
+    nbytes = src.numel() * src.element_size()
+    if dst.numel() * dst.element_size() < nbytes:
+        raise ValueError("dst is smaller than src")
+    check(lib.prox_copy(_ptr(src), _ptr(dst), nbytes, _stream(stream)))
+
+
+class Layer:
+    """One Prox FFN layer resident on the current CUDA device.
+
+    w_gate, w_up: bf16 [d_model, d_ff]; w_down: bf16 [d_ff, d_model] (math
+    layout, CUDA tensors).  The library repacks them into its own buffers, so
+    the tensors may be freed afterwards.
+    """
+
+    def __init__(self, w_gate, w_up, w_down, tau: float, k: int, max_batch: int = 1,
+                 stream=None):
+        _dev(w_gate, torch.bfloat16, "w_gate")
+        _dev(w_up, torch.bfloat16, "w_up")
+        _dev(w_down, torch.bfloat16, "w_down")
+        d, f = w_gate.shape
+        if tuple(w_up.shape) != (d, f) or tuple(w_down.shape) != (f, d):
+            raise ValueError("inconsistent weight shapes")
+        self.d_model, self.d_ff = d, f
+        self.device = w_gate.device
+        h = ctypes.c_void_p(0)
+        check(lib.prox_layer_create(_ptr(w_gate), _ptr(w_up), _ptr(w_down), d, f, float(tau),
+                                    int(k), int(max_batch), _stream(stream), ctypes.byref(h)))
+        self._h = h
+
+    # -- lifetime --------------------------------------------------------
+    def close(self):
+        if getattr(self, "_h", None) is not None and self._h.value:
+            with torch.cuda.device(self.device):
+                lib.prox_layer_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    @property
+    def handle(self) -> ctypes.c_void_p:
+        if self._h is None:
+            raise RuntimeError("layer is closed")
+        return self._h
+
+    # -- parameters ------------------------------------------------------
+    def info(self) -> dict:
+        inf = LayerInfo()
+        check(lib.prox_layer_get_info(self.handle, ctypes.byref(inf)))
+        return {name: getattr(inf, name) for name, _ in LayerInfo._fields_}
+
+    @property
+    def k(self) -> int:
+        return self.info()["k"]
+
+    @property
+    def tau(self) -> float:
+        return self.info()["tau_x"]
+
+    def set_tau(self, tau: float) -> None:
+        check(lib.prox_layer_set_tau(self.handle, float(tau)))
+
+    def set_k(self, k: int) -> None:
+        check(lib.prox_layer_set_k(self.handle, int(k)))
+
+    def error_word(self, stream=None) -> int:
+        v = ctypes.c_int32(0)
+        check(lib.prox_layer_error(self.handle, ctypes.byref(v), _stream(stream)))
+        return int(v.value)
+
+    def stats(self, stream=None):
+        """(sum of n_x, tokens) since the last call."""
+        s, t = ctypes.c_int64(0), ctypes.c_int64(0)
+        check(lib.prox_layer_stats(self.handle, ctypes.byref(s), ctypes.byref(t), _stream(stream)))
+        return int(s.value), int(t.value)
+
+    # -- compute ---------------------------------------------------------
+    def _io(self, x, out):
+        _dev(x, torch.float32, "x")
+        x2 = x.reshape(-1, self.d_model)
+        if out is None:
+            out = torch.empty_like(x2)
+        else:
+            _dev(out, torch.float32, "out")
+        return x2, out
+
+    def forward(self, x: torch.Tensor, out: torch.Tensor | None = None, stream=None):
+        x2, out = self._io(x, out)
+        check(lib.prox_ffn_forward(self.handle, _ptr(x2), _ptr(out), x2.shape[0], _stream(stream)))
+        return out
+
+    __call__ = forward
+
+    def dense(self, x: torch.Tensor, out: torch.Tensor | None = None, stream=None):
+        x2, out = self._io(x, out)
+        check(lib.prox_dense_ffn(self.handle, _ptr(x2), _ptr(out), x2.shape[0], _stream(stream)))
+        return out
+
+    def forward_host(self, x_host: torch.Tensor, out_host: torch.Tensor | None = None,
+                     stream=None):
+        """Tokens whose inputs/outputs live in host memory (pinned for async copies)."""
+        if x_host.is_cuda or x_host.dtype != torch.float32 or not x_host.is_contiguous():
+            raise TypeError("x_host must be a contiguous fp32 CPU tensor")
+        x2 = x_host.reshape(-1, self.d_model)
+        if out_host is None:
+            out_host = torch.empty_like(x2)
+        check(lib.prox_ffn_forward_host(self.handle, _ptr(x2), _ptr(out_host), x2.shape[0],
+                                        _stream(stream)))
+        return out_host
+
+    def forward_profiled(self, x: torch.Tensor, out: torch.Tensor, events, stream=None):
+        """One token, kernels serialised, with 4 torch.cuda.Event(enable_timing=True)."""
+        arr = (ctypes.c_void_p * 4)(*[ctypes.c_void_p(e.cuda_event) for e in events])
+        check(lib.prox_ffn_forward_profiled(self.handle, _ptr(x), _ptr(out), arr, _stream(stream)))
+
+    def debug_stage1(self, x: torch.Tensor, stream=None) -> dict:
+        """Stage 1 of one token: idx_x, n_x, g_tilde, u_tilde, idx_s (CUDA tensors)."""
+        _dev(x, torch.float32, "x")
+        dev = x.device
+        k = self.k
+        idx_x = torch.full((self.d_model,), -1, dtype=torch.int32, device=dev)
+        n_x = torch.zeros(1, dtype=torch.int32, device=dev)
+        g = torch.empty(self.d_ff, dtype=torch.float32, device=dev)
+        u = torch.empty(self.d_ff, dtype=torch.float32, device=dev)
+        idx_s = torch.empty(k, dtype=torch.int32, device=dev)
+        check(lib.prox_debug_stage1(self.handle, _ptr(x), _ptr(idx_x), _ptr(n_x), _ptr(g), _ptr(u),
+                                    _ptr(idx_s), _stream(stream)))
+        return dict(idx_x=idx_x, n_x=n_x, g_tilde=g, u_tilde=u, idx_s=idx_s)
+
+    def forward_with_mask(self, x: torch.Tensor, idx_s: torch.Tensor,
+                          out: torch.Tensor | None = None, want_s: bool = False, stream=None):
+        """Stage 2 on a given channel list (int32 CUDA tensor)."""
+        _dev(x, torch.float32, "x")
+        _dev(idx_s, torch.int32, "idx_s")
+        if out is None:
+            out = torch.empty(self.d_model, dtype=torch.float32, device=x.device)
+        s_sp = torch.empty(idx_s.numel(), dtype=torch.float32, device=x.device) if want_s else None
+        check(lib.prox_forward_with_mask(self.handle, _ptr(x), _ptr(idx_s), idx_s.numel(), _ptr(out),
+                                         _ptr(s_sp), _stream(stream)))
+        return (out, s_sp) if want_s else out

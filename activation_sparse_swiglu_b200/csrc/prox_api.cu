@@ -1,0 +1,492 @@
+// C ABI of the Prox library: argument checks, the layer handle, and the
+// stream-ordered kernel chains of the decode step.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <string>
+
+#include "prox_device.cuh"
+#include "prox_internal.h"
+
+namespace prox {
+cudaError_t setup_stage1_kernels();
+cudaError_t setup_stage2_kernels();
+}  // namespace prox
+
+namespace {
+
+thread_local std::string g_last_error;
+
+prox_status fail(prox_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+prox_status cuda_fail(cudaError_t e, const char* what) {
+  cudaGetLastError();  // clear the sticky-free error state of the runtime
+  return fail(e == cudaErrorMemoryAllocation ? PROX_ENOMEM : PROX_ECUDA, "%s: %s", what,
+              cudaGetErrorString(e));
+}
+
+#define PROX_CUDA(call, what)                         \
+  do {                                                \
+    cudaError_t e_ = (call);                          \
+    if (e_ != cudaSuccess) return cuda_fail(e_, what); \
+  } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+prox_status check_shape(int d, int F) {
+  if (d <= 0 || d % prox::kGroup != 0 || d > prox::kMaxDModel)
+    return fail(PROX_EINVAL, "d_model=%d must be a positive multiple of 128 and <= %d", d,
+                prox::kMaxDModel);
+  if (F <= 0 || F % 32 != 0 || F > prox::kMaxDff)
+    return fail(PROX_EINVAL, "d_ff=%d must be a positive multiple of 32 and <= %d", F,
+                prox::kMaxDff);
+  return PROX_OK;
+}
+
+prox_status check_device(int* dev, int* sms) {
+  PROX_CUDA(cudaGetDevice(dev), "cudaGetDevice");
+  int major = 0;
+  PROX_CUDA(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, *dev),
+            "cudaDeviceGetAttribute");
+  if (major != 10) return fail(PROX_EUNSUPPORTED, "device %d is not sm_100 (major=%d)", *dev, major);
+  PROX_CUDA(cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, *dev),
+            "cudaDeviceGetAttribute");
+  return PROX_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+void free_layer_buffers(prox_layer* L) {
+  if (L->wgu) cudaFree(L->wgu);
+  if (L->wd) cudaFree(L->wd);
+  if (L->pq) cudaFree(L->pq);
+  if (L->ps) cudaFree(L->ps);
+  if (L->ws.base) cudaFree(L->ws.base);
+  L->wgu = L->wd = nullptr;
+  L->pq = nullptr;
+  L->ps = nullptr;
+  L->ws = prox::Workspace{};
+}
+
+prox_status alloc_workspace(prox_layer* L) {
+  using prox::kHostChunkTokens;
+  const size_t d = L->d, F = L->F;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align256(bytes);
+    return o;
+  };
+  const size_t o_part = take((size_t)L->R * L->C * 1024 * 4);
+  const size_t o_scores = take(F * 4);
+  const size_t o_g = take(F * 4);
+  const size_t o_u = take(F * 4);
+  const size_t o_hist = take(prox::kHistBins * 4);
+  const size_t o_cnt = take((size_t)L->C * 4);
+  const size_t o_idx = take(F * 4);
+  const size_t o_k = take(4);
+  const size_t o_slab = take(d * 4);
+  const size_t o_slabc = take((size_t)L->R * 4);
+  const size_t o_ypart = take((size_t)L->P * d * 4);
+  const size_t o_stats = take(16);
+  const size_t o_err = take(4);
+  const size_t o_in = take((size_t)kHostChunkTokens * d * 4);
+  const size_t o_out = take((size_t)kHostChunkTokens * d * 4);
+  void* base = nullptr;
+  PROX_CUDA(cudaMalloc(&base, off), "cudaMalloc(workspace)");
+  PROX_CUDA(cudaMemset(base, 0, off), "cudaMemset(workspace)");
+  char* b = static_cast<char*>(base);
+  prox::Workspace& w = L->ws;
+  w.base = base;
+  w.bytes = off;
+  w.part = reinterpret_cast<float*>(b + o_part);
+  w.scores = reinterpret_cast<float*>(b + o_scores);
+  w.g_dbg = reinterpret_cast<float*>(b + o_g);
+  w.u_dbg = reinterpret_cast<float*>(b + o_u);
+  w.hist = reinterpret_cast<uint32_t*>(b + o_hist);
+  w.slice_cnt = reinterpret_cast<uint32_t*>(b + o_cnt);
+  w.idx_s = reinterpret_cast<int32_t*>(b + o_idx);
+  w.k_dev = reinterpret_cast<int32_t*>(b + o_k);
+  w.slab_idx = reinterpret_cast<int32_t*>(b + o_slab);
+  w.slab_cnt = reinterpret_cast<int32_t*>(b + o_slabc);
+  w.ypart = reinterpret_cast<float*>(b + o_ypart);
+  w.stats = reinterpret_cast<unsigned long long*>(b + o_stats);
+  w.err = reinterpret_cast<int*>(b + o_err);
+  w.stage_in = reinterpret_cast<float*>(b + o_in);
+  w.stage_out = reinterpret_cast<float*>(b + o_out);
+  return PROX_OK;
+}
+
+// Stage 1 -> select -> Stage 2 -> reduce for one token.
+cudaError_t enqueue_token(const prox_layer* L, const float* x, float* out, cudaStream_t s) {
+  cudaError_t e;
+  if ((e = prox::launch_stage1(L, x, prox::Stage1Taps{}, s, true)) != cudaSuccess) return e;
+  if ((e = prox::launch_select(L, prox::SelectTaps{}, s, true)) != cudaSuccess) return e;
+  if ((e = prox::launch_stage2(L, x, L->ws.idx_s, L->ws.k_dev, L->k, nullptr, s, true, true)) !=
+      cudaSuccess)
+    return e;
+  return prox::launch_reduce(L, out, s, true);
+}
+
+cudaError_t enqueue_dense(const prox_layer* L, const float* x, float* out, cudaStream_t s) {
+  cudaError_t e = prox::launch_stage2(L, x, nullptr, nullptr, L->F, nullptr, s, false, true);
+  if (e != cudaSuccess) return e;
+  return prox::launch_reduce(L, out, s, true);
+}
+
+prox_status check_layer(const prox_layer* L) {
+  if (L == nullptr) return fail(PROX_EINVAL, "layer handle is NULL");
+  int dev = -1;
+  PROX_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  if (dev != L->device)
+    return fail(PROX_EINVAL, "layer lives on device %d but device %d is current", L->device, dev);
+  return PROX_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* prox_version(void) { return "prox-b200 0.1 (sm_100a)"; }
+
+size_t prox_last_error(char* msg_host, size_t n) {
+  if (msg_host && n) {
+    const size_t m = g_last_error.size() < n - 1 ? g_last_error.size() : n - 1;
+    memcpy(msg_host, g_last_error.data(), m);
+    msg_host[m] = '\0';
+  }
+  return g_last_error.size();
+}
+
+prox_status prox_pack_proxy(const uint16_t* W, int d_model, int d_ff, int group, uint8_t* codes,
+                            uint16_t* scales, void* stream) {
+  prox_status st = check_shape(d_model, d_ff);
+  if (st != PROX_OK) return st;
+  if (group != prox::kGroup) return fail(PROX_EINVAL, "group must be 128 (got %d)", group);
+  if (!W || !codes || !scales) return fail(PROX_EINVAL, "NULL pointer");
+  if (!aligned16(W) || !aligned16(codes) || !aligned16(scales))
+    return fail(PROX_EINVAL, "pointers must be 16-byte aligned");
+  int dev, sms;
+  if ((st = check_device(&dev, &sms)) != PROX_OK) return st;
+  PROX_CUDA(prox::launch_pack_proxy(W, d_model, d_ff, codes, scales, as_stream(stream)),
+            "pack_proxy launch");
+  return PROX_OK;
+}
+
+prox_status prox_calibrate_thresholds(const float* X_cal, int n_tok, int d_model, float s1,
+                                      float* tau_host, void* stream) {
+  if (!tau_host) return fail(PROX_EINVAL, "tau_host is NULL");
+  if (!(s1 >= 0.f && s1 <= 1.f)) return fail(PROX_EINVAL, "s1=%g must be in [0, 1]", (double)s1);
+  if (n_tok <= 0 || d_model <= 0) return fail(PROX_EINVAL, "n_tok and d_model must be positive");
+  const size_t n = (size_t)n_tok * (size_t)d_model;
+  if (n >= (size_t)1 << 31) return fail(PROX_EINVAL, "at most 2^31-1 calibration values");
+  if (!X_cal || !aligned16(X_cal)) return fail(PROX_EINVAL, "X_cal must be a 16-byte aligned pointer");
+  if (s1 == 0.f) {
+    *tau_host = 0.f;
+    return PROX_OK;
+  }
+  int dev, sms;
+  prox_status st = check_device(&dev, &sms);
+  if (st != PROX_OK) return st;
+  unsigned long long rank = (unsigned long long)std::floor((double)s1 * (double)n);
+  if (rank >= n) rank = n - 1;
+  cudaStream_t s = as_stream(stream);
+  void* scratch = nullptr;
+  PROX_CUDA(cudaMallocAsync(&scratch, (prox::kHistBins + 4) * 4 + 16, s), "cudaMallocAsync");
+  uint32_t* sc = static_cast<uint32_t*>(scratch);
+  float* tau_dev = reinterpret_cast<float*>(sc + prox::kHistBins + 4);
+  cudaError_t e = prox::launch_calibrate(X_cal, n, rank, sc, tau_dev, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(tau_host, tau_dev, 4, cudaMemcpyDeviceToHost, s);
+  cudaFreeAsync(scratch, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "calibrate");
+  return PROX_OK;
+}
+
+prox_status prox_layer_create(const uint16_t* W_gate, const uint16_t* W_up, const uint16_t* W_down,
+                              int d_model, int d_ff, float tau_x, int k, int max_batch,
+                              void* stream, prox_layer** out_host) {
+  if (!out_host) return fail(PROX_EINVAL, "out_host is NULL");
+  *out_host = nullptr;
+  prox_status st = check_shape(d_model, d_ff);
+  if (st != PROX_OK) return st;
+  if (k < 1 || k > d_ff) return fail(PROX_EINVAL, "k=%d must be in [1, d_ff=%d]", k, d_ff);
+  if (max_batch < 1) return fail(PROX_EINVAL, "max_batch must be >= 1");
+  if (!(tau_x >= 0.f) || std::isinf(tau_x)) return fail(PROX_EINVAL, "tau_x must be finite and >= 0");
+  if (!W_gate || !W_up || !W_down) return fail(PROX_EINVAL, "NULL weight pointer");
+  if (!aligned16(W_gate) || !aligned16(W_up) || !aligned16(W_down))
+    return fail(PROX_EINVAL, "weight pointers must be 16-byte aligned");
+  int dev, sms;
+  if ((st = check_device(&dev, &sms)) != PROX_OK) return st;
+
+  prox_layer* L = new (std::nothrow) prox_layer();
+  if (!L) return fail(PROX_ENOMEM, "host allocation failed");
+  L->d = d_model;
+  L->F = d_ff;
+  L->G = d_model / prox::kGroup;
+  L->k = k;
+  L->max_batch = max_batch;
+  L->tau = tau_x;
+  L->device = dev;
+  L->num_sms = sms;
+  prox::choose_stage1_grid(L->d, L->F, sms, &L->C, &L->R, &L->gps);
+  prox::choose_stage2(L->d, L->F, sms, &L->P, &L->ring_slots, &L->stage2_smem);
+  L->stage1_smem = prox::stage1_smem_bytes(L->gps);
+  L->select_smem = prox::select_smem_bytes(L->F);
+
+  cudaStream_t s = as_stream(stream);
+  const size_t d = d_model, F = d_ff;
+  uint8_t *cg = nullptr, *cu = nullptr;
+  uint16_t *sg = nullptr, *su = nullptr;
+  cudaError_t e = cudaSuccess;
+  auto step = [&](cudaError_t r) {
+    if (e == cudaSuccess) e = r;
+  };
+  step(prox::setup_stage1_kernels());
+  step(prox::setup_stage2_kernels());
+  step(cudaMalloc(&L->wgu, 2 * F * d * 2));
+  step(cudaMalloc(&L->wd, F * d * 2));
+  step(cudaMalloc(&L->pq, d * F));
+  step(cudaMalloc(&L->ps, (size_t)L->G * F * 2 * 2));
+  step(cudaMalloc(&cg, d * F / 2));
+  step(cudaMalloc(&cu, d * F / 2));
+  step(cudaMalloc(&sg, (size_t)L->G * F * 2));
+  step(cudaMalloc(&su, (size_t)L->G * F * 2));
+  if (e == cudaSuccess) {
+    step(prox::launch_pack_proxy(W_gate, L->d, L->F, cg, sg, s));
+    step(prox::launch_pack_proxy(W_up, L->d, L->F, cu, su, s));
+    step(prox::launch_interleave_proxy(cg, cu, sg, su, L->d, L->F, L->pq, L->ps, s));
+    step(prox::launch_gateup_records(W_gate, W_up, L->d, L->F, L->wgu, s));
+    step(cudaMemcpyAsync(L->wd, W_down, F * d * 2, cudaMemcpyDeviceToDevice, s));
+    step(cudaStreamSynchronize(s));
+  }
+  if (cg) cudaFree(cg);
+  if (cu) cudaFree(cu);
+  if (sg) cudaFree(sg);
+  if (su) cudaFree(su);
+  if (e != cudaSuccess) {
+    free_layer_buffers(L);
+    delete L;
+    return cuda_fail(e, "prox_layer_create");
+  }
+  if ((st = alloc_workspace(L)) != PROX_OK) {
+    free_layer_buffers(L);
+    delete L;
+    return st;
+  }
+  *out_host = L;
+  return PROX_OK;
+}
+
+prox_status prox_layer_destroy(prox_layer* L) {
+  if (!L) return PROX_OK;
+  int cur = 0;
+  cudaGetDevice(&cur);
+  if (cur != L->device) cudaSetDevice(L->device);
+  free_layer_buffers(L);
+  if (cur != L->device) cudaSetDevice(cur);
+  delete L;
+  return PROX_OK;
+}
+
+prox_status prox_layer_set_tau(prox_layer* L, float tau_x) {
+  if (!L) return fail(PROX_EINVAL, "layer handle is NULL");
+  if (!(tau_x >= 0.f) || std::isinf(tau_x)) return fail(PROX_EINVAL, "tau_x must be finite and >= 0");
+  L->tau = tau_x;
+  return PROX_OK;
+}
+
+prox_status prox_layer_set_k(prox_layer* L, int k) {
+  if (!L) return fail(PROX_EINVAL, "layer handle is NULL");
+  if (k < 1 || k > L->F) return fail(PROX_EINVAL, "k=%d must be in [1, d_ff=%d]", k, L->F);
+  L->k = k;
+  return PROX_OK;
+}
+
+prox_status prox_layer_get_info(const prox_layer* L, prox_layer_info* info) {
+  if (!L || !info) return fail(PROX_EINVAL, "NULL argument");
+  info->d_model = L->d;
+  info->d_ff = L->F;
+  info->group = prox::kGroup;
+  info->k = L->k;
+  info->max_batch = L->max_batch;
+  info->tau_x = L->tau;
+  info->stage1_col_slices = L->C;
+  info->stage1_row_slabs = L->R;
+  info->stage2_ctas = L->P;
+  info->stage2_ring_slots = L->ring_slots;
+  info->weight_bytes = (size_t)3 * L->F * L->d * 2;
+  info->proxy_bytes = (size_t)L->d * L->F + (size_t)L->G * L->F * 4;
+  info->workspace_bytes = L->ws.bytes;
+  return PROX_OK;
+}
+
+prox_status prox_layer_error(prox_layer* L, int32_t* word_host, void* stream) {
+  prox_status st = check_layer(L);
+  if (st != PROX_OK) return st;
+  if (!word_host) return fail(PROX_EINVAL, "word_host is NULL");
+  cudaStream_t s = as_stream(stream);
+  int32_t v = 0;
+  PROX_CUDA(cudaMemcpyAsync(&v, L->ws.err, 4, cudaMemcpyDeviceToHost, s), "read error word");
+  PROX_CUDA(cudaMemsetAsync(L->ws.err, 0, 4, s), "clear error word");
+  PROX_CUDA(cudaStreamSynchronize(s), "cudaStreamSynchronize");
+  *word_host = v;
+  return PROX_OK;
+}
+
+prox_status prox_layer_stats(prox_layer* L, int64_t* sum_nx_host, int64_t* tokens_host,
+                             void* stream) {
+  prox_status st = check_layer(L);
+  if (st != PROX_OK) return st;
+  cudaStream_t s = as_stream(stream);
+  unsigned long long v[2] = {0, 0};
+  PROX_CUDA(cudaMemcpyAsync(v, L->ws.stats, 16, cudaMemcpyDeviceToHost, s), "read stats");
+  PROX_CUDA(cudaMemsetAsync(L->ws.stats, 0, 16, s), "clear stats");
+  PROX_CUDA(cudaStreamSynchronize(s), "cudaStreamSynchronize");
+  if (sum_nx_host) *sum_nx_host = (int64_t)v[0];
+  if (tokens_host) *tokens_host = (int64_t)v[1];
+  return PROX_OK;
+}
+
+prox_status prox_ffn_forward(const prox_layer* L, const float* x, float* out, int B,
+                             void* stream) {
+  prox_status st = check_layer(L);
+  if (st != PROX_OK) return st;
+  if (B < 1 || B > L->max_batch) return fail(PROX_EINVAL, "B=%d must be in [1, %d]", B, L->max_batch);
+  if (!x || !out || !aligned16(x) || !aligned16(out))
+    return fail(PROX_EINVAL, "x and out must be non-NULL 16-byte aligned pointers");
+  if (x == out) return fail(PROX_EINVAL, "out may not alias x");
+  cudaStream_t s = as_stream(stream);
+  for (int b = 0; b < B; ++b) {
+    cudaError_t e = enqueue_token(L, x + (size_t)b * L->d, out + (size_t)b * L->d, s);
+    if (e != cudaSuccess) return cuda_fail(e, "prox_ffn_forward launch");
+  }
+  return PROX_OK;
+}
+
+prox_status prox_dense_ffn(const prox_layer* L, const float* x, float* out, int B, void* stream) {
+  prox_status st = check_layer(L);
+  if (st != PROX_OK) return st;
+  if (B < 1 || B > L->max_batch) return fail(PROX_EINVAL, "B=%d must be in [1, %d]", B, L->max_batch);
+  if (!x || !out || !aligned16(x) || !aligned16(out))
+    return fail(PROX_EINVAL, "x and out must be non-NULL 16-byte aligned pointers");
+  cudaStream_t s = as_stream(stream);
+  for (int b = 0; b < B; ++b) {
+    cudaError_t e = enqueue_dense(L, x + (size_t)b * L->d, out + (size_t)b * L->d, s);
+    if (e != cudaSuccess) return cuda_fail(e, "prox_dense_ffn launch");
+  }
+  return PROX_OK;
+}
+
+prox_status prox_ffn_forward_host(prox_layer* L, const float* x_host, float* out_host, int n_tok,
+                                  void* stream) {
+  prox_status st = check_layer(L);
+  if (st != PROX_OK) return st;
+  if (!x_host || !out_host || n_tok < 0) return fail(PROX_EINVAL, "bad host buffers");
+  cudaStream_t s = as_stream(stream);
+  const size_t d = L->d;
+  for (int t0 = 0; t0 < n_tok; t0 += prox::kHostChunkTokens) {
+    const int n = n_tok - t0 < prox::kHostChunkTokens ? n_tok - t0 : prox::kHostChunkTokens;
+    PROX_CUDA(cudaMemcpyAsync(L->ws.stage_in, x_host + t0 * d, n * d * 4,
+                              cudaMemcpyHostToDevice, s),
+              "H2D copy");
+    for (int t = 0; t < n; ++t) {
+      cudaError_t e = enqueue_token(L, L->ws.stage_in + t * d, L->ws.stage_out + t * d, s);
+      if (e != cudaSuccess) return cuda_fail(e, "prox_ffn_forward_host launch");
+    }
+    PROX_CUDA(cudaMemcpyAsync(out_host + t0 * d, L->ws.stage_out, n * d * 4,
+                              cudaMemcpyDeviceToHost, s),
+              "D2H copy");
+  }
+  PROX_CUDA(cudaStreamSynchronize(s), "cudaStreamSynchronize");
+  return PROX_OK;
+}
+
+prox_status prox_ffn_forward_profiled(const prox_layer* L, const float* x, float* out,
+                                      void* const* events, void* stream) {
+  prox_status st = check_layer(L);
+  if (st != PROX_OK) return st;
+  if (!events || !x || !out) return fail(PROX_EINVAL, "NULL argument");
+  cudaStream_t s = as_stream(stream);
+  auto ev = [&](int i) { return reinterpret_cast<cudaEvent_t>(events[i]); };
+  PROX_CUDA(cudaEventRecord(ev(0), s), "cudaEventRecord");
+  PROX_CUDA(prox::launch_stage1(L, x, prox::Stage1Taps{}, s, false), "stage1 launch");
+  PROX_CUDA(prox::launch_select(L, prox::SelectTaps{}, s, false), "select launch");
+  PROX_CUDA(cudaEventRecord(ev(1), s), "cudaEventRecord");
+  PROX_CUDA(prox::launch_stage2(L, x, L->ws.idx_s, L->ws.k_dev, L->k, nullptr, s, false, true),
+            "stage2 launch");
+  PROX_CUDA(cudaEventRecord(ev(2), s), "cudaEventRecord");
+  PROX_CUDA(prox::launch_reduce(L, out, s, false), "reduce launch");
+  PROX_CUDA(cudaEventRecord(ev(3), s), "cudaEventRecord");
+  return PROX_OK;
+}
+
+prox_status prox_debug_stage1(prox_layer* L, const float* x, int32_t* idx_x, int32_t* n_x,
+                              float* g_tilde, float* u_tilde, int32_t* idx_s, void* stream) {
+  prox_status st = check_layer(L);
+  if (st != PROX_OK) return st;
+  if (!x || !aligned16(x)) return fail(PROX_EINVAL, "x must be a 16-byte aligned pointer");
+  cudaStream_t s = as_stream(stream);
+  prox::Stage1Taps t1;
+  t1.g = g_tilde;
+  t1.u = u_tilde;
+  t1.slabs = idx_x != nullptr || n_x != nullptr;
+  prox::SelectTaps t2;
+  int32_t* nx_dev = n_x;
+  if (t1.slabs) {
+    t2.idx_x = idx_x ? idx_x : L->ws.slab_idx;  // idx_x NULL: only count
+    t2.n_x = nx_dev;
+  }
+  if (t1.slabs && !idx_x) {
+    // Without an idx_x buffer the concatenation would overwrite the slab lists
+    // it reads; write it to the (unused) staging area instead.
+    t2.idx_x = reinterpret_cast<int32_t*>(L->ws.stage_in);
+  }
+  PROX_CUDA(prox::launch_stage1(L, x, t1, s, false), "stage1 launch");
+  PROX_CUDA(prox::launch_select(L, t2, s, false), "select launch");
+  if (idx_s)
+    PROX_CUDA(cudaMemcpyAsync(idx_s, L->ws.idx_s, (size_t)L->k * 4, cudaMemcpyDeviceToDevice, s),
+              "copy idx_s");
+  return PROX_OK;
+}
+
+prox_status prox_forward_with_mask(prox_layer* L, const float* x, const int32_t* idx_s, int k,
+                                   float* out, float* s_sp, void* stream) {
+  prox_status st = check_layer(L);
+  if (st != PROX_OK) return st;
+  if (k < 1 || k > L->F) return fail(PROX_EINVAL, "k=%d must be in [1, d_ff=%d]", k, L->F);
+  if (!x || !out || !idx_s || !aligned16(x) || !aligned16(out))
+    return fail(PROX_EINVAL, "bad pointer");
+  cudaStream_t s = as_stream(stream);
+  PROX_CUDA(prox::launch_stage2(L, x, idx_s, nullptr, k, s_sp, s, false, true), "stage2 launch");
+  PROX_CUDA(prox::launch_reduce(L, out, s, true), "reduce launch");
+  return PROX_OK;
+}
+
+prox_status prox_rmsnorm(const float* y, float* x_out, int rows, int d, float eps, void* stream) {
+  if (!y || !x_out || rows < 1 || d < 1 || !(eps >= 0.f))
+    return fail(PROX_EINVAL, "bad rmsnorm arguments");
+  PROX_CUDA(prox::launch_rmsnorm(y, x_out, rows, d, eps, as_stream(stream)), "rmsnorm launch");
+  return PROX_OK;
+}
+
+prox_status prox_copy(const void* src, void* dst, size_t bytes, void* stream) {
+  if (!src || !dst || (bytes & 15u) || !aligned16(src) || !aligned16(dst))
+    return fail(PROX_EINVAL, "copy needs 16-byte aligned pointers and a multiple of 16 bytes");
+  PROX_CUDA(prox::launch_copy(src, dst, bytes, as_stream(stream)), "copy launch");
+  return PROX_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,112 @@
+// Host-side internals of the Prox library: the layer handle, its buffers and
+// the kernel launchers that the C ABI (prox_api.cu) strings together.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "prox.h"
+
+namespace prox {
+
+constexpr int kGroup = 128;          // proxy quantisation group (input rows)
+constexpr int kHistBins = 2048;      // first radix level: score bits [30:20]
+constexpr int kStage1Warps = 4;      // Stage-1 CTA = 4 warps on one column slice
+constexpr int kMaxGroupsPerSlab = 32; // bounds Stage-1 shared memory (115 KB)
+constexpr int kSelectThreads = 1024; // top-k select CTA
+constexpr int kStage2Consumers = 8;  // Stage-2 consumer warps (+1 producer warp)
+constexpr int kReduceWarps = 8;      // output reduction: warps per 32 columns
+constexpr int kMaxDModel = 16384;
+constexpr int kMaxDff = 49152;       // select keeps all scores in shared memory
+constexpr int kHostChunkTokens = 64; // staging chunk of prox_ffn_forward_host
+
+// Per-token scratch of one layer (device memory owned by the handle).
+struct Workspace {
+  float* part = nullptr;          // Stage-1 partial sums [R][C][1024]
+  float* scores = nullptr;        // |SiLU(g~) u~| [F]
+  float* g_dbg = nullptr;         // debug g~ [F]
+  float* u_dbg = nullptr;         // debug u~ [F]
+  uint32_t* hist = nullptr;       // [kHistBins], zero between tokens
+  uint32_t* slice_cnt = nullptr;  // [C] tickets, zero between tokens
+  int32_t* idx_s = nullptr;       // [F] selected channels (first k valid)
+  int32_t* k_dev = nullptr;       // [1] number of selected channels
+  int32_t* slab_idx = nullptr;    // [d] kept input rows, per slab (debug)
+  int32_t* slab_cnt = nullptr;    // [R] kept rows per slab (debug)
+  float* ypart = nullptr;         // Stage-2 output partials [P][d]
+  unsigned long long* stats = nullptr;  // [2] sum n_x, tokens
+  int* err = nullptr;             // device error word
+  float* stage_in = nullptr;      // host-path staging [kHostChunkTokens][d]
+  float* stage_out = nullptr;
+  void* base = nullptr;           // single allocation holding all of the above
+  size_t bytes = 0;
+};
+
+}  // namespace prox
+
+struct prox_layer {
+  int d = 0, F = 0, G = 0, k = 0, max_batch = 0;
+  float tau = 0.f;
+  int device = 0, num_sms = 0;
+  // Stage-1 geometry
+  int C = 0, R = 0, gps = 0;
+  // Stage-2 geometry
+  int P = 0, ring_slots = 0;
+  size_t stage2_smem = 0, stage1_smem = 0, select_smem = 0;
+  // library-owned weights
+  uint16_t* wgu = nullptr;   // bf16 [F][2d]: gate column j | up column j
+  uint16_t* wd = nullptr;    // bf16 [F][d]
+  uint8_t* pq = nullptr;     // INT4 codes [d][F], gate/up interleaved per 16 B
+  uint16_t* ps = nullptr;    // fp16 scales [G][F/32][2][32]
+  prox::Workspace ws;
+};
+
+namespace prox {
+
+// ---- launchers (each returns the CUDA error of its launch) ----------------
+struct Stage1Taps {
+  float* g = nullptr;
+  float* u = nullptr;
+  bool slabs = false;  // write per-slab kept-row lists
+};
+struct SelectTaps {
+  int32_t* idx_x = nullptr;  // concatenated kept rows
+  int32_t* n_x = nullptr;
+};
+
+cudaError_t launch_stage1(const prox_layer* L, const float* x, const Stage1Taps& taps,
+                          cudaStream_t s, bool pdl);
+cudaError_t launch_select(const prox_layer* L, const SelectTaps& taps, cudaStream_t s,
+                          bool pdl);
+// idx == nullptr: dense (every channel, k = F).  k_dev != nullptr: k is read
+// on the device after the dependency wait; otherwise k_host is used.
+cudaError_t launch_stage2(const prox_layer* L, const float* x, const int32_t* idx,
+                          const int32_t* k_dev, int k_host, float* s_sp, cudaStream_t s,
+                          bool pdl, bool x_ready);
+cudaError_t launch_reduce(const prox_layer* L, float* out, cudaStream_t s, bool pdl);
+
+cudaError_t launch_pack_proxy(const uint16_t* W, int d, int F, uint8_t* codes,
+                              uint16_t* scales, cudaStream_t s);
+cudaError_t launch_interleave_proxy(const uint8_t* cg, const uint8_t* cu, const uint16_t* sg,
+                                    const uint16_t* su, int d, int F, uint8_t* pq,
+                                    uint16_t* ps, cudaStream_t s);
+cudaError_t launch_gateup_records(const uint16_t* Wg, const uint16_t* Wu, int d, int F,
+                                  uint16_t* wgu, cudaStream_t s);
+
+// Calibration: exact order statistic of |X| at 0-based ascending rank `rank`.
+// `scratch` holds kHistBins + 4 uint32 (zeroed by the caller).
+cudaError_t launch_calibrate(const float* X, size_t n, unsigned long long rank,
+                             uint32_t* scratch, float* tau_dev, cudaStream_t s);
+
+cudaError_t launch_rmsnorm(const float* y, float* x, int rows, int d, float eps,
+                           cudaStream_t s);
+cudaError_t launch_copy(const void* src, void* dst, size_t bytes, cudaStream_t s);
+
+// Stage-1 column slices and row slabs for a shape on `num_sms` SMs.
+void choose_stage1_grid(int d, int F, int num_sms, int* C, int* R, int* gps);
+size_t stage1_smem_bytes(int gps);
+size_t select_smem_bytes(int F);
+// Stage-2 ring depth and dynamic shared memory for d_model = d.
+void choose_stage2(int d, int F, int num_sms, int* P, int* slots, size_t* smem);
+
+}  // namespace prox

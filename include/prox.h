@@ -1,0 +1,214 @@
+/*
+ * prox.h -- C ABI of the B200 (sm_100a) Prox sparse SwiGLU FFN decode step.
+ *
+ * Source of every operation below: "Prox: Training-Free FFN Activation
+ * Sparsity via Approximate Intermediate-Channel Salience in LLMs" (Liu et al.),
+ * cited as *Prox* with its section or equation.
+ *
+ * Conventions shared by all entry points
+ * --------------------------------------
+ *  - Pointers are DEVICE pointers unless the parameter name ends in `_host`.
+ *  - bf16 and fp16 values are passed as their uint16_t bit patterns.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    All work is enqueued on it in stream order; functions whose comment says
+ *    "synchronises" wait for the stream before returning.
+ *  - The caller owns every buffer it passes and must keep it alive until the
+ *    enqueued work has finished.  The library owns the layer handle, its
+ *    repacked weights and its workspace (allocated in prox_layer_create, freed
+ *    in prox_layer_destroy); prox_ffn_forward and prox_dense_ffn allocate
+ *    nothing and never synchronise.
+ *  - Weight shapes are in math layout: W_gate, W_up are [d_model, d_ff] and
+ *    W_down is [d_ff, d_model], all row-major.  Activations are fp32.
+ *  - Shape rules (else PROX_EINVAL, checked before any launch):
+ *    d_model > 0 and d_model % 128 == 0; d_ff > 0 and d_ff % 32 == 0;
+ *    d_model <= 16384; d_ff <= 49152; 1 <= k <= d_ff; pointers 16-byte aligned.
+ *  - Errors: every call returns a prox_status; prox_last_error() copies a
+ *    message for the calling thread's last failure.  No C++ exception crosses
+ *    this boundary.  Device-side checks (an index out of range in a caller's
+ *    mask, a bounded wait that ran out) never trap: they set the layer's error
+ *    word, read with prox_layer_error().
+ *  - A layer handle is used by one stream at a time (its workspace is shared
+ *    by the calls on it).
+ */
+#ifndef PROX_H_
+#define PROX_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PROX_API __attribute__((visibility("default")))
+#else
+#define PROX_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum prox_status {
+  PROX_OK = 0,
+  PROX_EINVAL = 1,       /* bad argument (shape, pointer, k, s1 ...) */
+  PROX_ENOMEM = 2,       /* device allocation failed */
+  PROX_ECUDA = 3,        /* a CUDA runtime call failed */
+  PROX_EUNSUPPORTED = 4, /* device is not sm_100 or a limit is exceeded */
+  PROX_EDEVICE = 5       /* a device-side check fired (see prox_layer_error) */
+} prox_status;
+
+/* Device error word bits (prox_layer_error). */
+#define PROX_DEVERR_MASK_INDEX 0x1  /* a channel index outside [0, d_ff) */
+#define PROX_DEVERR_WAIT_TIMEOUT 0x2 /* a bounded pipeline wait ran out */
+
+typedef struct prox_layer prox_layer; /* opaque */
+
+/* Static description of a created layer (all host values). */
+typedef struct prox_layer_info {
+  int d_model, d_ff, group, k, max_batch;
+  float tau_x;
+  int stage1_col_slices, stage1_row_slabs; /* Stage-1 grid (C x R)          */
+  int stage2_ctas, stage2_ring_slots;      /* Stage-2 grid and TMA ring depth */
+  size_t weight_bytes;    /* bf16 gate/up records + bf16 W_down             */
+  size_t proxy_bytes;     /* INT4 codes + fp16 scales                        */
+  size_t workspace_bytes; /* scratch owned by the handle                     */
+} prox_layer_info;
+
+/* ------------------------------------------------------------------------
+ * Offline preparation
+ * ------------------------------------------------------------------------ */
+
+/* INT4 proxy of one weight matrix (Prox §4.3 "Hardware-Aware Implementation":
+ * symmetric INT4 proxies of W_up and W_gate kept resident on the GPU; this
+ * build quantises in groups of `group` consecutive input rows per channel).
+ *
+ * For every group g of rows and channel j:
+ *   amax = max_{i in g} |W[i,j]|,  S[g,j] = fp16_nearest_even(amax / 7),
+ *   Q[i,j] = clamp(round_half_even(W[i,j] / S[g,j]), -7, 7)   (0 when S = 0).
+ * W: bf16 [d_model, d_ff].  codes: uint8 [d_model, d_ff/2]; byte b of row i
+ * holds channel 2b in its low nibble and 2b+1 in its high nibble, each stored
+ * as Q + 8.  scales: fp16 [d_model/group, d_ff].  group must be 128.
+ * amax/7 must be finite in fp16 (|W| < 458752).  Stream-ordered; no sync. */
+PROX_API prox_status prox_pack_proxy(const uint16_t* W, int d_model, int d_ff, int group,
+                            uint8_t* codes, uint16_t* scales, void* stream);
+
+/* Per-layer Stage-1 input threshold (Prox App. A.7 "Calibration data and
+ * scale": the threshold is the empirical quantile of the calibration
+ * activations; §4.1 uses it as tau_x).
+ *
+ * tau = the order statistic of rank floor(s1 * n) (0-based, ascending) of the
+ * n = n_tok * d_model values |X_cal|; s1 = 0 gives tau = 0.  Exact (radix
+ * select on the fp32 bit patterns).  X_cal: fp32 [n_tok, d_model] on the
+ * device.  tau_host: one float written on return.  Allocates its scratch
+ * (a few KB) stream-ordered and synchronises the stream. */
+PROX_API prox_status prox_calibrate_thresholds(const float* X_cal, int n_tok, int d_model, float s1,
+                                      float* tau_host, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Layer handle
+ * ------------------------------------------------------------------------ */
+
+/* Repack one SwiGLU FFN layer into library-owned buffers:
+ *  - gate/up channel records: record j = [W_gate[:, j] | W_up[:, j]], bf16;
+ *  - W_down rows (bf16 [d_ff, d_model], unchanged);
+ *  - INT4 proxies of W_gate and W_up (prox_pack_proxy), interleaved so that
+ *    one input row i of both proxies is a single contiguous run of d_ff bytes;
+ *  - workspace for max_batch tokens.
+ * tau_x: Stage-1 threshold; k: channels kept per token by the top-k mask.
+ * Inputs may be freed once the call returns (it synchronises `stream`). */
+PROX_API prox_status prox_layer_create(const uint16_t* W_gate, const uint16_t* W_up,
+                              const uint16_t* W_down, int d_model, int d_ff, float tau_x,
+                              int k, int max_batch, void* stream, prox_layer** out_host);
+
+PROX_API prox_status prox_layer_destroy(prox_layer* layer);
+
+/* Change the threshold or k of an existing layer (host-side; affects calls
+ * enqueued afterwards). */
+PROX_API prox_status prox_layer_set_tau(prox_layer* layer, float tau_x);
+PROX_API prox_status prox_layer_set_k(prox_layer* layer, int k);
+
+PROX_API prox_status prox_layer_get_info(const prox_layer* layer, prox_layer_info* info_host);
+
+/* Reads (and clears) the layer's device error word; synchronises `stream`. */
+PROX_API prox_status prox_layer_error(prox_layer* layer, int32_t* word_host, void* stream);
+
+/* Realised Stage-1 statistics accumulated since the last call: the sum of
+ * n_x over tokens and the number of tokens (realised s1 = 1 - sum/(tokens*d)),
+ * Prox App. A.7 "Runtime sparsity".  Synchronises `stream` and resets. */
+PROX_API prox_status prox_layer_stats(prox_layer* layer, int64_t* sum_nx_host, int64_t* tokens_host,
+                             void* stream);
+
+/* ------------------------------------------------------------------------
+ * The decode step
+ * ------------------------------------------------------------------------ */
+
+/* Prox two-stage sparse FFN (Prox §4.1), B tokens each with its own masks:
+ *   Stage 1: m_x = 1[|x_i| >= tau_x]; g~ = Π_in(x, W~_gate, m_x),
+ *            u~ = Π_in(x, W~_up, m_x); score_j = |SiLU(g~_j) u~_j|;
+ *            idx_s = the k channels of largest score, ties to the lower
+ *            index (Prox App. A.6, per-token top-k), ascending.
+ *   Stage 2: for j in idx_s: s_j = SiLU(x W_gate[:, j]) (x W_up[:, j]) with the
+ *            full x; out = sum_j s_j W_down[j, :].
+ * x, out: fp32 [B, d_model] (out may not alias x).  B <= max_batch.
+ * Three kernels per token, chained with programmatic dependent launch. */
+PROX_API prox_status prox_ffn_forward(const prox_layer* layer, const float* x, float* out, int B,
+                             void* stream);
+
+/* Dense SwiGLU baseline FFN(x) = (x W_up ⊙ SiLU(x W_gate)) W_down (Prox §2.1),
+ * on the same bf16 buffers (Stage 2 with every channel kept). */
+PROX_API prox_status prox_dense_ffn(const prox_layer* layer, const float* x, float* out, int B,
+                           void* stream);
+
+/* Same as prox_ffn_forward for n_tok tokens whose inputs and outputs live in
+ * HOST memory (pinned memory makes the copies asynchronous): copies each
+ * chunk of tokens to the device, runs the step and copies the results back.
+ * Synchronises `stream` before returning. */
+PROX_API prox_status prox_ffn_forward_host(prox_layer* layer, const float* x_host, float* out_host,
+                                  int n_tok, void* stream);
+
+/* prox_ffn_forward for one token with cudaEvent_t events[4] (passed as void*)
+ * recorded before Stage 1, between Stage 1 and Stage 2, between Stage 2 and
+ * the output reduction, and after it; the kernels are then serialised
+ * (no programmatic overlap) so each interval is one kernel's duration. */
+PROX_API prox_status prox_ffn_forward_profiled(const prox_layer* layer, const float* x, float* out,
+                                      void* const* events_host, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Test taps: the same kernels, exposing intermediate results
+ * ------------------------------------------------------------------------ */
+
+/* Stage 1 of one token.  idx_x: int32 [d_model] (first n_x entries valid,
+ * ascending); n_x: one int32; g_tilde, u_tilde: fp32 [d_ff] proxy
+ * pre-activations; idx_s: int32 [k], ascending.  Any output may be NULL. */
+PROX_API prox_status prox_debug_stage1(prox_layer* layer, const float* x, int32_t* idx_x, int32_t* n_x,
+                              float* g_tilde, float* u_tilde, int32_t* idx_s, void* stream);
+
+/* Stage 2 of one token on a caller-given channel list idx_s (int32 [k], any
+ * order, entries in [0, d_ff)); s_sp (fp32 [k], may be NULL) receives
+ * SiLU(g) u for each listed channel. */
+PROX_API prox_status prox_forward_with_mask(prox_layer* layer, const float* x, const int32_t* idx_s,
+                                   int k, float* out, float* s_sp, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Harness kernels
+ * ------------------------------------------------------------------------ */
+
+/* Unit-gain RMSNorm y / sqrt(mean(y^2) + eps) of `rows` vectors of length d,
+ * used to chain stacked layers (not part of the paper's FFN). */
+PROX_API prox_status prox_rmsnorm(const float* y, float* x_out, int rows, int d, float eps,
+                         void* stream);
+
+/* Streaming device copy of `bytes` (multiple of 16, 16-byte aligned) used to
+ * measure the HBM copy bandwidth that rooflines are quoted against. */
+PROX_API prox_status prox_copy(const void* src, void* dst, size_t bytes, void* stream);
+
+/* Copies the calling thread's last error message into msg_host (NUL-terminated,
+ * at most n bytes); returns the full message length. */
+PROX_API size_t prox_last_error(char* msg_host, size_t n);
+
+/* Library version string (static storage). */
+PROX_API const char* prox_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PROX_H_ */

@@ -77,13 +77,13 @@ def pi_in(x, w, idx):
     ``idx`` is I(m), the retained input indices.
     """
     idx = np.asarray(idx, dtype=np.int64)
-    return np.asarray(x, dtype=F64)[idx] @ np.asarray(w, dtype=F64)[idx, :]
+    return np.asarray(x, dtype=F64)[idx] @ np.asarray(w)[idx, :].astype(F64)
 
 
 def pi_out(x, w, idx):
     """Output sparsity Π_out(x, W, m) = x W[:, I(m)]  (Prox §2.2)."""
     idx = np.asarray(idx, dtype=np.int64)
-    return np.asarray(x, dtype=F64) @ np.asarray(w, dtype=F64)[:, idx]
+    return np.asarray(x, dtype=F64) @ np.asarray(w)[:, idx].astype(F64)
 
 
 # ---------------------------------------------------------------------------
@@ -244,7 +244,7 @@ def stage2(x, w_gate, w_up, w_down, idx_s):
     u_sp = pi_out(x, w_up, idx_s)
     h_sp = silu(pi_out(x, w_gate, idx_s))
     s_sp = u_sp * h_sp
-    y = s_sp @ np.asarray(w_down, dtype=F64)[idx_s, :]
+    y = s_sp @ np.asarray(w_down)[idx_s, :].astype(F64)
     return y, s_sp
 
 

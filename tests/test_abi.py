@@ -1,0 +1,72 @@
+"""The C-ABI library loads, exports every symbol include/prox.h declares, and
+rejects bad arguments on the host before touching a GPU."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "prox.h")).read()
+    return sorted(set(re.findall(r"PROX_API\s+[\w\s\*]+?\b(prox_\w+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def plib():
+    from activation_sparse_swiglu_b200 import _lib
+    return _lib
+
+
+def test_header_symbols_are_exported(plib):
+    declared = _declared()
+    assert len(declared) >= 15
+    raw = ctypes.CDLL(plib.LIB_PATH)
+    for name in declared:
+        assert hasattr(raw, name), name
+    assert set(declared) == set(plib.SIGNATURES)
+
+
+def test_version(plib):
+    assert b"sm_100a" in plib.lib.prox_version()
+
+
+def test_host_side_argument_checks(plib):
+    lib = plib.lib
+    h = ctypes.c_void_p(0)
+    p = ctypes.c_void_p(16)
+    # d_model not a multiple of 128
+    st = lib.prox_layer_create(p, p, p, 100, 64, 0.5, 8, 1, None, ctypes.byref(h))
+    assert st == plib.PROX_EINVAL and "d_model" in plib.last_error()
+    # d_ff not a multiple of 32
+    st = lib.prox_layer_create(p, p, p, 128, 40, 0.5, 8, 1, None, ctypes.byref(h))
+    assert st == plib.PROX_EINVAL and "d_ff" in plib.last_error()
+    # k out of range
+    st = lib.prox_layer_create(p, p, p, 128, 64, 0.5, 65, 1, None, ctypes.byref(h))
+    assert st == plib.PROX_EINVAL and "k=" in plib.last_error()
+    st = lib.prox_layer_create(p, p, p, 128, 64, 0.5, 0, 1, None, ctypes.byref(h))
+    assert st == plib.PROX_EINVAL
+    # negative threshold, unaligned pointer
+    st = lib.prox_layer_create(p, p, p, 128, 64, -1.0, 8, 1, None, ctypes.byref(h))
+    assert st == plib.PROX_EINVAL
+    st = lib.prox_layer_create(ctypes.c_void_p(18), p, p, 128, 64, 0.5, 8, 1, None,
+                               ctypes.byref(h))
+    assert st == plib.PROX_EINVAL and "aligned" in plib.last_error()
+    # packer: only group 128
+    assert lib.prox_pack_proxy(p, 128, 64, 64, p, p, None) == plib.PROX_EINVAL
+    # calibration: s1 outside [0, 1]
+    tau = ctypes.c_float(1.0)
+    assert lib.prox_calibrate_thresholds(p, 4, 128, 1.5, ctypes.byref(tau), None) == plib.PROX_EINVAL
+    # s1 = 0 needs no device work and gives tau = 0
+    assert lib.prox_calibrate_thresholds(p, 4, 128, 0.0, ctypes.byref(tau), None) == plib.PROX_OK
+    assert tau.value == 0.0
+    # NULL handles
+    assert lib.prox_ffn_forward(None, p, p, 1, None) == plib.PROX_EINVAL
+    assert lib.prox_dense_ffn(None, p, p, 1, None) == plib.PROX_EINVAL
+    assert lib.prox_layer_set_k(None, 3) == plib.PROX_EINVAL
+    assert lib.prox_layer_destroy(None) == plib.PROX_OK
+    # copy: size must be a multiple of 16
+    assert lib.prox_copy(p, p, 20, None) == plib.PROX_EINVAL
