@@ -89,14 +89,16 @@ prox_status alloc_workspace(prox_layer* L) {
     off += align256(bytes);
     return o;
   };
-  const size_t o_part = take((size_t)L->R * L->C * 1024 * 4);
   const size_t o_scores = take(F * 4);
   const size_t o_g = take(F * 4);
   const size_t o_u = take(F * 4);
   const size_t o_hist = take(prox::kHistBins * 4);
-  const size_t o_cnt = take((size_t)L->C * 4);
+  const size_t o_sst = take(8 * 4);
+  const size_t o_ck = take(prox::kSelectCand * 4);
+  const size_t o_ci = take(prox::kSelectCand * 4);
+  const size_t o_gt1 = take(prox::kMaxSlices * 4);
+  const size_t o_off = take((prox::kMaxSlices + 1) * 4);
   const size_t o_idx = take(F * 4);
-  const size_t o_k = take(4);
   const size_t o_slab = take(d * 4);
   const size_t o_slabc = take((size_t)L->R * 4);
   const size_t o_ypart = take((size_t)L->P * d * 4);
@@ -111,14 +113,17 @@ prox_status alloc_workspace(prox_layer* L) {
   prox::Workspace& w = L->ws;
   w.base = base;
   w.bytes = off;
-  w.part = reinterpret_cast<float*>(b + o_part);
   w.scores = reinterpret_cast<float*>(b + o_scores);
   w.g_dbg = reinterpret_cast<float*>(b + o_g);
   w.u_dbg = reinterpret_cast<float*>(b + o_u);
   w.hist = reinterpret_cast<uint32_t*>(b + o_hist);
-  w.slice_cnt = reinterpret_cast<uint32_t*>(b + o_cnt);
+  w.sel.hist = w.hist;
+  w.sel.state = reinterpret_cast<uint32_t*>(b + o_sst);
+  w.sel.cand_key = reinterpret_cast<uint32_t*>(b + o_ck);
+  w.sel.cand_idx = reinterpret_cast<int32_t*>(b + o_ci);
+  w.sel.sl_gt1 = reinterpret_cast<int32_t*>(b + o_gt1);
+  w.sel.sl_off = reinterpret_cast<int32_t*>(b + o_off);
   w.idx_s = reinterpret_cast<int32_t*>(b + o_idx);
-  w.k_dev = reinterpret_cast<int32_t*>(b + o_k);
   w.slab_idx = reinterpret_cast<int32_t*>(b + o_slab);
   w.slab_cnt = reinterpret_cast<int32_t*>(b + o_slabc);
   w.ypart = reinterpret_cast<float*>(b + o_ypart);
@@ -129,19 +134,28 @@ prox_status alloc_workspace(prox_layer* L) {
   return PROX_OK;
 }
 
-// Stage 1 -> select -> Stage 2 -> reduce for one token.
+prox::Stage2Launch topk_launch(const prox_layer* L) {
+  prox::Stage2Launch m;
+  m.mode = 1;
+  m.k = L->k;
+  m.idx_out = L->ws.idx_s;
+  return m;
+}
+
+// Stage 1 -> select -> Stage 2 (gate/up + down) -> output reduction, one token.
 cudaError_t enqueue_token(const prox_layer* L, const float* x, float* out, cudaStream_t s) {
   cudaError_t e;
   if ((e = prox::launch_stage1(L, x, prox::Stage1Taps{}, s, true)) != cudaSuccess) return e;
-  if ((e = prox::launch_select(L, prox::SelectTaps{}, s, true)) != cudaSuccess) return e;
-  if ((e = prox::launch_stage2(L, x, L->ws.idx_s, L->ws.k_dev, L->k, nullptr, s, true, true)) !=
-      cudaSuccess)
-    return e;
+  if ((e = prox::launch_select(L, s, true)) != cudaSuccess) return e;
+  if ((e = prox::launch_stage2(L, x, topk_launch(L), s, true, true)) != cudaSuccess) return e;
   return prox::launch_reduce(L, out, s, true);
 }
 
 cudaError_t enqueue_dense(const prox_layer* L, const float* x, float* out, cudaStream_t s) {
-  cudaError_t e = prox::launch_stage2(L, x, nullptr, nullptr, L->F, nullptr, s, false, true);
+  prox::Stage2Launch m;
+  m.mode = 2;
+  m.k = L->F;
+  cudaError_t e = prox::launch_stage2(L, x, m, s, false, true);
   if (e != cudaSuccess) return e;
   return prox::launch_reduce(L, out, s, true);
 }
@@ -242,9 +256,9 @@ prox_status prox_layer_create(const uint16_t* W_gate, const uint16_t* W_up, cons
   L->device = dev;
   L->num_sms = sms;
   prox::choose_stage1_grid(L->d, L->F, sms, &L->C, &L->R, &L->gps);
-  prox::choose_stage2(L->d, L->F, sms, &L->P, &L->ring_slots, &L->stage2_smem);
+  prox::choose_stage2(L->d, L->F, sms, &L->P, &L->ring_slots, &L->stage2_producers,
+                     &L->stage2_smem);
   L->stage1_smem = prox::stage1_smem_bytes(L->gps);
-  L->select_smem = prox::select_smem_bytes(L->F);
 
   cudaStream_t s = as_stream(stream);
   const size_t d = d_model, F = d_ff;
@@ -423,10 +437,9 @@ prox_status prox_ffn_forward_profiled(const prox_layer* L, const float* x, float
   auto ev = [&](int i) { return reinterpret_cast<cudaEvent_t>(events[i]); };
   PROX_CUDA(cudaEventRecord(ev(0), s), "cudaEventRecord");
   PROX_CUDA(prox::launch_stage1(L, x, prox::Stage1Taps{}, s, false), "stage1 launch");
-  PROX_CUDA(prox::launch_select(L, prox::SelectTaps{}, s, false), "select launch");
+  PROX_CUDA(prox::launch_select(L, s, false), "select launch");
   PROX_CUDA(cudaEventRecord(ev(1), s), "cudaEventRecord");
-  PROX_CUDA(prox::launch_stage2(L, x, L->ws.idx_s, L->ws.k_dev, L->k, nullptr, s, false, true),
-            "stage2 launch");
+  PROX_CUDA(prox::launch_stage2(L, x, topk_launch(L), s, false, true), "stage2 launch");
   PROX_CUDA(cudaEventRecord(ev(2), s), "cudaEventRecord");
   PROX_CUDA(prox::launch_reduce(L, out, s, false), "reduce launch");
   PROX_CUDA(cudaEventRecord(ev(3), s), "cudaEventRecord");
@@ -443,19 +456,17 @@ prox_status prox_debug_stage1(prox_layer* L, const float* x, int32_t* idx_x, int
   t1.g = g_tilde;
   t1.u = u_tilde;
   t1.slabs = idx_x != nullptr || n_x != nullptr;
-  prox::SelectTaps t2;
-  int32_t* nx_dev = n_x;
-  if (t1.slabs) {
-    t2.idx_x = idx_x ? idx_x : L->ws.slab_idx;  // idx_x NULL: only count
-    t2.n_x = nx_dev;
-  }
-  if (t1.slabs && !idx_x) {
-    // Without an idx_x buffer the concatenation would overwrite the slab lists
-    // it reads; write it to the (unused) staging area instead.
-    t2.idx_x = reinterpret_cast<int32_t*>(L->ws.stage_in);
-  }
   PROX_CUDA(prox::launch_stage1(L, x, t1, s, false), "stage1 launch");
-  PROX_CUDA(prox::launch_select(L, t2, s, false), "select launch");
+  PROX_CUDA(prox::launch_select(L, s, false), "select launch");
+  // the rank-to-channel step of the forward path, stopped before the weight streaming
+  prox::Stage2Launch m = topk_launch(L);
+  m.select_only = true;
+  PROX_CUDA(prox::launch_stage2(L, x, m, s, false, true), "stage2 launch");
+  PROX_CUDA(cudaMemsetAsync(L->ws.hist, 0, prox::kHistBins * 4, s), "clear histogram");
+  if (t1.slabs) {
+    int32_t* ix = idx_x ? idx_x : reinterpret_cast<int32_t*>(L->ws.stage_in);
+    PROX_CUDA(prox::launch_concat_slabs(L, ix, n_x, s), "concat launch");
+  }
   if (idx_s)
     PROX_CUDA(cudaMemcpyAsync(idx_s, L->ws.idx_s, (size_t)L->k * 4, cudaMemcpyDeviceToDevice, s),
               "copy idx_s");
@@ -470,7 +481,12 @@ prox_status prox_forward_with_mask(prox_layer* L, const float* x, const int32_t*
   if (!x || !out || !idx_s || !aligned16(x) || !aligned16(out))
     return fail(PROX_EINVAL, "bad pointer");
   cudaStream_t s = as_stream(stream);
-  PROX_CUDA(prox::launch_stage2(L, x, idx_s, nullptr, k, s_sp, s, false, true), "stage2 launch");
+  prox::Stage2Launch m;
+  m.mode = 0;
+  m.idx = idx_s;
+  m.k = k;
+  m.s_sp = s_sp;
+  PROX_CUDA(prox::launch_stage2(L, x, m, s, false, true), "stage2 launch");
   PROX_CUDA(prox::launch_reduce(L, out, s, true), "reduce launch");
   return PROX_OK;
 }

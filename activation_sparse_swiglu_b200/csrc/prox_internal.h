@@ -12,25 +12,37 @@ namespace prox {
 
 constexpr int kGroup = 128;          // proxy quantisation group (input rows)
 constexpr int kHistBins = 2048;      // first radix level: score bits [30:20]
-constexpr int kStage1Warps = 4;      // Stage-1 CTA = 4 warps on one column slice
-constexpr int kMaxGroupsPerSlab = 32; // bounds Stage-1 shared memory (115 KB)
-constexpr int kSelectThreads = 1024; // top-k select CTA
+constexpr int kStage1Warps = 4;      // Stage-1 warps per CTA
+constexpr int kMaxGroupsPerSlab = 32; // bounds Stage-1 shared memory
+constexpr int kMaxCluster = 16;       // Stage-1 cluster size limit (row slabs per slice)
+constexpr int kSelectCand = 4096;    // candidate buffer of the select (level-1 bin)
+constexpr int kSelectSlice = 256;    // channels per select CTA (and per rank-offset entry)
+constexpr int kMaxSlices = 160;      // >= d_ff / kSelectSlice + 1
 constexpr int kStage2Consumers = 8;  // Stage-2 consumer warps (+1 producer warp)
-constexpr int kReduceWarps = 8;      // output reduction: warps per 32 columns
+constexpr int kReduceWarps = 16;     // output reduction: warps per 32 columns
 constexpr int kMaxDModel = 16384;
-constexpr int kMaxDff = 49152;       // select keeps all scores in shared memory
+constexpr int kMaxDff = 32768;       // the select keeps all scores in registers
 constexpr int kHostChunkTokens = 64; // staging chunk of prox_ffn_forward_host
+
+// Select state shared by the select kernel and Stage 2.
+enum { kSelCandCount = 0, kSelTicket = 1, kSelT = 2, kSelTieCut = 3 };
+struct SelectState {
+  uint32_t* hist = nullptr;      // [kHistBins] score bits 30..20, zero between tokens
+  uint32_t* state = nullptr;     // [8] candidate count, ticket, T, tie cut
+  uint32_t* cand_key = nullptr;  // [kSelectCand] keys of the boundary bin
+  int32_t* cand_idx = nullptr;   // [kSelectCand] their channels
+  int32_t* sl_gt1 = nullptr;     // [kMaxSlices] keys above the boundary bin, per slice
+  int32_t* sl_off = nullptr;     // [kMaxSlices + 1] rank offset of each slice's selected channels
+};
 
 // Per-token scratch of one layer (device memory owned by the handle).
 struct Workspace {
-  float* part = nullptr;          // Stage-1 partial sums [R][C][1024]
   float* scores = nullptr;        // |SiLU(g~) u~| [F]
   float* g_dbg = nullptr;         // debug g~ [F]
   float* u_dbg = nullptr;         // debug u~ [F]
-  uint32_t* hist = nullptr;       // [kHistBins], zero between tokens
-  uint32_t* slice_cnt = nullptr;  // [C] tickets, zero between tokens
+  uint32_t* hist = nullptr;       // [kHistBins], zero between tokens (== sel.hist)
+  SelectState sel;
   int32_t* idx_s = nullptr;       // [F] selected channels (first k valid)
-  int32_t* k_dev = nullptr;       // [1] number of selected channels
   int32_t* slab_idx = nullptr;    // [d] kept input rows, per slab (debug)
   int32_t* slab_cnt = nullptr;    // [R] kept rows per slab (debug)
   float* ypart = nullptr;         // Stage-2 output partials [P][d]
@@ -51,8 +63,8 @@ struct prox_layer {
   // Stage-1 geometry
   int C = 0, R = 0, gps = 0;
   // Stage-2 geometry
-  int P = 0, ring_slots = 0;
-  size_t stage2_smem = 0, stage1_smem = 0, select_smem = 0;
+  int P = 0, ring_slots = 0, stage2_producers = 1;
+  size_t stage2_smem = 0, stage1_smem = 0;
   // library-owned weights
   uint16_t* wgu = nullptr;   // bf16 [F][2d]: gate column j | up column j
   uint16_t* wd = nullptr;    // bf16 [F][d]
@@ -69,20 +81,23 @@ struct Stage1Taps {
   float* u = nullptr;
   bool slabs = false;  // write per-slab kept-row lists
 };
-struct SelectTaps {
-  int32_t* idx_x = nullptr;  // concatenated kept rows
-  int32_t* n_x = nullptr;
+// How Stage 2 obtains its channels.
+struct Stage2Launch {
+  int mode = 1;               // 0: given list `idx`, 1: top-k select, 2: dense
+  const int32_t* idx = nullptr;
+  int k = 0;
+  int32_t* idx_out = nullptr;  // top-k: selected channels (ascending) written here
+  float* s_sp = nullptr;       // optional SiLU(g) u per listed channel
+  bool select_only = false;    // top-k: stop after selecting
 };
 
 cudaError_t launch_stage1(const prox_layer* L, const float* x, const Stage1Taps& taps,
                           cudaStream_t s, bool pdl);
-cudaError_t launch_select(const prox_layer* L, const SelectTaps& taps, cudaStream_t s,
-                          bool pdl);
-// idx == nullptr: dense (every channel, k = F).  k_dev != nullptr: k is read
-// on the device after the dependency wait; otherwise k_host is used.
-cudaError_t launch_stage2(const prox_layer* L, const float* x, const int32_t* idx,
-                          const int32_t* k_dev, int k_host, float* s_sp, cudaStream_t s,
-                          bool pdl, bool x_ready);
+cudaError_t launch_select(const prox_layer* L, cudaStream_t s, bool pdl);
+cudaError_t launch_concat_slabs(const prox_layer* L, int32_t* idx_x, int32_t* n_x,
+                                cudaStream_t s);
+cudaError_t launch_stage2(const prox_layer* L, const float* x, const Stage2Launch& m,
+                          cudaStream_t s, bool pdl, bool x_ready);
 cudaError_t launch_reduce(const prox_layer* L, float* out, cudaStream_t s, bool pdl);
 
 cudaError_t launch_pack_proxy(const uint16_t* W, int d, int F, uint8_t* codes,
@@ -105,8 +120,7 @@ cudaError_t launch_copy(const void* src, void* dst, size_t bytes, cudaStream_t s
 // Stage-1 column slices and row slabs for a shape on `num_sms` SMs.
 void choose_stage1_grid(int d, int F, int num_sms, int* C, int* R, int* gps);
 size_t stage1_smem_bytes(int gps);
-size_t select_smem_bytes(int F);
 // Stage-2 ring depth and dynamic shared memory for d_model = d.
-void choose_stage2(int d, int F, int num_sms, int* P, int* slots, size_t* smem);
+void choose_stage2(int d, int F, int num_sms, int* P, int* slots, int* nprod, size_t* smem);
 
 }  // namespace prox

@@ -4,14 +4,22 @@
 // kernel with every channel kept.
 //
 // stage2_kernel -- persistent: one CTA per SM, each CTA owning a contiguous,
-// balanced range of the k selected channels.  A producer warp streams, with
-// 1-D bulk async copies (TMA engine) into a ring of shared-memory slots, first
-// the gate/up channel records of its channels (gate column then up column,
-// d_model bf16 each, contiguous per channel), then their W_down rows.  Eight
-// consumer warps:
-//   phase A: one warp per channel computes g = x . W_gate[:, j] and
-//            u = x . W_up[:, j] over the full x (fp32, packed f32x2 FMAs,
-//            warp-shuffle reduction) and keeps s_j = SiLU(g) u;
+// balanced range [t0, t1) of the k selected channels (ranked by channel
+// index).  In top-k mode the CTA turns its ranks into channels from the
+// select kernel's per-slice rank offsets, threshold T and tie cut, reading
+// only the one or two 256-channel slices of scores that hold its ranks.  Four producer lanes stream, with
+// 1-D bulk async copies (TMA engine) into a ring of 16 KB-class shared-memory
+// slots, first the gate/up channel records of its channels (gate column then
+// up column, d_model bf16 each: one copy per channel), then their W_down rows
+// (two rows per slot).  Eight consumer warps take every ring item in order (so
+// each mbarrier wait is for the phase right after one the waiting thread has
+// already seen complete):
+//   phase A: for each channel every warp forms partial dot products of its
+//            share of the column with the full x (x kept in registers; fp32,
+//            packed f32x2 FMAs, warp-shuffle reduction) and parks them in
+//            shared memory; after the last channel the partials are summed in
+//            a fixed order into g = x . W_gate[:, j], u = x . W_up[:, j] and
+//            s_j = SiLU(g) u;
 //   phase B: all warps accumulate y_part += s_j W_down[j, :] for the CTA's
 //            channels, each thread owning 8-column groups of the output.
 // Each CTA writes its fp32 partial y; reduce_kernel sums the partials in a
@@ -24,21 +32,77 @@ namespace {
 
 constexpr int NCW = kStage2Consumers;
 constexpr int S2_THREADS = (NCW + 1) * 32;
-constexpr size_t kStage2SmemBudget = 200 * 1024;
+constexpr size_t kStage2SmemBudget = 208 * 1024;
+
+enum Stage2Mode { kGivenList = 0, kTopK = 1, kDense = 2 };
 
 struct Stage2Args {
   const float* x;
   const uint16_t* wgu;
   const uint16_t* wd;
-  const int32_t* idx;
-  const int32_t* k_dev;
-  int k_host;
+  const int32_t* idx;      // kGivenList: channel list [k]
+  const float* scores;     // kTopK: Stage-1 scores [F]
+  const int32_t* sl_off;   // kTopK: rank offsets per 256-channel slice
+  const uint32_t* sel_state;  // kTopK: threshold T and tie cut
+  int32_t* idx_out;        // kTopK: selected channels, ascending (each CTA its ranks)
+  int mode, select_only;
+  int k;
   int d, F, P, slots, max_rec;
+  int nprod;  // producer lanes; slots is a multiple of it
   float* ypart;
   float* s_sp;
   int* err;
   int x_ready;
 };
+
+// Top-k mode: the selected channels of ranks [t0, t1) (ascending channel
+// order) into s_idx and idx_out, from the rank offsets of the slices.
+__device__ void ranks_to_channels(const Stage2Args& a, int t0, int t1, int* s_idx, int* s_tmp) {
+  constexpr int NTH = (kStage2Consumers + 1) * 32;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nsl = (a.F + kSelectSlice - 1) / kSelectSlice;
+  int* s_off = s_tmp;                      // [nsl + 1]
+  int* s_w = s_tmp + kMaxSlices + 1;       // [8] per-warp counts
+  int* s_m = s_w + 8;                      // [4]
+  for (int i = tid; i <= nsl; i += NTH) s_off[i] = __ldcg(a.sl_off + i);
+  if (tid == 0) {
+    s_m[0] = (int)__ldcg(a.sel_state + kSelT);
+    s_m[1] = (int)__ldcg(a.sel_state + kSelTieCut);
+  }
+  __syncthreads();
+  const uint32_t T = (uint32_t)s_m[0];
+  const int cut = s_m[1];
+  if (tid == 0) {
+    int lo = 0;
+    while (lo < nsl - 1 && s_off[lo + 1] <= t0) ++lo;
+    int hi = lo;
+    while (hi < nsl - 1 && s_off[hi + 1] < t1) ++hi;
+    s_m[2] = lo;
+    s_m[3] = hi;
+  }
+  __syncthreads();
+  const int lo = s_m[2], hi = s_m[3];
+  const unsigned lt = (1u << lane) - 1u;
+  for (int sl = lo; sl <= hi && t0 < t1; ++sl) {
+    const int e = sl * kSelectSlice + tid;
+    bool take = false;
+    if (tid < kSelectSlice && e < a.F) {
+      const uint32_t key = __float_as_uint(__ldcg(a.scores + e));
+      take = key > T || (key == T && e <= cut);
+    }
+    const unsigned m = __ballot_sync(0xffffffffu, take);
+    if (lane == 0 && warp < 8) s_w[warp] = __popc(m);
+    __syncthreads();
+    int before = s_off[sl];
+    for (int w = 0; w < warp && w < 8; ++w) before += s_w[w];
+    const int rank = before + __popc(m & lt);
+    if (take && rank >= t0 && rank < t1) {
+      s_idx[rank - t0] = e;
+      if (a.idx_out) a.idx_out[rank] = e;
+    }
+    __syncthreads();
+  }
+}
 
 __device__ __forceinline__ void load_x(float* xs, const float* x, int d, int tid, int nt) {
   for (int e = tid * 4; e < d; e += nt * 4)
@@ -60,21 +124,22 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
+// MAXM = ceil(d_model / 2048): 8-element chunks per thread and column.
 template <int MAXM>
 __global__ void __launch_bounds__(S2_THREADS, 1) stage2_kernel(Stage2Args a) {
   extern __shared__ __align__(128) unsigned char smem[];
   const int d = a.d, slots = a.slots;
-  const uint32_t slot_bytes = 2u * (uint32_t)d;
+  const uint32_t col_bytes = 2u * (uint32_t)d;     // one bf16 column / row
+  const uint32_t slot_bytes = 2u * col_bytes;      // a gate/up record, or two W_down rows
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);
   uint64_t* empty = full + slots;
-  float* s_val = reinterpret_cast<float*>(empty + slots);
-  int* s_idx = reinterpret_cast<int*>(s_val + a.max_rec);
-  size_t off = (size_t)slots * 16 + (size_t)a.max_rec * 8;
-  off = (off + 15) & ~(size_t)15;
-  float* xs = reinterpret_cast<float*>(smem + off);
-  off += (size_t)d * 4;
+  float* s_val = reinterpret_cast<float*>(empty + slots);        // [max_rec]
+  int* s_idx = reinterpret_cast<int*>(s_val + a.max_rec);        // [max_rec]
+  float* s_pg = reinterpret_cast<float*>(s_idx + a.max_rec);     // [max_rec][NCW]
+  float* s_pu = s_pg + (size_t)a.max_rec * NCW;                  // [max_rec][NCW]
+  size_t off = (size_t)slots * 16 + (size_t)a.max_rec * (8 + 8 * NCW);
   off = (off + 127) & ~(size_t)127;
   unsigned char* ring = smem + off;
 
@@ -85,137 +150,218 @@ __global__ void __launch_bounds__(S2_THREADS, 1) stage2_kernel(Stage2Args a) {
     }
     fence_barrier_init();
   }
-  if (a.x_ready) load_x(xs, a.x, d, tid, S2_THREADS);
+  // this thread's share of x (chunks c8 = tid + 256 m), kept in registers
+  float4 xr[MAXM][2];
+  if (a.x_ready && warp < NCW) {
+#pragma unroll
+    for (int m = 0; m < MAXM; ++m) {
+      const int e = (tid + m * NCW * 32) * 8;
+      xr[m][0] = e < d ? __ldg(reinterpret_cast<const float4*>(a.x + e)) : make_float4(0, 0, 0, 0);
+      xr[m][1] = e < d ? __ldg(reinterpret_cast<const float4*>(a.x + e + 4)) : make_float4(0, 0, 0, 0);
+    }
+  }
   __syncthreads();
 
   pdl_wait();
   pdl_trigger();
 
-  if (!a.x_ready) load_x(xs, a.x, d, tid, S2_THREADS);
-  const int k = a.k_dev ? __ldcg(a.k_dev) : a.k_host;
+  if (!a.x_ready && warp < NCW) {
+#pragma unroll
+    for (int m = 0; m < MAXM; ++m) {
+      const int e = (tid + m * NCW * 32) * 8;
+      xr[m][0] = e < d ? __ldg(reinterpret_cast<const float4*>(a.x + e)) : make_float4(0, 0, 0, 0);
+      xr[m][1] = e < d ? __ldg(reinterpret_cast<const float4*>(a.x + e + 4)) : make_float4(0, 0, 0, 0);
+    }
+  }
+  const int k = a.mode == kDense ? a.F : a.k;
   const int cta = blockIdx.x;
   const int t0 = (int)(((long long)k * cta) / a.P);
   const int t1 = (int)(((long long)k * (cta + 1)) / a.P);
   const int n = t1 - t0;
-  for (int i = tid; i < n; i += S2_THREADS) {
-    int j = a.idx ? __ldcg(a.idx + t0 + i) : t0 + i;
-    if (j < 0 || j >= a.F) {
-      atomicOr(a.err, PROX_DEVERR_MASK_INDEX);
-      j = 0;
+  if (a.mode == kTopK) {
+    ranks_to_channels(a, t0, t1, s_idx, reinterpret_cast<int*>(ring));
+    __syncthreads();
+  } else {
+    for (int i = tid; i < n; i += S2_THREADS) {
+      int j = a.mode == kGivenList ? __ldcg(a.idx + t0 + i) : t0 + i;
+      if (j < 0 || j >= a.F) {
+        atomicOr(a.err, PROX_DEVERR_MASK_INDEX);
+        j = 0;
+      }
+      s_idx[i] = j;
     }
-    s_idx[i] = j;
+    __syncthreads();
   }
-  __syncthreads();
+  if (a.select_only) return;
 
-  // Ring schedule.  Phase A: record r (gate column, up column) goes to slot
-  // pair r % npa and is consumed by warp (r % npa) % na, so every slot pair
-  // has one owning warp that consumes its uses in order.  Phase B: W_down row
-  // i goes to slot i % slots and is consumed by every warp in order.  Each
-  // mbarrier wait is therefore for the next phase of a barrier whose earlier
-  // phases this thread has already seen complete, so parity waits cannot alias.
+  // Ring items q = 0 .. nA + nB - 1: q < n is the gate/up record of channel q;
+  // q >= n holds W_down rows 2(q-n) and 2(q-n)+1.  Item q lives in slot
+  // q % slots as that slot's use q / slots.
+  const int nB = (n + 1) >> 1;
+  const int total = n + nB;
   bool dead = false;  // set once a wait of this thread ran out
-  const int npairs = slots / 2;
-  const int na = npairs < NCW ? npairs : NCW;   // phase-A consumer warps
-  const int npa = na * (npairs / na);           // phase-A slot pairs in use
-  // uses of slot s by phase A
-  auto uses_a = [&](int slot) -> int {
-    const int p = slot >> 1;
-    if (p >= npa || p >= n) return 0;
-    return (n - p + npa - 1) / npa;
-  };
   if (warp == NCW) {
-    // ---------------- producer ----------------
-    if (lane == 0 && n > 0) {
+    // ---------------- producer lanes 0..nprod-1: lane l issues items q = l + j*nprod.
+    // slots is a multiple of nprod, so every slot is refilled by one lane, in order.
+    const int np = a.nprod;
+    if (lane < np && lane < total) {
       const uint64_t pol = l2_policy_evict_first();
-      for (int r = 0; r < n; ++r) {
-        const int p = r % npa, use = r / npa;
-        const size_t rec = (size_t)s_idx[r] * 2;
-        for (int h = 0; h < 2; ++h) {
-          const int slot = 2 * p + h;
-          if (use > 0) mbar_wait(&empty[slot], (uint32_t)((use - 1) & 1), a.err, &dead);
+      int q = lane;
+      int slot = q % slots;
+      int use = q / slots;
+      for (; q < total; q += np) {
+        if (use > 0) mbar_wait(&empty[slot], (uint32_t)((use - 1) & 1), a.err, &dead);
+        unsigned char* dst = ring + (size_t)slot * slot_bytes;
+        if (q < n) {
           mbar_arrive_expect_tx(&full[slot], slot_bytes);
-          bulk_copy_g2s(ring + (size_t)slot * slot_bytes, a.wgu + (rec + h) * (size_t)d,
-                        slot_bytes, &full[slot], pol);
+          bulk_copy_g2s(dst, a.wgu + (size_t)s_idx[q] * 2 * (size_t)d, slot_bytes, &full[slot], pol);
+        } else {
+          const int r0 = 2 * (q - n);
+          const int nr = r0 + 1 < n ? 2 : 1;
+          mbar_arrive_expect_tx(&full[slot], (uint32_t)nr * col_bytes);
+          bulk_copy_g2s(dst, a.wd + (size_t)s_idx[r0] * (size_t)d, col_bytes, &full[slot], pol);
+          if (nr == 2)
+            bulk_copy_g2s(dst + col_bytes, a.wd + (size_t)s_idx[r0 + 1] * (size_t)d, col_bytes,
+                          &full[slot], pol);
+        }
+        slot += np;
+        while (slot >= slots) {
+          slot -= slots;
+          ++use;
         }
       }
-      for (int i = 0; i < n; ++i) {
-        const int slot = i % slots, use = uses_a(slot) + i / slots;
-        if (use > 0) mbar_wait(&empty[slot], (uint32_t)((use - 1) & 1), a.err, &dead);
-        mbar_arrive_expect_tx(&full[slot], slot_bytes);
-        bulk_copy_g2s(ring + (size_t)slot * slot_bytes, a.wd + (size_t)s_idx[i] * (size_t)d,
-                      slot_bytes, &full[slot], pol);
-      }
-      // Every issued copy must land before this CTA's shared memory is released.
-      for (int slot = 0; slot < slots; ++slot) {
-        const int uses = uses_a(slot) + (slot < n ? (n - slot + slots - 1) / slots : 0);
-        if (uses > 0) mbar_wait(&full[slot], (uint32_t)((uses - 1) & 1), a.err);
+      // Every issued copy must land before this CTA's shared memory is released:
+      // wait for the last use of each slot this lane filled.
+      for (int s2 = 0; s2 < slots; ++s2) {
+        int last = -1;  // last item of this lane in slot s2
+        for (int qq = s2; qq < total; qq += slots)
+          if (qq % np == lane) last = qq;
+        if (last >= 0) mbar_wait(&full[s2], (uint32_t)((last / slots) & 1), a.err);
       }
     }
     return;
   }
 
-  // ---------------- phase A: gate/up, one warp per channel ----------------
-  if (warp < na) {
-    // npa is a multiple of na, so slot pair r % npa is always owned by warp r % na
-    for (int r = warp; r < n; r += na) {
-      const int p = r % npa, use = r / npa;
-      const int sl0 = 2 * p, sl1 = sl0 + 1;
-      mbar_wait(&full[sl0], (uint32_t)(use & 1), a.err, &dead);
-      mbar_wait(&full[sl1], (uint32_t)(use & 1), a.err, &dead);
-      const unsigned char* wg = ring + (size_t)sl0 * slot_bytes;
-      const unsigned char* wu = ring + (size_t)sl1 * slot_bytes;
-      float2 ag[4], au[4];
+  int cs = 0;        // consumer: slot of the next item
+  uint32_t cp = 0;   // and the parity of its use
+
+  // ---------------- phase A: partial gate/up dot products ----------------
+  // Records are taken RB at a time so that the 2*RB warp reductions of a batch
+  // run interleaved.
+  constexpr int RB = 4;
+  const int rbn = slots < RB ? slots : RB;  // a batch never holds more than the ring
+  for (int r0 = 0; r0 < n; r0 += rbn) {
+    int sl[RB];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) ag[i] = au[i] = make_float2(0.f, 0.f);
-      for (int e = lane * 8; e < d; e += 256) {
-        const uint4 g4 = lds_v4(wg + (size_t)e * 2);
-        const uint4 u4 = lds_v4(wu + (size_t)e * 2);
-        const float4 xa = lds_f4(xs + e);
-        const float4 xb = lds_f4(xs + e + 4);
-        dot8(ag, g4, xa, xb);
-        dot8(au, u4, xa, xb);
+    for (int b = 0; b < RB; ++b) {
+      sl[b] = cs;
+      if (b < rbn && r0 + b < n) {
+        mbar_wait(&full[cs], cp, a.err, &dead);
+        if (++cs == slots) { cs = 0; cp ^= 1u; }
       }
-      float g = (ag[0].x + ag[0].y) + (ag[1].x + ag[1].y) + (ag[2].x + ag[2].y) +
-                (ag[3].x + ag[3].y);
-      float u = (au[0].x + au[0].y) + (au[1].x + au[1].y) + (au[2].x + au[2].y) +
-                (au[3].x + au[3].y);
-      g = warp_sum(g);
-      u = warp_sum(u);
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&empty[sl0], NCW);
-        mbar_arrive(&empty[sl1], NCW);
-        const float sv = silu_f32(g) * u;
-        s_val[r] = sv;
-        if (a.s_sp) a.s_sp[t0 + r] = sv;
+    }
+    float g[RB], u[RB];
+#pragma unroll
+    for (int b = 0; b < RB; ++b) {
+      float2 ag = make_float2(0.f, 0.f), au = make_float2(0.f, 0.f);
+      if (b < rbn && r0 + b < n) {
+        const unsigned char* wg = ring + (size_t)sl[b] * slot_bytes;
+        const unsigned char* wu = wg + col_bytes;
+#pragma unroll
+        for (int m = 0; m < MAXM; ++m) {
+          const int e = (tid + m * NCW * 32) * 8;
+          if (e < d) {
+            const uint4 g4 = *reinterpret_cast<const uint4*>(wg + (size_t)e * 2);
+            const uint4 u4 = *reinterpret_cast<const uint4*>(wu + (size_t)e * 2);
+            const float4 xa = xr[m][0], xb = xr[m][1];
+            ag = __ffma2_rn(bf16x2_to_f2(g4.x), make_float2(xa.x, xa.y), ag);
+            au = __ffma2_rn(bf16x2_to_f2(u4.x), make_float2(xa.x, xa.y), au);
+            ag = __ffma2_rn(bf16x2_to_f2(g4.y), make_float2(xa.z, xa.w), ag);
+            au = __ffma2_rn(bf16x2_to_f2(u4.y), make_float2(xa.z, xa.w), au);
+            ag = __ffma2_rn(bf16x2_to_f2(g4.z), make_float2(xb.x, xb.y), ag);
+            au = __ffma2_rn(bf16x2_to_f2(u4.z), make_float2(xb.x, xb.y), au);
+            ag = __ffma2_rn(bf16x2_to_f2(g4.w), make_float2(xb.z, xb.w), ag);
+            au = __ffma2_rn(bf16x2_to_f2(u4.w), make_float2(xb.z, xb.w), au);
+          }
+        }
+      }
+      g[b] = ag.x + ag.y;
+      u[b] = au.x + au.y;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+      for (int b = 0; b < RB; ++b) {
+        g[b] += __shfl_xor_sync(0xffffffffu, g[b], o);
+        u[b] += __shfl_xor_sync(0xffffffffu, u[b], o);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) {
+#pragma unroll
+      for (int b = 0; b < RB; ++b) {
+        if (b < rbn && r0 + b < n) {
+          mbar_arrive(&empty[sl[b]], 1);
+          s_pg[(r0 + b) * NCW + warp] = g[b];
+          s_pu[(r0 + b) * NCW + warp] = u[b];
+        }
       }
     }
   }
   asm volatile("bar.sync 1, %0;" ::"r"(NCW * 32) : "memory");
+  for (int r = tid; r < n; r += NCW * 32) {
+    float g = 0.f, u = 0.f;
+#pragma unroll
+    for (int w = 0; w < NCW; ++w) {
+      g += s_pg[r * NCW + w];
+      u += s_pu[r * NCW + w];
+    }
+    const float sv = silu_f32(g) * u;
+    s_val[r] = sv;
+    if (a.s_sp) a.s_sp[t0 + r] = sv;
+  }
+  asm volatile("bar.sync 1, %0;" ::"r"(NCW * 32) : "memory");
 
   // ---------------- phase B: y_part = sum_t s_t W_down[j_t, :] ----------------
+  // Items (two rows each) are taken two at a time.
   float2 acc[MAXM * 4];
 #pragma unroll
   for (int i = 0; i < MAXM * 4; ++i) acc[i] = make_float2(0.f, 0.f);
-  for (int rr = 0; rr < n; ++rr) {
-    const int sl = rr % slots, use = uses_a(sl) + rr / slots;
-    mbar_wait(&full[sl], (uint32_t)(use & 1), a.err, &dead);
-    const float sv = s_val[rr];
-    const float2 s2 = make_float2(sv, sv);
-    const unsigned char* w = ring + (size_t)sl * slot_bytes;
+  for (int rb0 = 0; rb0 < nB; rb0 += 2) {
+    int sl[2];
 #pragma unroll
-    for (int m = 0; m < MAXM; ++m) {
-      const int e = tid * 8 + m * (NCW * 32 * 8);
-      if (e < d) {
-        const uint4 w4 = lds_v4(w + (size_t)e * 2);
-        acc[4 * m + 0] = __ffma2_rn(bf16x2_to_f2(w4.x), s2, acc[4 * m + 0]);
-        acc[4 * m + 1] = __ffma2_rn(bf16x2_to_f2(w4.y), s2, acc[4 * m + 1]);
-        acc[4 * m + 2] = __ffma2_rn(bf16x2_to_f2(w4.z), s2, acc[4 * m + 2]);
-        acc[4 * m + 3] = __ffma2_rn(bf16x2_to_f2(w4.w), s2, acc[4 * m + 3]);
+    for (int b = 0; b < 2; ++b) {
+      sl[b] = cs;
+      if (rb0 + b < nB) {
+        mbar_wait(&full[cs], cp, a.err, &dead);
+        if (++cs == slots) { cs = 0; cp ^= 1u; }
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      const int rr = 2 * rb0 + h;  // W_down row (channel slot) of this CTA
+      if (rr < n) {
+        const float sv = s_val[rr];
+        const float2 s2 = make_float2(sv, sv);
+        const unsigned char* w = ring + (size_t)sl[h >> 1] * slot_bytes + (h & 1) * col_bytes;
+#pragma unroll
+        for (int m = 0; m < MAXM; ++m) {
+          const int e = tid * 8 + m * (NCW * 32 * 8);
+          if (e < d) {
+            const uint4 w4 = *reinterpret_cast<const uint4*>(w + (size_t)e * 2);
+            acc[4 * m + 0] = __ffma2_rn(bf16x2_to_f2(w4.x), s2, acc[4 * m + 0]);
+            acc[4 * m + 1] = __ffma2_rn(bf16x2_to_f2(w4.y), s2, acc[4 * m + 1]);
+            acc[4 * m + 2] = __ffma2_rn(bf16x2_to_f2(w4.z), s2, acc[4 * m + 2]);
+            acc[4 * m + 3] = __ffma2_rn(bf16x2_to_f2(w4.w), s2, acc[4 * m + 3]);
+          }
+        }
       }
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[sl], 1);
+    if (lane == 0) {
+      mbar_arrive(&empty[sl[0]], 1);
+      if (rb0 + 1 < nB) mbar_arrive(&empty[sl[1]], 1);
+    }
   }
   float* dst = a.ypart + (size_t)cta * d;
 #pragma unroll
@@ -230,28 +376,30 @@ __global__ void __launch_bounds__(S2_THREADS, 1) stage2_kernel(Stage2Args a) {
   }
 }
 
-// out[c] = sum_p ypart[p][c], p in increasing order.
+// out[c] = sum_p ypart[p][c]: warp w sums partials p = w, w + W, ... (all its
+// loads in flight at once), then the warps' sums are added in warp order.
 __global__ void __launch_bounds__(kReduceWarps * 32) reduce_kernel(const float* ypart, int P, int d,
-                                                                   float* out) {
+                                                                   float* out, uint32_t* hist) {
   __shared__ float s_part[kReduceWarps][32];
   pdl_wait();
   pdl_trigger();
+  // Stage 2 is complete: clear the level-1 histogram for the next token.
+  if (hist && blockIdx.x == 0)
+    for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) hist[i] = 0u;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int col = blockIdx.x * 32 + lane;
   float s = 0.f;
   if (col < d) {
-    int p = warp;
-    for (; p + 3 * kReduceWarps < P; p += 4 * kReduceWarps) {
-      const float v0 = __ldcg(ypart + (size_t)p * d + col);
-      const float v1 = __ldcg(ypart + (size_t)(p + kReduceWarps) * d + col);
-      const float v2 = __ldcg(ypart + (size_t)(p + 2 * kReduceWarps) * d + col);
-      const float v3 = __ldcg(ypart + (size_t)(p + 3 * kReduceWarps) * d + col);
-      s += v0;
-      s += v1;
-      s += v2;
-      s += v3;
+    for (int p0 = warp; p0 < P; p0 += 16 * kReduceWarps) {
+      float v[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int p = p0 + u * kReduceWarps;
+        v[u] = p < P ? __ldcg(ypart + (size_t)p * d + col) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 16; ++u) s += v[u];
     }
-    for (; p < P; p += kReduceWarps) s += __ldcg(ypart + (size_t)p * d + col);
   }
   s_part[warp][lane] = s;
   __syncthreads();
@@ -276,20 +424,28 @@ cudaError_t set_stage2_attr() {
 
 }  // namespace
 
-void choose_stage2(int d, int F, int num_sms, int* P, int* slots, size_t* smem) {
+void choose_stage2(int d, int F, int num_sms, int* P, int* slots, int* nprod, size_t* smem) {
   *P = num_sms;
   const int max_rec = (F + num_sms - 1) / num_sms + 1;
-  size_t fixed = (size_t)max_rec * 8 + 16 + (size_t)d * 4 + 128;
-  const size_t slot_bytes = 2 * (size_t)d;
-  int s = (int)((kStage2SmemBudget - fixed) / (slot_bytes + 16));
+  size_t off = (size_t)max_rec * (8 + 8 * NCW) + 128;
+  const size_t slot_bytes = 4 * (size_t)d;  // gate + up column, or two W_down rows
+  int s = (int)((kStage2SmemBudget - off) / (slot_bytes + 16));
   if (s > 32) s = 32;
-  if (s < 3) s = 3;
+  if (s < 2) s = 2;
+  // producer lanes: the slot count must be a multiple of them
+  if (s >= 8) {
+    s -= s % 4;
+    *nprod = 4;
+  } else {
+    s -= s % 2;
+    *nprod = 2;
+  }
   *slots = s;
-  size_t off = (size_t)s * 16 + (size_t)max_rec * 8;
-  off = (off + 15) & ~(size_t)15;
-  off += (size_t)d * 4;
+  off = (size_t)s * 16 + (size_t)max_rec * (8 + 8 * NCW);
   off = (off + 127) & ~(size_t)127;
-  *smem = off + (size_t)s * slot_bytes;
+  size_t region = (size_t)s * slot_bytes;
+  if (region < 4096) region = 4096;  // scratch of ranks_to_channels
+  *smem = off + region;
 }
 
 cudaError_t setup_stage2_kernels() {
@@ -301,23 +457,28 @@ cudaError_t setup_stage2_kernels() {
   return set_stage2_attr<8>();
 }
 
-cudaError_t launch_stage2(const prox_layer* L, const float* x, const int32_t* idx,
-                          const int32_t* k_dev, int k_host, float* s_sp, cudaStream_t s,
-                          bool pdl, bool x_ready) {
+cudaError_t launch_stage2(const prox_layer* L, const float* x, const Stage2Launch& m,
+                          cudaStream_t s, bool pdl, bool x_ready) {
   Stage2Args a;
   a.x = x;
   a.wgu = L->wgu;
   a.wd = L->wd;
-  a.idx = idx;
-  a.k_dev = k_dev;
-  a.k_host = idx ? k_host : L->F;
+  a.idx = m.idx;
+  a.scores = L->ws.scores;
+  a.sl_off = L->ws.sel.sl_off;
+  a.sel_state = L->ws.sel.state;
+  a.idx_out = m.idx_out;
+  a.mode = m.mode;
+  a.select_only = m.select_only ? 1 : 0;
+  a.k = m.k;
   a.d = L->d;
   a.F = L->F;
   a.P = L->P;
   a.slots = L->ring_slots;
+  a.nprod = L->stage2_producers;
   a.max_rec = (L->F + L->P - 1) / L->P + 1;
   a.ypart = L->ws.ypart;
-  a.s_sp = s_sp;
+  a.s_sp = m.s_sp;
   a.err = L->ws.err;
   a.x_ready = x_ready ? 1 : 0;
 
@@ -331,11 +492,11 @@ cudaError_t launch_stage2(const prox_layer* L, const float* x, const int32_t* id
   attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const int m = (L->d + 2047) / 2048;
-  if (m <= 1) return launch_stage2_t<1>(cfg, a);
-  if (m == 2) return launch_stage2_t<2>(cfg, a);
-  if (m == 3) return launch_stage2_t<3>(cfg, a);
-  if (m == 4) return launch_stage2_t<4>(cfg, a);
+  const int mm = (L->d + 2047) / 2048;
+  if (mm <= 1) return launch_stage2_t<1>(cfg, a);
+  if (mm == 2) return launch_stage2_t<2>(cfg, a);
+  if (mm == 3) return launch_stage2_t<3>(cfg, a);
+  if (mm == 4) return launch_stage2_t<4>(cfg, a);
   return launch_stage2_t<8>(cfg, a);
 }
 
@@ -350,7 +511,8 @@ cudaError_t launch_reduce(const prox_layer* L, float* out, cudaStream_t s, bool 
   attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, reduce_kernel, (const float*)L->ws.ypart, L->P, L->d, out);
+  return cudaLaunchKernelEx(&cfg, reduce_kernel, (const float*)L->ws.ypart, L->P, L->d, out,
+                            L->ws.hist);
 }
 
 }  // namespace prox

@@ -21,7 +21,7 @@
  *    W_down is [d_ff, d_model], all row-major.  Activations are fp32.
  *  - Shape rules (else PROX_EINVAL, checked before any launch):
  *    d_model > 0 and d_model % 128 == 0; d_ff > 0 and d_ff % 32 == 0;
- *    d_model <= 16384; d_ff <= 49152; 1 <= k <= d_ff; pointers 16-byte aligned.
+ *    d_model <= 16384; d_ff <= 32768; 1 <= k <= d_ff; pointers 16-byte aligned.
  *  - Errors: every call returns a prox_status; prox_last_error() copies a
  *    message for the calling thread's last failure.  No C++ exception crosses
  *    this boundary.  Device-side checks (an index out of range in a caller's

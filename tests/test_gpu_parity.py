@@ -153,14 +153,21 @@ def test_stage1_llama3_8b_sampled(prox):
         _stage1_case(prox, lay, olay, tau, lay.config.k(s2), range(3))
 
 
-def test_stage1_no_input_kept(prox):
-    # tau above every |x|: n_x = 0, all proxy scores are 0, ties go to the lowest indices
-    lay, olay = _layer(_custom(384, 96))
-    layer = device_layer(lay, 1e30, 10)
-    taps = layer.debug_stage1(torch.from_numpy(lay.x_eval[0]).cuda())
+@pytest.mark.parametrize("shape,k", [((384, 96), 10), ((256, 8192), 3001)])
+def test_stage1_no_input_kept(prox, shape, k):
+    # tau above every |x|: n_x = 0, all proxy scores are 0, ties go to the lowest
+    # indices (the second shape has more tied keys than the candidate buffer)
+    lay, olay = _layer(_custom(*shape))
+    layer = device_layer(lay, 1e30, k)
+    x = torch.from_numpy(lay.x_eval[0]).cuda()
+    taps = layer.debug_stage1(x)
     assert int(taps["n_x"].item()) == 0
     np.testing.assert_array_equal(taps["g_tilde"].cpu().numpy(), 0.0)
-    np.testing.assert_array_equal(taps["idx_s"].cpu().numpy(), np.arange(10))
+    np.testing.assert_array_equal(taps["idx_s"].cpu().numpy(), np.arange(k))
+    # the full step selects the same channels
+    ref_y, _ = orc.stage2(lay.x_eval[0], lay.w_gate, lay.w_up, lay.w_down, np.arange(k))
+    assert rel_l2(layer.forward(x).cpu().numpy().reshape(-1), ref_y) <= OUT_RTOL
+    assert layer.error_word() == 0
 
 
 # ---------------------------------------------------------------------------
