@@ -29,7 +29,7 @@ class LayerInfo(ctypes.Structure):
     _fields_ = [
         ("d_model", ctypes.c_int), ("d_ff", ctypes.c_int), ("group", ctypes.c_int),
         ("k", ctypes.c_int), ("max_batch", ctypes.c_int), ("tau_x", ctypes.c_float),
-        ("stage1_col_slices", ctypes.c_int), ("stage1_row_slabs", ctypes.c_int),
+        ("stage1_col_slices", ctypes.c_int), ("stage1_ctas", ctypes.c_int),
         ("stage2_ctas", ctypes.c_int), ("stage2_ring_slots", ctypes.c_int),
         ("weight_bytes", ctypes.c_size_t), ("proxy_bytes", ctypes.c_size_t),
         ("workspace_bytes", ctypes.c_size_t),

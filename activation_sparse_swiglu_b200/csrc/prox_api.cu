@@ -99,8 +99,8 @@ prox_status alloc_workspace(prox_layer* L) {
   const size_t o_gt1 = take(prox::kMaxSlices * 4);
   const size_t o_off = take((prox::kMaxSlices + 1) * 4);
   const size_t o_idx = take(F * 4);
-  const size_t o_slab = take(d * 4);
-  const size_t o_slabc = take((size_t)L->R * 4);
+  const size_t o_s1p = take(prox::stage1_part_floats(L->P1) * 4);
+  const size_t o_s1c = take((size_t)L->C * 4);
   const size_t o_ypart = take((size_t)L->P * d * 4);
   const size_t o_stats = take(16);
   const size_t o_err = take(4);
@@ -124,8 +124,8 @@ prox_status alloc_workspace(prox_layer* L) {
   w.sel.sl_gt1 = reinterpret_cast<int32_t*>(b + o_gt1);
   w.sel.sl_off = reinterpret_cast<int32_t*>(b + o_off);
   w.idx_s = reinterpret_cast<int32_t*>(b + o_idx);
-  w.slab_idx = reinterpret_cast<int32_t*>(b + o_slab);
-  w.slab_cnt = reinterpret_cast<int32_t*>(b + o_slabc);
+  w.s1_part = reinterpret_cast<float*>(b + o_s1p);
+  w.s1_cnt = reinterpret_cast<int*>(b + o_s1c);
   w.ypart = reinterpret_cast<float*>(b + o_ypart);
   w.stats = reinterpret_cast<unsigned long long*>(b + o_stats);
   w.err = reinterpret_cast<int*>(b + o_err);
@@ -255,10 +255,15 @@ prox_status prox_layer_create(const uint16_t* W_gate, const uint16_t* W_up, cons
   L->tau = tau_x;
   L->device = dev;
   L->num_sms = sms;
-  prox::choose_stage1_grid(L->d, L->F, sms, &L->C, &L->R, &L->gps);
+  prox::choose_stage1_grid(L->d, L->F, sms, &L->C, &L->P1, &L->s1_lmax);
   prox::choose_stage2(L->d, L->F, sms, &L->P, &L->ring_slots, &L->stage2_producers,
                      &L->stage2_smem);
-  L->stage1_smem = prox::stage1_smem_bytes(L->gps);
+  L->stage1_smem = prox::stage1_smem_bytes(L->s1_lmax);
+  if (L->stage1_smem > (size_t)prox::kMaxSmemPerBlock) {
+    const size_t need = L->stage1_smem;
+    delete L;
+    return fail(PROX_EUNSUPPORTED, "Stage-1 shared memory %zu exceeds the per-CTA limit", need);
+  }
 
   cudaStream_t s = as_stream(stream);
   const size_t d = d_model, F = d_ff;
@@ -338,7 +343,7 @@ prox_status prox_layer_get_info(const prox_layer* L, prox_layer_info* info) {
   info->max_batch = L->max_batch;
   info->tau_x = L->tau;
   info->stage1_col_slices = L->C;
-  info->stage1_row_slabs = L->R;
+  info->stage1_ctas = L->P1;
   info->stage2_ctas = L->P;
   info->stage2_ring_slots = L->ring_slots;
   info->weight_bytes = (size_t)3 * L->F * L->d * 2;
@@ -455,7 +460,8 @@ prox_status prox_debug_stage1(prox_layer* L, const float* x, int32_t* idx_x, int
   prox::Stage1Taps t1;
   t1.g = g_tilde;
   t1.u = u_tilde;
-  t1.slabs = idx_x != nullptr || n_x != nullptr;
+  t1.idx_x = idx_x;
+  t1.n_x = n_x;
   PROX_CUDA(prox::launch_stage1(L, x, t1, s, false), "stage1 launch");
   PROX_CUDA(prox::launch_select(L, s, false), "select launch");
   // the rank-to-channel step of the forward path, stopped before the weight streaming
@@ -463,10 +469,6 @@ prox_status prox_debug_stage1(prox_layer* L, const float* x, int32_t* idx_x, int
   m.select_only = true;
   PROX_CUDA(prox::launch_stage2(L, x, m, s, false, true), "stage2 launch");
   PROX_CUDA(cudaMemsetAsync(L->ws.hist, 0, prox::kHistBins * 4, s), "clear histogram");
-  if (t1.slabs) {
-    int32_t* ix = idx_x ? idx_x : reinterpret_cast<int32_t*>(L->ws.stage_in);
-    PROX_CUDA(prox::launch_concat_slabs(L, ix, n_x, s), "concat launch");
-  }
   if (idx_s)
     PROX_CUDA(cudaMemcpyAsync(idx_s, L->ws.idx_s, (size_t)L->k * 4, cudaMemcpyDeviceToDevice, s),
               "copy idx_s");

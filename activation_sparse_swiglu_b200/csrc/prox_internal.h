@@ -2,6 +2,7 @@
 // the kernel launchers that the C ABI (prox_api.cu) strings together.
 #pragma once
 
+#include <algorithm>
 #include <cstddef>
 #include <cstdint>
 #include <cuda_runtime.h>
@@ -12,16 +13,16 @@ namespace prox {
 
 constexpr int kGroup = 128;          // proxy quantisation group (input rows)
 constexpr int kHistBins = 2048;      // first radix level: score bits [30:20]
-constexpr int kStage1Warps = 4;      // Stage-1 warps per CTA
-constexpr int kMaxGroupsPerSlab = 32; // bounds Stage-1 shared memory
-constexpr int kMaxCluster = 16;       // Stage-1 cluster size limit (row slabs per slice)
+constexpr int kStage1Warps = 16;     // Stage-1 warps per CTA (one CTA per SM)
 constexpr int kSelectCand = 4096;    // candidate buffer of the select (level-1 bin)
 constexpr int kSelectSlice = 256;    // channels per select CTA (and per rank-offset entry)
 constexpr int kMaxSlices = 160;      // >= d_ff / kSelectSlice + 1
 constexpr int kStage2Consumers = 8;  // Stage-2 consumer warps (+1 producer warp)
 constexpr int kReduceWarps = 16;     // output reduction: warps per 32 columns
 constexpr int kMaxDModel = 16384;
-constexpr int kMaxDff = 32768;       // the select keeps all scores in registers
+constexpr int kMaxDff = 32768;       // bounds the select's slice table (kMaxSlices)
+constexpr int kSmemPerSm = 233472;   // shared memory per SM on sm_100 (228 KB)
+constexpr int kMaxSmemPerBlock = 232448;  // opt-in dynamic shared memory per CTA (227 KB)
 constexpr int kHostChunkTokens = 64; // staging chunk of prox_ffn_forward_host
 
 // Select state shared by the select kernel and Stage 2.
@@ -43,8 +44,8 @@ struct Workspace {
   uint32_t* hist = nullptr;       // [kHistBins], zero between tokens (== sel.hist)
   SelectState sel;
   int32_t* idx_s = nullptr;       // [F] selected channels (first k valid)
-  int32_t* slab_idx = nullptr;    // [d] kept input rows, per slab (debug)
-  int32_t* slab_cnt = nullptr;    // [R] kept rows per slab (debug)
+  float* s1_part = nullptr;        // Stage-1 partial sums [P1][2][1024]
+  int* s1_cnt = nullptr;          // [C] Stage-1 row slices reported per slice, zero between tokens
   float* ypart = nullptr;         // Stage-2 output partials [P][d]
   unsigned long long* stats = nullptr;  // [2] sum n_x, tokens
   int* err = nullptr;             // device error word
@@ -60,8 +61,8 @@ struct prox_layer {
   int d = 0, F = 0, G = 0, k = 0, max_batch = 0;
   float tau = 0.f;
   int device = 0, num_sms = 0;
-  // Stage-1 geometry
-  int C = 0, R = 0, gps = 0;
+  // Stage-1 geometry: C column slices, P1 CTAs, at most s1_lmax rows per CTA
+  int C = 0, P1 = 0, s1_lmax = 0;
   // Stage-2 geometry
   int P = 0, ring_slots = 0, stage2_producers = 1;
   size_t stage2_smem = 0, stage1_smem = 0;
@@ -77,9 +78,10 @@ namespace prox {
 
 // ---- launchers (each returns the CUDA error of its launch) ----------------
 struct Stage1Taps {
-  float* g = nullptr;
-  float* u = nullptr;
-  bool slabs = false;  // write per-slab kept-row lists
+  float* g = nullptr;       // g~ [F]
+  float* u = nullptr;       // u~ [F]
+  int32_t* idx_x = nullptr; // kept input rows, ascending [d]
+  int32_t* n_x = nullptr;   // their number
 };
 // How Stage 2 obtains its channels.
 struct Stage2Launch {
@@ -94,8 +96,6 @@ struct Stage2Launch {
 cudaError_t launch_stage1(const prox_layer* L, const float* x, const Stage1Taps& taps,
                           cudaStream_t s, bool pdl);
 cudaError_t launch_select(const prox_layer* L, cudaStream_t s, bool pdl);
-cudaError_t launch_concat_slabs(const prox_layer* L, int32_t* idx_x, int32_t* n_x,
-                                cudaStream_t s);
 cudaError_t launch_stage2(const prox_layer* L, const float* x, const Stage2Launch& m,
                           cudaStream_t s, bool pdl, bool x_ready);
 cudaError_t launch_reduce(const prox_layer* L, float* out, cudaStream_t s, bool pdl);
@@ -117,9 +117,10 @@ cudaError_t launch_rmsnorm(const float* y, float* x, int rows, int d, float eps,
                            cudaStream_t s);
 cudaError_t launch_copy(const void* src, void* dst, size_t bytes, cudaStream_t s);
 
-// Stage-1 column slices and row slabs for a shape on `num_sms` SMs.
-void choose_stage1_grid(int d, int F, int num_sms, int* C, int* R, int* gps);
-size_t stage1_smem_bytes(int gps);
+// Stage-1 column slices, CTAs and per-CTA row capacity for a shape on `num_sms` SMs.
+void choose_stage1_grid(int d, int F, int num_sms, int* C, int* P1, int* lmax);
+size_t stage1_smem_bytes(int lmax);
+size_t stage1_part_floats(int P1);
 // Stage-2 ring depth and dynamic shared memory for d_model = d.
 void choose_stage2(int d, int F, int num_sms, int* P, int* slots, int* nprod, size_t* smem);
 

@@ -46,7 +46,8 @@ __device__ __forceinline__ void for_each_cand(const SelectArgs& a, bool listed, 
 }
 
 __global__ void __launch_bounds__(SEL_NT) select_kernel(SelectArgs a) {
-  __shared__ __align__(16) uint32_t s_h[1024];
+  __shared__ __align__(16) uint32_t s_h[kHistBins];
+  __shared__ unsigned long long s_c64[kSelectDirect];
   __shared__ uint32_t s_ck[kSelectCand];
   __shared__ int32_t s_ci[kSelectCand];
   __shared__ int s_sel[kMaxSlices + 1];
@@ -60,9 +61,13 @@ __global__ void __launch_bounds__(SEL_NT) select_kernel(SelectArgs a) {
   const int e = s * SEL_NT + tid;
   const bool valid = e < a.F;
   const uint32_t key = valid ? __float_as_uint(__ldcg(a.scores + e)) : 0u;
+  // the level-1 histogram (built by Stage 1) into shared memory: one round trip
+  for (int i = tid; i < kHistBins / 4; i += SEL_NT)
+    reinterpret_cast<uint4*>(s_h)[i] = __ldcg(reinterpret_cast<const uint4*>(a.st.hist) + i);
+  __syncthreads();
   if (warp == 0) {
     int b1, krem, n1;
-    warp_find_bin<kHistBins / 32, true>(a.st.hist, a.k, &b1, &krem, &n1);
+    warp_find_bin<kHistBins / 32, false>(s_h, a.k, &b1, &krem, &n1);
     if (lane == 0) {
       s_misc[0] = b1;
       s_misc[1] = krem;
@@ -115,18 +120,25 @@ __global__ void __launch_bounds__(SEL_NT) select_kernel(SelectArgs a) {
   uint32_t T;
   int tie_cut;
   if (listed && n1 <= kSelectDirect) {
-    // direct ranks: O(n1^2 / threads) comparisons, one phase
+    // Direct ranks.  The order (key descending, index ascending) is that of
+    // the composite key << 32 | (~index) descending, so a candidate's rank is
+    // the number of larger composites.  Padding with 0 (below every real
+    // composite) lets the comparison loop run in blocks of 8.
+    const int n8 = (n1 + 7) & ~7;
+    for (int i = tid; i < n8; i += SEL_NT)
+      s_c64[i] = i < n1 ? ((unsigned long long)s_ck[i] << 32) | (uint32_t)~(uint32_t)s_ci[i] : 0ull;
+    __syncthreads();
     for (int i = tid; i < n1; i += SEL_NT) {
-      const uint32_t ki = s_ck[i];
-      const int ii = s_ci[i];
+      const unsigned long long ci = s_c64[i];
       int rank = 0;
-      for (int j = 0; j < n1; ++j) {
-        const uint32_t kj = s_ck[j];
-        rank += kj > ki || (kj == ki && s_ci[j] < ii);
+      for (int j = 0; j < n8; j += 8) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) rank += s_c64[j + u] > ci;
       }
+      const int ii = s_ci[i];
       if (rank < krem) atomicAdd(&s_sel[ii / kSelectSlice], 1);
       if (rank == krem - 1) {
-        s_misc[7] = (int)ki;
+        s_misc[7] = (int)s_ck[i];
         s_misc[12] = ii;
       }
     }

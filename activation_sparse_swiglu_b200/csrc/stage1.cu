@@ -1,26 +1,30 @@
 // Stage 1 of the Prox decode step (Prox §4.1 "Stage 1: lightweight proxy
 // construction", §4.3 fused split-N proxy kernel).
 //
-// stage1_kernel -- one CTA per (column slice c, row slab r); the R slabs of a
-// column slice form one thread-block cluster:
-//   * a column slice is 512 bytes of an interleaved proxy row (16 blocks of 32
-//     channels; each block is 16 B of gate codes then 16 B of up codes), i.e.
-//     512 channels of both proxies; a warp reads one kept row's slice per load
-//     instruction (512 contiguous bytes), a lane owning one 16-byte chunk (32
-//     channels of one branch);
-//   * a row slab is `gps` whole quantisation groups (gps * 128 input rows).
-//   The CTA thresholds its slab of x (|x_i| >= tau) and compacts the kept rows
-//   in ascending order; its 4 warps stream those rows through a per-warp
-//   shared-memory ring with asynchronous 16-byte copies (cp.async, L2 only;
-//   each lane copies and later reads back its own chunk, so no barrier is
-//   needed), three batches of 8 rows in flight, and dequantise the INT4 codes
-//   in registers with fp32 (packed f32x2) arithmetic, accumulating per group
-//   and scaling once per group by the fp16 group scale.  The cluster's CTAs
-//   then add their partial sums through distributed shared memory in rank
-//   order (deterministic), each CTA scoring a share of the slice's channels:
-//   score_j = |SiLU(g~_j) u~_j|, also added to a 2048-bin histogram of its top
-//   bits -- the first level of the radix select.
+// stage1_kernel -- persistent, one CTA (16 warps) per SM.  The work is the set
+// of (column slice, kept input row) pairs: a column slice is 512 bytes of an
+// interleaved proxy row (16 blocks of 32 channels, each block 16 B of gate
+// codes then 16 B of up codes), i.e. 512 channels of both proxies.  Every CTA
+// thresholds all of x (|x_i| >= tau) and compacts the kept rows in ascending
+// order; the C * n_x pairs, slice-major, are then split into equal contiguous
+// ranges, one per CTA and, inside it, one per warp, so every warp streams the
+// same number of 512-byte row slices whatever the mask looks like.  A CTA's
+// range lies in at most two adjacent slices.
 //
+// A warp streams its rows through a shared-memory ring with asynchronous
+// 16-byte copies (cp.async, L2 only; each lane copies and later reads back its
+// own chunk, so no barrier is needed), four batches of four rows in flight,
+// and dequantises the INT4 codes in registers with fp32 (packed f32x2)
+// arithmetic, accumulating per quantisation group and scaling once per group
+// by the fp16 group scale.  A batch whose rows share one slice and one group
+// takes a path without any boundary checks.
+//
+// The warps' partial sums are combined in warp order into one partial vector
+// per touched slice and written to global memory.  Each CTA then adds its row
+// count to the slice's counter; the CTA that completes a slice adds that
+// slice's partials in CTA order (deterministic), scores the channels,
+// score_j = |SiLU(g~_j) u~_j|, and adds them to a 2048-bin histogram of
+// their top bits -- the first level of the radix select.
 #include "prox_device.cuh"
 #include "prox_internal.h"
 
@@ -29,46 +33,58 @@ namespace {
 
 constexpr int S1_NW = kStage1Warps;
 constexpr int S1_NT = S1_NW * 32;
+static_assert(kMaxDModel % S1_NT == 0, "rows per thread");
 constexpr int S1_SLICE = 512;   // bytes (= channels of both proxies) per column slice
-constexpr int S1_CHUNKS = 32;   // 16-byte chunks per slice (one per lane)
-constexpr int S1_PART = 1024;   // partial values per CTA: 32 chunks x 32 channels
-constexpr int S1_U = 8;         // rows per batch
-constexpr int S1_NB = 3;        // batches in flight per warp
-constexpr int S1_RING = S1_NB * S1_U * S1_SLICE;  // ring bytes per warp
+constexpr int S1_PART = 1024;   // partial values per slice: 32 chunks x 32 channels
+constexpr int S1_U = 4;         // rows per batch
+constexpr int S1_BATCH = S1_U * S1_SLICE;
+
+// Exponent words for the nibble decode: 2^23, 2^19, 2^15, 2^11, 2^7.
+struct Magic {
+  uint32_t e23, e19, e15, e11, e7;
+};
 
 struct Stage1Args {
   const float* x;
   const uint8_t* pq;
   const __half* ps;
   float tau;
-  int d, F, R, gps;
+  int d, F, C, lmax;
   float* scores;
   uint32_t* hist;
   unsigned long long* stats;
   float* g_dbg;
   float* u_dbg;
-  int32_t* slab_idx;
-  int32_t* slab_cnt;
+  int32_t* idx_x;   // optional: the kept rows, ascending
+  int32_t* n_x;     // optional: their number
+  float* part;      // [gridDim.x][2][S1_PART] partial sums per CTA and touched slice
+  int* cnt;         // [C] row slices reported per slice; zero between tokens
+  Magic mg;
 };
+
+// (w & M) | e in one instruction; e is a register (the exponents come from
+// kernel parameters, so they are not folded into a second immediate).
+template <uint32_t M>
+__device__ __forceinline__ float andor(uint32_t w, uint32_t e) {
+  uint32_t r;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(w), "n"(M), "r"(e));
+  return __uint_as_float(r);
+}
 
 // Eight INT4 codes of one 32-bit word (nibble p is channel 8w+p of the lane's
 // chunk, stored as q+8) into four float2 accumulators.  Each nibble is OR-ed
 // into the mantissa of a float whose exponent makes the nibble's lowest bit
-// worth exactly 1, so subtracting (2^e + 8) leaves q - 8 exactly; nibbles 5..7
+// worth exactly 1, so subtracting (2^e + 8) leaves q exactly; nibbles 5..7
 // are first shifted down by 12 bits.
-__device__ __forceinline__ void acc_word(float2* a, uint32_t w, float2 x2) {
+__device__ __forceinline__ void acc_word(float2* a, uint32_t w, float2 x2, const Magic& mg) {
   const uint32_t h = w >> 12;
-  const float2 v0 = __fadd2_rn(make_float2(__uint_as_float((w & 0x0000000Fu) | 0x4B000000u),
-                                           __uint_as_float((w & 0x000000F0u) | 0x49000000u)),
+  const float2 v0 = __fadd2_rn(make_float2(andor<0x0000000Fu>(w, mg.e23), andor<0x000000F0u>(w, mg.e19)),
                                make_float2(-8388616.0f, -524296.0f));
-  const float2 v1 = __fadd2_rn(make_float2(__uint_as_float((w & 0x00000F00u) | 0x47000000u),
-                                           __uint_as_float((w & 0x0000F000u) | 0x45000000u)),
+  const float2 v1 = __fadd2_rn(make_float2(andor<0x00000F00u>(w, mg.e15), andor<0x0000F000u>(w, mg.e11)),
                                make_float2(-32776.0f, -2056.0f));
-  const float2 v2 = __fadd2_rn(make_float2(__uint_as_float((w & 0x000F0000u) | 0x43000000u),
-                                           __uint_as_float((h & 0x00000F00u) | 0x47000000u)),
+  const float2 v2 = __fadd2_rn(make_float2(andor<0x000F0000u>(w, mg.e7), andor<0x00000F00u>(h, mg.e15)),
                                make_float2(-136.0f, -32776.0f));
-  const float2 v3 = __fadd2_rn(make_float2(__uint_as_float((h & 0x0000F000u) | 0x45000000u),
-                                           __uint_as_float((h & 0x000F0000u) | 0x43000000u)),
+  const float2 v3 = __fadd2_rn(make_float2(andor<0x0000F000u>(h, mg.e11), andor<0x000F0000u>(h, mg.e7)),
                                make_float2(-2056.0f, -136.0f));
   a[0] = __ffma2_rn(v0, x2, a[0]);
   a[1] = __ffma2_rn(v1, x2, a[1]);
@@ -88,291 +104,332 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-// All threads of all CTAs of the cluster: release our shared-memory writes,
-// acquire the others'.
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
-}
-__device__ __forceinline__ float ld_peer_f32(const float* local, uint32_t rank) {
-  uint32_t remote;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
-  return v;
+// CTA holding pair t of T pairs split over P CTAs (CTA i holds
+// [floor(T i / P), floor(T (i + 1) / P))); never an empty CTA.  T * P < 2^31
+// (T <= 64 * 16384, P <= 1024).
+__device__ __forceinline__ int cta_of(int t, int T, int P) {
+  return (int)(((unsigned)(t + 1) * (unsigned)P + (unsigned)T - 1u) / (unsigned)T) - 1;
 }
 
-__global__ void __launch_bounds__(S1_NT, 4) stage1_kernel(Stage1Args a) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  const int c = blockIdx.x, r = blockIdx.y;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int cl = lane;
-  const int gps = a.gps, slab_rows = gps * kGroup, row0 = r * slab_rows;
-  const int n16 = a.F >> 4, nblk = a.F >> 5;
-  const int c16 = c * S1_CHUNKS + cl;  // this lane's 16-byte chunk of a proxy row
-  const bool lane_ok = c16 < n16;
-
-  unsigned char* ring = smem;                                            // [NW][NB][U][512]
-  float* s_red = reinterpret_cast<float*>(smem + S1_NW * S1_RING);       // [NW][1024]
-  float* s_part = s_red + S1_NW * S1_PART;                               // [512]
-  uint4* s_scale = reinterpret_cast<uint4*>(s_part + S1_PART);           // [gps][32][4]
-  int2* s_rx = reinterpret_cast<int2*>(s_scale + gps * S1_CHUNKS * 4);   // [slab_rows]
-  int* s_scan = reinterpret_cast<int*>(s_rx + slab_rows);                // [33]
-
-  // Prologue (constant weights only): this slice's fp16 scales for the slab's
-  // groups, 64 bytes per chunk and group, loaded in batches of 8.
-  {
-    const int n = gps * S1_CHUNKS * 4;
-    for (int base = tid; base < n; base += 8 * S1_NT) {
-      uint4 v[8];
+// Sums the partials of slice c over the CTAs that hold its pairs (CTA order),
+// scores its channels and adds them to the histogram.  n_x == 0: all zero.
+// s_src: shared scratch for the contributors' partial offsets.
+__device__ void finish_slice(const Stage1Args& a, int c, int n_x, int P, int* s_src) {
+  const int t = threadIdx.x;
+  int nsrc = 0;
+  if (n_x > 0) {
+    const int T = a.C * n_x;
+    const int i_lo = cta_of(c * n_x, T, P);
+    nsrc = cta_of((c + 1) * n_x - 1, T, P) - i_lo + 1;
+    __syncthreads();  // s_src may still be read by a previous call
+    if (t < nsrc) {
+      const int i = i_lo + t;
+      const unsigned tlo = (unsigned)T * (unsigned)i / (unsigned)P;
+      const unsigned thi = (unsigned)T * (unsigned)(i + 1) / (unsigned)P;
+      // partial of CTA i for slice c (its first or second slice); -1: empty CTA
+      s_src[t] = thi > tlo ? (i * 2 + (c - (int)(tlo / (unsigned)n_x))) * S1_PART : -1;
+    }
+    __syncthreads();
+  }
+  // Thread t takes block blk = t % 16, channel j = t / 16 of the block: its gate
+  // and up sums are the adjacent partial elements j*32 + 2*blk and + 1, so a
+  // warp reads 256 contiguous bytes per contributor.
+  const int j = t >> 4, blk = t & 15;
+  const int m = blk * 32 + j;  // channel of the slice
+  const int ch = c * S1_SLICE + m;
+  if (t >= S1_SLICE || ch >= a.F) return;
+  const int e = j * 32 + 2 * blk;
+  float g = 0.f, u = 0.f;
+  for (int j0 = 0; j0 < nsrc; j0 += 8) {
+    float2 v[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int e = base + u * S1_NT;
-        v[u] = make_uint4(0u, 0u, 0u, 0u);
-        const int gl = e / (S1_CHUNKS * 4), ck = (e >> 2) % S1_CHUNKS, qd = e & 3;
-        const int cc = c * S1_CHUNKS + ck;
-        if (e < n && cc < n16) {
-          const int g = row0 / kGroup + gl;
-          const __half* src = a.ps + ((size_t)g * nblk + (cc >> 1)) * 64 + (cc & 1) * 32 + qd * 8;
-          v[u] = __ldg(reinterpret_cast<const uint4*>(src));
-        }
-      }
+    for (int q = 0; q < 8; ++q) {
+      const int off = j0 + q < nsrc ? s_src[j0 + q] : -1;
+      v[q] = off >= 0 ? __ldcg(reinterpret_cast<const float2*>(a.part + off + e))
+                      : make_float2(0.f, 0.f);
+    }
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int e = base + u * S1_NT;
-        if (e < n) s_scale[e] = v[u];
-      }
+    for (int q = 0; q < 8; ++q) {
+      g += v[q].x;
+      u += v[q].y;
     }
   }
+  const float sc = fabsf(silu_f32(g) * u);
+  a.scores[ch] = sc;
+  if (a.g_dbg) a.g_dbg[ch] = g;
+  if (a.u_dbg) a.u_dbg[ch] = u;
+  atomicAdd(a.hist + (__float_as_uint(sc) >> 20), 1u);
+}
+
+// Shared memory: per-warp rings of NB batches, per-warp group-scaled sums,
+// the CTA's kept rows, the stash of the warp that crosses a slice boundary.
+template <int NB>
+constexpr size_t stage1_smem(int lmax) {
+  return (size_t)S1_NW * NB * S1_BATCH + (size_t)S1_NW * S1_PART * 4 + (size_t)lmax * 12 +
+         (size_t)S1_PART * 4 + (37 + S1_NT) * 4;
+}
+
+template <int NB>
+__global__ void __launch_bounds__(S1_NT, 1) stage1_kernel(Stage1Args a) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  constexpr int S1_RING = NB * S1_BATCH;  // ring bytes per warp
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int P = gridDim.x, cta = blockIdx.x;
+  const int n16 = a.F >> 4, nblk = a.F >> 5;
+  const Magic mg = a.mg;
+
+  unsigned char* ring = smem;                                             // [NW][S1_RING]
+  float* s_tot = reinterpret_cast<float*>(smem + S1_NW * S1_RING);        // [NW][S1_PART]
+  int2* s_rx = reinterpret_cast<int2*>(s_tot + S1_NW * S1_PART);          // [lmax] (offset, x)
+  int* s_key = reinterpret_cast<int*>(s_rx + a.lmax);                     // [lmax] segment key
+  float* s_stash = reinterpret_cast<float*>(s_key + a.lmax);              // [S1_PART]
+  int* s_scan = reinterpret_cast<int*>(s_stash + S1_PART);                // [33]
+  int* s_m = s_scan + 33;                                                 // [4]
+  int* s_src = s_m + 4;                                                   // [S1_NT]
 
   pdl_wait();     // x and the workspace now belong to this token
-  pdl_trigger();  // let Stage 2 become resident
+  pdl_trigger();  // let the next kernel become resident
 
-  // Kept rows of this slab, ascending: thread t owns rows [t*rpt, (t+1)*rpt).
-  const int rpt = slab_rows / S1_NT;
-  const float* xs = a.x + row0 + tid * rpt;
+  // ---- kept rows of x, ascending: thread t owns rows [t*rpt, (t+1)*rpt) ----
+  const int rpt = (a.d + S1_NT - 1) / S1_NT;
+  const int r0 = tid * rpt;
+  const int r1 = min(r0 + rpt, a.d);
+  const bool vec = (rpt & 3) == 0;  // rows r0.. are 16-byte aligned
+  auto x_at = [&](int row) -> float4 {  // rows row..row+3 (those < r1)
+    if (vec) return __ldg(reinterpret_cast<const float4*>(a.x + row));
+    float4 v;
+    v.x = __ldg(a.x + row);
+    v.y = row + 1 < r1 ? __ldg(a.x + row + 1) : 0.f;
+    v.z = row + 2 < r1 ? __ldg(a.x + row + 2) : 0.f;
+    v.w = row + 3 < r1 ? __ldg(a.x + row + 3) : 0.f;
+    return v;
+  };
   int cnt = 0;
-  for (int i0 = 0; i0 < rpt; i0 += 8) {
-    float v[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) v[u] = (i0 + u < rpt) ? __ldg(xs + i0 + u) : 0.f;
-#pragma unroll
-    for (int u = 0; u < 8; ++u) cnt += (i0 + u < rpt) && (fabsf(v[u]) >= a.tau);
+  for (int row = r0; row < r1; row += 4) {
+    const float4 v = x_at(row);
+    cnt += (fabsf(v.x) >= a.tau) + (row + 1 < r1 && fabsf(v.y) >= a.tau) +
+           (row + 2 < r1 && fabsf(v.z) >= a.tau) + (row + 3 < r1 && fabsf(v.w) >= a.tau);
   }
-  int total;
-  int pos = block_exclusive_scan(cnt, s_scan, &total);
-  for (int i = 0; i < rpt; ++i) {
-    const float xv = __ldg(xs + i);
-    if (fabsf(xv) >= a.tau) s_rx[pos++] = make_int2(row0 + tid * rpt + i, __float_as_int(xv));
+  int n_x;
+  int pos = block_exclusive_scan(cnt, s_scan, &n_x);
+  if (n_x == 0) {
+    // nothing kept: g~ = u~ = 0 everywhere; CTA i scores slices i, i + P, ...
+    if (cta == 0 && tid == 0) {
+      if (a.n_x) *a.n_x = 0;
+    }
+    for (int c = cta; c < a.C; c += P) finish_slice(a, c, 0, P, s_src);
+    return;
   }
-  __syncthreads();
-  if (c == 0) {
-    if (tid == 0) atomicAdd(a.stats, (unsigned long long)total);
-    if (a.slab_idx) {
-      for (int e = tid; e < total; e += S1_NT) a.slab_idx[row0 + e] = s_rx[e].x;
-      if (tid == 0) a.slab_cnt[r] = total;
+  const unsigned T = (unsigned)a.C * (unsigned)n_x;   // T * P < 2^31
+  const unsigned tlo = T * (unsigned)cta / (unsigned)P, thi = T * (unsigned)(cta + 1) / (unsigned)P;
+  const int len = (int)(thi - tlo);      // <= n_x, since C < P
+  const int cA = (int)(tlo / (unsigned)n_x), pA = (int)(tlo % (unsigned)n_x);
+  const int l_split = n_x - pA;          // local rows l >= l_split lie in slice cA + 1
+  // local row l of this CTA is compacted position (pA + l) mod n_x
+  for (int row0 = r0; row0 < r1; row0 += 4) {
+    const float4 v4 = x_at(row0);
+    const float vv[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int row = row0 + q;
+      if (row < r1 && fabsf(vv[q]) >= a.tau) {
+        int l = pos - pA;
+        if (l < 0) l += n_x;
+        if (l < len) {
+          // the row slice's byte offset in the proxy, and its segment key
+          // (slice, quantisation group), nondecreasing over the CTA's rows
+          const int sl = l >= l_split ? 1 : 0;
+          s_rx[l] = make_int2(row * a.F + (cA + sl) * S1_SLICE, __float_as_int(vv[q]));
+          s_key[l] = sl * 128 + (row >> 7);
+        }
+        if (cta == 0 && a.idx_x) a.idx_x[pos] = row;
+        ++pos;
+      }
     }
   }
+  if (cta == 0 && tid == 0) {
+    atomicAdd(a.stats, (unsigned long long)n_x);
+    if (a.n_x) *a.n_x = n_x;
+  }
+  __syncthreads();
 
-  // Warp w takes positions w, w + 4, w + 8, ... of the compacted list, in
-  // batches of 8 rows through its ring (NB batches in flight).
-  const int nw = total > warp ? (total - warp + S1_NW - 1) / S1_NW : 0;
-  const int nbw = (nw + S1_U - 1) / S1_U;
+  // ---- this warp's local rows [wl0, wl1) ----
+  const int wl0 = (int)((long long)len * warp / S1_NW);
+  const int wl1 = (int)((long long)len * (warp + 1) / S1_NW);
+  const int nbw = (wl1 - wl0 + S1_U - 1) / S1_U;
   unsigned char* wring = ring + warp * S1_RING + lane * 16;
-  const uint8_t* colp = a.pq + (size_t)(lane_ok ? c16 : 0) * 16;
-  auto issue = [&](int j) {
-    if (j < nbw && lane_ok) {
-      unsigned char* dst = wring + (j % S1_NB) * (S1_U * S1_SLICE);
+  const uint8_t* pq_lane = a.pq + lane * 16;
+  float* wtot = s_tot + warp * S1_PART + lane;  // element j*32 + lane: channel j of the chunk
 #pragma unroll
-      for (int u = 0; u < S1_U; ++u) {
-        const int jj = j * S1_U + u;
-        if (jj < nw) cp_async16(dst + u * S1_SLICE, colp + (size_t)s_rx[warp + S1_NW * jj].x * a.F);
+  for (int j = 0; j < 32; ++j) wtot[j * 32] = 0.f;
+  // Only the last slice can be narrower than 512 bytes; a warp with rows there
+  // checks each lane's chunk before copying it.
+  const bool checked = (a.F % S1_SLICE) != 0 && wl1 > wl0 &&
+                       cA + (wl1 - 1 >= l_split ? 1 : 0) == a.C - 1;
+  auto issue = [&](int j) {
+    if (j < nbw) {
+      unsigned char* dst = wring + (j % NB) * S1_BATCH;
+      const int l0 = wl0 + j * S1_U;
+      if (!checked && l0 + S1_U <= wl1) {
+#pragma unroll
+        for (int u = 0; u < S1_U; ++u)
+          cp_async16(dst + u * S1_SLICE, pq_lane + (uint32_t)s_rx[l0 + u].x);
+      } else {
+        for (int u = 0; u < S1_U && l0 + u < wl1; ++u) {
+          const int l = l0 + u;
+          const int c16 = (cA + (l >= l_split ? 1 : 0)) * 32 + lane;
+          if (c16 < n16) cp_async16(dst + u * S1_SLICE, pq_lane + (uint32_t)s_rx[l].x);
+        }
       }
     }
     cp_async_commit();
   };
-  float2 acc[16], tot[16];
+  float2 acc[16];
 #pragma unroll
-  for (int h = 0; h < 16; ++h) acc[h] = tot[h] = make_float2(0.f, 0.f);
-  int cur_g = -1;
+  for (int h = 0; h < 16; ++h) acc[h] = make_float2(0.f, 0.f);
+  uint4 sc[4];            // fp16 scales of the current (slice, group) for this lane's chunk
+  int cur_key = -1, cur_g = -1;
+  float okf = 0.f;        // 1 when this lane's chunk exists in the current slice
+  // group end: tot += scale * acc (tot in shared memory), acc = 0
+  auto flush = [&]() {
 #pragma unroll
-  for (int j = 0; j < S1_NB - 1; ++j) issue(j);
+    for (int qd = 0; qd < 4; ++qd) {
+      const uint32_t sw[4] = {sc[qd].x, sc[qd].y, sc[qd].z, sc[qd].w};
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int h = qd * 4 + m;
+        const float2 s2 = __half22float2(*reinterpret_cast<const __half2*>(&sw[m]));
+        wtot[(2 * h) * 32] = fmaf(s2.x, acc[h].x, wtot[(2 * h) * 32]);
+        wtot[(2 * h + 1) * 32] = fmaf(s2.y, acc[h].y, wtot[(2 * h + 1) * 32]);
+        acc[h] = make_float2(0.f, 0.f);
+      }
+    }
+  };
+  auto row_fma = [&](const unsigned char* src, float xv) {
+    const uint4 v = *reinterpret_cast<const uint4*>(src);
+    const float2 x2 = make_float2(xv * okf, xv * okf);
+    acc_word(acc + 0, v.x, x2, mg);
+    acc_word(acc + 4, v.y, x2, mg);
+    acc_word(acc + 8, v.z, x2, mg);
+    acc_word(acc + 12, v.w, x2, mg);
+  };
+#pragma unroll
+  for (int j = 0; j < NB - 1; ++j) issue(j);
   for (int j = 0; j < nbw; ++j) {
-    issue(j + S1_NB - 1);
-    cp_async_wait<S1_NB - 1>();  // this lane's copies of batch j have landed
-    const unsigned char* src = wring + (j % S1_NB) * (S1_U * S1_SLICE);
+    issue(j + NB - 1);
+    cp_async_wait<NB - 1>();  // this lane's copies of batch j have landed
+    const unsigned char* src = wring + (j % NB) * S1_BATCH;
+    const int first = wl0 + j * S1_U;
+    const int last = min(first + S1_U, wl1);
+    if (last - first == S1_U && s_key[first] == cur_key && s_key[last - 1] == cur_key) {
+      // one segment: no boundary checks
 #pragma unroll
-    for (int u = 0; u < S1_U; ++u) {
-      const int jj = j * S1_U + u;
-      if (jj < nw) {
-        const int2 rx = s_rx[warp + S1_NW * jj];
-        const int gl = (rx.x - row0) >> 7;
-        if (gl != cur_g) {
-          if (cur_g >= 0) {
-            const uint4* sc = s_scale + (cur_g * S1_CHUNKS + cl) * 4;
+      for (int u = 0; u < S1_U; ++u)
+        row_fma(src + u * S1_SLICE, __int_as_float(s_rx[first + u].y));
+    } else {
+      for (int l = first; l < last; ++l) {
+        const int key = s_key[l];
+        if (key != cur_key) {
+          if (cur_g >= 0) flush();
+          if (cur_key >= 0 && (key >> 7) != (cur_key >> 7)) {
+            // the warp crosses into the next slice: park the first slice's sums
 #pragma unroll
-            for (int qd = 0; qd < 4; ++qd) {
-              const uint4 s4 = sc[qd];
-              const uint32_t sw[4] = {s4.x, s4.y, s4.z, s4.w};
-#pragma unroll
-              for (int m = 0; m < 4; ++m) {
-                const float2 s2 = __half22float2(*reinterpret_cast<const __half2*>(&sw[m]));
-                tot[qd * 4 + m] = __ffma2_rn(s2, acc[qd * 4 + m], tot[qd * 4 + m]);
-                acc[qd * 4 + m] = make_float2(0.f, 0.f);
-              }
+            for (int j2 = 0; j2 < 32; ++j2) {
+              s_stash[j2 * 32 + lane] = wtot[j2 * 32];
+              wtot[j2 * 32] = 0.f;
             }
           }
-          cur_g = gl;
+          cur_key = key;
+          cur_g = key & 127;
+          const int c16 = (cA + (key >> 7)) * 32 + lane;
+          okf = c16 < n16 ? 1.f : 0.f;
+#pragma unroll
+          for (int qd = 0; qd < 4; ++qd) sc[qd] = make_uint4(0u, 0u, 0u, 0u);
+          if (c16 < n16) {
+            const uint4* sp = reinterpret_cast<const uint4*>(
+                a.ps + ((size_t)cur_g * nblk + (c16 >> 1)) * 64 + (c16 & 1) * 32);
+#pragma unroll
+            for (int qd = 0; qd < 4; ++qd) sc[qd] = __ldg(sp + qd);
+          }
         }
-        const uint4 v = lane_ok ? *reinterpret_cast<const uint4*>(src + u * S1_SLICE)
-                                : make_uint4(0x88888888u, 0x88888888u, 0x88888888u, 0x88888888u);
-        const float xv = __int_as_float(rx.y);
-        const float2 x2 = make_float2(xv, xv);
-        acc_word(acc + 0, v.x, x2);
-        acc_word(acc + 4, v.y, x2);
-        acc_word(acc + 8, v.z, x2);
-        acc_word(acc + 12, v.w, x2);
+        row_fma(src + (l - first) * S1_SLICE, __int_as_float(s_rx[l].y));
       }
     }
   }
   cp_async_wait<0>();
-  if (cur_g >= 0) {
-    const uint4* sc = s_scale + (cur_g * S1_CHUNKS + cl) * 4;
-#pragma unroll
-    for (int qd = 0; qd < 4; ++qd) {
-      const uint4 s4 = sc[qd];
-      const uint32_t sw[4] = {s4.x, s4.y, s4.z, s4.w};
-#pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const float2 s2 = __half22float2(*reinterpret_cast<const __half2*>(&sw[m]));
-        tot[qd * 4 + m] = __ffma2_rn(s2, acc[qd * 4 + m], tot[qd * 4 + m]);
-      }
-    }
-  }
-  // Combine the warps in a fixed order.  Partial element e = j*32 + chunk for
-  // channel j of a chunk.
-  {
-    float* red = s_red + warp * S1_PART;
-#pragma unroll
-    for (int h = 0; h < 16; ++h) {
-      red[(2 * h) * 32 + cl] = tot[h].x;
-      red[(2 * h + 1) * 32 + cl] = tot[h].y;
-    }
+  if (cur_g >= 0) flush();
+  __syncthreads();
+
+  // ---- the CTA's partials per touched slice (warp order), then report ----
+  // warp w's share: bit 0 -> its sums belong to the CTA's first slice, bit 1 ->
+  // to the second, both -> it crossed (first-slice sums in the stash)
+  if (tid < S1_NW) {
+    const int l0 = (int)((long long)len * tid / S1_NW), l1 = (int)((long long)len * (tid + 1) / S1_NW);
+    s_src[tid] = l1 <= l0 ? 0 : (l1 <= l_split ? 1 : (l0 >= l_split ? 2 : 3));
   }
   __syncthreads();
+  const int nsl = len > l_split ? 2 : 1;
   for (int e = tid; e < S1_PART; e += S1_NT) {
-    float sum = s_red[e];
+    float p0 = 0.f, p1 = 0.f;
 #pragma unroll
-    for (int w = 1; w < S1_NW; ++w) sum += s_red[w * S1_PART + e];
-    s_part[e] = sum;
-  }
-
-  // Slab partials -> channel scores: the CTA of cluster rank q scores channels
-  // [q*CH, (q+1)*CH) of the slice.  TPC threads share a channel, thread
-  // `sub` adding peers sub, sub+TPC, ... (all loads in flight); the TPC sums
-  // are then added in a fixed order.
-  cluster_sync_all();
-  const uint32_t q = cluster_rank();
-  const int CH = (S1_SLICE + a.R - 1) / a.R;
-  const int TPC = CH * 4 <= S1_NT ? 4 : (CH * 2 <= S1_NT ? 2 : 1);
-  for (int base = 0; base < CH; base += S1_NT / TPC) {
-    const int mc = base + tid / TPC, sub = tid % TPC;
-    const int m = (int)q * CH + mc;
-    const int ch = c * S1_SLICE + m;
-    const bool ok = mc < CH && m < S1_SLICE && ch < a.F;
-    float g = 0.f, u = 0.f;
-    if (ok) {
-      const int blk = m >> 5, jj = m & 31;
-      const int eg = jj * 32 + 2 * blk, eu = eg + 1;
-      float vg[kMaxCluster / 1], vu[kMaxCluster / 1];
-#pragma unroll
-      for (int i = 0; i < kMaxCluster; ++i) {
-        const int rr = sub + i * TPC;
-        vg[i] = rr < a.R ? ld_peer_f32(s_part + eg, (uint32_t)rr) : 0.f;
-        vu[i] = rr < a.R ? ld_peer_f32(s_part + eu, (uint32_t)rr) : 0.f;
-      }
-#pragma unroll
-      for (int i = 0; i < kMaxCluster; ++i) {
-        g += vg[i];
-        u += vu[i];
+    for (int w = 0; w < S1_NW; ++w) {
+      const int kind = s_src[w];
+      const float v = s_tot[w * S1_PART + e];
+      if (kind == 1) p0 += v;
+      if (kind == 2) p1 += v;
+      if (kind == 3) {
+        p0 += s_stash[e];
+        p1 += v;
       }
     }
-    // lanes sub = 0..TPC-1 of a channel are adjacent: combine in a fixed order
-    if (TPC >= 2) {
-      g += __shfl_xor_sync(0xffffffffu, g, 1);
-      u += __shfl_xor_sync(0xffffffffu, u, 1);
-    }
-    if (TPC >= 4) {
-      g += __shfl_xor_sync(0xffffffffu, g, 2);
-      u += __shfl_xor_sync(0xffffffffu, u, 2);
-    }
-    if (ok && sub == 0) {
-      const float sc = fabsf(silu_f32(g) * u);
-      a.scores[ch] = sc;
-      if (a.g_dbg) a.g_dbg[ch] = g;
-      if (a.u_dbg) a.u_dbg[ch] = u;
-      atomicAdd(a.hist + (__float_as_uint(sc) >> 20), 1u);
-    }
+    a.part[((size_t)cta * 2) * S1_PART + e] = p0;
+    if (nsl == 2) a.part[((size_t)cta * 2 + 1) * S1_PART + e] = p1;
   }
-  cluster_sync_all();  // keep our shared memory alive until the peers have read it
-}
-
-// Debug tap: concatenate the per-slab kept-row lists written by stage1_kernel
-// into one ascending list idx_x (and its length n_x).
-__global__ void __launch_bounds__(256) concat_slabs_kernel(const int32_t* slab_idx,
-                                                           const int32_t* slab_cnt, int R,
-                                                           int slab_rows, int32_t* idx_x,
-                                                           int32_t* n_x) {
-  __shared__ int s_off[kMaxGroupsPerSlab * 4 + 1];
-  if (threadIdx.x == 0) {
-    int off = 0;
-    for (int r = 0; r < R; ++r) {
-      s_off[r] = off;
-      off += slab_cnt[r];
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    const int rows0 = min(len, l_split);
+    int done = 0;
+    if (len > 0) {
+      if (atomicAdd(a.cnt + cA, rows0) + rows0 == n_x) done |= 1;
+      if (nsl == 2 && atomicAdd(a.cnt + cA + 1, len - rows0) + (len - rows0) == n_x) done |= 2;
     }
-    s_off[R] = off;
-    if (n_x) *n_x = off;
+    __threadfence();
+    s_m[0] = done;
   }
   __syncthreads();
-  for (int r = 0; r < R; ++r) {
-    const int n = s_off[r + 1] - s_off[r];
-    for (int e = threadIdx.x; e < n; e += blockDim.x)
-      idx_x[s_off[r] + e] = slab_idx[(size_t)r * slab_rows + e];
+  const int done = s_m[0];
+  for (int k = 0; k < 2; ++k) {
+    if (done & (1 << k)) {
+      finish_slice(a, cA + k, n_x, P, s_src);
+      if (tid == 0) a.cnt[cA + k] = 0;  // ready for the next token
+    }
   }
 }
 
 }  // namespace
 
-void choose_stage1_grid(int d, int F, int num_sms, int* C, int* R, int* gps) {
-  const int G = d / kGroup;
+void choose_stage1_grid(int d, int F, int num_sms, int* C, int* P, int* lmax) {
   *C = (F + S1_SLICE - 1) / S1_SLICE;
-  // The row slabs of a column slice form one cluster (at most 16 CTAs).  Take
-  // the most slabs that still keep the grid within one wave of 4 CTAs per SM.
-  const int cap = 4 * num_sms;
-  int best = 1;
-  for (int r = 1; r <= kMaxCluster && r <= G; ++r) {
-    if (G % r || G / r > kMaxGroupsPerSlab) continue;
-    if (r == 1 || (long)(*C) * r <= cap) best = r;
-  }
-  *R = best;
-  *gps = G / best;
+  *P = std::max(num_sms, *C + 1);  // a CTA's range then never spans more than two slices
+  // a CTA's share of the C * n_x pairs, n_x <= d
+  *lmax = (int)(((long long)(*C) * d + *P - 1) / *P) + 1;
 }
 
-size_t stage1_smem_bytes(int gps) {
-  return (size_t)S1_NW * S1_RING + (size_t)(S1_NW + 1) * S1_PART * 4 +
-         (size_t)gps * S1_CHUNKS * 64 + (size_t)gps * kGroup * 8 + 33 * 4;
+size_t stage1_smem_bytes(int lmax) {
+  // four batches in flight when they fit, else three
+  const size_t s4 = stage1_smem<4>(lmax);
+  return s4 <= (size_t)kMaxSmemPerBlock ? s4 : stage1_smem<3>(lmax);
 }
+
+size_t stage1_part_floats(int P) { return (size_t)P * 2 * S1_PART; }
 
 cudaError_t setup_stage1_kernels() {
-  cudaError_t e = cudaFuncSetAttribute(stage1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)stage1_smem_bytes(kMaxGroupsPerSlab));
+  cudaError_t e = cudaFuncSetAttribute(stage1_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kMaxSmemPerBlock);
   if (e != cudaSuccess) return e;
-  // clusters of up to 16 CTAs (a size B200 supports beyond the portable 8)
-  return cudaFuncSetAttribute(stage1_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  return cudaFuncSetAttribute(stage1_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              kMaxSmemPerBlock);
 }
 
 cudaError_t launch_stage1(const prox_layer* L, const float* x, const Stage1Taps& taps,
@@ -384,38 +441,32 @@ cudaError_t launch_stage1(const prox_layer* L, const float* x, const Stage1Taps&
   a.tau = L->tau;
   a.d = L->d;
   a.F = L->F;
-  a.R = L->R;
-  a.gps = L->gps;
+  a.C = L->C;
+  a.lmax = L->s1_lmax;
   a.scores = L->ws.scores;
   a.hist = L->ws.hist;
   a.stats = L->ws.stats;
   a.g_dbg = taps.g;
   a.u_dbg = taps.u;
-  a.slab_idx = taps.slabs ? L->ws.slab_idx : nullptr;
-  a.slab_cnt = L->ws.slab_cnt;
+  a.idx_x = taps.idx_x;
+  a.n_x = taps.n_x;
+  a.part = L->ws.s1_part;
+  a.cnt = L->ws.s1_cnt;
+  a.mg = Magic{0x4B000000u, 0x49000000u, 0x47000000u, 0x45000000u, 0x43000000u};
 
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(L->C, L->R, 1);
+  cfg.gridDim = dim3(L->P1, 1, 1);
   cfg.blockDim = dim3(S1_NT, 1, 1);
   cfg.dynamicSmemBytes = L->stage1_smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[2];
+  cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
-  attr[1].id = cudaLaunchAttributeClusterDimension;
-  attr[1].val.clusterDim.x = 1;
-  attr[1].val.clusterDim.y = (unsigned)L->R;
-  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, stage1_kernel, a);
-}
-
-cudaError_t launch_concat_slabs(const prox_layer* L, int32_t* idx_x, int32_t* n_x,
-                                cudaStream_t s) {
-  concat_slabs_kernel<<<1, 256, 0, s>>>(L->ws.slab_idx, L->ws.slab_cnt, L->R, L->gps * kGroup,
-                                        idx_x, n_x);
-  return cudaGetLastError();
+  cfg.numAttrs = 1;
+  if (L->stage1_smem == stage1_smem<4>(L->s1_lmax))
+    return cudaLaunchKernelEx(&cfg, stage1_kernel<4>, a);
+  return cudaLaunchKernelEx(&cfg, stage1_kernel<3>, a);
 }
 
 }  // namespace prox

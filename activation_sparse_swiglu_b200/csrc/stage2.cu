@@ -104,26 +104,6 @@ __device__ void ranks_to_channels(const Stage2Args& a, int t0, int t1, int* s_id
   }
 }
 
-__device__ __forceinline__ void load_x(float* xs, const float* x, int d, int tid, int nt) {
-  for (int e = tid * 4; e < d; e += nt * 4)
-    *reinterpret_cast<float4*>(xs + e) = __ldg(reinterpret_cast<const float4*>(x + e));
-}
-
-// Dot products of 8 consecutive bf16 weights (one uint4) with 8 fp32 x values.
-__device__ __forceinline__ void dot8(float2 (&acc)[4], const uint4& w, const float4& xa,
-                                     const float4& xb) {
-  acc[0] = __ffma2_rn(bf16x2_to_f2(w.x), make_float2(xa.x, xa.y), acc[0]);
-  acc[1] = __ffma2_rn(bf16x2_to_f2(w.y), make_float2(xa.z, xa.w), acc[1]);
-  acc[2] = __ffma2_rn(bf16x2_to_f2(w.z), make_float2(xb.x, xb.y), acc[2]);
-  acc[3] = __ffma2_rn(bf16x2_to_f2(w.w), make_float2(xb.z, xb.w), acc[3]);
-}
-
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
-
 // MAXM = ceil(d_model / 2048): 8-element chunks per thread and column.
 template <int MAXM>
 __global__ void __launch_bounds__(S2_THREADS, 1) stage2_kernel(Stage2Args a) {

@@ -65,7 +65,7 @@ typedef struct prox_layer prox_layer; /* opaque */
 typedef struct prox_layer_info {
   int d_model, d_ff, group, k, max_batch;
   float tau_x;
-  int stage1_col_slices, stage1_row_slabs; /* Stage-1 grid (C x R)          */
+  int stage1_col_slices, stage1_ctas; /* Stage-1 column slices and CTAs */
   int stage2_ctas, stage2_ring_slots;      /* Stage-2 grid and TMA ring depth */
   size_t weight_bytes;    /* bf16 gate/up records + bf16 W_down             */
   size_t proxy_bytes;     /* INT4 codes + fp16 scales                        */
