@@ -17,9 +17,9 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libprox.so")
 
-SOURCES = ["prox_api.cu", "stage1.cu", "select.cu", "stage2.cu", "pack.cu", "calibrate.cu",
+SOURCES = ["prox_api.cu", "stage1.cu", "stage2.cu", "pack.cu", "calibrate.cu",
            "misc.cu"]
-HEADERS = ["prox_device.cuh", "prox_internal.h"]
+HEADERS = ["prox_device.cuh", "prox_internal.h", "select.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

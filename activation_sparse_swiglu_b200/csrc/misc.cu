@@ -1,5 +1,6 @@
-// Harness kernels: unit-gain RMSNorm between stacked layers, and a streaming
-// copy used to measure the HBM bandwidth that rooflines are quoted against.
+// Harness kernels: unit-gain RMSNorm between stacked layers, a streaming copy
+// used to measure the HBM bandwidth that rooflines are quoted against, and the
+// debug compaction of a per-channel selection mask into an ascending list.
 #include "prox_device.cuh"
 #include "prox_internal.h"
 
@@ -48,7 +49,26 @@ __global__ void __launch_bounds__(256) copy_kernel(const uint4* __restrict__ src
   for (; i < n; i += stride) dst[i] = ld_stream_v4(src + i);
 }
 
+// One CTA of 1024 threads: thread t owns entries [t*per, (t+1)*per).
+__global__ void __launch_bounds__(1024) mask_to_list_kernel(const int32_t* __restrict__ mask,
+                                                            int n, int32_t* __restrict__ list) {
+  __shared__ int s_scan[33];
+  const int per = (n + 1023) / 1024;
+  const int lo = min((int)threadIdx.x * per, n), hi = min(lo + per, n);
+  int c = 0;
+  for (int i = lo; i < hi; ++i) c += mask[i] != 0;
+  int total;
+  int pos = block_exclusive_scan(c, s_scan, &total);
+  for (int i = lo; i < hi; ++i)
+    if (mask[i] != 0) list[pos++] = i;
+}
+
 }  // namespace
+
+cudaError_t launch_mask_to_list(const int32_t* mask, int n, int32_t* list, cudaStream_t s) {
+  mask_to_list_kernel<<<1, 1024, 0, s>>>(mask, n, list);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_rmsnorm(const float* y, float* x, int rows, int d, float eps,
                            cudaStream_t s) {

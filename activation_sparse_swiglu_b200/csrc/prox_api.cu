@@ -92,12 +92,9 @@ prox_status alloc_workspace(prox_layer* L) {
   const size_t o_scores = take(F * 4);
   const size_t o_g = take(F * 4);
   const size_t o_u = take(F * 4);
-  const size_t o_hist = take(prox::kHistBins * 4);
-  const size_t o_sst = take(8 * 4);
-  const size_t o_ck = take(prox::kSelectCand * 4);
-  const size_t o_ci = take(prox::kSelectCand * 4);
-  const size_t o_gt1 = take(prox::kMaxSlices * 4);
-  const size_t o_off = take((prox::kMaxSlices + 1) * 4);
+  const size_t o_hist = take(prox::kScoreBins * 4);
+  const size_t o_bucket = take((size_t)prox::kScoreBins * prox::kBucketCap * 8);
+  const size_t o_mask = take(F * 4);
   const size_t o_idx = take(F * 4);
   const size_t o_s1p = take(prox::stage1_part_floats(L->P1) * 4);
   const size_t o_s1c = take((size_t)L->C * 4);
@@ -117,12 +114,8 @@ prox_status alloc_workspace(prox_layer* L) {
   w.g_dbg = reinterpret_cast<float*>(b + o_g);
   w.u_dbg = reinterpret_cast<float*>(b + o_u);
   w.hist = reinterpret_cast<uint32_t*>(b + o_hist);
-  w.sel.hist = w.hist;
-  w.sel.state = reinterpret_cast<uint32_t*>(b + o_sst);
-  w.sel.cand_key = reinterpret_cast<uint32_t*>(b + o_ck);
-  w.sel.cand_idx = reinterpret_cast<int32_t*>(b + o_ci);
-  w.sel.sl_gt1 = reinterpret_cast<int32_t*>(b + o_gt1);
-  w.sel.sl_off = reinterpret_cast<int32_t*>(b + o_off);
+  w.bucket = reinterpret_cast<uint2*>(b + o_bucket);
+  w.sel_mask = reinterpret_cast<int32_t*>(b + o_mask);
   w.idx_s = reinterpret_cast<int32_t*>(b + o_idx);
   w.s1_part = reinterpret_cast<float*>(b + o_s1p);
   w.s1_cnt = reinterpret_cast<int*>(b + o_s1c);
@@ -138,7 +131,6 @@ prox::Stage2Launch topk_launch(const prox_layer* L) {
   prox::Stage2Launch m;
   m.mode = 1;
   m.k = L->k;
-  m.idx_out = L->ws.idx_s;
   return m;
 }
 
@@ -146,7 +138,6 @@ prox::Stage2Launch topk_launch(const prox_layer* L) {
 cudaError_t enqueue_token(const prox_layer* L, const float* x, float* out, cudaStream_t s) {
   cudaError_t e;
   if ((e = prox::launch_stage1(L, x, prox::Stage1Taps{}, s, true)) != cudaSuccess) return e;
-  if ((e = prox::launch_select(L, s, true)) != cudaSuccess) return e;
   if ((e = prox::launch_stage2(L, x, topk_launch(L), s, true, true)) != cudaSuccess) return e;
   return prox::launch_reduce(L, out, s, true);
 }
@@ -442,7 +433,6 @@ prox_status prox_ffn_forward_profiled(const prox_layer* L, const float* x, float
   auto ev = [&](int i) { return reinterpret_cast<cudaEvent_t>(events[i]); };
   PROX_CUDA(cudaEventRecord(ev(0), s), "cudaEventRecord");
   PROX_CUDA(prox::launch_stage1(L, x, prox::Stage1Taps{}, s, false), "stage1 launch");
-  PROX_CUDA(prox::launch_select(L, s, false), "select launch");
   PROX_CUDA(cudaEventRecord(ev(1), s), "cudaEventRecord");
   PROX_CUDA(prox::launch_stage2(L, x, topk_launch(L), s, false, true), "stage2 launch");
   PROX_CUDA(cudaEventRecord(ev(2), s), "cudaEventRecord");
@@ -463,15 +453,14 @@ prox_status prox_debug_stage1(prox_layer* L, const float* x, int32_t* idx_x, int
   t1.idx_x = idx_x;
   t1.n_x = n_x;
   PROX_CUDA(prox::launch_stage1(L, x, t1, s, false), "stage1 launch");
-  PROX_CUDA(prox::launch_select(L, s, false), "select launch");
-  // the rank-to-channel step of the forward path, stopped before the weight streaming
+  // the selection step of the forward path, stopped before the weight streaming
   prox::Stage2Launch m = topk_launch(L);
   m.select_only = true;
+  m.sel_mask = L->ws.sel_mask;
   PROX_CUDA(prox::launch_stage2(L, x, m, s, false, true), "stage2 launch");
-  PROX_CUDA(cudaMemsetAsync(L->ws.hist, 0, prox::kHistBins * 4, s), "clear histogram");
+  PROX_CUDA(cudaMemsetAsync(L->ws.hist, 0, prox::kScoreBins * 4, s), "clear histogram");
   if (idx_s)
-    PROX_CUDA(cudaMemcpyAsync(idx_s, L->ws.idx_s, (size_t)L->k * 4, cudaMemcpyDeviceToDevice, s),
-              "copy idx_s");
+    PROX_CUDA(prox::launch_mask_to_list(L->ws.sel_mask, L->F, idx_s, s), "mask compaction launch");
   return PROX_OK;
 }
 

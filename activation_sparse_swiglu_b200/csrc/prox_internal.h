@@ -12,7 +12,10 @@
 namespace prox {
 
 constexpr int kGroup = 128;          // proxy quantisation group (input rows)
-constexpr int kHistBins = 2048;      // first radix level: score bits [30:20]
+constexpr int kHistBins = 2048;      // calibration radix levels: 11 bits
+constexpr int kScoreShift = 18;      // top-k select, first radix level: score bits [30:18]
+constexpr int kScoreBins = 8192;
+constexpr int kBucketCap = 64;       // (key, channel) entries kept per histogram bin
 constexpr int kStage1Warps = 16;     // Stage-1 warps per CTA (one CTA per SM)
 constexpr int kSelectCand = 4096;    // candidate buffer of the select (level-1 bin)
 constexpr int kSelectSlice = 256;    // channels per select CTA (and per rank-offset entry)
@@ -25,25 +28,15 @@ constexpr int kSmemPerSm = 233472;   // shared memory per SM on sm_100 (228 KB)
 constexpr int kMaxSmemPerBlock = 232448;  // opt-in dynamic shared memory per CTA (227 KB)
 constexpr int kHostChunkTokens = 64; // staging chunk of prox_ffn_forward_host
 
-// Select state shared by the select kernel and Stage 2.
-enum { kSelCandCount = 0, kSelTicket = 1, kSelT = 2, kSelTieCut = 3 };
-struct SelectState {
-  uint32_t* hist = nullptr;      // [kHistBins] score bits 30..20, zero between tokens
-  uint32_t* state = nullptr;     // [8] candidate count, ticket, T, tie cut
-  uint32_t* cand_key = nullptr;  // [kSelectCand] keys of the boundary bin
-  int32_t* cand_idx = nullptr;   // [kSelectCand] their channels
-  int32_t* sl_gt1 = nullptr;     // [kMaxSlices] keys above the boundary bin, per slice
-  int32_t* sl_off = nullptr;     // [kMaxSlices + 1] rank offset of each slice's selected channels
-};
-
 // Per-token scratch of one layer (device memory owned by the handle).
 struct Workspace {
   float* scores = nullptr;        // |SiLU(g~) u~| [F]
   float* g_dbg = nullptr;         // debug g~ [F]
   float* u_dbg = nullptr;         // debug u~ [F]
-  uint32_t* hist = nullptr;       // [kHistBins], zero between tokens (== sel.hist)
-  SelectState sel;
-  int32_t* idx_s = nullptr;       // [F] selected channels (first k valid)
+  uint32_t* hist = nullptr;       // [kScoreBins] score bits 30..18, zero between tokens
+  uint2* bucket = nullptr;        // [kScoreBins][kBucketCap] (key, channel) per bin
+  int32_t* sel_mask = nullptr;    // [F] debug: 1 where the channel is selected
+  int32_t* idx_s = nullptr;       // [F] debug: selected channels (first k valid)
   float* s1_part = nullptr;        // Stage-1 partial sums [P1][2][1024]
   int* s1_cnt = nullptr;          // [C] Stage-1 row slices reported per slice, zero between tokens
   float* ypart = nullptr;         // Stage-2 output partials [P][d]
@@ -88,14 +81,13 @@ struct Stage2Launch {
   int mode = 1;               // 0: given list `idx`, 1: top-k select, 2: dense
   const int32_t* idx = nullptr;
   int k = 0;
-  int32_t* idx_out = nullptr;  // top-k: selected channels (ascending) written here
+  int32_t* sel_mask = nullptr;  // top-k: 1/0 per channel written here (debug)
   float* s_sp = nullptr;       // optional SiLU(g) u per listed channel
   bool select_only = false;    // top-k: stop after selecting
 };
 
 cudaError_t launch_stage1(const prox_layer* L, const float* x, const Stage1Taps& taps,
                           cudaStream_t s, bool pdl);
-cudaError_t launch_select(const prox_layer* L, cudaStream_t s, bool pdl);
 cudaError_t launch_stage2(const prox_layer* L, const float* x, const Stage2Launch& m,
                           cudaStream_t s, bool pdl, bool x_ready);
 cudaError_t launch_reduce(const prox_layer* L, float* out, cudaStream_t s, bool pdl);
@@ -116,6 +108,7 @@ cudaError_t launch_calibrate(const float* X, size_t n, unsigned long long rank,
 cudaError_t launch_rmsnorm(const float* y, float* x, int rows, int d, float eps,
                            cudaStream_t s);
 cudaError_t launch_copy(const void* src, void* dst, size_t bytes, cudaStream_t s);
+cudaError_t launch_mask_to_list(const int32_t* mask, int n, int32_t* list, cudaStream_t s);
 
 // Stage-1 column slices, CTAs and per-CTA row capacity for a shape on `num_sms` SMs.
 void choose_stage1_grid(int d, int F, int num_sms, int* C, int* P1, int* lmax);

@@ -23,8 +23,9 @@
 // per touched slice and written to global memory.  Each CTA then adds its row
 // count to the slice's counter; the CTA that completes a slice adds that
 // slice's partials in CTA order (deterministic), scores the channels,
-// score_j = |SiLU(g~_j) u~_j|, and adds them to a 2048-bin histogram of
-// their top bits -- the first level of the radix select.
+// score_j = |SiLU(g~_j) u~_j|, counts them in an 8192-bin histogram of their
+// top bits -- the first level of the radix select -- and appends (key,
+// channel) to the bin's bucket at the slot the count returned.
 #include "prox_device.cuh"
 #include "prox_internal.h"
 
@@ -52,6 +53,7 @@ struct Stage1Args {
   int d, F, C, lmax;
   float* scores;
   uint32_t* hist;
+  uint2* bucket;    // [kScoreBins][kBucketCap] (key, channel) per histogram bin
   unsigned long long* stats;
   float* g_dbg;
   float* u_dbg;
@@ -158,7 +160,9 @@ __device__ void finish_slice(const Stage1Args& a, int c, int n_x, int P, int* s_
   a.scores[ch] = sc;
   if (a.g_dbg) a.g_dbg[ch] = g;
   if (a.u_dbg) a.u_dbg[ch] = u;
-  atomicAdd(a.hist + (__float_as_uint(sc) >> 20), 1u);
+  const uint32_t key = __float_as_uint(sc), bin = key >> kScoreShift;
+  const uint32_t slot = atomicAdd(a.hist + bin, 1u);
+  if (slot < (uint32_t)kBucketCap) a.bucket[bin * kBucketCap + slot] = make_uint2(key, (uint32_t)ch);
 }
 
 // Shared memory: per-warp rings of NB batches, per-warp group-scaled sums,
@@ -445,6 +449,7 @@ cudaError_t launch_stage1(const prox_layer* L, const float* x, const Stage1Taps&
   a.lmax = L->s1_lmax;
   a.scores = L->ws.scores;
   a.hist = L->ws.hist;
+  a.bucket = L->ws.bucket;
   a.stats = L->ws.stats;
   a.g_dbg = taps.g;
   a.u_dbg = taps.u;

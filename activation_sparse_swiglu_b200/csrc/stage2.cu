@@ -3,13 +3,15 @@
 // down GEMV), and the dense SwiGLU baseline (Prox §2.1), which is the same
 // kernel with every channel kept.
 //
-// stage2_kernel -- persistent: one CTA per SM, each CTA owning a contiguous,
-// balanced range [t0, t1) of the k selected channels (ranked by channel
-// index).  In top-k mode the CTA turns its ranks into channels from the
-// select kernel's per-slice rank offsets, threshold T and tie cut, reading
-// only the one or two 256-channel slices of scores that hold its ranks.  Four producer lanes stream, with
-// 1-D bulk async copies (TMA engine) into a ring of 16 KB-class shared-memory
-// slots, first the gate/up channel records of its channels (gate column then
+// stage2_kernel -- persistent: one CTA per SM, each CTA owning the channels
+// [c0, c1) of an even split of d_ff.  In top-k mode every CTA computes the
+// exact cut of the token (select.cuh: T and the tie cut, from the Stage-1
+// histogram and the boundary bin's bucket) and keeps the channels of its range
+// past the cut; with a given list it keeps the list's channels in its range;
+// the dense baseline keeps all of them.  The uneven record counts this leaves
+// are absorbed by the deep ring (each SM may stream above its average share).
+// Four producer lanes stream, with 1-D bulk async copies (TMA engine) into a
+// ring of 16 KB-class shared-memory slots, first the gate/up channel records of its channels (gate column then
 // up column, d_model bf16 each: one copy per channel), then their W_down rows
 // (two rows per slot).  Eight consumer warps take every ring item in order (so
 // each mbarrier wait is for the phase right after one the waiting thread has
@@ -26,6 +28,7 @@
 // fixed order (deterministic, no atomics on floats).
 #include "prox_device.cuh"
 #include "prox_internal.h"
+#include "select.cuh"
 
 namespace prox {
 namespace {
@@ -42,9 +45,10 @@ struct Stage2Args {
   const uint16_t* wd;
   const int32_t* idx;      // kGivenList: channel list [k]
   const float* scores;     // kTopK: Stage-1 scores [F]
-  const int32_t* sl_off;   // kTopK: rank offsets per 256-channel slice
-  const uint32_t* sel_state;  // kTopK: threshold T and tie cut
-  int32_t* idx_out;        // kTopK: selected channels, ascending (each CTA its ranks)
+  const uint32_t* hist;    // kTopK: Stage-1 histogram of the scores' bits 30..20
+  unsigned long long* stats;
+  const uint2* bucket;     // kTopK: Stage-1 (key, channel) buckets per histogram bin
+  int32_t* sel_mask;       // kTopK: 1/0 per channel (debug)
   int mode, select_only;
   int k;
   int d, F, P, slots, max_rec;
@@ -54,55 +58,6 @@ struct Stage2Args {
   int* err;
   int x_ready;
 };
-
-// Top-k mode: the selected channels of ranks [t0, t1) (ascending channel
-// order) into s_idx and idx_out, from the rank offsets of the slices.
-__device__ void ranks_to_channels(const Stage2Args& a, int t0, int t1, int* s_idx, int* s_tmp) {
-  constexpr int NTH = (kStage2Consumers + 1) * 32;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int nsl = (a.F + kSelectSlice - 1) / kSelectSlice;
-  int* s_off = s_tmp;                      // [nsl + 1]
-  int* s_w = s_tmp + kMaxSlices + 1;       // [8] per-warp counts
-  int* s_m = s_w + 8;                      // [4]
-  for (int i = tid; i <= nsl; i += NTH) s_off[i] = __ldcg(a.sl_off + i);
-  if (tid == 0) {
-    s_m[0] = (int)__ldcg(a.sel_state + kSelT);
-    s_m[1] = (int)__ldcg(a.sel_state + kSelTieCut);
-  }
-  __syncthreads();
-  const uint32_t T = (uint32_t)s_m[0];
-  const int cut = s_m[1];
-  if (tid == 0) {
-    int lo = 0;
-    while (lo < nsl - 1 && s_off[lo + 1] <= t0) ++lo;
-    int hi = lo;
-    while (hi < nsl - 1 && s_off[hi + 1] < t1) ++hi;
-    s_m[2] = lo;
-    s_m[3] = hi;
-  }
-  __syncthreads();
-  const int lo = s_m[2], hi = s_m[3];
-  const unsigned lt = (1u << lane) - 1u;
-  for (int sl = lo; sl <= hi && t0 < t1; ++sl) {
-    const int e = sl * kSelectSlice + tid;
-    bool take = false;
-    if (tid < kSelectSlice && e < a.F) {
-      const uint32_t key = __float_as_uint(__ldcg(a.scores + e));
-      take = key > T || (key == T && e <= cut);
-    }
-    const unsigned m = __ballot_sync(0xffffffffu, take);
-    if (lane == 0 && warp < 8) s_w[warp] = __popc(m);
-    __syncthreads();
-    int before = s_off[sl];
-    for (int w = 0; w < warp && w < 8; ++w) before += s_w[w];
-    const int rank = before + __popc(m & lt);
-    if (take && rank >= t0 && rank < t1) {
-      s_idx[rank - t0] = e;
-      if (a.idx_out) a.idx_out[rank] = e;
-    }
-    __syncthreads();
-  }
-}
 
 // MAXM = ceil(d_model / 2048): 8-element chunks per thread and column.
 template <int MAXM>
@@ -119,7 +74,8 @@ __global__ void __launch_bounds__(S2_THREADS, 1) stage2_kernel(Stage2Args a) {
   int* s_idx = reinterpret_cast<int*>(s_val + a.max_rec);        // [max_rec]
   float* s_pg = reinterpret_cast<float*>(s_idx + a.max_rec);     // [max_rec][NCW]
   float* s_pu = s_pg + (size_t)a.max_rec * NCW;                  // [max_rec][NCW]
-  size_t off = (size_t)slots * 16 + (size_t)a.max_rec * (8 + 8 * NCW);
+  int* s_lpos = reinterpret_cast<int*>(s_pu + (size_t)a.max_rec * NCW);  // [max_rec]
+  size_t off = (size_t)slots * 16 + (size_t)a.max_rec * (12 + 8 * NCW);
   off = (off + 127) & ~(size_t)127;
   unsigned char* ring = smem + off;
 
@@ -155,21 +111,61 @@ __global__ void __launch_bounds__(S2_THREADS, 1) stage2_kernel(Stage2Args a) {
   }
   const int k = a.mode == kDense ? a.F : a.k;
   const int cta = blockIdx.x;
-  const int t0 = (int)(((long long)k * cta) / a.P);
-  const int t1 = (int)(((long long)k * (cta + 1)) / a.P);
-  const int n = t1 - t0;
+  int t0 = 0, n = 0;
   if (a.mode == kTopK) {
-    ranks_to_channels(a, t0, t1, s_idx, reinterpret_cast<int*>(ring));
+    // This CTA's channels are [c0, c1); those past the exact cut are its records.
+    const int c0 = (int)(((long long)a.F * cta) / a.P);
+    const int c1 = (int)(((long long)a.F * (cta + 1)) / a.P);
+    SelectScratch& sc = *reinterpret_cast<SelectScratch*>(ring);
+    const uint32_t key0 = c0 + tid < c1 ? __float_as_uint(__ldcg(a.scores + c0 + tid)) : 0u;
+    const TopkCut cut = select_cut_cta(a.scores, a.hist, a.bucket, a.F, a.k, sc);
+    for (int b = c0; b < c1; b += S2_THREADS) {
+      const int e = b + tid;
+      const uint32_t key =
+          b == c0 ? key0 : (e < c1 ? __float_as_uint(__ldcg(a.scores + e)) : 0u);
+      const bool sel = e < c1 && selected(key, e, cut);
+      int total;
+      const int pos = n + block_exclusive_scan(sel ? 1 : 0, sc.scan, &total);
+      if (sel) s_idx[pos] = e;
+      if (a.sel_mask && e < c1) a.sel_mask[e] = sel ? 1 : 0;
+      n += total;
+    }
+    if (cta == 0 && tid == 0 && a.stats) atomicAdd(a.stats + 1, 1ull);
+    __syncthreads();
+  } else if (a.mode == kGivenList) {
+    // Entries of the list whose channel lies in [c0, c1), in list order -- the
+    // same split of the channels as the top-k step, so that a sorted list
+    // reproduces it exactly.  Thread t scans entries [t*per, (t+1)*per).
+    const int c0 = (int)(((long long)a.F * cta) / a.P);
+    const int c1 = (int)(((long long)a.F * (cta + 1)) / a.P);
+    const int per = (k + S2_THREADS - 1) / S2_THREADS;
+    const int lo = min(tid * per, k), hi = min(lo + per, k);
+    int cnt = 0;
+    for (int i = lo; i < hi; ++i) {
+      const int j = __ldcg(a.idx + i);
+      if (j < 0 || j >= a.F) atomicOr(a.err, PROX_DEVERR_MASK_INDEX);
+      cnt += j >= c0 && j < c1;
+    }
+    int total;
+    int pos = block_exclusive_scan(cnt, reinterpret_cast<SelectScratch*>(ring)->scan, &total);
+    for (int i = lo; i < hi; ++i) {
+      const int j = __ldcg(a.idx + i);
+      if (j >= c0 && j < c1) {
+        if (pos < a.max_rec) {  // more only with repeated channels
+          s_lpos[pos] = i;      // list position (for s_sp)
+          s_idx[pos] = j;
+        } else {
+          atomicOr(a.err, PROX_DEVERR_MASK_INDEX);
+        }
+        ++pos;
+      }
+    }
+    n = min(total, a.max_rec);
     __syncthreads();
   } else {
-    for (int i = tid; i < n; i += S2_THREADS) {
-      int j = a.mode == kGivenList ? __ldcg(a.idx + t0 + i) : t0 + i;
-      if (j < 0 || j >= a.F) {
-        atomicOr(a.err, PROX_DEVERR_MASK_INDEX);
-        j = 0;
-      }
-      s_idx[i] = j;
-    }
+    t0 = (int)(((long long)k * cta) / a.P);
+    n = (int)(((long long)k * (cta + 1)) / a.P) - t0;
+    for (int i = tid; i < n; i += S2_THREADS) s_idx[i] = t0 + i;
     __syncthreads();
   }
   if (a.select_only) return;
@@ -298,7 +294,7 @@ __global__ void __launch_bounds__(S2_THREADS, 1) stage2_kernel(Stage2Args a) {
     }
     const float sv = silu_f32(g) * u;
     s_val[r] = sv;
-    if (a.s_sp) a.s_sp[t0 + r] = sv;
+    if (a.s_sp) a.s_sp[a.mode == kGivenList ? s_lpos[r] : t0 + r] = sv;
   }
   asm volatile("bar.sync 1, %0;" ::"r"(NCW * 32) : "memory");
 
@@ -365,7 +361,7 @@ __global__ void __launch_bounds__(kReduceWarps * 32) reduce_kernel(const float* 
   pdl_trigger();
   // Stage 2 is complete: clear the level-1 histogram for the next token.
   if (hist && blockIdx.x == 0)
-    for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) hist[i] = 0u;
+    for (int i = threadIdx.x; i < kScoreBins; i += blockDim.x) hist[i] = 0u;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int col = blockIdx.x * 32 + lane;
   float s = 0.f;
@@ -407,7 +403,7 @@ cudaError_t set_stage2_attr() {
 void choose_stage2(int d, int F, int num_sms, int* P, int* slots, int* nprod, size_t* smem) {
   *P = num_sms;
   const int max_rec = (F + num_sms - 1) / num_sms + 1;
-  size_t off = (size_t)max_rec * (8 + 8 * NCW) + 128;
+  size_t off = (size_t)max_rec * (12 + 8 * NCW) + 128;
   const size_t slot_bytes = 4 * (size_t)d;  // gate + up column, or two W_down rows
   int s = (int)((kStage2SmemBudget - off) / (slot_bytes + 16));
   if (s > 32) s = 32;
@@ -421,10 +417,10 @@ void choose_stage2(int d, int F, int num_sms, int* P, int* slots, int* nprod, si
     *nprod = 2;
   }
   *slots = s;
-  off = (size_t)s * 16 + (size_t)max_rec * (8 + 8 * NCW);
+  off = (size_t)s * 16 + (size_t)max_rec * (12 + 8 * NCW);
   off = (off + 127) & ~(size_t)127;
   size_t region = (size_t)s * slot_bytes;
-  if (region < 4096) region = 4096;  // scratch of ranks_to_channels
+  if (region < sizeof(SelectScratch)) region = sizeof(SelectScratch);  // the select's scratch
   *smem = off + region;
 }
 
@@ -445,9 +441,10 @@ cudaError_t launch_stage2(const prox_layer* L, const float* x, const Stage2Launc
   a.wd = L->wd;
   a.idx = m.idx;
   a.scores = L->ws.scores;
-  a.sl_off = L->ws.sel.sl_off;
-  a.sel_state = L->ws.sel.state;
-  a.idx_out = m.idx_out;
+  a.hist = L->ws.hist;
+  a.stats = L->ws.stats;
+  a.bucket = L->ws.bucket;
+  a.sel_mask = m.sel_mask;
   a.mode = m.mode;
   a.select_only = m.select_only ? 1 : 0;
   a.k = m.k;
