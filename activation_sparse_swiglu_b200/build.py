@@ -1,6 +1,7 @@
 """Builds libprox.so (all CUDA sources, sm_100a) next to this file.
 
-Usage: python -m activation_sparse_swiglu_b200.build [--force] [--verbose]
+Usage: python activation_sparse_swiglu_b200/build.py [--force] [--verbose] [--ptxas-info]
+(run by path: importing the package loads libprox.so, which may be missing or stale)
 """
 
 from __future__ import annotations
