@@ -74,6 +74,21 @@ def calibrate_thresholds(x_cal: torch.Tensor, s1: float, stream=None) -> float:
     return float(tau.value)
 
 
+def calibrate_thresholds_noalloc(x_cal: torch.Tensor, s1: float, tau: torch.Tensor,
+                                 stream=None) -> torch.Tensor:
+    """The same quantile written to the 1-element fp32 device tensor `tau` in
+    stream order, with no allocation (fixed static scratch; concurrent calls on
+    one device race)."""
+    _dev(x_cal, torch.float32, "x_cal")
+    _dev(tau, torch.float32, "tau")
+    if tau.numel() < 1:
+        raise ValueError("tau needs one element")
+    n, d = x_cal.shape
+    check(lib.prox_calibrate_thresholds_noalloc(_ptr(x_cal), n, d, float(s1), _ptr(tau),
+                                                _stream(stream)))
+    return tau
+
+
 def rmsnorm(y: torch.Tensor, eps: float = 1e-6, out: torch.Tensor | None = None, stream=None):
     _dev(y, torch.float32, "y")
     y2 = y.reshape(-1, y.shape[-1])

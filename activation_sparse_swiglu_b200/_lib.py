@@ -45,6 +45,7 @@ _S = ctypes.c_size_t
 SIGNATURES = {
     "prox_pack_proxy": (_I, [_P, _I, _I, _I, _P, _P, _P]),
     "prox_calibrate_thresholds": (_I, [_P, _I, _I, _F, ctypes.POINTER(_F), _P]),
+    "prox_calibrate_thresholds_noalloc": (_I, [_P, _I, _I, _F, _P, _P]),
     "prox_layer_create": (_I, [_P, _P, _P, _I, _I, _F, _I, _I, _P, ctypes.POINTER(_P)]),
     "prox_layer_destroy": (_I, [_P]),
     "prox_layer_set_tau": (_I, [_P, _F]),

@@ -96,7 +96,20 @@ __global__ void calib_init_kernel(uint32_t* scratch, unsigned long long rank) {
   }
 }
 
+// Fixed scratch of the allocation-free calibration entry point: the histogram,
+// the key prefix and the remaining rank (as in the allocated scratch), then
+// room for spare words.  One per device; every call rewrites all of it.
+constexpr int kStaticScratchWords = kHistBins + 8;
+static __device__ __align__(256) uint32_t g_calib_scratch[kStaticScratchWords];
+
 }  // namespace
+
+cudaError_t calibrate_static_scratch(uint32_t** ptr) {
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_calib_scratch);
+  *ptr = static_cast<uint32_t*>(p);
+  return e;
+}
 
 cudaError_t launch_calibrate(const float* X, size_t n, unsigned long long rank,
                              uint32_t* scratch, float* tau_dev, cudaStream_t s) {

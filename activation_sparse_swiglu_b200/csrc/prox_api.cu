@@ -1,6 +1,8 @@
 // C ABI of the Prox library: argument checks, the layer handle, and the
 // stream-ordered kernel chains of the decode step.
+#include <atomic>
 #include <cmath>
+#include <mutex>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -16,6 +18,11 @@ cudaError_t setup_stage2_kernels();
 }  // namespace prox
 
 namespace {
+
+constexpr int kMaxDevices = 64;
+// Device address of the static calibration scratch, per device, set once.
+std::atomic<uint32_t*> g_calib_scratch_addr[kMaxDevices];
+std::mutex g_calib_scratch_mu;
 
 thread_local std::string g_last_error;
 
@@ -42,6 +49,7 @@ prox_status cuda_fail(cudaError_t e, const char* what) {
   } while (0)
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
@@ -217,6 +225,41 @@ prox_status prox_calibrate_thresholds(const float* X_cal, int n_tok, int d_model
   cudaFreeAsync(scratch, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_fail(e, "calibrate");
+  return PROX_OK;
+}
+
+prox_status prox_calibrate_thresholds_noalloc(const float* X_cal, int n_tok, int d_model,
+                                              float s1, float* tau_dev, void* stream) {
+  if (!tau_dev || !aligned4(tau_dev)) return fail(PROX_EINVAL, "tau_dev must be a 4-byte aligned device pointer");
+  if (!(s1 >= 0.f && s1 <= 1.f)) return fail(PROX_EINVAL, "s1=%g must be in [0, 1]", (double)s1);
+  if (n_tok <= 0 || d_model <= 0) return fail(PROX_EINVAL, "n_tok and d_model must be positive");
+  const size_t n = (size_t)n_tok * (size_t)d_model;
+  if (n >= (size_t)1 << 31)
+    return fail(PROX_EINVAL, "n_tok * d_model = %zu exceeds the 2^31-1 values the fixed scratch counts", n);
+  if (!X_cal || !aligned16(X_cal)) return fail(PROX_EINVAL, "X_cal must be a 16-byte aligned pointer");
+  int dev, sms;
+  prox_status st = check_device(&dev, &sms);
+  if (st != PROX_OK) return st;
+  if (dev < 0 || dev >= kMaxDevices) return fail(PROX_EUNSUPPORTED, "device ordinal %d out of range", dev);
+  // The scratch address is looked up once per device, with that device
+  // current (it is the caller's current device here).
+  uint32_t* scratch = g_calib_scratch_addr[dev].load(std::memory_order_acquire);
+  if (!scratch) {
+    std::lock_guard<std::mutex> lock(g_calib_scratch_mu);
+    scratch = g_calib_scratch_addr[dev].load(std::memory_order_relaxed);
+    if (!scratch) {
+      PROX_CUDA(prox::calibrate_static_scratch(&scratch), "cudaGetSymbolAddress(calibration scratch)");
+      g_calib_scratch_addr[dev].store(scratch, std::memory_order_release);
+    }
+  }
+  cudaStream_t s = as_stream(stream);
+  if (s1 == 0.f) {
+    PROX_CUDA(cudaMemsetAsync(tau_dev, 0, 4, s), "cudaMemsetAsync(tau)");
+    return PROX_OK;
+  }
+  unsigned long long rank = (unsigned long long)std::floor((double)s1 * (double)n);
+  if (rank >= n) rank = n - 1;
+  PROX_CUDA(prox::launch_calibrate(X_cal, n, rank, scratch, tau_dev, s), "calibrate launch");
   return PROX_OK;
 }
 

@@ -102,6 +102,9 @@ cudaError_t launch_gateup_records(const uint16_t* Wg, const uint16_t* Wu, int d,
 
 // Calibration: exact order statistic of |X| at 0-based ascending rank `rank`.
 // `scratch` holds kHistBins + 4 uint32 (zeroed by the caller).
+// Device address of the calibration scratch kept in a static __device__
+// array (kHistBins + 8 words) of the current device.
+cudaError_t calibrate_static_scratch(uint32_t** ptr);
 cudaError_t launch_calibrate(const float* X, size_t n, unsigned long long rank,
                              uint32_t* scratch, float* tau_dev, cudaStream_t s);
 

@@ -102,6 +102,22 @@ PROX_API prox_status prox_pack_proxy(const uint16_t* W, int d_model, int d_ff, i
 PROX_API prox_status prox_calibrate_thresholds(const float* X_cal, int n_tok, int d_model, float s1,
                                       float* tau_host, void* stream);
 
+/* The calibration above without any allocation (the Prox pages have no
+ * counterpart: this is an engineering variant for allocation-free hosts and
+ * CUDA graphs).  Same quantile, same exactness.  Its scratch is a fixed
+ * static __device__ array of 2056 uint32 (8 KB) per device, found with
+ * cudaGetSymbolAddress on the first call made on that device (with it
+ * current): make that first call before any stream capture.  Every call
+ * zeroes the histogram it needs before counting, so nothing has to start at
+ * zero.  Calls that overlap on one device (other streams, other threads)
+ * share that scratch and race: serialise them.  X_cal: fp32 [n_tok, d_model]
+ * on the current device, 16-byte aligned; n_tok * d_model must stay below
+ * 2^31 (the counters are 32-bit), else PROX_EINVAL with a message.  tau_dev:
+ * one float on the device, written in stream order (nothing synchronises).
+ * Allocates nothing: no cudaMalloc, cudaMallocAsync or cudaFree. */
+PROX_API prox_status prox_calibrate_thresholds_noalloc(const float* X_cal, int n_tok, int d_model,
+                                                       float s1, float* tau_dev, void* stream);
+
 /* ------------------------------------------------------------------------
  * Layer handle
  * ------------------------------------------------------------------------ */

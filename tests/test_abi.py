@@ -63,6 +63,13 @@ def test_host_side_argument_checks(plib):
     # s1 = 0 needs no device work and gives tau = 0
     assert lib.prox_calibrate_thresholds(p, 4, 128, 0.0, ctypes.byref(tau), None) == plib.PROX_OK
     assert tau.value == 0.0
+    # allocation-free calibration: oversize input, bad s1, misaligned outputs,
+    # all refused on the host before any device work
+    assert lib.prox_calibrate_thresholds_noalloc(p, 65536, 32768, 0.5, p, None) == plib.PROX_EINVAL
+    assert "2^31" in plib.last_error()
+    assert lib.prox_calibrate_thresholds_noalloc(p, 4, 128, -0.1, p, None) == plib.PROX_EINVAL
+    assert lib.prox_calibrate_thresholds_noalloc(p, 4, 128, 0.5, ctypes.c_void_p(18), None) == plib.PROX_EINVAL
+    assert lib.prox_calibrate_thresholds_noalloc(ctypes.c_void_p(20), 4, 128, 0.5, p, None) == plib.PROX_EINVAL
     # NULL handles
     assert lib.prox_ffn_forward(None, p, p, 1, None) == plib.PROX_EINVAL
     assert lib.prox_dense_ffn(None, p, p, 1, None) == plib.PROX_EINVAL
