@@ -1,0 +1,51 @@
+"""bench.py's replica plumbing (barrier, max over ranks, whole-job value) on
+two CPU processes with the gloo backend."""
+
+import os
+import socket
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, q):
+    os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), LOCAL_RANK=str(rank),
+                      MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(ROOT, "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    d = bench.Dist(world, backend="gloo")
+    d.barrier()
+    # each rank "timed" a different duration; the job's time is the slowest
+    t = d.max(10.0 + 5.0 * rank)
+    units = 256 * d.world  # every rank processed the same units (weak scaling)
+    q.put((rank, t, units / (t / 1e3)))
+    d.barrier()
+    d.close()
+
+
+def test_two_rank_max_and_value():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+    assert all(p.exitcode == 0 for p in procs)
+    res = sorted(q.get(timeout=5) for _ in range(2))
+    for rank, t, value in res:
+        assert t == pytest.approx(15.0)
+        assert value == pytest.approx(512 / 0.015)
