@@ -290,7 +290,7 @@ prox_status prox_layer_create(const uint16_t* W_gate, const uint16_t* W_up, cons
   L->device = dev;
   L->num_sms = sms;
   prox::choose_stage1_grid(L->d, L->F, sms, &L->C, &L->P1, &L->s1_lmax);
-  prox::choose_stage2(L->d, L->F, sms, &L->P, &L->ring_slots, &L->stage2_producers,
+  prox::choose_stage2(L->d, L->F, sms, &L->P, &L->ring_slots, &L->stage2_groups,
                      &L->stage2_smem);
   L->stage1_smem = prox::stage1_smem_bytes(L->s1_lmax);
   if (L->stage1_smem > (size_t)prox::kMaxSmemPerBlock) {

@@ -20,7 +20,7 @@ constexpr int kStage1Warps = 16;     // Stage-1 warps per CTA (one CTA per SM)
 constexpr int kSelectCand = 4096;    // candidate buffer of the select (level-1 bin)
 constexpr int kSelectSlice = 256;    // channels per select CTA (and per rank-offset entry)
 constexpr int kMaxSlices = 160;      // >= d_ff / kSelectSlice + 1
-constexpr int kStage2Consumers = 8;  // Stage-2 consumer warps (+1 producer warp)
+constexpr int kStage2Consumers = 16;  // Stage-2 consumer warps (+1 producer warp)
 constexpr int kReduceWarps = 16;     // output reduction: warps per 32 columns
 constexpr int kMaxDModel = 16384;
 constexpr int kMaxDff = 32768;       // bounds the select's slice table (kMaxSlices)
@@ -57,7 +57,7 @@ struct prox_layer {
   // Stage-1 geometry: C column slices, P1 CTAs, at most s1_lmax rows per CTA
   int C = 0, P1 = 0, s1_lmax = 0;
   // Stage-2 geometry
-  int P = 0, ring_slots = 0, stage2_producers = 1;
+  int P = 0, ring_slots = 0, stage2_groups = 1;
   size_t stage2_smem = 0, stage1_smem = 0;
   // library-owned weights
   uint16_t* wgu = nullptr;   // bf16 [F][2d]: gate column j | up column j
@@ -118,6 +118,6 @@ void choose_stage1_grid(int d, int F, int num_sms, int* C, int* P1, int* lmax);
 size_t stage1_smem_bytes(int lmax);
 size_t stage1_part_floats(int P1);
 // Stage-2 ring depth and dynamic shared memory for d_model = d.
-void choose_stage2(int d, int F, int num_sms, int* P, int* slots, int* nprod, size_t* smem);
+void choose_stage2(int d, int F, int num_sms, int* P, int* slots, int* groups, size_t* smem);
 
 }  // namespace prox

@@ -13,7 +13,7 @@
 // Four producer lanes stream, with 1-D bulk async copies (TMA engine) into a
 // ring of 16 KB-class shared-memory slots, first the gate/up channel records of its channels (gate column then
 // up column, d_model bf16 each: one copy per channel), then their W_down rows
-// (two rows per slot).  Eight consumer warps take every ring item in order (so
+// (two rows per slot).  The consumer warps take every ring item in order (so
 // each mbarrier wait is for the phase right after one the waiting thread has
 // already seen complete):
 //   phase A: for each channel every warp forms partial dot products of its
@@ -52,14 +52,14 @@ struct Stage2Args {
   int mode, select_only;
   int k;
   int d, F, P, slots, max_rec;
-  int nprod;  // producer lanes; slots is a multiple of it
+  int groups;  // consumer groups NG (= producer lanes); slots is a multiple of it
   float* ypart;
   float* s_sp;
   int* err;
   int x_ready;
 };
 
-// MAXM = ceil(d_model / 2048): 8-element chunks per thread and column.
+// MAXM = ceil(d_model / (8 * consumer threads)): 8-element chunks per thread and column.
 template <int MAXM>
 __global__ void __launch_bounds__(S2_THREADS, 1) stage2_kernel(Stage2Args a) {
   extern __shared__ __align__(128) unsigned char smem[];
@@ -82,33 +82,34 @@ __global__ void __launch_bounds__(S2_THREADS, 1) stage2_kernel(Stage2Args a) {
   if (tid == 0) {
     for (int s = 0; s < slots; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], NCW);
+      mbar_init(&empty[s], NCW / a.groups);
     }
     fence_barrier_init();
   }
-  // this thread's share of x (chunks c8 = tid + 256 m), kept in registers
+  // Consumer warps form NG groups of WPG; a group takes whole ring items, warp
+  // wi of a group the elements [wi*qd, (wi+1)*qd) of each column / row
+  // (qd = d / WPG), lane chunks e8 = m*32 + lane of 8 elements.
+  const int NG = a.groups, WPG = NCW / NG, qd = d / WPG;
+  const int grp = warp / WPG, wi = warp % WPG;
+  auto elem = [&](int m) { return wi * qd + (m * 32 + lane) * 8; };
+  auto elem_ok = [&](int m) { return (m * 32 + lane) * 8 < qd; };
+  // this thread's x elements, kept in registers
   float4 xr[MAXM][2];
-  if (a.x_ready && warp < NCW) {
+  auto load_x = [&]() {
 #pragma unroll
     for (int m = 0; m < MAXM; ++m) {
-      const int e = (tid + m * NCW * 32) * 8;
-      xr[m][0] = e < d ? __ldg(reinterpret_cast<const float4*>(a.x + e)) : make_float4(0, 0, 0, 0);
-      xr[m][1] = e < d ? __ldg(reinterpret_cast<const float4*>(a.x + e + 4)) : make_float4(0, 0, 0, 0);
+      const int e = elem(m);
+      xr[m][0] = elem_ok(m) ? __ldg(reinterpret_cast<const float4*>(a.x + e)) : make_float4(0, 0, 0, 0);
+      xr[m][1] = elem_ok(m) ? __ldg(reinterpret_cast<const float4*>(a.x + e + 4)) : make_float4(0, 0, 0, 0);
     }
-  }
+  };
+  if (a.x_ready && warp < NCW) load_x();
   __syncthreads();
 
   pdl_wait();
   pdl_trigger();
 
-  if (!a.x_ready && warp < NCW) {
-#pragma unroll
-    for (int m = 0; m < MAXM; ++m) {
-      const int e = (tid + m * NCW * 32) * 8;
-      xr[m][0] = e < d ? __ldg(reinterpret_cast<const float4*>(a.x + e)) : make_float4(0, 0, 0, 0);
-      xr[m][1] = e < d ? __ldg(reinterpret_cast<const float4*>(a.x + e + 4)) : make_float4(0, 0, 0, 0);
-    }
-  }
+  if (!a.x_ready && warp < NCW) load_x();
   const int k = a.mode == kDense ? a.F : a.k;
   const int cta = blockIdx.x;
   int t0 = 0, n = 0;
@@ -170,29 +171,32 @@ __global__ void __launch_bounds__(S2_THREADS, 1) stage2_kernel(Stage2Args a) {
   }
   if (a.select_only) return;
 
-  // Ring items q = 0 .. nA + nB - 1: q < n is the gate/up record of channel q;
-  // q >= n holds W_down rows 2(q-n) and 2(q-n)+1.  Item q lives in slot
-  // q % slots as that slot's use q / slots.
+  // Ring items: channel records q < n (gate column | up column), then W_down
+  // row pairs (rows 2p, 2p+1).  Group g takes records g, g+NG, ... and pairs
+  // g, g+NG, ...; its items, records first, use the group's own SPG slots
+  // [g*SPG, (g+1)*SPG) round robin, so every slot's waiter is one group that
+  // takes its uses in order.  Producer lane g fills group g's slots.
   const int nB = (n + 1) >> 1;
-  const int total = n + nB;
+  const int SPG = slots / NG;
+  auto group_items = [&](int g, int cnt) { return cnt > g ? (cnt - g + NG - 1) / NG : 0; };
   bool dead = false;  // set once a wait of this thread ran out
   if (warp == NCW) {
-    // ---------------- producer lanes 0..nprod-1: lane l issues items q = l + j*nprod.
-    // slots is a multiple of nprod, so every slot is refilled by one lane, in order.
-    const int np = a.nprod;
-    if (lane < np && lane < total) {
+    // ---------------- producer lanes 0..NG-1 ----------------
+    if (lane < NG) {
+      const int g = lane;
       const uint64_t pol = l2_policy_evict_first();
-      int q = lane;
-      int slot = q % slots;
-      int use = q / slots;
-      for (; q < total; q += np) {
+      const int nA_g = group_items(g, n), nB_g = group_items(g, nB);
+      const int tot_g = nA_g + nB_g;
+      for (int li = 0; li < tot_g; ++li) {
+        const int slot = g * SPG + li % SPG, use = li / SPG;
         if (use > 0) mbar_wait(&empty[slot], (uint32_t)((use - 1) & 1), a.err, &dead);
         unsigned char* dst = ring + (size_t)slot * slot_bytes;
-        if (q < n) {
+        if (li < nA_g) {
+          const int r = g + li * NG;
           mbar_arrive_expect_tx(&full[slot], slot_bytes);
-          bulk_copy_g2s(dst, a.wgu + (size_t)s_idx[q] * 2 * (size_t)d, slot_bytes, &full[slot], pol);
+          bulk_copy_g2s(dst, a.wgu + (size_t)s_idx[r] * 2 * (size_t)d, slot_bytes, &full[slot], pol);
         } else {
-          const int r0 = 2 * (q - n);
+          const int r0 = 2 * (g + (li - nA_g) * NG);
           const int nr = r0 + 1 < n ? 2 : 1;
           mbar_arrive_expect_tx(&full[slot], (uint32_t)nr * col_bytes);
           bulk_copy_g2s(dst, a.wd + (size_t)s_idx[r0] * (size_t)d, col_bytes, &full[slot], pol);
@@ -200,95 +204,65 @@ __global__ void __launch_bounds__(S2_THREADS, 1) stage2_kernel(Stage2Args a) {
             bulk_copy_g2s(dst + col_bytes, a.wd + (size_t)s_idx[r0 + 1] * (size_t)d, col_bytes,
                           &full[slot], pol);
         }
-        slot += np;
-        while (slot >= slots) {
-          slot -= slots;
-          ++use;
-        }
       }
       // Every issued copy must land before this CTA's shared memory is released:
-      // wait for the last use of each slot this lane filled.
-      for (int s2 = 0; s2 < slots; ++s2) {
-        int last = -1;  // last item of this lane in slot s2
-        for (int qq = s2; qq < total; qq += slots)
-          if (qq % np == lane) last = qq;
-        if (last >= 0) mbar_wait(&full[s2], (uint32_t)((last / slots) & 1), a.err);
+      // wait for the last use of each slot of the group.
+      for (int j = 0; j < SPG && j < tot_g; ++j) {
+        const int last = j + ((tot_g - 1 - j) / SPG) * SPG;  // last li with li % SPG == j
+        mbar_wait(&full[g * SPG + j], (uint32_t)((last / SPG) & 1), a.err);
       }
     }
     return;
   }
 
-  int cs = 0;        // consumer: slot of the next item
-  uint32_t cp = 0;   // and the parity of its use
-
-  // ---------------- phase A: partial gate/up dot products ----------------
-  // Records are taken RB at a time so that the 2*RB warp reductions of a batch
-  // run interleaved.
-  constexpr int RB = 4;
-  const int rbn = slots < RB ? slots : RB;  // a batch never holds more than the ring
-  for (int r0 = 0; r0 < n; r0 += rbn) {
-    int sl[RB];
+  // ---------------- phase A: gate/up partial dot products ----------------
+  // The warp's share of an item goes into registers, the slot goes back to the
+  // producer, then the FMAs.
+  const int nA_g = group_items(grp, n);
+  for (int li = 0; li < nA_g; ++li) {
+    const int r = grp + li * NG;
+    const int slot = grp * SPG + li % SPG;
+    mbar_wait(&full[slot], (uint32_t)((li / SPG) & 1), a.err, &dead);
+    const unsigned char* wg = ring + (size_t)slot * slot_bytes;
+    const unsigned char* wu = wg + col_bytes;
+    uint4 gv[MAXM], uv[MAXM];
 #pragma unroll
-    for (int b = 0; b < RB; ++b) {
-      sl[b] = cs;
-      if (b < rbn && r0 + b < n) {
-        mbar_wait(&full[cs], cp, a.err, &dead);
-        if (++cs == slots) { cs = 0; cp ^= 1u; }
-      }
-    }
-    float g[RB], u[RB];
-#pragma unroll
-    for (int b = 0; b < RB; ++b) {
-      float2 ag = make_float2(0.f, 0.f), au = make_float2(0.f, 0.f);
-      if (b < rbn && r0 + b < n) {
-        const unsigned char* wg = ring + (size_t)sl[b] * slot_bytes;
-        const unsigned char* wu = wg + col_bytes;
-#pragma unroll
-        for (int m = 0; m < MAXM; ++m) {
-          const int e = (tid + m * NCW * 32) * 8;
-          if (e < d) {
-            const uint4 g4 = *reinterpret_cast<const uint4*>(wg + (size_t)e * 2);
-            const uint4 u4 = *reinterpret_cast<const uint4*>(wu + (size_t)e * 2);
-            const float4 xa = xr[m][0], xb = xr[m][1];
-            ag = __ffma2_rn(bf16x2_to_f2(g4.x), make_float2(xa.x, xa.y), ag);
-            au = __ffma2_rn(bf16x2_to_f2(u4.x), make_float2(xa.x, xa.y), au);
-            ag = __ffma2_rn(bf16x2_to_f2(g4.y), make_float2(xa.z, xa.w), ag);
-            au = __ffma2_rn(bf16x2_to_f2(u4.y), make_float2(xa.z, xa.w), au);
-            ag = __ffma2_rn(bf16x2_to_f2(g4.z), make_float2(xb.x, xb.y), ag);
-            au = __ffma2_rn(bf16x2_to_f2(u4.z), make_float2(xb.x, xb.y), au);
-            ag = __ffma2_rn(bf16x2_to_f2(g4.w), make_float2(xb.z, xb.w), ag);
-            au = __ffma2_rn(bf16x2_to_f2(u4.w), make_float2(xb.z, xb.w), au);
-          }
-        }
-      }
-      g[b] = ag.x + ag.y;
-      u[b] = au.x + au.y;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-#pragma unroll
-      for (int b = 0; b < RB; ++b) {
-        g[b] += __shfl_xor_sync(0xffffffffu, g[b], o);
-        u[b] += __shfl_xor_sync(0xffffffffu, u[b], o);
-      }
+    for (int m = 0; m < MAXM; ++m) {
+      const int e = elem(m);
+      gv[m] = elem_ok(m) ? *reinterpret_cast<const uint4*>(wg + (size_t)e * 2) : make_uint4(0u, 0u, 0u, 0u);
+      uv[m] = elem_ok(m) ? *reinterpret_cast<const uint4*>(wu + (size_t)e * 2) : make_uint4(0u, 0u, 0u, 0u);
     }
     __syncwarp();
-    if (lane == 0) {
+    if (lane == 0) mbar_arrive(&empty[slot], 1);
+    float2 ag0 = make_float2(0.f, 0.f), ag1 = ag0, au0 = ag0, au1 = ag0;
 #pragma unroll
-      for (int b = 0; b < RB; ++b) {
-        if (b < rbn && r0 + b < n) {
-          mbar_arrive(&empty[sl[b]], 1);
-          s_pg[(r0 + b) * NCW + warp] = g[b];
-          s_pu[(r0 + b) * NCW + warp] = u[b];
-        }
-      }
+    for (int m = 0; m < MAXM; ++m) {
+      const float4 xa = xr[m][0], xb = xr[m][1];
+      ag0 = __ffma2_rn(bf16x2_to_f2(gv[m].x), make_float2(xa.x, xa.y), ag0);
+      au0 = __ffma2_rn(bf16x2_to_f2(uv[m].x), make_float2(xa.x, xa.y), au0);
+      ag1 = __ffma2_rn(bf16x2_to_f2(gv[m].y), make_float2(xa.z, xa.w), ag1);
+      au1 = __ffma2_rn(bf16x2_to_f2(uv[m].y), make_float2(xa.z, xa.w), au1);
+      ag0 = __ffma2_rn(bf16x2_to_f2(gv[m].z), make_float2(xb.x, xb.y), ag0);
+      au0 = __ffma2_rn(bf16x2_to_f2(uv[m].z), make_float2(xb.x, xb.y), au0);
+      ag1 = __ffma2_rn(bf16x2_to_f2(gv[m].w), make_float2(xb.z, xb.w), ag1);
+      au1 = __ffma2_rn(bf16x2_to_f2(uv[m].w), make_float2(xb.z, xb.w), au1);
+    }
+    float g = (ag0.x + ag0.y) + (ag1.x + ag1.y);
+    float u = (au0.x + au0.y) + (au1.x + au1.y);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      g += __shfl_xor_sync(0xffffffffu, g, o);
+      u += __shfl_xor_sync(0xffffffffu, u, o);
+    }
+    if (lane == 0) {
+      s_pg[r * NCW + wi] = g;
+      s_pu[r * NCW + wi] = u;
     }
   }
   asm volatile("bar.sync 1, %0;" ::"r"(NCW * 32) : "memory");
   for (int r = tid; r < n; r += NCW * 32) {
     float g = 0.f, u = 0.f;
-#pragma unroll
-    for (int w = 0; w < NCW; ++w) {
+    for (int w = 0; w < WPG; ++w) {
       g += s_pg[r * NCW + w];
       u += s_pu[r * NCW + w];
     }
@@ -299,56 +273,71 @@ __global__ void __launch_bounds__(S2_THREADS, 1) stage2_kernel(Stage2Args a) {
   asm volatile("bar.sync 1, %0;" ::"r"(NCW * 32) : "memory");
 
   // ---------------- phase B: y_part = sum_t s_t W_down[j_t, :] ----------------
-  // Items (two rows each) are taken two at a time.
+  // The group's row pairs; warp wi accumulates its columns [wi*qd, (wi+1)*qd).
   float2 acc[MAXM * 4];
 #pragma unroll
   for (int i = 0; i < MAXM * 4; ++i) acc[i] = make_float2(0.f, 0.f);
-  for (int rb0 = 0; rb0 < nB; rb0 += 2) {
-    int sl[2];
+  const int nB_g = group_items(grp, nB);
+  for (int lb = 0; lb < nB_g; ++lb) {
+    const int li = nA_g + lb;
+    const int p = grp + lb * NG;  // row pair
+    const int slot = grp * SPG + li % SPG;
+    mbar_wait(&full[slot], (uint32_t)((li / SPG) & 1), a.err, &dead);
+    const unsigned char* w = ring + (size_t)slot * slot_bytes;
+    const bool two = 2 * p + 1 < n;
+    uint4 wv[2][MAXM];
 #pragma unroll
-    for (int b = 0; b < 2; ++b) {
-      sl[b] = cs;
-      if (rb0 + b < nB) {
-        mbar_wait(&full[cs], cp, a.err, &dead);
-        if (++cs == slots) { cs = 0; cp ^= 1u; }
-      }
-    }
+    for (int h = 0; h < 2; ++h) {
 #pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      const int rr = 2 * rb0 + h;  // W_down row (channel slot) of this CTA
-      if (rr < n) {
-        const float sv = s_val[rr];
-        const float2 s2 = make_float2(sv, sv);
-        const unsigned char* w = ring + (size_t)sl[h >> 1] * slot_bytes + (h & 1) * col_bytes;
-#pragma unroll
-        for (int m = 0; m < MAXM; ++m) {
-          const int e = tid * 8 + m * (NCW * 32 * 8);
-          if (e < d) {
-            const uint4 w4 = *reinterpret_cast<const uint4*>(w + (size_t)e * 2);
-            acc[4 * m + 0] = __ffma2_rn(bf16x2_to_f2(w4.x), s2, acc[4 * m + 0]);
-            acc[4 * m + 1] = __ffma2_rn(bf16x2_to_f2(w4.y), s2, acc[4 * m + 1]);
-            acc[4 * m + 2] = __ffma2_rn(bf16x2_to_f2(w4.z), s2, acc[4 * m + 2]);
-            acc[4 * m + 3] = __ffma2_rn(bf16x2_to_f2(w4.w), s2, acc[4 * m + 3]);
-          }
-        }
+      for (int m = 0; m < MAXM; ++m) {
+        const int e = elem(m);
+        wv[h][m] = (elem_ok(m) && (h == 0 || two))
+                       ? *reinterpret_cast<const uint4*>(w + h * col_bytes + (size_t)e * 2)
+                       : make_uint4(0u, 0u, 0u, 0u);
       }
     }
     __syncwarp();
-    if (lane == 0) {
-      mbar_arrive(&empty[sl[0]], 1);
-      if (rb0 + 1 < nB) mbar_arrive(&empty[sl[1]], 1);
+    if (lane == 0) mbar_arrive(&empty[slot], 1);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const float sv = (h == 0 || two) ? s_val[2 * p + h] : 0.f;
+      const float2 s2 = make_float2(sv, sv);
+#pragma unroll
+      for (int m = 0; m < MAXM; ++m) {
+        const uint4 w4 = wv[h][m];
+        acc[4 * m + 0] = __ffma2_rn(bf16x2_to_f2(w4.x), s2, acc[4 * m + 0]);
+        acc[4 * m + 1] = __ffma2_rn(bf16x2_to_f2(w4.y), s2, acc[4 * m + 1]);
+        acc[4 * m + 2] = __ffma2_rn(bf16x2_to_f2(w4.z), s2, acc[4 * m + 2]);
+        acc[4 * m + 3] = __ffma2_rn(bf16x2_to_f2(w4.w), s2, acc[4 * m + 3]);
+      }
     }
   }
-  float* dst = a.ypart + (size_t)cta * d;
+  // The groups' partial rows are added in group order (deterministic).  Every
+  // copy has landed (each item was waited for), so the ring holds them.
+  asm volatile("bar.sync 1, %0;" ::"r"(NCW * 32) : "memory");
+  float* s_y = reinterpret_cast<float*>(ring);  // [NG][d]
 #pragma unroll
   for (int m = 0; m < MAXM; ++m) {
-    const int e = tid * 8 + m * (NCW * 32 * 8);
-    if (e < d) {
-      *reinterpret_cast<float4*>(dst + e) =
+    if (elem_ok(m)) {
+      float* dst = s_y + (size_t)grp * d + elem(m);
+      *reinterpret_cast<float4*>(dst) =
           make_float4(acc[4 * m].x, acc[4 * m].y, acc[4 * m + 1].x, acc[4 * m + 1].y);
-      *reinterpret_cast<float4*>(dst + e + 4) =
+      *reinterpret_cast<float4*>(dst + 4) =
           make_float4(acc[4 * m + 2].x, acc[4 * m + 2].y, acc[4 * m + 3].x, acc[4 * m + 3].y);
     }
+  }
+  asm volatile("bar.sync 1, %0;" ::"r"(NCW * 32) : "memory");
+  float* out = a.ypart + (size_t)cta * d;
+  for (int e = tid * 4; e < d; e += NCW * 32 * 4) {
+    float4 v = *reinterpret_cast<const float4*>(s_y + e);
+    for (int g = 1; g < NG; ++g) {
+      const float4 t = *reinterpret_cast<const float4*>(s_y + (size_t)g * d + e);
+      v.x += t.x;
+      v.y += t.y;
+      v.z += t.z;
+      v.w += t.w;
+    }
+    *reinterpret_cast<float4*>(out + e) = v;
   }
 }
 
@@ -400,7 +389,7 @@ cudaError_t set_stage2_attr() {
 
 }  // namespace
 
-void choose_stage2(int d, int F, int num_sms, int* P, int* slots, int* nprod, size_t* smem) {
+void choose_stage2(int d, int F, int num_sms, int* P, int* slots, int* groups, size_t* smem) {
   *P = num_sms;
   const int max_rec = (F + num_sms - 1) / num_sms + 1;
   size_t off = (size_t)max_rec * (12 + 8 * NCW) + 128;
@@ -408,19 +397,25 @@ void choose_stage2(int d, int F, int num_sms, int* P, int* slots, int* nprod, si
   int s = (int)((kStage2SmemBudget - off) / (slot_bytes + 16));
   if (s > 32) s = 32;
   if (s < 2) s = 2;
-  // producer lanes: the slot count must be a multiple of them
-  if (s >= 8) {
-    s -= s % 4;
-    *nprod = 4;
-  } else {
-    s -= s % 2;
-    *nprod = 2;
+  // Consumer groups: the most groups (4, 2, 1) whose slot share is at least
+  // two and whose warps hold at most 4 chunks of 8 elements per lane.
+  int ng = 1;
+  for (int cand : {4, 2}) {
+    const int wpg = NCW / cand;
+    const int maxm = (d + wpg * 256 - 1) / (wpg * 256);
+    if ((s - s % cand) / cand >= 2 && maxm <= 4) {
+      ng = cand;
+      break;
+    }
   }
+  s -= s % ng;
+  *groups = ng;
   *slots = s;
   off = (size_t)s * 16 + (size_t)max_rec * (12 + 8 * NCW);
   off = (off + 127) & ~(size_t)127;
   size_t region = (size_t)s * slot_bytes;
   if (region < sizeof(SelectScratch)) region = sizeof(SelectScratch);  // the select's scratch
+  if (region < (size_t)ng * d * 4) region = (size_t)ng * d * 4;         // the groups' partial rows
   *smem = off + region;
 }
 
@@ -429,8 +424,7 @@ cudaError_t setup_stage2_kernels() {
   if ((e = set_stage2_attr<1>()) != cudaSuccess) return e;
   if ((e = set_stage2_attr<2>()) != cudaSuccess) return e;
   if ((e = set_stage2_attr<3>()) != cudaSuccess) return e;
-  if ((e = set_stage2_attr<4>()) != cudaSuccess) return e;
-  return set_stage2_attr<8>();
+  return set_stage2_attr<4>();
 }
 
 cudaError_t launch_stage2(const prox_layer* L, const float* x, const Stage2Launch& m,
@@ -452,7 +446,7 @@ cudaError_t launch_stage2(const prox_layer* L, const float* x, const Stage2Launc
   a.F = L->F;
   a.P = L->P;
   a.slots = L->ring_slots;
-  a.nprod = L->stage2_producers;
+  a.groups = L->stage2_groups;
   a.max_rec = (L->F + L->P - 1) / L->P + 1;
   a.ypart = L->ws.ypart;
   a.s_sp = m.s_sp;
@@ -469,12 +463,12 @@ cudaError_t launch_stage2(const prox_layer* L, const float* x, const Stage2Launc
   attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const int mm = (L->d + 2047) / 2048;
+  const int wpg = NCW / L->stage2_groups;
+  const int mm = (L->d + wpg * 256 - 1) / (wpg * 256);
   if (mm <= 1) return launch_stage2_t<1>(cfg, a);
   if (mm == 2) return launch_stage2_t<2>(cfg, a);
   if (mm == 3) return launch_stage2_t<3>(cfg, a);
-  if (mm == 4) return launch_stage2_t<4>(cfg, a);
-  return launch_stage2_t<8>(cfg, a);
+  return launch_stage2_t<4>(cfg, a);  // choose_stage2 keeps mm <= 4
 }
 
 cudaError_t launch_reduce(const prox_layer* L, float* out, cudaStream_t s, bool pdl) {

@@ -281,3 +281,51 @@ def rmsnorm(y, eps=1e-6):
     """
     y = np.asarray(y, dtype=F64)
     return y / np.sqrt(np.mean(y * y) + eps)
+
+
+# ---------------------------------------------------------------------------
+# A stack of layers (the synthetic multi-layer workload)
+# ---------------------------------------------------------------------------
+
+def stack_next_input(y, eps=1e-6):
+    """Input of the next stacked layer: RMSNorm of the output, held in fp32 like
+    every layer input."""
+    return np.asarray(rmsnorm(y, eps), dtype=np.float32)
+
+
+def calibrate_stack(layers, x_cal, s1, k, group=GROUP, eps=1e-6):
+    """Sequential threshold calibration (Prox App. A.7, Algorithm 1) with the
+    top-k Stage-2 rule: layer l's threshold is the s1-quantile of its own
+    inputs, which are the calibration tokens run through layers 1..l-1 with
+    their finalised thresholds (the current layer's inputs are collected before
+    its own rule is fixed).
+
+    ``layers``: sequence of (w_gate, w_up, w_down, q_gate, s_gate, q_up, s_up).
+    Returns (taus, inputs): the threshold of every layer and the calibration
+    inputs each layer saw (n_cal x d_model fp32 arrays).
+    """
+    x = np.asarray(x_cal, dtype=np.float32)
+    taus, inputs = [], []
+    for li, (wg, wu, wd, qg, sg, qu, su) in enumerate(layers):
+        inputs.append(x)
+        tau = calibrate_tau(x, s1)
+        taus.append(tau)
+        if li + 1 < len(layers):
+            ys = [prox_ffn(xt, wg, wu, wd, qg, sg, qu, su, tau=tau, k=k, group=group)["y"]
+                  for xt in x]
+            x = np.stack([stack_next_input(yt, eps) for yt in ys])
+    return taus, inputs
+
+
+def stack_forward(layers, taus, x, k, group=GROUP, eps=1e-6):
+    """One token through the stack: the Prox step of every layer, RMSNorm in
+    between.  Returns the per-layer inputs and the last layer's output."""
+    xs = []
+    x = np.asarray(x, dtype=np.float32)
+    y = None
+    for li, ((wg, wu, wd, qg, sg, qu, su), tau) in enumerate(zip(layers, taus)):
+        xs.append(x)
+        y = prox_ffn(x, wg, wu, wd, qg, sg, qu, su, tau=tau, k=k, group=group)["y"]
+        if li + 1 < len(layers):
+            x = stack_next_input(y, eps)
+    return xs, y

@@ -1,0 +1,142 @@
+"""GPU parity on the remaining workloads: the Qwen3-14B-shaped layer at three
+input sparsities, the Llama-3-70B-shaped layer at batch 1..16 (independent
+per-token masks), and layer stacks chained through RMSNorm with sequential
+threshold calibration (Prox App. A.7, Algorithm 1).
+
+Bars as in test_gpu_parity.py.  Stacks are checked teacher-forced: each GPU
+layer gets the oracle's inputs for that layer; the free-running GPU stack is
+checked only loosely (its earlier layers round differently).
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import prox_oracle as orc
+from tests.gpu_helpers import (OUT_RTOL, OracleLayer, bits_to_bf16, check_mask,
+                               close_with_floor, device_layer, rel_l2)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def prox():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import activation_sparse_swiglu_b200 as p
+    return p
+
+
+def _step_checks(layer, olay, x, tau, k):
+    """Stage-1 taps, the mask rule and the output (given the oracle's mask)."""
+    ref = olay.step(x, tau, k)
+    xd = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).cuda()
+    taps = layer.debug_stage1(xd)
+    y_m, s_sp = layer.forward_with_mask(
+        xd, torch.from_numpy(ref["idx_s"].astype(np.int32)).cuda(), want_s=True)
+    torch.cuda.synchronize()
+    n_x = int(taps["n_x"].item())
+    np.testing.assert_array_equal(taps["idx_x"].cpu().numpy()[:n_x], ref["idx_x"])
+    ok, nbad = close_with_floor(taps["g_tilde"].cpu().numpy(), ref["g_tilde"])
+    assert ok, f"g~ off at {nbad} channels"
+    ok, nbad = close_with_floor(taps["u_tilde"].cpu().numpy(), ref["u_tilde"])
+    assert ok, f"u~ off at {nbad} channels"
+    check_mask(taps["idx_s"].cpu().numpy(), ref["idx_s"], ref["scores"], k)
+    assert rel_l2(y_m.cpu().numpy(), ref["y"]) <= OUT_RTOL
+    assert rel_l2(s_sp.cpu().numpy(), ref["s_sp"]) <= OUT_RTOL
+    return ref
+
+
+# ---------------------------------------------------------------------------
+# Qwen3-14B shape: s1 in {40, 50, 60} %
+# ---------------------------------------------------------------------------
+
+def test_qwen3_14b_three_input_sparsities(prox):
+    lay = synth.make_layer("qwen3_14b", n_tokens=2, n_cal=64)
+    olay = OracleLayer(lay)
+    k = lay.config.k()
+    layer = device_layer(lay, 0.0, k)
+    xc = torch.from_numpy(lay.x_cal).cuda()
+    for s1 in lay.config.s1_percent:
+        tau = orc.calibrate_tau(lay.x_cal, s1 / 100)
+        assert np.float32(prox.calibrate_thresholds(xc, s1 / 100)) == tau
+        layer.set_tau(tau)
+        _step_checks(layer, olay, lay.x_eval[0], tau, k)
+    assert layer.error_word() == 0
+    layer.close()
+
+
+# ---------------------------------------------------------------------------
+# Llama-3-70B shape at batch 1..16, per-token masks
+# ---------------------------------------------------------------------------
+
+def test_llama3_70b_batches(prox):
+    lay = synth.make_layer("llama3_70b", n_cal=32)
+    olay = OracleLayer(lay)
+    k = lay.config.k()
+    tau = orc.calibrate_tau(lay.x_cal, 0.5)
+    layer = device_layer(lay, tau, k, max_batch=16)
+    x = torch.from_numpy(lay.x_eval).cuda()
+    singles = torch.stack([layer.forward(x[i]).reshape(-1) for i in range(16)])
+    for b in lay.config.batch_sizes:
+        yb = layer.forward(x[:b])
+        torch.cuda.synchronize()
+        assert torch.equal(yb, singles[:b])  # each token keeps its own mask
+    for t in range(2):
+        ref = _step_checks(layer, olay, lay.x_eval[t], tau, k)
+        y_full = singles[t].cpu().numpy()
+        if np.array_equal(layer.debug_stage1(x[t])["idx_s"].cpu().numpy(), ref["idx_s"]):
+            assert rel_l2(y_full, ref["y"]) <= OUT_RTOL
+    assert layer.error_word() == 0
+    layer.close()
+
+
+# ---------------------------------------------------------------------------
+# Stacks with sequential calibration
+# ---------------------------------------------------------------------------
+
+def _stack_case(prox, cfg, n_layers, n_cal, n_tok):
+    from activation_sparse_swiglu_b200.stack import Stack
+    lays = [synth.make_layer(cfg, li, draw_tokens=(li == 0), n_cal=n_cal, n_tokens=n_tok)
+            for li in range(n_layers)]
+    x_cal, x_eval = lays[0].x_cal, lays[0].x_eval
+    olays = [OracleLayer(lay) for lay in lays]
+    layers = [(l.w_gate, l.w_up, l.w_down, o.qg, o.sg, o.qu, o.su) for l, o in zip(lays, olays)]
+    k = cfg.k()
+    taus, cal_inputs = orc.calibrate_stack(layers, x_cal, 0.5, k)
+    weights = [(bits_to_bf16(l.w_gate_bits), bits_to_bf16(l.w_up_bits), bits_to_bf16(l.w_down_bits))
+               for l in lays]
+    stack = Stack(weights, k, max_batch=max(n_cal, n_tok))
+    del weights
+    # free-running GPU calibration: thresholds close to the oracle's
+    g_taus, _ = stack.calibrate(torch.from_numpy(x_cal).cuda(), 0.5)
+    for gt, ot in zip(g_taus, taus):
+        assert abs(gt - ot) <= 1e-4 * ot, (gt, ot)
+    # teacher-forced: every layer on the oracle's own inputs
+    for li, (layer, olay) in enumerate(zip(stack.layers, olays)):
+        tau_g = prox.calibrate_thresholds(torch.from_numpy(cal_inputs[li]).cuda(), 0.5)
+        assert np.float32(tau_g) == taus[li]
+        layer.set_tau(taus[li])
+    for t in range(n_tok):
+        xs, y_ref = orc.stack_forward(layers, taus, x_eval[t], k)
+        for li, (layer, olay) in enumerate(zip(stack.layers, olays)):
+            _step_checks(layer, olay, xs[li], taus[li], k)
+        # free-running output, reported loosely
+        _, y = stack.forward(torch.from_numpy(x_eval[t:t + 1]).cuda())
+        assert rel_l2(y.cpu().numpy().reshape(-1), y_ref) <= 5e-2
+    for layer in stack.layers:
+        assert layer.error_word() == 0
+    stack.close()
+
+
+def test_stack_of_eight_small_layers(prox):
+    cfg = synth.WorkloadConfig(name="stack_small", index=62, d_model=512, d_ff=1376, sigma=0.02,
+                               outlier_frac=0.01, outlier_scale=20.0, s1_percent=(50,),
+                               s2_percent=(70,), n_tokens=2, n_cal=32, n_layers=8)
+    _stack_case(prox, cfg, n_layers=8, n_cal=32, n_tok=2)
+
+
+def test_stack32_first_two_layers_full_size(prox):
+    # the 32-layer workload's own seeds and shapes, first two layers
+    _stack_case(prox, synth.get_config("stack32"), n_layers=2, n_cal=16, n_tok=1)

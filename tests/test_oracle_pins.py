@@ -408,3 +408,51 @@ def test_rmsnorm_closed_form():
     np.testing.assert_allclose(orc.rmsnorm(y, eps), c / np.sqrt(c * c + eps), rtol=1e-15)
     z = np.random.default_rng(8).standard_normal(4096) * 3
     assert abs(np.sqrt(np.mean(orc.rmsnorm(z, 0.0) ** 2)) - 1) < 1e-14
+
+
+# ---------------------------------------------------------------------------
+# the layer stack (sequential calibration, Prox App. A.7 Algorithm 1)
+# ---------------------------------------------------------------------------
+
+def _small_stack(n_layers=3, d=256, f=384, n_cal=24, n_tok=2):
+    from synth.configs import WorkloadConfig
+    cfg = WorkloadConfig(name="stack_small", index=61, d_model=d, d_ff=f, sigma=0.05,
+                         outlier_frac=0.01, outlier_scale=20.0, s1_percent=(50,),
+                         s2_percent=(70,), n_tokens=n_tok, n_cal=n_cal, n_layers=n_layers)
+    layers = []
+    x_cal = x_eval = None
+    for li in range(n_layers):
+        lay = synth.make_layer(cfg, li, draw_tokens=(li == 0))
+        if li == 0:
+            x_cal, x_eval = lay.x_cal, lay.x_eval
+        qg, sg = orc.quantize_proxy(lay.w_gate)
+        qu, su = orc.quantize_proxy(lay.w_up)
+        layers.append((lay.w_gate, lay.w_up, lay.w_down, qg, sg, qu, su))
+    return cfg, layers, x_cal, x_eval
+
+
+def test_stack_keep_all_is_the_dense_chain():
+    # s1 = 0 and k = d_ff: every layer is the dense SwiGLU, chained by RMSNorm
+    cfg, layers, x_cal, x_eval = _small_stack()
+    taus, _ = orc.calibrate_stack(layers, x_cal, 0.0, cfg.d_ff)
+    assert taus == [0.0] * len(layers)
+    _, y = orc.stack_forward(layers, taus, x_eval[0], cfg.d_ff)
+    x = x_eval[0].astype(np.float64)
+    for li, (wg, wu, wd, *_rest) in enumerate(layers):
+        h = orc.dense_ffn(x, wg, wu, wd)
+        if li + 1 < len(layers):
+            x = (h / np.sqrt(np.mean(h * h) + 1e-6)).astype(np.float32).astype(np.float64)
+    np.testing.assert_allclose(y, h, rtol=1e-12, atol=1e-12)
+
+
+def test_stack_every_layer_keeps_the_target_fraction_of_its_own_inputs():
+    cfg, layers, x_cal, _ = _small_stack()
+    taus, inputs = orc.calibrate_stack(layers, x_cal, 0.5, cfg.k())
+    n = x_cal.size
+    r = int(np.floor(0.5 * n))
+    for tau, xin in zip(taus, inputs):
+        # tau is the order statistic of rank r of this layer's own |x|
+        a = np.abs(xin.astype(np.float64)).ravel()
+        assert np.count_nonzero(a < tau) <= r < np.count_nonzero(a <= tau)
+    # later layers see the earlier sparse layers' outputs, not the raw tokens
+    assert not np.array_equal(inputs[1], inputs[0])
