@@ -389,9 +389,11 @@ __global__ void __launch_bounds__(S1_NT, 1) stage1_kernel(Stage1Args a) {
     a.part[((size_t)cta * 2) * S1_PART + e] = p0;
     if (nsl == 2) a.part[((size_t)cta * 2 + 1) * S1_PART + e] = p1;
   }
-  __threadfence();
+  // The barrier orders every thread's partial writes before thread 0's fence,
+  // which (cumulatively) orders them before its counter updates at GPU scope.
   __syncthreads();
   if (tid == 0) {
+    __threadfence();
     const int rows0 = min(len, l_split);
     int done = 0;
     if (len > 0) {
