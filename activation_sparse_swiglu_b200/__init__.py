@@ -16,11 +16,13 @@ import ctypes
 
 import torch
 
-from ._lib import (DEVERR_MASK_INDEX, DEVERR_WAIT_TIMEOUT, LayerInfo, ProxError, check,
+from ._lib import (DEVERR_MASK_INDEX, DEVERR_WAIT_TIMEOUT, MASK_THRESHOLD, MASK_TOPK, LayerInfo,
+                   ProxError, check,
                    last_error, lib)
 
 __all__ = ["Layer", "pack_proxy", "calibrate_thresholds", "rmsnorm", "copy", "version",
-           "ProxError", "DEVERR_MASK_INDEX", "DEVERR_WAIT_TIMEOUT", "last_error", "lib"]
+           "ProxError", "DEVERR_MASK_INDEX", "DEVERR_WAIT_TIMEOUT", "MASK_TOPK", "MASK_THRESHOLD",
+           "last_error", "lib"]
 
 GROUP = 128
 
@@ -168,16 +170,40 @@ class Layer:
     def set_k(self, k: int) -> None:
         check(lib.prox_layer_set_k(self.handle, int(k)))
 
+    def set_mask(self, mode: int, tau_s: float = 0.0) -> None:
+        """Stage-2 rule: MASK_TOPK (uses k) or MASK_THRESHOLD (score >= tau_s)."""
+        check(lib.prox_layer_set_mask(self.handle, int(mode), float(tau_s)))
+
     def error_word(self, stream=None) -> int:
         v = ctypes.c_int32(0)
         check(lib.prox_layer_error(self.handle, ctypes.byref(v), _stream(stream)))
         return int(v.value)
 
-    def stats(self, stream=None):
-        """(sum of n_x, tokens) since the last call."""
-        s, t = ctypes.c_int64(0), ctypes.c_int64(0)
-        check(lib.prox_layer_stats(self.handle, ctypes.byref(s), ctypes.byref(t), _stream(stream)))
+    def stats(self, stream=None, with_selected: bool = False):
+        """(sum of n_x, tokens[, sum of selected Stage-2 channels]) since the last call."""
+        s, t, c = ctypes.c_int64(0), ctypes.c_int64(0), ctypes.c_int64(0)
+        check(lib.prox_layer_stats(self.handle, ctypes.byref(s), ctypes.byref(t), ctypes.byref(c),
+                                   _stream(stream)))
+        if with_selected:
+            return int(s.value), int(t.value), int(c.value)
         return int(s.value), int(t.value)
+
+    def proxy_scores(self, x: torch.Tensor, stream=None) -> torch.Tensor:
+        """Stage-1 scores |SiLU(g~) u~| of tokens x [B, d] as fp32 [B, d_ff]."""
+        _dev(x, torch.float32, "x")
+        x2 = x.reshape(-1, self.d_model)
+        out = torch.empty((x2.shape[0], self.d_ff), dtype=torch.float32, device=x.device)
+        check(lib.prox_layer_proxy_scores(self.handle, _ptr(x2), x2.shape[0], _ptr(out),
+                                          _stream(stream)))
+        return out
+
+    def debug_mask(self, x: torch.Tensor, stream=None) -> torch.Tensor:
+        """The Stage-2 channels one token selects under the current rule (int32, ascending)."""
+        _dev(x, torch.float32, "x")
+        idx = torch.empty(self.d_ff, dtype=torch.int32, device=x.device)
+        n = torch.zeros(1, dtype=torch.int32, device=x.device)
+        check(lib.prox_debug_mask(self.handle, _ptr(x), _ptr(idx), _ptr(n), _stream(stream)))
+        return idx[: int(n.item())]
 
     # -- compute ---------------------------------------------------------
     def _io(self, x, out):

@@ -33,7 +33,12 @@ class LayerInfo(ctypes.Structure):
         ("stage2_ctas", ctypes.c_int), ("stage2_ring_slots", ctypes.c_int),
         ("weight_bytes", ctypes.c_size_t), ("proxy_bytes", ctypes.c_size_t),
         ("workspace_bytes", ctypes.c_size_t),
+        ("mask_mode", ctypes.c_int), ("tau_s", ctypes.c_float),
     ]
+
+
+MASK_TOPK = 0
+MASK_THRESHOLD = 1
 
 
 _P = ctypes.c_void_p
@@ -50,15 +55,18 @@ SIGNATURES = {
     "prox_layer_destroy": (_I, [_P]),
     "prox_layer_set_tau": (_I, [_P, _F]),
     "prox_layer_set_k": (_I, [_P, _I]),
+    "prox_layer_set_mask": (_I, [_P, _I, _F]),
     "prox_layer_get_info": (_I, [_P, ctypes.POINTER(LayerInfo)]),
     "prox_layer_error": (_I, [_P, ctypes.POINTER(ctypes.c_int32), _P]),
     "prox_layer_stats": (_I, [_P, ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int64),
-                              _P]),
+                              ctypes.POINTER(ctypes.c_int64), _P]),
     "prox_ffn_forward": (_I, [_P, _P, _P, _I, _P]),
     "prox_dense_ffn": (_I, [_P, _P, _P, _I, _P]),
     "prox_ffn_forward_host": (_I, [_P, _P, _P, _I, _P]),
     "prox_ffn_forward_profiled": (_I, [_P, _P, _P, ctypes.POINTER(_P), _P]),
     "prox_debug_stage1": (_I, [_P, _P, _P, _P, _P, _P, _P, _P]),
+    "prox_layer_proxy_scores": (_I, [_P, _P, _I, _P, _P]),
+    "prox_debug_mask": (_I, [_P, _P, _P, _P, _P]),
     "prox_forward_with_mask": (_I, [_P, _P, _P, _I, _P, _P, _P]),
     "prox_rmsnorm": (_I, [_P, _P, _I, _I, _F, _P]),
     "prox_copy": (_I, [_P, _P, _S, _P]),

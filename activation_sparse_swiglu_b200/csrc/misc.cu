@@ -51,7 +51,8 @@ __global__ void __launch_bounds__(256) copy_kernel(const uint4* __restrict__ src
 
 // One CTA of 1024 threads: thread t owns entries [t*per, (t+1)*per).
 __global__ void __launch_bounds__(1024) mask_to_list_kernel(const int32_t* __restrict__ mask,
-                                                            int n, int32_t* __restrict__ list) {
+                                                            int n, int32_t* __restrict__ list,
+                                                            int32_t* count) {
   __shared__ int s_scan[33];
   const int per = (n + 1023) / 1024;
   const int lo = min((int)threadIdx.x * per, n), hi = min(lo + per, n);
@@ -61,12 +62,14 @@ __global__ void __launch_bounds__(1024) mask_to_list_kernel(const int32_t* __res
   int pos = block_exclusive_scan(c, s_scan, &total);
   for (int i = lo; i < hi; ++i)
     if (mask[i] != 0) list[pos++] = i;
+  if (count && threadIdx.x == 0) *count = total;
 }
 
 }  // namespace
 
-cudaError_t launch_mask_to_list(const int32_t* mask, int n, int32_t* list, cudaStream_t s) {
-  mask_to_list_kernel<<<1, 1024, 0, s>>>(mask, n, list);
+cudaError_t launch_mask_to_list(const int32_t* mask, int n, int32_t* list, int32_t* count,
+                                cudaStream_t s) {
+  mask_to_list_kernel<<<1, 1024, 0, s>>>(mask, n, list, count);
   return cudaGetLastError();
 }
 

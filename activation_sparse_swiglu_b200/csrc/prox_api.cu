@@ -1,6 +1,7 @@
 // C ABI of the Prox library: argument checks, the layer handle, and the
 // stream-ordered kernel chains of the decode step.
 #include <atomic>
+#include <cfloat>
 #include <cmath>
 #include <mutex>
 #include <cstdarg>
@@ -107,7 +108,7 @@ prox_status alloc_workspace(prox_layer* L) {
   const size_t o_s1p = take(prox::stage1_part_floats(L->P1) * 4);
   const size_t o_s1c = take((size_t)L->C * 4);
   const size_t o_ypart = take((size_t)L->P * d * 4);
-  const size_t o_stats = take(16);
+  const size_t o_stats = take(24);
   const size_t o_err = take(4);
   const size_t o_in = take((size_t)kHostChunkTokens * d * 4);
   const size_t o_out = take((size_t)kHostChunkTokens * d * 4);
@@ -135,10 +136,13 @@ prox_status alloc_workspace(prox_layer* L) {
   return PROX_OK;
 }
 
+// The Stage-2 selection of the forward step: the layer's rule (top-k or the
+// score threshold).
 prox::Stage2Launch topk_launch(const prox_layer* L) {
   prox::Stage2Launch m;
-  m.mode = 1;
+  m.mode = L->mask_mode == PROX_MASK_THRESHOLD ? 3 : 1;
   m.k = L->k;
+  m.tau_s = L->tau_s;
   return m;
 }
 
@@ -368,6 +372,17 @@ prox_status prox_layer_set_k(prox_layer* L, int k) {
   return PROX_OK;
 }
 
+prox_status prox_layer_set_mask(prox_layer* L, int mode, float tau_s) {
+  if (!L) return fail(PROX_EINVAL, "layer handle is NULL");
+  if (mode != PROX_MASK_TOPK && mode != PROX_MASK_THRESHOLD)
+    return fail(PROX_EINVAL, "mask mode %d is neither PROX_MASK_TOPK nor PROX_MASK_THRESHOLD", mode);
+  if (mode == PROX_MASK_THRESHOLD && !(tau_s >= 0.f && tau_s <= FLT_MAX))
+    return fail(PROX_EINVAL, "tau_s=%g must be finite and >= 0", (double)tau_s);
+  L->mask_mode = mode;
+  L->tau_s = mode == PROX_MASK_THRESHOLD ? tau_s : 0.f;
+  return PROX_OK;
+}
+
 prox_status prox_layer_get_info(const prox_layer* L, prox_layer_info* info) {
   if (!L || !info) return fail(PROX_EINVAL, "NULL argument");
   info->d_model = L->d;
@@ -383,6 +398,8 @@ prox_status prox_layer_get_info(const prox_layer* L, prox_layer_info* info) {
   info->weight_bytes = (size_t)3 * L->F * L->d * 2;
   info->proxy_bytes = (size_t)L->d * L->F + (size_t)L->G * L->F * 4;
   info->workspace_bytes = L->ws.bytes;
+  info->mask_mode = L->mask_mode;
+  info->tau_s = L->tau_s;
   return PROX_OK;
 }
 
@@ -400,16 +417,17 @@ prox_status prox_layer_error(prox_layer* L, int32_t* word_host, void* stream) {
 }
 
 prox_status prox_layer_stats(prox_layer* L, int64_t* sum_nx_host, int64_t* tokens_host,
-                             void* stream) {
+                             int64_t* sum_sel_host, void* stream) {
   prox_status st = check_layer(L);
   if (st != PROX_OK) return st;
   cudaStream_t s = as_stream(stream);
-  unsigned long long v[2] = {0, 0};
-  PROX_CUDA(cudaMemcpyAsync(v, L->ws.stats, 16, cudaMemcpyDeviceToHost, s), "read stats");
-  PROX_CUDA(cudaMemsetAsync(L->ws.stats, 0, 16, s), "clear stats");
+  unsigned long long v[3] = {0, 0, 0};
+  PROX_CUDA(cudaMemcpyAsync(v, L->ws.stats, 24, cudaMemcpyDeviceToHost, s), "read stats");
+  PROX_CUDA(cudaMemsetAsync(L->ws.stats, 0, 24, s), "clear stats");
   PROX_CUDA(cudaStreamSynchronize(s), "cudaStreamSynchronize");
   if (sum_nx_host) *sum_nx_host = (int64_t)v[0];
   if (tokens_host) *tokens_host = (int64_t)v[1];
+  if (sum_sel_host) *sum_sel_host = (int64_t)v[2];
   return PROX_OK;
 }
 
@@ -489,6 +507,8 @@ prox_status prox_debug_stage1(prox_layer* L, const float* x, int32_t* idx_x, int
   prox_status st = check_layer(L);
   if (st != PROX_OK) return st;
   if (!x || !aligned16(x)) return fail(PROX_EINVAL, "x must be a 16-byte aligned pointer");
+  if (idx_s && L->mask_mode != PROX_MASK_TOPK)
+    return fail(PROX_EINVAL, "idx_s holds k channels under top-k only; use prox_debug_mask");
   cudaStream_t s = as_stream(stream);
   prox::Stage1Taps t1;
   t1.g = g_tilde;
@@ -503,7 +523,42 @@ prox_status prox_debug_stage1(prox_layer* L, const float* x, int32_t* idx_x, int
   PROX_CUDA(prox::launch_stage2(L, x, m, s, false, true), "stage2 launch");
   PROX_CUDA(cudaMemsetAsync(L->ws.hist, 0, prox::kScoreBins * 4, s), "clear histogram");
   if (idx_s)
-    PROX_CUDA(prox::launch_mask_to_list(L->ws.sel_mask, L->F, idx_s, s), "mask compaction launch");
+    PROX_CUDA(prox::launch_mask_to_list(L->ws.sel_mask, L->F, idx_s, nullptr, s),
+              "mask compaction launch");
+  return PROX_OK;
+}
+
+prox_status prox_debug_mask(const prox_layer* L, const float* x, int32_t* idx_s, int32_t* n_s,
+                            void* stream) {
+  prox_status st = check_layer(L);
+  if (st != PROX_OK) return st;
+  if (!x || !aligned16(x) || !idx_s || !n_s)
+    return fail(PROX_EINVAL, "x (16-byte aligned), idx_s and n_s must be non-NULL");
+  cudaStream_t s = as_stream(stream);
+  PROX_CUDA(prox::launch_stage1(L, x, prox::Stage1Taps{}, s, false), "stage1 launch");
+  prox::Stage2Launch m = topk_launch(L);
+  m.select_only = true;
+  m.sel_mask = L->ws.sel_mask;
+  PROX_CUDA(prox::launch_stage2(L, x, m, s, false, true), "stage2 launch");
+  PROX_CUDA(cudaMemsetAsync(L->ws.hist, 0, prox::kScoreBins * 4, s), "clear histogram");
+  PROX_CUDA(prox::launch_mask_to_list(L->ws.sel_mask, L->F, idx_s, n_s, s), "mask compaction launch");
+  return PROX_OK;
+}
+
+prox_status prox_layer_proxy_scores(const prox_layer* L, const float* x, int B, float* scores,
+                                    void* stream) {
+  prox_status st = check_layer(L);
+  if (st != PROX_OK) return st;
+  if (B < 1 || B > L->max_batch) return fail(PROX_EINVAL, "B=%d must be in [1, %d]", B, L->max_batch);
+  if (!x || !scores || !aligned16(x)) return fail(PROX_EINVAL, "x (16-byte aligned) and scores must be non-NULL");
+  cudaStream_t s = as_stream(stream);
+  for (int b = 0; b < B; ++b) {
+    PROX_CUDA(prox::launch_stage1(L, x + (size_t)b * L->d, prox::Stage1Taps{}, s, false),
+              "stage1 launch");
+    PROX_CUDA(cudaMemcpyAsync(scores + (size_t)b * L->F, L->ws.scores, (size_t)L->F * 4,
+                              cudaMemcpyDeviceToDevice, s), "copy scores");
+    PROX_CUDA(cudaMemsetAsync(L->ws.hist, 0, prox::kScoreBins * 4, s), "clear histogram");
+  }
   return PROX_OK;
 }
 

@@ -40,7 +40,7 @@ struct Workspace {
   float* s1_part = nullptr;        // Stage-1 partial sums [P1][2][1024]
   int* s1_cnt = nullptr;          // [C] Stage-1 row slices reported per slice, zero between tokens
   float* ypart = nullptr;         // Stage-2 output partials [P][d]
-  unsigned long long* stats = nullptr;  // [2] sum n_x, tokens
+  unsigned long long* stats = nullptr;  // [3] sum n_x, tokens, sum of selected channels
   int* err = nullptr;             // device error word
   float* stage_in = nullptr;      // host-path staging [kHostChunkTokens][d]
   float* stage_out = nullptr;
@@ -53,6 +53,8 @@ struct Workspace {
 struct prox_layer {
   int d = 0, F = 0, G = 0, k = 0, max_batch = 0;
   float tau = 0.f;
+  int mask_mode = 0;     // PROX_MASK_TOPK or PROX_MASK_THRESHOLD
+  float tau_s = 0.f;     // Stage-2 score threshold (threshold mode)
   int device = 0, num_sms = 0;
   // Stage-1 geometry: C column slices, P1 CTAs, at most s1_lmax rows per CTA
   int C = 0, P1 = 0, s1_lmax = 0;
@@ -78,7 +80,8 @@ struct Stage1Taps {
 };
 // How Stage 2 obtains its channels.
 struct Stage2Launch {
-  int mode = 1;               // 0: given list `idx`, 1: top-k select, 2: dense
+  int mode = 1;               // 0: given list `idx`, 1: top-k select, 2: dense, 3: score threshold
+  float tau_s = 0.f;          // mode 3: channels with score >= tau_s
   const int32_t* idx = nullptr;
   int k = 0;
   int32_t* sel_mask = nullptr;  // top-k: 1/0 per channel written here (debug)
@@ -111,7 +114,8 @@ cudaError_t launch_calibrate(const float* X, size_t n, unsigned long long rank,
 cudaError_t launch_rmsnorm(const float* y, float* x, int rows, int d, float eps,
                            cudaStream_t s);
 cudaError_t launch_copy(const void* src, void* dst, size_t bytes, cudaStream_t s);
-cudaError_t launch_mask_to_list(const int32_t* mask, int n, int32_t* list, cudaStream_t s);
+cudaError_t launch_mask_to_list(const int32_t* mask, int n, int32_t* list, int32_t* count,
+                                cudaStream_t s);
 
 // Stage-1 column slices, CTAs and per-CTA row capacity for a shape on `num_sms` SMs.
 void choose_stage1_grid(int d, int F, int num_sms, int* C, int* P1, int* lmax);

@@ -37,7 +37,7 @@ constexpr int NCW = kStage2Consumers;
 constexpr int S2_THREADS = (NCW + 1) * 32;
 constexpr size_t kStage2SmemBudget = 208 * 1024;
 
-enum Stage2Mode { kGivenList = 0, kTopK = 1, kDense = 2 };
+enum Stage2Mode { kGivenList = 0, kTopK = 1, kDense = 2, kThreshold = 3 };
 
 struct Stage2Args {
   const float* x;
@@ -48,7 +48,8 @@ struct Stage2Args {
   const uint32_t* hist;    // kTopK: Stage-1 histogram of the scores' bits 30..20
   unsigned long long* stats;
   const uint2* bucket;     // kTopK: Stage-1 (key, channel) buckets per histogram bin
-  int32_t* sel_mask;       // kTopK: 1/0 per channel (debug)
+  int32_t* sel_mask;       // kTopK / kThreshold: 1/0 per channel (debug)
+  float tau_s;             // kThreshold: channels with score >= tau_s
   int mode, select_only;
   int k;
   int d, F, P, slots, max_rec;
@@ -113,13 +114,21 @@ __global__ void __launch_bounds__(S2_THREADS, 1) stage2_kernel(Stage2Args a) {
   const int k = a.mode == kDense ? a.F : a.k;
   const int cta = blockIdx.x;
   int t0 = 0, n = 0;
-  if (a.mode == kTopK) {
-    // This CTA's channels are [c0, c1); those past the exact cut are its records.
+  if (a.mode == kTopK || a.mode == kThreshold) {
+    // This CTA's channels are [c0, c1); those past the cut are its records.
+    // Top-k: the exact cut of the token; threshold (Prox §4.1): score >= tau_s,
+    // i.e. key >= bits(tau_s) with every tie kept.
     const int c0 = (int)(((long long)a.F * cta) / a.P);
     const int c1 = (int)(((long long)a.F * (cta + 1)) / a.P);
     SelectScratch& sc = *reinterpret_cast<SelectScratch*>(ring);
     const uint32_t key0 = c0 + tid < c1 ? __float_as_uint(__ldcg(a.scores + c0 + tid)) : 0u;
-    const TopkCut cut = select_cut_cta(a.scores, a.hist, a.bucket, a.F, a.k, sc);
+    TopkCut cut;
+    if (a.mode == kTopK) {
+      cut = select_cut_cta(a.scores, a.hist, a.bucket, a.F, a.k, sc);
+    } else {
+      cut.T = __float_as_uint(a.tau_s);
+      cut.tie_cut = a.F;
+    }
     for (int b = c0; b < c1; b += S2_THREADS) {
       const int e = b + tid;
       const uint32_t key =
@@ -131,7 +140,10 @@ __global__ void __launch_bounds__(S2_THREADS, 1) stage2_kernel(Stage2Args a) {
       if (a.sel_mask && e < c1) a.sel_mask[e] = sel ? 1 : 0;
       n += total;
     }
-    if (cta == 0 && tid == 0 && a.stats) atomicAdd(a.stats + 1, 1ull);
+    if (tid == 0 && a.stats && !a.select_only) {
+      if (cta == 0) atomicAdd(a.stats + 1, 1ull);
+      atomicAdd(a.stats + 2, (unsigned long long)n);
+    }
     __syncthreads();
   } else if (a.mode == kGivenList) {
     // Entries of the list whose channel lies in [c0, c1), in list order -- the
@@ -439,6 +451,7 @@ cudaError_t launch_stage2(const prox_layer* L, const float* x, const Stage2Launc
   a.stats = L->ws.stats;
   a.bucket = L->ws.bucket;
   a.sel_mask = m.sel_mask;
+  a.tau_s = m.tau_s;
   a.mode = m.mode;
   a.select_only = m.select_only ? 1 : 0;
   a.k = m.k;

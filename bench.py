@@ -404,6 +404,30 @@ def run_ours(args, dist):
             L.set_k(k)
         result["sweep"] = sorted(sweep, key=lambda r: r["s2_percent"])
 
+        # ---- the paper's Stage-2 threshold rule (Prox §4.1, App. A.7) --------------
+        # tau_s = the s2-quantile of the calibration tokens' proxy scores; the
+        # channel count then varies per token.
+        ncal = min(64, lay.x_cal.shape[0])
+        cal_scores = torch.cat([layers[0].proxy_scores(x_cal[i:i + 1]) for i in range(ncal)])
+        tau_s = prox.calibrate_thresholds(cal_scores, args.s2 / 100.0)
+        del cal_scores
+        for L in layers:
+            L.set_mask(prox.MASK_THRESHOLD, tau_s)
+            L.stats()
+        tstep, tgraph = make_step(prox_fn)
+        tms, _ = timed(tstep, dsteps, 2)
+        del tgraph
+        sel = [L.stats(with_selected=True) for L in layers]
+        ntk = max(1, sum(r[1] for r in sel))
+        k_hat = sum(r[2] for r in sel) / ntk
+        for L in layers:
+            L.set_mask(prox.MASK_TOPK)
+        ttok = dist.world * n_tok * dsteps / (tms / 1e3)
+        result["threshold_rule"] = {
+            "tau_s": tau_s, "calibration_tokens": ncal, "mean_channels": round(k_hat, 1),
+            "realised_s2": round(1 - k_hat / f, 4), "tokens_per_s": round(ttok, 1),
+            "speedup_vs_dense": round(ttok / dense_tok_s, 3)}
+
         # ---- end to end through the host-buffer entry point ----------------------
         xh = [torch.from_numpy(np.ascontiguousarray(lay.x_eval[c::n_copies])).pin_memory()
               for c in range(n_copies)]

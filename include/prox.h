@@ -70,7 +70,15 @@ typedef struct prox_layer_info {
   size_t weight_bytes;    /* bf16 gate/up records + bf16 W_down             */
   size_t proxy_bytes;     /* INT4 codes + fp16 scales                        */
   size_t workspace_bytes; /* scratch owned by the handle                     */
+  int mask_mode;          /* PROX_MASK_TOPK or PROX_MASK_THRESHOLD           */
+  float tau_s;            /* Stage-2 score threshold (threshold mode)        */
 } prox_layer_info;
+
+/* Stage-2 channel rule: per-token top-k (Prox App. A.6), or the fixed
+ * layer-wise score threshold m_s = 1[|s~_j| >= tau_s] of Prox §4.1 (a
+ * token-adaptive channel count). */
+#define PROX_MASK_TOPK 0
+#define PROX_MASK_THRESHOLD 1
 
 /* ------------------------------------------------------------------------
  * Offline preparation
@@ -141,16 +149,22 @@ PROX_API prox_status prox_layer_destroy(prox_layer* layer);
 PROX_API prox_status prox_layer_set_tau(prox_layer* layer, float tau_x);
 PROX_API prox_status prox_layer_set_k(prox_layer* layer, int k);
 
+/* Chooses the Stage-2 rule: PROX_MASK_TOPK (uses k) or PROX_MASK_THRESHOLD
+ * (uses tau_s, a finite value >= 0; Prox §4.1).  Host only. */
+PROX_API prox_status prox_layer_set_mask(prox_layer* layer, int mode, float tau_s);
+
 PROX_API prox_status prox_layer_get_info(const prox_layer* layer, prox_layer_info* info_host);
 
 /* Reads (and clears) the layer's device error word; synchronises `stream`. */
 PROX_API prox_status prox_layer_error(prox_layer* layer, int32_t* word_host, void* stream);
 
-/* Realised Stage-1 statistics accumulated since the last call: the sum of
- * n_x over tokens and the number of tokens (realised s1 = 1 - sum/(tokens*d)),
- * Prox App. A.7 "Runtime sparsity".  Synchronises `stream` and resets. */
+/* Realised statistics accumulated since the last call (Prox App. A.7
+ * "Runtime sparsity"): the sum of n_x over tokens, the number of tokens and
+ * the sum of selected Stage-2 channels (realised s1 = 1 - sum_nx/(tokens*d),
+ * s2 = 1 - sum_sel/(tokens*d_ff)).  Any output may be NULL.  Synchronises
+ * `stream` and resets. */
 PROX_API prox_status prox_layer_stats(prox_layer* layer, int64_t* sum_nx_host, int64_t* tokens_host,
-                             void* stream);
+                             int64_t* sum_sel_host, void* stream);
 
 /* ------------------------------------------------------------------------
  * The decode step
@@ -196,6 +210,20 @@ PROX_API prox_status prox_ffn_forward_profiled(const prox_layer* layer, const fl
  * pre-activations; idx_s: int32 [k], ascending.  Any output may be NULL. */
 PROX_API prox_status prox_debug_stage1(prox_layer* layer, const float* x, int32_t* idx_x, int32_t* n_x,
                               float* g_tilde, float* u_tilde, int32_t* idx_s, void* stream);
+
+/* Proxy scores |SiLU(g~) u~| (Prox §4.1, Stage 1) of B tokens x [B, d_model]
+ * into scores [B, d_ff] (fp32, device), with the layer's tau_x.  The input to
+ * calibrating tau_s (Prox App. A.7, Algorithm 1: the s2-quantile of these
+ * scores over the calibration tokens, e.g. with prox_calibrate_thresholds).
+ * Stream-ordered; B <= max_batch. */
+PROX_API prox_status prox_layer_proxy_scores(const prox_layer* layer, const float* x, int B,
+                                             float* scores, void* stream);
+
+/* Test tap: the Stage-2 channels one token selects under the layer's current
+ * rule, ascending, into idx_s [d_ff] (device) and their number into n_s (one
+ * int32 on the device).  Same kernels as the forward step. */
+PROX_API prox_status prox_debug_mask(const prox_layer* layer, const float* x, int32_t* idx_s,
+                                     int32_t* n_s, void* stream);
 
 /* Stage 2 of one token on a caller-given channel list idx_s (int32 [k], any
  * order, entries in [0, d_ff)); s_sp (fp32 [k], may be NULL) receives

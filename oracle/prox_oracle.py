@@ -229,6 +229,18 @@ def threshold_channels(scores, tau_s):
     return np.nonzero(np.asarray(scores, dtype=F64) >= F64(tau_s))[0].astype(np.int64)
 
 
+def calibrate_tau_s(x_cal, tau_x, q_gate, s_gate, q_up, s_up, s2, group=GROUP):
+    """Stage-2 score threshold (Prox App. A.7, Algorithm 1, steps 5-6): with the
+    layer's input threshold fixed, the proxy scores |s~| of every calibration
+    token, and their s2-quantile (the same exact lower order statistic as the
+    input threshold, over the scores held as fp32)."""
+    rows = []
+    for x in np.asarray(x_cal):
+        _, g_t, u_t, _ = proxy_intermediate(x, tau_x, q_gate, s_gate, q_up, s_up, group)
+        rows.append(proxy_scores(g_t, u_t))
+    return calibrate_tau(np.asarray(rows, dtype=np.float32), s2)
+
+
 # ---------------------------------------------------------------------------
 # Stage 2: exact computation of the selected channels (Prox §4.1)
 # ---------------------------------------------------------------------------
@@ -293,27 +305,34 @@ def stack_next_input(y, eps=1e-6):
     return np.asarray(rmsnorm(y, eps), dtype=np.float32)
 
 
-def calibrate_stack(layers, x_cal, s1, k, group=GROUP, eps=1e-6):
-    """Sequential threshold calibration (Prox App. A.7, Algorithm 1) with the
-    top-k Stage-2 rule: layer l's threshold is the s1-quantile of its own
-    inputs, which are the calibration tokens run through layers 1..l-1 with
-    their finalised thresholds (the current layer's inputs are collected before
-    its own rule is fixed).
+def calibrate_stack(layers, x_cal, s1, k, group=GROUP, eps=1e-6, s2=None):
+    """Sequential threshold calibration (Prox App. A.7, Algorithm 1): layer l's
+    input threshold is the s1-quantile of its own inputs, which are the
+    calibration tokens run through layers 1..l-1 with their finalised rules
+    (the current layer's inputs are collected before its own rule is fixed).
+    With ``s2`` given, the layer's Stage-2 rule is the score threshold tau_s,
+    the s2-quantile of its proxy scores (steps 5-6); otherwise it is top-k.
 
     ``layers``: sequence of (w_gate, w_up, w_down, q_gate, s_gate, q_up, s_up).
-    Returns (taus, inputs): the threshold of every layer and the calibration
-    inputs each layer saw (n_cal x d_model fp32 arrays).
+    Returns (taus, inputs) -- or (taus, taus_s, inputs) with ``s2`` -- the
+    thresholds of every layer and the calibration inputs each layer saw.
     """
     x = np.asarray(x_cal, dtype=np.float32)
-    taus, inputs = [], []
+    taus, taus_s, inputs = [], [], []
     for li, (wg, wu, wd, qg, sg, qu, su) in enumerate(layers):
         inputs.append(x)
         tau = calibrate_tau(x, s1)
         taus.append(tau)
+        tau_s = None
+        if s2 is not None:
+            tau_s = calibrate_tau_s(x, tau, qg, sg, qu, su, s2, group)
+            taus_s.append(tau_s)
         if li + 1 < len(layers):
-            ys = [prox_ffn(xt, wg, wu, wd, qg, sg, qu, su, tau=tau, k=k, group=group)["y"]
-                  for xt in x]
+            ys = [prox_ffn(xt, wg, wu, wd, qg, sg, qu, su, tau=tau, k=k, group=group,
+                           tau_s=tau_s)["y"] for xt in x]
             x = np.stack([stack_next_input(yt, eps) for yt in ys])
+    if s2 is not None:
+        return taus, taus_s, inputs
     return taus, inputs
 
 

@@ -456,3 +456,42 @@ def test_stack_every_layer_keeps_the_target_fraction_of_its_own_inputs():
         assert np.count_nonzero(a < tau) <= r < np.count_nonzero(a <= tau)
     # later layers see the earlier sparse layers' outputs, not the raw tokens
     assert not np.array_equal(inputs[1], inputs[0])
+
+
+# ---------------------------------------------------------------------------
+# the Stage-2 score threshold (Prox §4.1 mask, App. A.7 calibration)
+# ---------------------------------------------------------------------------
+
+def test_threshold_rule_keeps_ties_at_tau():
+    s = np.array([0.5, 0.25, 0.5, 0.75, 0.0])
+    np.testing.assert_array_equal(orc.threshold_channels(s, 0.5), [0, 2, 3])
+    np.testing.assert_array_equal(orc.threshold_channels(s, 0.0), [0, 1, 2, 3, 4])
+    assert orc.threshold_channels(s, 0.8).size == 0
+
+
+def test_tau_s_is_the_order_statistic_of_the_calibration_scores():
+    lay = synth.make_layer("tiny", n_tokens=1, n_cal=16)
+    qg, sg = orc.quantize_proxy(lay.w_gate)
+    qu, su = orc.quantize_proxy(lay.w_up)
+    tau_x = orc.calibrate_tau(lay.x_cal, 0.5)
+    tau_s = orc.calibrate_tau_s(lay.x_cal, tau_x, qg, sg, qu, su, 0.7)
+    scores = []
+    for x in lay.x_cal:
+        _, g, u, _ = orc.proxy_intermediate(x, tau_x, qg, sg, qu, su)
+        scores.append(orc.proxy_scores(g, u))
+    v = np.asarray(scores, dtype=np.float32).ravel().astype(np.float64)
+    r = int(np.floor(np.float64(np.float32(0.7)) * v.size))
+    assert np.count_nonzero(v < tau_s) <= r < np.count_nonzero(v <= tau_s)
+    # the threshold rule then keeps about 30 % of the calibration channels
+    kept = np.count_nonzero(v >= tau_s) / v.size
+    assert abs(kept - 0.3) < 0.01
+
+
+def test_stack_with_threshold_rule_calibrates_both_thresholds():
+    cfg, layers, x_cal, _ = _small_stack()
+    taus, taus_s, inputs = orc.calibrate_stack(layers, x_cal, 0.5, cfg.k(), s2=0.7)
+    assert len(taus) == len(taus_s) == len(inputs) == len(layers)
+    assert all(t > 0 for t in taus_s)
+    # layer 1's thresholds depend only on the raw calibration tokens
+    wg, wu, wd, qg, sg, qu, su = layers[0]
+    assert taus_s[0] == orc.calibrate_tau_s(x_cal, taus[0], qg, sg, qu, su, 0.7)
