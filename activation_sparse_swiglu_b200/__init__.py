@@ -16,11 +16,13 @@ import ctypes
 
 import torch
 
-from ._lib import (DEVERR_MASK_INDEX, DEVERR_WAIT_TIMEOUT, MASK_THRESHOLD, MASK_TOPK, LayerInfo,
-                   ProxError, check,
-                   last_error, lib)
+from ._lib import (ACT_GELU_ERF, ACT_GELU_TANH, ACT_SILU, DEVERR_MASK_INDEX, DEVERR_WAIT_TIMEOUT,
+                   MASK_THRESHOLD, MASK_TOPK, STAGE2_EXACT, STAGE2_PROXY_VALUES, LayerInfo,
+                   ProxError, check, last_error, lib)
 
 __all__ = ["Layer", "pack_proxy", "calibrate_thresholds", "rmsnorm", "copy", "version",
+           "effective_sparsity", "allocate_sparsity", "runtime_sparsity", "ALPHA",
+           "ACT_SILU", "ACT_GELU_TANH", "ACT_GELU_ERF", "STAGE2_EXACT", "STAGE2_PROXY_VALUES",
            "ProxError", "DEVERR_MASK_INDEX", "DEVERR_WAIT_TIMEOUT", "MASK_TOPK", "MASK_THRESHOLD",
            "last_error", "lib"]
 
@@ -108,6 +110,34 @@ def copy(src: torch.Tensor, dst: torch.Tensor, stream=None) -> None:
     check(lib.prox_copy(_ptr(src), _ptr(dst), nbytes, _stream(stream)))
 
 
+ALPHA = 1.0 / 3.0  # proxy-projection cost the paper allocates with (Prox §4.2)
+
+
+def effective_sparsity(s1: float, s2: float, alpha: float = ALPHA) -> float:
+    """e = s2 - 2 alpha (1 - s1) / 3 (Prox §4.2 cost model)."""
+    e = ctypes.c_double(0.0)
+    check(lib.prox_effective_sparsity(float(s1), float(s2), float(alpha), ctypes.byref(e)))
+    return e.value
+
+
+def allocate_sparsity(e: float, alpha: float = ALPHA, s_ref: float = 0.7,
+                      s1_bounds: tuple[float, float] = (0.0, 0.7)) -> tuple[float, float]:
+    """(s1, s2) for a target effective sparsity e (Prox §4.2 allocation policy)."""
+    s1, s2 = ctypes.c_double(0.0), ctypes.c_double(0.0)
+    check(lib.prox_allocate_sparsity(float(e), float(alpha), float(s_ref), float(s1_bounds[0]),
+                                     float(s1_bounds[1]), ctypes.byref(s1), ctypes.byref(s2)))
+    return s1.value, s2.value
+
+
+def runtime_sparsity(sum_nx: int, sum_sel: int, tokens: int, d_model: int, d_ff: int,
+                     alpha: float = ALPHA) -> tuple[float, float, float]:
+    """(s1^, s2^, e^) from accumulated mask counts (Prox App. A.7)."""
+    a, b, c = ctypes.c_double(0.0), ctypes.c_double(0.0), ctypes.c_double(0.0)
+    check(lib.prox_runtime_sparsity(int(sum_nx), int(sum_sel), int(tokens), int(d_model), int(d_ff),
+                                    float(alpha), ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)))
+    return a.value, b.value, c.value
+
+
 class Layer:
     """One Prox FFN layer resident on the current CUDA device.
 
@@ -174,6 +204,14 @@ class Layer:
         """Stage-2 rule: MASK_TOPK (uses k) or MASK_THRESHOLD (score >= tau_s)."""
         check(lib.prox_layer_set_mask(self.handle, int(mode), float(tau_s)))
 
+    def set_activation(self, act: int) -> None:
+        """Gate activation: ACT_SILU (SwiGLU), ACT_GELU_TANH or ACT_GELU_ERF (GeGLU)."""
+        check(lib.prox_layer_set_activation(self.handle, int(act)))
+
+    def set_stage2(self, source: int) -> None:
+        """STAGE2_EXACT (the method) or STAGE2_PROXY_VALUES (ablation A3)."""
+        check(lib.prox_layer_set_stage2(self.handle, int(source)))
+
     def error_word(self, stream=None) -> int:
         v = ctypes.c_int32(0)
         check(lib.prox_layer_error(self.handle, ctypes.byref(v), _stream(stream)))
@@ -188,8 +226,16 @@ class Layer:
             return int(s.value), int(t.value), int(c.value)
         return int(s.value), int(t.value)
 
+    def runtime_sparsity(self, alpha: float = ALPHA, stream=None) -> dict:
+        """Realised s1^, s2^ and e^ of the tokens run since the last stats read
+        (Prox App. A.7 "Runtime sparsity"); resets the counters."""
+        s, t, c = self.stats(stream, with_selected=True)
+        inf = self.info()
+        s1, s2, e = runtime_sparsity(s, c, t, inf["d_model"], inf["d_ff"], alpha)
+        return {"tokens": t, "s1": s1, "s2": s2, "e": e}
+
     def proxy_scores(self, x: torch.Tensor, stream=None) -> torch.Tensor:
-        """Stage-1 scores |SiLU(g~) u~| of tokens x [B, d] as fp32 [B, d_ff]."""
+        """Stage-1 scores |act(g~) u~| of tokens x [B, d] as fp32 [B, d_ff]."""
         _dev(x, torch.float32, "x")
         x2 = x.reshape(-1, self.d_model)
         out = torch.empty((x2.shape[0], self.d_ff), dtype=torch.float32, device=x.device)

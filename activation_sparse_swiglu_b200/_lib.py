@@ -34,17 +34,22 @@ class LayerInfo(ctypes.Structure):
         ("weight_bytes", ctypes.c_size_t), ("proxy_bytes", ctypes.c_size_t),
         ("workspace_bytes", ctypes.c_size_t),
         ("mask_mode", ctypes.c_int), ("tau_s", ctypes.c_float),
+        ("activation", ctypes.c_int), ("stage2_source", ctypes.c_int),
     ]
 
 
 MASK_TOPK = 0
 MASK_THRESHOLD = 1
+ACT_SILU, ACT_GELU_TANH, ACT_GELU_ERF = 0, 1, 2
+STAGE2_EXACT, STAGE2_PROXY_VALUES = 0, 1
 
 
 _P = ctypes.c_void_p
 _I = ctypes.c_int
 _F = ctypes.c_float
 _S = ctypes.c_size_t
+_D = ctypes.c_double
+_L = ctypes.c_int64
 
 # name -> (restype, argtypes); the order follows include/prox.h
 SIGNATURES = {
@@ -56,10 +61,16 @@ SIGNATURES = {
     "prox_layer_set_tau": (_I, [_P, _F]),
     "prox_layer_set_k": (_I, [_P, _I]),
     "prox_layer_set_mask": (_I, [_P, _I, _F]),
+    "prox_layer_set_activation": (_I, [_P, _I]),
+    "prox_layer_set_stage2": (_I, [_P, _I]),
     "prox_layer_get_info": (_I, [_P, ctypes.POINTER(LayerInfo)]),
     "prox_layer_error": (_I, [_P, ctypes.POINTER(ctypes.c_int32), _P]),
     "prox_layer_stats": (_I, [_P, ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int64),
                               ctypes.POINTER(ctypes.c_int64), _P]),
+    "prox_effective_sparsity": (_I, [_D, _D, _D, ctypes.POINTER(_D)]),
+    "prox_allocate_sparsity": (_I, [_D, _D, _D, _D, _D, ctypes.POINTER(_D), ctypes.POINTER(_D)]),
+    "prox_runtime_sparsity": (_I, [_L, _L, _L, _I, _I, _D, ctypes.POINTER(_D), ctypes.POINTER(_D),
+                                   ctypes.POINTER(_D)]),
     "prox_ffn_forward": (_I, [_P, _P, _P, _I, _P]),
     "prox_dense_ffn": (_I, [_P, _P, _P, _I, _P]),
     "prox_ffn_forward_host": (_I, [_P, _P, _P, _I, _P]),

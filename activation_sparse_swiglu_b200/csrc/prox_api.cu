@@ -99,6 +99,7 @@ prox_status alloc_workspace(prox_layer* L) {
     return o;
   };
   const size_t o_scores = take(F * 4);
+  const size_t o_st = take(F * 4);
   const size_t o_g = take(F * 4);
   const size_t o_u = take(F * 4);
   const size_t o_hist = take(prox::kScoreBins * 4);
@@ -120,6 +121,7 @@ prox_status alloc_workspace(prox_layer* L) {
   w.base = base;
   w.bytes = off;
   w.scores = reinterpret_cast<float*>(b + o_scores);
+  w.s_tilde = reinterpret_cast<float*>(b + o_st);
   w.g_dbg = reinterpret_cast<float*>(b + o_g);
   w.u_dbg = reinterpret_cast<float*>(b + o_u);
   w.hist = reinterpret_cast<uint32_t*>(b + o_hist);
@@ -143,6 +145,7 @@ prox::Stage2Launch topk_launch(const prox_layer* L) {
   m.mode = L->mask_mode == PROX_MASK_THRESHOLD ? 3 : 1;
   m.k = L->k;
   m.tau_s = L->tau_s;
+  m.proxy_values = L->stage2_source == PROX_STAGE2_PROXY_VALUES;
   return m;
 }
 
@@ -383,6 +386,22 @@ prox_status prox_layer_set_mask(prox_layer* L, int mode, float tau_s) {
   return PROX_OK;
 }
 
+prox_status prox_layer_set_activation(prox_layer* L, int act) {
+  if (!L) return fail(PROX_EINVAL, "layer handle is NULL");
+  if (act != PROX_ACT_SILU && act != PROX_ACT_GELU_TANH && act != PROX_ACT_GELU_ERF)
+    return fail(PROX_EINVAL, "activation %d is not one of PROX_ACT_*", act);
+  L->act = act;
+  return PROX_OK;
+}
+
+prox_status prox_layer_set_stage2(prox_layer* L, int source) {
+  if (!L) return fail(PROX_EINVAL, "layer handle is NULL");
+  if (source != PROX_STAGE2_EXACT && source != PROX_STAGE2_PROXY_VALUES)
+    return fail(PROX_EINVAL, "Stage-2 source %d is not one of PROX_STAGE2_*", source);
+  L->stage2_source = source;
+  return PROX_OK;
+}
+
 prox_status prox_layer_get_info(const prox_layer* L, prox_layer_info* info) {
   if (!L || !info) return fail(PROX_EINVAL, "NULL argument");
   info->d_model = L->d;
@@ -400,6 +419,8 @@ prox_status prox_layer_get_info(const prox_layer* L, prox_layer_info* info) {
   info->workspace_bytes = L->ws.bytes;
   info->mask_mode = L->mask_mode;
   info->tau_s = L->tau_s;
+  info->activation = L->act;
+  info->stage2_source = L->stage2_source;
   return PROX_OK;
 }
 
@@ -428,6 +449,57 @@ prox_status prox_layer_stats(prox_layer* L, int64_t* sum_nx_host, int64_t* token
   if (sum_nx_host) *sum_nx_host = (int64_t)v[0];
   if (tokens_host) *tokens_host = (int64_t)v[1];
   if (sum_sel_host) *sum_sel_host = (int64_t)v[2];
+  return PROX_OK;
+}
+
+// ---- cost model (Prox §4.2) and runtime sparsity (Prox App. A.7) ------------
+
+prox_status prox_effective_sparsity(double s1, double s2, double alpha, double* e_host) {
+  if (!e_host) return fail(PROX_EINVAL, "e_host is NULL");
+  if (!(s1 >= 0.0 && s1 <= 1.0) || !(s2 >= 0.0 && s2 <= 1.0))
+    return fail(PROX_EINVAL, "s1=%g and s2=%g must lie in [0, 1]", s1, s2);
+  if (!(alpha >= 0.0) || std::isinf(alpha)) return fail(PROX_EINVAL, "alpha=%g must be finite and >= 0", alpha);
+  *e_host = s2 - 2.0 * alpha * (1.0 - s1) / 3.0;
+  return PROX_OK;
+}
+
+prox_status prox_allocate_sparsity(double e, double alpha, double s_ref, double s1_min,
+                                   double s1_max, double* s1_host, double* s2_host) {
+  if (!s1_host || !s2_host) return fail(PROX_EINVAL, "NULL output pointer");
+  if (!std::isfinite(e)) return fail(PROX_EINVAL, "e must be finite");
+  if (!(alpha > 0.0) || std::isinf(alpha)) return fail(PROX_EINVAL, "alpha=%g must be finite and > 0", alpha);
+  if (!(s_ref >= 0.0 && s_ref <= 1.0)) return fail(PROX_EINVAL, "s_ref=%g must lie in [0, 1]", s_ref);
+  if (!(s1_min >= 0.0 && s1_min <= s1_max && s1_max <= 1.0))
+    return fail(PROX_EINVAL, "need 0 <= s1_min (%g) <= s1_max (%g) <= 1", s1_min, s1_max);
+  // s2 = s_ref first; e = s2 - 2 alpha (1 - s1) / 3 then fixes s1.
+  double s1 = 1.0 - 3.0 * (s_ref - e) / (2.0 * alpha);
+  double s2 = s_ref;
+  if (s1 < s1_min || s1 > s1_max) {
+    s1 = s1 < s1_min ? s1_min : s1_max;
+    s2 = e + 2.0 * alpha * (1.0 - s1) / 3.0;
+    if (!(s2 >= 0.0 && s2 <= 1.0))
+      return fail(PROX_EINVAL, "target e=%g is out of reach: s1 clamped to %g needs s2=%g", e, s1, s2);
+  }
+  *s1_host = s1;
+  *s2_host = s2;
+  return PROX_OK;
+}
+
+prox_status prox_runtime_sparsity(int64_t sum_nx, int64_t sum_sel, int64_t tokens, int d_model,
+                                  int d_ff, double alpha, double* s1_host, double* s2_host,
+                                  double* e_host) {
+  if (tokens < 1 || d_model < 1 || d_ff < 1)
+    return fail(PROX_EINVAL, "tokens, d_model and d_ff must be >= 1");
+  if (tokens > INT64_MAX / (d_model > d_ff ? d_model : d_ff))
+    return fail(PROX_EINVAL, "tokens=%lld too large", (long long)tokens);
+  if (sum_nx < 0 || sum_nx > tokens * d_model || sum_sel < 0 || sum_sel > tokens * d_ff)
+    return fail(PROX_EINVAL, "counts outside [0, tokens * width]");
+  if (!(alpha >= 0.0) || std::isinf(alpha)) return fail(PROX_EINVAL, "alpha=%g must be finite and >= 0", alpha);
+  const double s1 = 1.0 - (double)sum_nx / ((double)tokens * d_model);
+  const double s2 = 1.0 - (double)sum_sel / ((double)tokens * d_ff);
+  if (s1_host) *s1_host = s1;
+  if (s2_host) *s2_host = s2;
+  if (e_host) *e_host = s2 - 2.0 * alpha * (1.0 - s1) / 3.0;
   return PROX_OK;
 }
 

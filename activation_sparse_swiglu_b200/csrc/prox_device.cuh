@@ -137,6 +137,21 @@ __device__ __forceinline__ float2 bf16x2_to_f2(uint32_t w) {
 // SiLU(z) = z / (1 + e^{-z}) in fp32.
 __device__ __forceinline__ float silu_f32(float z) { return z / (1.0f + expf(-z)); }
 
+// Gate activations of the GLU: SiLU (SwiGLU, Prox §2.1) or GELU (GeGLU, the
+// FFN family Prox §5 also sparsifies), the latter either as z Phi(z) or in the
+// tanh form of Hendrycks & Gimpel, "Gaussian Error Linear Units", §2:
+//   0.5 z (1 + tanh(sqrt(2/pi) (z + 0.044715 z^3))).
+// `act` is uniform across the grid (a kernel argument), so the branch costs
+// nothing.  Values follow PROX_ACT_* of prox.h.
+__device__ __forceinline__ float act_f32(float z, int act) {
+  if (act == 1) {
+    const float c = 0.7978845608028654f;  // sqrt(2/pi)
+    return 0.5f * z * (1.0f + tanhf(c * fmaf(0.044715f * z, z * z, z)));
+  }
+  if (act == 2) return 0.5f * z * erfcf(-z * 0.7071067811865476f);  // z Phi(z)
+  return silu_f32(z);
+}
+
 // ---- block-wide scans (blockDim.x a multiple of 32, at most 1024) ---------------
 // Exclusive prefix sum of `v` over the threads of the block in thread order.
 // `scratch` needs 33 words of shared memory.  Returns the block total in *total.

@@ -30,7 +30,8 @@ constexpr int kHostChunkTokens = 64; // staging chunk of prox_ffn_forward_host
 
 // Per-token scratch of one layer (device memory owned by the handle).
 struct Workspace {
-  float* scores = nullptr;        // |SiLU(g~) u~| [F]
+  float* scores = nullptr;        // |act(g~) u~| [F]
+  float* s_tilde = nullptr;       // act(g~) u~ [F], signed (proxy-values Stage 2 only)
   float* g_dbg = nullptr;         // debug g~ [F]
   float* u_dbg = nullptr;         // debug u~ [F]
   uint32_t* hist = nullptr;       // [kScoreBins] score bits 30..18, zero between tokens
@@ -55,6 +56,8 @@ struct prox_layer {
   float tau = 0.f;
   int mask_mode = 0;     // PROX_MASK_TOPK or PROX_MASK_THRESHOLD
   float tau_s = 0.f;     // Stage-2 score threshold (threshold mode)
+  int act = 0;           // PROX_ACT_*: gate activation of the GLU
+  int stage2_source = 0; // PROX_STAGE2_EXACT or PROX_STAGE2_PROXY_VALUES
   int device = 0, num_sms = 0;
   // Stage-1 geometry: C column slices, P1 CTAs, at most s1_lmax rows per CTA
   int C = 0, P1 = 0, s1_lmax = 0;
@@ -77,6 +80,7 @@ struct Stage1Taps {
   float* u = nullptr;       // u~ [F]
   int32_t* idx_x = nullptr; // kept input rows, ascending [d]
   int32_t* n_x = nullptr;   // their number
+  float* s_tilde = nullptr; // signed proxy values act(g~) u~ [F]
 };
 // How Stage 2 obtains its channels.
 struct Stage2Launch {
@@ -85,7 +89,8 @@ struct Stage2Launch {
   const int32_t* idx = nullptr;
   int k = 0;
   int32_t* sel_mask = nullptr;  // top-k: 1/0 per channel written here (debug)
-  float* s_sp = nullptr;       // optional SiLU(g) u per listed channel
+  float* s_sp = nullptr;       // optional act(g) u per listed channel
+  bool proxy_values = false;   // ablation: s~ of Stage 1 instead of the exact s
   bool select_only = false;    // top-k: stop after selecting
 };
 

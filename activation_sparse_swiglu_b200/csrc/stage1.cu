@@ -61,6 +61,8 @@ struct Stage1Args {
   int32_t* n_x;     // optional: their number
   float* part;      // [gridDim.x][2][S1_PART] partial sums per CTA and touched slice
   int* cnt;         // [C] row slices reported per slice; zero between tokens
+  float* s_tilde;   // optional: signed proxy values act(g~) u~ [F]
+  int act;          // gate activation (PROX_ACT_*)
   Magic mg;
 };
 
@@ -156,8 +158,10 @@ __device__ void finish_slice(const Stage1Args& a, int c, int n_x, int P, int* s_
       u += v[q].y;
     }
   }
-  const float sc = fabsf(silu_f32(g) * u);
+  const float sv = act_f32(g, a.act) * u;
+  const float sc = fabsf(sv);
   a.scores[ch] = sc;
+  if (a.s_tilde) a.s_tilde[ch] = sv;
   if (a.g_dbg) a.g_dbg[ch] = g;
   if (a.u_dbg) a.u_dbg[ch] = u;
   const uint32_t key = __float_as_uint(sc), bin = key >> kScoreShift;
@@ -459,6 +463,9 @@ cudaError_t launch_stage1(const prox_layer* L, const float* x, const Stage1Taps&
   a.n_x = taps.n_x;
   a.part = L->ws.s1_part;
   a.cnt = L->ws.s1_cnt;
+  a.s_tilde = taps.s_tilde ? taps.s_tilde
+                           : (L->stage2_source == PROX_STAGE2_PROXY_VALUES ? L->ws.s_tilde : nullptr);
+  a.act = L->act;
   a.mg = Magic{0x4B000000u, 0x49000000u, 0x47000000u, 0x45000000u, 0x43000000u};
 
   cudaLaunchConfig_t cfg = {};

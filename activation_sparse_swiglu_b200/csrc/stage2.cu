@@ -56,6 +56,9 @@ struct Stage2Args {
   int groups;  // consumer groups NG (= producer lanes); slots is a multiple of it
   float* ypart;
   float* s_sp;
+  const float* s_tilde;  // proxy_values: Stage-1 act(g~) u~ [F]
+  int proxy_values;      // ablation: skip the gate/up records, use s~ as s
+  int act;               // gate activation (PROX_ACT_*)
   int* err;
   int x_ready;
 };
@@ -197,7 +200,7 @@ __global__ void __launch_bounds__(S2_THREADS, 1) stage2_kernel(Stage2Args a) {
     if (lane < NG) {
       const int g = lane;
       const uint64_t pol = l2_policy_evict_first();
-      const int nA_g = group_items(g, n), nB_g = group_items(g, nB);
+      const int nA_g = a.proxy_values ? 0 : group_items(g, n), nB_g = group_items(g, nB);
       const int tot_g = nA_g + nB_g;
       for (int li = 0; li < tot_g; ++li) {
         const int slot = g * SPG + li % SPG, use = li / SPG;
@@ -230,7 +233,7 @@ __global__ void __launch_bounds__(S2_THREADS, 1) stage2_kernel(Stage2Args a) {
   // ---------------- phase A: gate/up partial dot products ----------------
   // The warp's share of an item goes into registers, the slot goes back to the
   // producer, then the FMAs.
-  const int nA_g = group_items(grp, n);
+  const int nA_g = a.proxy_values ? 0 : group_items(grp, n);
   for (int li = 0; li < nA_g; ++li) {
     const int r = grp + li * NG;
     const int slot = grp * SPG + li % SPG;
@@ -273,12 +276,17 @@ __global__ void __launch_bounds__(S2_THREADS, 1) stage2_kernel(Stage2Args a) {
   }
   asm volatile("bar.sync 1, %0;" ::"r"(NCW * 32) : "memory");
   for (int r = tid; r < n; r += NCW * 32) {
-    float g = 0.f, u = 0.f;
-    for (int w = 0; w < WPG; ++w) {
-      g += s_pg[r * NCW + w];
-      u += s_pu[r * NCW + w];
+    float sv;
+    if (a.proxy_values) {
+      sv = __ldcg(a.s_tilde + s_idx[r]);
+    } else {
+      float g = 0.f, u = 0.f;
+      for (int w = 0; w < WPG; ++w) {
+        g += s_pg[r * NCW + w];
+        u += s_pu[r * NCW + w];
+      }
+      sv = act_f32(g, a.act) * u;
     }
-    const float sv = silu_f32(g) * u;
     s_val[r] = sv;
     if (a.s_sp) a.s_sp[a.mode == kGivenList ? s_lpos[r] : t0 + r] = sv;
   }
@@ -463,6 +471,9 @@ cudaError_t launch_stage2(const prox_layer* L, const float* x, const Stage2Launc
   a.max_rec = (L->F + L->P - 1) / L->P + 1;
   a.ypart = L->ws.ypart;
   a.s_sp = m.s_sp;
+  a.s_tilde = L->ws.s_tilde;
+  a.proxy_values = m.proxy_values ? 1 : 0;
+  a.act = L->act;
   a.err = L->ws.err;
   a.x_ready = x_ready ? 1 : 0;
 

@@ -423,10 +423,91 @@ def run_ours(args, dist):
         for L in layers:
             L.set_mask(prox.MASK_TOPK)
         ttok = dist.world * n_tok * dsteps / (tms / 1e3)
+        r_s1, r_s2, r_e = prox.runtime_sparsity(sum(r[0] for r in sel), sum(r[2] for r in sel),
+                                                ntk, d, f)
         result["threshold_rule"] = {
             "tau_s": tau_s, "calibration_tokens": ncal, "mean_channels": round(k_hat, 1),
-            "realised_s2": round(1 - k_hat / f, 4), "tokens_per_s": round(ttok, 1),
+            "realised_s1": round(r_s1, 4), "realised_s2": round(r_s2, 4),
+            "realised_e": round(r_e, 4), "tokens_per_s": round(ttok, 1),
             "speedup_vs_dense": round(ttok / dense_tok_s, 3)}
+
+        # ---- variants: GeGLU gate (Prox §5) and ablation A3 (Prox §5.2) ------------
+        variants = {}
+        for vname, setup in (("geglu_tanh", lambda L: L.set_activation(prox.ACT_GELU_TANH)),
+                             ("geglu_erf", lambda L: L.set_activation(prox.ACT_GELU_ERF)),
+                             ("a3_proxy_values", lambda L: L.set_stage2(prox.STAGE2_PROXY_VALUES))):
+            for L in layers:
+                setup(L)
+            vstep, vgraph = make_step(prox_fn)
+            vms, _ = timed(vstep, dsteps, 2)
+            del vgraph
+            for L in layers:
+                L.set_activation(prox.ACT_SILU)
+                L.set_stage2(prox.STAGE2_EXACT)
+            variants[vname] = round(dist.world * n_tok * dsteps / (vms / 1e3), 1)
+        result["variants_tokens_per_s"] = variants
+
+        # ---- the paper's operating points (Prox §4.2 allocation, App. A.4) -------
+        # (s1, s2) from the target e with alpha = 1/3, s_ref = 0.7, s1 in [0, 0.7];
+        # tau_x calibrated for s1, top-k with k = round((1 - s2) d_ff).
+        ops = []
+        for e_t in (0.4, 0.5, 0.6, 0.7):
+            o_s1, o_s2 = prox.allocate_sparsity(e_t)
+            o_tau = prox.calibrate_thresholds(x_cal, o_s1)
+            o_k = max(1, int(round((1.0 - o_s2) * f)))
+            for L in layers:
+                L.set_tau(o_tau)
+                L.set_k(o_k)
+                L.stats()
+            ostep, ograph = make_step(prox_fn)
+            oms, _ = timed(ostep, dsteps, 2)
+            del ograph
+            rs = [L.stats(with_selected=True) for L in layers]
+            _, _, o_e = prox.runtime_sparsity(sum(r[0] for r in rs), sum(r[2] for r in rs),
+                                              max(1, sum(r[1] for r in rs)), d, f)
+            otok = dist.world * n_tok * dsteps / (oms / 1e3)
+            ops.append({"e_target": e_t, "s1": round(o_s1, 4), "s2": round(o_s2, 4), "k": o_k,
+                        "realised_e": round(o_e, 4), "tokens_per_s": round(otok, 1),
+                        "speedup_vs_dense": round(otok / dense_tok_s, 3)})
+        for L in layers:
+            L.set_tau(tau)
+            L.set_k(k)
+        result["operating_points"] = ops
+
+        # ---- alpha on B200 (Prox App. A.3): Stage 1 vs a bf16 GEMV over the same
+        # kept input rows.  Stage 1 runs both proxy projections, so
+        # alpha = t_stage1 / (2 t_gemv); the GEMV is cuBLAS (torch.matmul).
+        n_x = max(1, int(round(mean_nx)))
+        slice_bytes = 2 * n_x * f
+        n_win = max(2, math.ceil(2 * l2 / slice_bytes) + 1)
+        w_src = bf16_dev(lay.w_gate_bits)
+        wins = [w_src[:n_x].clone() for _ in range(n_win)]
+        del w_src
+        xs = torch.randn(1, n_x, device="cuda").to(torch.bfloat16)
+        ys = torch.empty(1, f, device="cuda", dtype=torch.bfloat16)
+        with torch.cuda.stream(stream):
+            for i in range(3 * n_win):
+                torch.matmul(xs, wins[i % n_win], out=ys)
+            g0 = torch.cuda.Event(enable_timing=True)
+            g1 = torch.cuda.Event(enable_timing=True)
+            reps = 20 * n_win
+            g0.record(stream)
+            for i in range(reps):
+                torch.matmul(xs, wins[i % n_win], out=ys)
+            g1.record(stream)
+        g1.synchronize()
+        gemv_us = g0.elapsed_time(g1) * 1e3 / reps
+        del wins, xs, ys
+        t1_us = result["kernel_us"]["stage1"]
+        proxy_bytes = n_x * f // 2 + 2 * f * g  # one projection: codes of the kept rows + scales
+        result["alpha"] = {
+            "n_x": n_x, "stage1_us": t1_us, "bf16_gemv_us": round(gemv_us, 2),
+            "alpha_time": round(t1_us / (2 * gemv_us), 4),
+            "alpha_bytes": round(proxy_bytes / (2 * n_x * f), 4),
+            "bf16_gemv_gbs": round(slice_bytes / (gemv_us * 1e-6) / 1e9, 1),
+            "note": ("Stage 1 (both INT4 proxies + scores) over 2 x one cuBLAS bf16 GEMV "
+                     f"[1 x {n_x}] @ [{n_x} x {f}] of the same kept rows, "
+                     f"{n_win} rotating weight windows (> L2)")}
 
         # ---- end to end through the host-buffer entry point ----------------------
         xh = [torch.from_numpy(np.ascontiguousarray(lay.x_eval[c::n_copies])).pin_memory()

@@ -72,6 +72,8 @@ typedef struct prox_layer_info {
   size_t workspace_bytes; /* scratch owned by the handle                     */
   int mask_mode;          /* PROX_MASK_TOPK or PROX_MASK_THRESHOLD           */
   float tau_s;            /* Stage-2 score threshold (threshold mode)        */
+  int activation;         /* PROX_ACT_*                                      */
+  int stage2_source;      /* PROX_STAGE2_EXACT or PROX_STAGE2_PROXY_VALUES   */
 } prox_layer_info;
 
 /* Stage-2 channel rule: per-token top-k (Prox App. A.6), or the fixed
@@ -79,6 +81,24 @@ typedef struct prox_layer_info {
  * token-adaptive channel count). */
 #define PROX_MASK_TOPK 0
 #define PROX_MASK_THRESHOLD 1
+
+/* Gate activation of the GLU, used by the Stage-1 score, Stage 2 and the
+ * dense baseline alike.  SwiGLU (Prox §2.1) is the default; Prox §5 applies
+ * the method unchanged to GeGLU FFNs, whose gate is GELU, here either
+ * GELU(z) = z Phi(z) (Phi the standard normal CDF) or its tanh form
+ * 0.5 z (1 + tanh(sqrt(2/pi) (z + 0.044715 z^3))) (Hendrycks & Gimpel,
+ * "Gaussian Error Linear Units", §2). */
+#define PROX_ACT_SILU 0
+#define PROX_ACT_GELU_TANH 1
+#define PROX_ACT_GELU_ERF 2
+
+/* Where Stage 2 takes the selected channels' values from.  EXACT is the
+ * method (Prox §4.1).  PROXY_VALUES is ablation A3 of Prox §5.2: Stage 2
+ * skips the exact gate/up projections and feeds the selected Stage-1 proxy
+ * values s~_j = act(g~_j) u~_j straight into the down projection,
+ * y = sum_{j in S} s~_j W_down[j, :]. */
+#define PROX_STAGE2_EXACT 0
+#define PROX_STAGE2_PROXY_VALUES 1
 
 /* ------------------------------------------------------------------------
  * Offline preparation
@@ -153,6 +173,15 @@ PROX_API prox_status prox_layer_set_k(prox_layer* layer, int k);
  * (uses tau_s, a finite value >= 0; Prox §4.1).  Host only. */
 PROX_API prox_status prox_layer_set_mask(prox_layer* layer, int mode, float tau_s);
 
+/* Chooses the gate activation (PROX_ACT_*; else PROX_EINVAL).  Host only;
+ * takes effect from the next enqueued call. */
+PROX_API prox_status prox_layer_set_activation(prox_layer* layer, int act);
+
+/* Chooses the Stage-2 value source of prox_ffn_forward and
+ * prox_ffn_forward_host (PROX_STAGE2_*; else PROX_EINVAL).  Host only.
+ * prox_forward_with_mask and prox_dense_ffn always compute exact values. */
+PROX_API prox_status prox_layer_set_stage2(prox_layer* layer, int source);
+
 PROX_API prox_status prox_layer_get_info(const prox_layer* layer, prox_layer_info* info_host);
 
 /* Reads (and clears) the layer's device error word; synchronises `stream`. */
@@ -167,22 +196,62 @@ PROX_API prox_status prox_layer_stats(prox_layer* layer, int64_t* sum_nx_host, i
                              int64_t* sum_sel_host, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Cost model and sparsity allocation (host only: no device work, no stream)
+ * ------------------------------------------------------------------------ */
+
+/* Effective FFN sparsity of a (s1, s2) pair under the normalised cost model
+ * of Prox §4.2: the dense gate, up and down projections cost one unit each
+ * (C_Dense = 3); Stage 1 runs two INT4 proxy projections over the kept
+ * (1 - s1) share of the inputs at alpha units each, Stage 2 three exact
+ * projections over the kept (1 - s2) share of the channels:
+ *   C_Prox = 2 alpha (1 - s1) + 3 (1 - s2),  e = 1 - C_Prox / 3
+ *          = s2 - 2 alpha (1 - s1) / 3.
+ * s1, s2 in [0, 1] and alpha >= 0 (finite), else PROX_EINVAL. */
+PROX_API prox_status prox_effective_sparsity(double s1, double s2, double alpha, double* e_host);
+
+/* The allocation policy of Prox §4.2 (operating points in App. A.4): for a
+ * target effective sparsity e, set s2 = s_ref and solve the relation above
+ * for s1; if that s1 lies outside [s1_min, s1_max], clamp it to the nearer
+ * bound and re-solve s2 = e + 2 alpha (1 - s1) / 3.  The paper's setting is
+ * alpha = 1/3, s_ref = 0.7, [s1_min, s1_max] = [0, 0.7].
+ * PROX_EINVAL when alpha <= 0, s_ref is outside [0, 1], the bounds are not
+ * 0 <= s1_min <= s1_max <= 1, any argument is not finite, or the re-solved
+ * s2 leaves [0, 1] (no allocation within the bounds reaches e). */
+PROX_API prox_status prox_allocate_sparsity(double e, double alpha, double s_ref, double s1_min,
+                                            double s1_max, double* s1_host, double* s2_host);
+
+/* Runtime sparsity from accumulated mask counts (Prox App. A.7, "Runtime
+ * sparsity"), with the counts prox_layer_stats returns:
+ *   s1^ = 1 - sum_nx / (tokens d_model),  s2^ = 1 - sum_sel / (tokens d_ff),
+ *   e^  = s2^ - 2 alpha (1 - s1^) / 3.
+ * tokens >= 1, 0 <= sum_nx <= tokens d_model, 0 <= sum_sel <= tokens d_ff,
+ * d_model, d_ff >= 1, alpha >= 0 (finite), else PROX_EINVAL.  Any output may
+ * be NULL. */
+PROX_API prox_status prox_runtime_sparsity(int64_t sum_nx, int64_t sum_sel, int64_t tokens,
+                                           int d_model, int d_ff, double alpha, double* s1_host,
+                                           double* s2_host, double* e_host);
+
+/* ------------------------------------------------------------------------
  * The decode step
  * ------------------------------------------------------------------------ */
 
-/* Prox two-stage sparse FFN (Prox §4.1), B tokens each with its own masks:
+/* Prox two-stage sparse FFN (Prox §4.1), B tokens each with its own masks;
+ * act is the layer's gate activation (SiLU unless prox_layer_set_activation
+ * chose GELU):
  *   Stage 1: m_x = 1[|x_i| >= tau_x]; g~ = Π_in(x, W~_gate, m_x),
- *            u~ = Π_in(x, W~_up, m_x); score_j = |SiLU(g~_j) u~_j|;
+ *            u~ = Π_in(x, W~_up, m_x); score_j = |act(g~_j) u~_j|;
  *            idx_s = the k channels of largest score, ties to the lower
- *            index (Prox App. A.6, per-token top-k), ascending.
- *   Stage 2: for j in idx_s: s_j = SiLU(x W_gate[:, j]) (x W_up[:, j]) with the
- *            full x; out = sum_j s_j W_down[j, :].
+ *            index (Prox App. A.6, per-token top-k), ascending; or, in
+ *            threshold mode, every channel with score_j >= tau_s.
+ *   Stage 2: for j in idx_s: s_j = act(x W_gate[:, j]) (x W_up[:, j]) with the
+ *            full x (or s~_j in PROX_STAGE2_PROXY_VALUES mode);
+ *            out = sum_j s_j W_down[j, :].
  * x, out: fp32 [B, d_model] (out may not alias x).  B <= max_batch.
  * Three kernels per token, chained with programmatic dependent launch. */
 PROX_API prox_status prox_ffn_forward(const prox_layer* layer, const float* x, float* out, int B,
                              void* stream);
 
-/* Dense SwiGLU baseline FFN(x) = (x W_up ⊙ SiLU(x W_gate)) W_down (Prox §2.1),
+/* Dense GLU baseline FFN(x) = (x W_up ⊙ act(x W_gate)) W_down (Prox §2.1),
  * on the same bf16 buffers (Stage 2 with every channel kept). */
 PROX_API prox_status prox_dense_ffn(const prox_layer* layer, const float* x, float* out, int B,
                            void* stream);
@@ -211,7 +280,7 @@ PROX_API prox_status prox_ffn_forward_profiled(const prox_layer* layer, const fl
 PROX_API prox_status prox_debug_stage1(prox_layer* layer, const float* x, int32_t* idx_x, int32_t* n_x,
                               float* g_tilde, float* u_tilde, int32_t* idx_s, void* stream);
 
-/* Proxy scores |SiLU(g~) u~| (Prox §4.1, Stage 1) of B tokens x [B, d_model]
+/* Proxy scores |act(g~) u~| (Prox §4.1, Stage 1) of B tokens x [B, d_model]
  * into scores [B, d_ff] (fp32, device), with the layer's tau_x.  The input to
  * calibrating tau_s (Prox App. A.7, Algorithm 1: the s2-quantile of these
  * scores over the calibration tokens, e.g. with prox_calibrate_thresholds).
@@ -227,7 +296,7 @@ PROX_API prox_status prox_debug_mask(const prox_layer* layer, const float* x, in
 
 /* Stage 2 of one token on a caller-given channel list idx_s (int32 [k], any
  * order, entries in [0, d_ff)); s_sp (fp32 [k], may be NULL) receives
- * SiLU(g) u for each listed channel. */
+ * act(g) u for each listed channel.  Always the exact Stage 2. */
 PROX_API prox_status prox_forward_with_mask(prox_layer* layer, const float* x, const int32_t* idx_s,
                                    int k, float* out, float* s_sp, void* stream);
 

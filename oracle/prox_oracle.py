@@ -31,6 +31,8 @@ Readings taken where the paper is silent or differs from the workload spec
 
 from __future__ import annotations
 
+import math
+
 import numpy as np
 
 F64 = np.float64
@@ -49,22 +51,43 @@ def silu(z):
         return z / (1.0 + np.exp(-z))
 
 
-def dense_ffn(x, w_gate, w_up, w_down):
-    """FFN(x) = (x W_up ⊙ SiLU(x W_gate)) W_down  (Prox §2.1, FFN equation).
+def gelu(z):
+    """GELU(z) = z Phi(z), Phi the standard normal CDF (Hendrycks & Gimpel,
+    "Gaussian Error Linear Units", §2); the gate of a GeGLU FFN, the family
+    Prox §5 sparsifies besides SwiGLU."""
+    z = np.asarray(z, dtype=F64)
+    # Phi(z) = erfc(-z / sqrt 2) / 2, which keeps its relative accuracy for z << 0
+    return z * 0.5 * np.vectorize(math.erfc, otypes=[F64])(-z / math.sqrt(2.0))
+
+
+def gelu_tanh(z):
+    """The tanh form of GELU from the same paper:
+    0.5 z (1 + tanh(sqrt(2/pi) (z + 0.044715 z^3)))."""
+    z = np.asarray(z, dtype=F64)
+    return 0.5 * z * (1.0 + np.tanh(math.sqrt(2.0 / math.pi) * (z + 0.044715 * z ** 3)))
+
+
+# gate activations by name; the library's PROX_ACT_* codes are 0, 1, 2 in this order
+ACTIVATIONS = {"silu": silu, "gelu_tanh": gelu_tanh, "gelu": gelu}
+
+
+def dense_ffn(x, w_gate, w_up, w_down, act="silu"):
+    """FFN(x) = (x W_up ⊙ SiLU(x W_gate)) W_down  (Prox §2.1, FFN equation);
+    ``act`` swaps the gate activation (GeGLU with "gelu" / "gelu_tanh").
 
     x: [d_model]; W_gate, W_up: [d_model, d_ff]; W_down: [d_ff, d_model].
     """
     x = np.asarray(x, dtype=F64)
     u = x @ np.asarray(w_up, dtype=F64)
-    h = silu(x @ np.asarray(w_gate, dtype=F64))
+    h = ACTIVATIONS[act](x @ np.asarray(w_gate, dtype=F64))
     s = u * h
     return s @ np.asarray(w_down, dtype=F64)
 
 
-def intermediate_state(x, w_gate, w_up):
+def intermediate_state(x, w_gate, w_up, act="silu"):
     """s = u ⊙ h with u = x W_up, h = SiLU(x W_gate)  (Prox §2.1)."""
     x = np.asarray(x, dtype=F64)
-    return (x @ np.asarray(w_up, dtype=F64)) * silu(x @ np.asarray(w_gate, dtype=F64))
+    return (x @ np.asarray(w_up, dtype=F64)) * ACTIVATIONS[act](x @ np.asarray(w_gate, dtype=F64))
 
 
 # ---------------------------------------------------------------------------
@@ -188,7 +211,7 @@ def input_mask(x, tau):
     return np.nonzero(np.abs(x) >= np.float32(tau))[0].astype(np.int64)
 
 
-def proxy_intermediate(x, tau, q_gate, s_gate, q_up, s_up, group=GROUP):
+def proxy_intermediate(x, tau, q_gate, s_gate, q_up, s_up, group=GROUP, act="silu"):
     """Stage-1 proxy (Prox §4.1):
     u~ = Π_in(x, W~_up, m_x),  h~ = SiLU(Π_in(x, W~_gate, m_x)),  s~ = u~ ⊙ h~.
 
@@ -201,13 +224,13 @@ def proxy_intermediate(x, tau, q_gate, s_gate, q_up, s_up, group=GROUP):
     wu = dequantize_proxy(q_up, s_up, group, rows=idx_x)
     g_t = x64[idx_x] @ wg
     u_t = x64[idx_x] @ wu
-    s_t = u_t * silu(g_t)
+    s_t = u_t * ACTIVATIONS[act](g_t)
     return idx_x, g_t, u_t, s_t
 
 
-def proxy_scores(g_tilde, u_tilde):
+def proxy_scores(g_tilde, u_tilde, act="silu"):
     """Channel salience |s~_j| = |SiLU(g~_j) u~_j|  (Prox §4.1)."""
-    return np.abs(silu(g_tilde) * np.asarray(u_tilde, dtype=F64))
+    return np.abs(ACTIVATIONS[act](g_tilde) * np.asarray(u_tilde, dtype=F64))
 
 
 def topk_channels(scores, k):
@@ -229,15 +252,15 @@ def threshold_channels(scores, tau_s):
     return np.nonzero(np.asarray(scores, dtype=F64) >= F64(tau_s))[0].astype(np.int64)
 
 
-def calibrate_tau_s(x_cal, tau_x, q_gate, s_gate, q_up, s_up, s2, group=GROUP):
+def calibrate_tau_s(x_cal, tau_x, q_gate, s_gate, q_up, s_up, s2, group=GROUP, act="silu"):
     """Stage-2 score threshold (Prox App. A.7, Algorithm 1, steps 5-6): with the
     layer's input threshold fixed, the proxy scores |s~| of every calibration
     token, and their s2-quantile (the same exact lower order statistic as the
     input threshold, over the scores held as fp32)."""
     rows = []
     for x in np.asarray(x_cal):
-        _, g_t, u_t, _ = proxy_intermediate(x, tau_x, q_gate, s_gate, q_up, s_up, group)
-        rows.append(proxy_scores(g_t, u_t))
+        _, g_t, u_t, _ = proxy_intermediate(x, tau_x, q_gate, s_gate, q_up, s_up, group, act)
+        rows.append(proxy_scores(g_t, u_t, act))
     return calibrate_tau(np.asarray(rows, dtype=np.float32), s2)
 
 
@@ -245,7 +268,7 @@ def calibrate_tau_s(x_cal, tau_x, q_gate, s_gate, q_up, s_up, s2, group=GROUP):
 # Stage 2: exact computation of the selected channels (Prox §4.1)
 # ---------------------------------------------------------------------------
 
-def stage2(x, w_gate, w_up, w_down, idx_s):
+def stage2(x, w_gate, w_up, w_down, idx_s, act="silu"):
     """Stage 2 (Prox §4.1):
     u_sp = Π_out(x, W_up, m_s), h_sp = SiLU(Π_out(x, W_gate, m_s)),
     s_sp = u_sp ⊙ h_sp,  y = Π_in(s_sp, W_down, m_s)  with the full x.
@@ -254,10 +277,19 @@ def stage2(x, w_gate, w_up, w_down, idx_s):
     """
     idx_s = np.asarray(idx_s, dtype=np.int64)
     u_sp = pi_out(x, w_up, idx_s)
-    h_sp = silu(pi_out(x, w_gate, idx_s))
+    h_sp = ACTIVATIONS[act](pi_out(x, w_gate, idx_s))
     s_sp = u_sp * h_sp
     y = s_sp @ np.asarray(w_down)[idx_s, :].astype(F64)
     return y, s_sp
+
+
+def stage2_proxy_values(w_down, idx_s, s_tilde):
+    """Ablation A3 of Prox §5.2: no exact recomputation; the selected proxy
+    values s~_j go straight into the down projection,
+    y = Π_in(s~, W_down, m_s) = sum_{j in idx_s} s~_j W_down[j, :]."""
+    idx_s = np.asarray(idx_s, dtype=np.int64)
+    s_sel = np.asarray(s_tilde, dtype=F64)[idx_s]
+    return s_sel @ np.asarray(w_down)[idx_s, :].astype(F64)
 
 
 def oracle_s_mask(x, w_gate, w_up, k):
@@ -271,18 +303,23 @@ def oracle_s_mask(x, w_gate, w_up, k):
 # ---------------------------------------------------------------------------
 
 def prox_ffn(x, w_gate, w_up, w_down, q_gate, s_gate, q_up, s_up, tau, k,
-             group=GROUP, tau_s=None):
+             group=GROUP, tau_s=None, act="silu", proxy_values=False):
     """One token through both stages (Prox §4.1, with the top-k mask of App. A.6
-    unless ``tau_s`` selects the §4.1 threshold rule).  Returns a dict with
-    idx_x, g_tilde, u_tilde, scores, idx_s, s_sp and y."""
-    idx_x, g_t, u_t, _ = proxy_intermediate(x, tau, q_gate, s_gate, q_up, s_up, group)
-    scores = proxy_scores(g_t, u_t)
+    unless ``tau_s`` selects the §4.1 threshold rule; ``act`` the gate
+    activation; ``proxy_values`` the A3 ablation of §5.2 in place of Stage 2).
+    Returns a dict with idx_x, g_tilde, u_tilde, s_tilde, scores, idx_s, s_sp
+    (None under A3) and y."""
+    idx_x, g_t, u_t, s_t = proxy_intermediate(x, tau, q_gate, s_gate, q_up, s_up, group, act)
+    scores = proxy_scores(g_t, u_t, act)
     if tau_s is None:
         idx_s = topk_channels(scores, k)
     else:
         idx_s = threshold_channels(scores, tau_s)
-    y, s_sp = stage2(x, w_gate, w_up, w_down, idx_s)
-    return dict(idx_x=idx_x, g_tilde=g_t, u_tilde=u_t, scores=scores,
+    if proxy_values:
+        y, s_sp = stage2_proxy_values(w_down, idx_s, s_t), None
+    else:
+        y, s_sp = stage2(x, w_gate, w_up, w_down, idx_s, act)
+    return dict(idx_x=idx_x, g_tilde=g_t, u_tilde=u_t, s_tilde=s_t, scores=scores,
                 idx_s=idx_s, s_sp=s_sp, y=y)
 
 
@@ -348,3 +385,55 @@ def stack_forward(layers, taus, x, k, group=GROUP, eps=1e-6):
         if li + 1 < len(layers):
             x = stack_next_input(y, eps)
     return xs, y
+
+
+# ---------------------------------------------------------------------------
+# Cost model, allocation policy and runtime sparsity (Prox §4.2, App. A.4, A.7)
+# ---------------------------------------------------------------------------
+
+C_DENSE = 3.0  # gate, up and down projections at one unit each (Prox §4.2)
+
+
+def prox_cost(s1, s2, alpha):
+    """Normalised Prox FFN cost (Prox §4.2): two INT4 proxy projections of
+    relative cost alpha over the kept (1 - s1) inputs plus three exact
+    projections over the kept (1 - s2) channels."""
+    return 2.0 * F64(alpha) * (1.0 - F64(s1)) + 3.0 * (1.0 - F64(s2))
+
+
+def effective_sparsity(s1, s2, alpha):
+    """e = 1 - C_Prox / C_Dense  (Prox §4.2)."""
+    return 1.0 - prox_cost(s1, s2, alpha) / C_DENSE
+
+
+def allocate_sparsity(e, alpha=1.0 / 3.0, s_ref=0.7, s1_min=0.0, s1_max=0.7):
+    """Allocation policy of Prox §4.2 (operating points of App. A.4).
+
+    Keep Stage 2 at the anchor s_ref and give Stage 1 whatever input sparsity
+    makes the cost meet the budget C_Prox = C_Dense (1 - e); when that s1 is
+    outside [s1_min, s1_max], pin s1 to the nearer bound and let s2 take up
+    the budget instead.  Raises ValueError when no s2 in [0, 1] does.
+    """
+    e, alpha = F64(e), F64(alpha)
+    if not alpha > 0:
+        raise ValueError("alpha must be > 0")
+    budget = C_DENSE * (1.0 - e)
+    # Stage-1 share of the budget with s2 = s_ref: 2 alpha (1 - s1) = budget - 3 (1 - s_ref)
+    s1 = 1.0 - (budget - 3.0 * (1.0 - F64(s_ref))) / (2.0 * alpha)
+    if s1_min <= s1 <= s1_max:
+        return float(s1), float(s_ref)
+    s1 = F64(s1_min) if s1 < s1_min else F64(s1_max)
+    # remaining budget for Stage 2: 3 (1 - s2) = budget - 2 alpha (1 - s1)
+    s2 = 1.0 - (budget - 2.0 * alpha * (1.0 - s1)) / 3.0
+    if not 0.0 <= s2 <= 1.0:
+        raise ValueError(f"target e={float(e)} is out of reach with s1={float(s1)}")
+    return float(s1), float(s2)
+
+
+def runtime_sparsity(sum_nx, sum_sel, tokens, d_model, d_ff, alpha=1.0 / 3.0):
+    """Realised (s1^, s2^, e^) from accumulated mask counts (Prox App. A.7,
+    "Runtime sparsity"): the kept fractions of inputs and channels over all
+    tokens, then the cost model of §4.2."""
+    s1 = 1.0 - F64(sum_nx) / (F64(tokens) * d_model)
+    s2 = 1.0 - F64(sum_sel) / (F64(tokens) * d_ff)
+    return float(s1), float(s2), float(effective_sparsity(s1, s2, alpha))

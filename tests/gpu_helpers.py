@@ -39,10 +39,11 @@ class OracleLayer:
         self.qg, self.sg = orc.quantize_proxy(lay.w_gate)
         self.qu, self.su = orc.quantize_proxy(lay.w_up)
 
-    def step(self, x, tau, k):
+    def step(self, x, tau, k, **kw):
+        """prox_ffn of the oracle; kw: tau_s, act, proxy_values."""
         lay = self.lay
         return orc.prox_ffn(x, lay.w_gate, lay.w_up, lay.w_down, self.qg, self.sg, self.qu,
-                            self.su, tau=tau, k=k)
+                            self.su, tau=tau, k=k, **kw)
 
     def stage1(self, x, tau):
         return orc.proxy_intermediate(x, tau, self.qg, self.sg, self.qu, self.su)

@@ -5,6 +5,7 @@ import ctypes
 import os
 import re
 
+import numpy as np
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -77,3 +78,40 @@ def test_host_side_argument_checks(plib):
     assert lib.prox_layer_destroy(None) == plib.PROX_OK
     # copy: size must be a multiple of 16
     assert lib.prox_copy(p, p, 20, None) == plib.PROX_EINVAL
+
+
+def test_cost_model_host_functions_match_the_oracle(plib):
+    """The library's host-only cost model (Prox §4.2, App. A.7) against the
+    oracle's restatement, and its argument checks."""
+    from oracle import prox_oracle as orc
+    lib = plib.lib
+    D = ctypes.c_double
+    a, b, c = D(), D(), D()
+    for alpha in (1.0 / 3.0, 0.285, 0.5):
+        for e in np.linspace(0.0, 0.9, 37):
+            try:
+                want = orc.allocate_sparsity(e, alpha)
+            except ValueError:
+                assert lib.prox_allocate_sparsity(e, alpha, 0.7, 0.0, 0.7, ctypes.byref(a),
+                                                  ctypes.byref(b)) == plib.PROX_EINVAL
+                continue
+            assert lib.prox_allocate_sparsity(e, alpha, 0.7, 0.0, 0.7, ctypes.byref(a),
+                                              ctypes.byref(b)) == plib.PROX_OK
+            assert a.value == pytest.approx(want[0], abs=1e-12)
+            assert b.value == pytest.approx(want[1], abs=1e-12)
+            assert lib.prox_effective_sparsity(a.value, b.value, alpha, ctypes.byref(c)) == plib.PROX_OK
+            assert c.value == pytest.approx(orc.effective_sparsity(a.value, b.value, alpha), abs=1e-12)
+    assert lib.prox_runtime_sparsity(1000, 300, 4, 512, 1024, 1.0 / 3.0, ctypes.byref(a),
+                                     ctypes.byref(b), ctypes.byref(c)) == plib.PROX_OK
+    want = orc.runtime_sparsity(1000, 300, 4, 512, 1024)
+    assert (a.value, b.value, c.value) == pytest.approx(want, abs=1e-15)
+    # bad arguments
+    assert lib.prox_allocate_sparsity(0.5, 0.0, 0.7, 0.0, 0.7, ctypes.byref(a), ctypes.byref(b)) == plib.PROX_EINVAL
+    assert lib.prox_allocate_sparsity(0.5, 1 / 3, 0.7, 0.5, 0.2, ctypes.byref(a), ctypes.byref(b)) == plib.PROX_EINVAL
+    assert lib.prox_allocate_sparsity(float("nan"), 1 / 3, 0.7, 0.0, 0.7, ctypes.byref(a),
+                                      ctypes.byref(b)) == plib.PROX_EINVAL
+    assert lib.prox_allocate_sparsity(0.99, 1 / 3, 0.7, 0.0, 0.7, ctypes.byref(a), ctypes.byref(b)) == plib.PROX_EINVAL
+    assert "out of reach" in plib.last_error()
+    assert lib.prox_effective_sparsity(1.2, 0.5, 1 / 3, ctypes.byref(c)) == plib.PROX_EINVAL
+    assert lib.prox_runtime_sparsity(5000, 0, 4, 512, 1024, 1 / 3, None, None, None) == plib.PROX_EINVAL
+    assert lib.prox_runtime_sparsity(0, 0, 0, 512, 1024, 1 / 3, None, None, None) == plib.PROX_EINVAL

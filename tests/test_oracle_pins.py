@@ -495,3 +495,187 @@ def test_stack_with_threshold_rule_calibrates_both_thresholds():
     # layer 1's thresholds depend only on the raw calibration tokens
     wg, wu, wd, qg, sg, qu, su = layers[0]
     assert taus_s[0] == orc.calibrate_tau_s(x_cal, taus[0], qg, sg, qu, su, 0.7)
+
+
+# ---------------------------------------------------------------------------
+# Cost model and allocation policy (§4.2, App. A.4, App. A.7)
+# ---------------------------------------------------------------------------
+
+def _allocation_table():
+    rows = []
+    with open(os.path.join(GOLDEN, "allocation_appendix_a4.txt")) as fh:
+        for line in fh:
+            line = line.split("#", 1)[0].strip()
+            if line:
+                e, s1, s2, clamp = line.split()
+                rows.append((float(e) / 100, None if s1 == "-" else float(s1) / 100,
+                             float(s2) / 100, clamp))
+    return rows
+
+
+def test_allocation_matches_the_printed_operating_points():
+    rows = _allocation_table()
+    assert len(rows) == 4
+    for e, s1_p, s2_p, clamp in rows:
+        s1, s2 = orc.allocate_sparsity(e)
+        assert abs(s2 - s2_p) <= 5e-4 + 1e-12, (e, s2, s2_p)  # printed to 0.1 %
+        if s1_p is not None:
+            assert abs(s1 - s1_p) <= 5e-4 + 1e-12, (e, s1, s1_p)
+        if clamp == "no":
+            assert 0.0 < s1 < 0.7 and s2 == 0.7
+        else:
+            assert s1 == (0.0 if clamp == "low" else 0.7)
+
+
+def test_cost_model_special_cases():
+    a = 1.0 / 3.0
+    # nothing skipped and no proxy: the dense cost, e = 0
+    assert orc.prox_cost(1.0, 0.0, a) == orc.C_DENSE
+    assert orc.effective_sparsity(1.0, 0.0, a) == 0.0
+    # every input dropped: the proxy is free and e is the Stage-2 sparsity
+    for s2 in (0.0, 0.3, 0.7, 1.0):
+        assert orc.effective_sparsity(1.0, s2, a) == pytest.approx(s2, abs=1e-15)
+    # keep every input and every channel: the proxy's two projections come on top
+    assert orc.effective_sparsity(0.0, 0.0, a) == pytest.approx(-2.0 / 9.0, abs=1e-15)
+    # each term on its own: one unit per dense projection, alpha per proxy projection
+    assert orc.prox_cost(0.0, 1.0, 0.25) == pytest.approx(0.5, abs=1e-15)
+    assert orc.prox_cost(1.0, 2.0 / 3.0, 0.25) == pytest.approx(1.0, abs=1e-15)
+
+
+def test_allocation_meets_the_budget_and_respects_the_bounds():
+    a = 1.0 / 3.0
+    for e in np.linspace(0.0, 0.9, 91):
+        s1, s2 = orc.allocate_sparsity(e)
+        assert 0.0 <= s1 <= 0.7 and 0.0 <= s2 <= 1.0
+        assert orc.effective_sparsity(s1, s2, a) == pytest.approx(e, abs=1e-12)
+        # s2 is the anchor unless s1 sits on a bound
+        assert s2 == 0.7 or s1 in (0.0, 0.7)
+    # the switch points: with s2 = 0.7, s1 = 0 at e = 0.7 - 2a/3 and s1 = 0.7 at e = 0.7 - 0.6a/3
+    lo = 0.7 - 2 * a / 3
+    hi = 0.7 - 2 * a * 0.3 / 3
+    assert orc.allocate_sparsity(lo) == pytest.approx((0.0, 0.7), abs=1e-12)
+    assert orc.allocate_sparsity(hi) == pytest.approx((0.7, 0.7), abs=1e-12)
+    # monotone: a larger target never lowers either sparsity
+    prev = (-1.0, -1.0)
+    for e in np.linspace(0.0, 0.9, 181):
+        cur = orc.allocate_sparsity(e)
+        assert cur[0] >= prev[0] - 1e-12 and cur[1] >= prev[1] - 1e-12
+        prev = cur
+    # out of reach: s2 would have to exceed 1
+    with pytest.raises(ValueError):
+        orc.allocate_sparsity(0.99)
+    with pytest.raises(ValueError):
+        orc.allocate_sparsity(-0.5)
+
+
+def test_runtime_sparsity_from_counted_masks():
+    rng = np.random.default_rng(7)
+    d, f, t = 256, 640, 37
+    mx = rng.random((t, d)) < 0.45
+    ms = rng.random((t, f)) < 0.28
+    s1, s2, e = orc.runtime_sparsity(int(mx.sum()), int(ms.sum()), t, d, f)
+    assert s1 == pytest.approx(np.mean(~mx), abs=1e-15)
+    assert s2 == pytest.approx(np.mean(~ms), abs=1e-15)
+    # e^ with the realised pair equals the budget identity of §4.2
+    assert e == pytest.approx(1.0 - orc.prox_cost(s1, s2, 1.0 / 3.0) / 3.0, abs=1e-15)
+
+
+# ---------------------------------------------------------------------------
+# GeGLU gate (§5: Gemma-3's GeGLU FFN) and the A3 ablation (§5.2)
+# ---------------------------------------------------------------------------
+
+def test_gelu_is_z_times_the_normal_cdf():
+    z = np.linspace(-12, 12, 2401)
+    np.testing.assert_allclose(orc.gelu(z), z * stats.norm.cdf(z), rtol=1e-13, atol=1e-300)
+    # textbook values: Phi(0) = 1/2, Phi(1) = 0.8413447460685429
+    assert orc.gelu(0.0) == 0.0
+    assert orc.gelu(1.0) == pytest.approx(0.8413447460685429, rel=1e-15)
+    assert orc.gelu(-1.0) == pytest.approx(-(1 - 0.8413447460685429), rel=1e-14)
+
+
+@pytest.mark.parametrize("act", ["gelu", "gelu_tanh", "silu"])
+def test_gate_activation_symmetry(act):
+    # z Phi(z) - (-z) Phi(-z) = z, and the same holds for the tanh form (tanh is
+    # odd) and for SiLU (the logistic function has the same symmetry)
+    f = orc.ACTIVATIONS[act]
+    z = np.linspace(-9, 9, 1801)
+    np.testing.assert_allclose(f(z) - f(-z), z, rtol=1e-13, atol=1e-13)
+
+
+def test_gelu_tanh_form_tracks_the_exact_gelu():
+    z = np.linspace(-8, 8, 16001)
+    err = np.abs(orc.gelu_tanh(z) - orc.gelu(z))
+    assert err.max() < 5e-4  # the tanh form's known accuracy, a few 1e-4
+    assert err.max() > 1e-5  # ... and it is an approximation, not a copy
+    # derivative 1/2 at 0 for both: (f(h) - f(-h)) / 2h -> 1/2 ... and f(h)/h -> 1/2
+    h = 1e-6
+    assert orc.gelu_tanh(h) / h == pytest.approx(0.5, abs=1e-6)
+
+
+def test_geglu_ffn_with_permutation_weights_is_elementwise():
+    rng = np.random.default_rng(1)
+    n = 9
+    x = rng.standard_normal(n)
+    p1, p2, p3 = (rng.permutation(n) for _ in range(3))
+    c = -0.8
+    w_up = np.zeros((n, n)); w_up[p1, np.arange(n)] = 1.0
+    w_gate = np.zeros((n, n)); w_gate[p2, np.arange(n)] = c
+    w_down = np.zeros((n, n)); w_down[np.arange(n), p3] = 1.0
+    for act in ("gelu", "gelu_tanh"):
+        y = orc.dense_ffn(x, w_gate, w_up, w_down, act=act)
+        expect = np.zeros(n)
+        for j in range(n):
+            z = c * x[p2[j]]
+            g = z * stats.norm.cdf(z) if act == "gelu" else \
+                0.5 * z * (1 + np.tanh(np.sqrt(2 / np.pi) * (z + 0.044715 * z ** 3)))
+            expect[p3[j]] = x[p1[j]] * g
+        np.testing.assert_allclose(y, expect, rtol=1e-12, atol=1e-15)
+
+
+@pytest.mark.parametrize("act", ["gelu", "gelu_tanh"])
+def test_geglu_keep_all_equals_dense(act):
+    lay = synth.make_layer(_small_cfg(256, 96), n_tokens=2)
+    qg, sg, qu, su = _packed(lay)
+    for x in lay.x_eval:
+        r = orc.prox_ffn(x, lay.w_gate, lay.w_up, lay.w_down, qg, sg, qu, su,
+                         tau=0.0, k=lay.d_ff, act=act)
+        np.testing.assert_allclose(
+            r["y"], orc.dense_ffn(x, lay.w_gate, lay.w_up, lay.w_down, act=act),
+            rtol=1e-12, atol=1e-14)
+
+
+def test_a3_equals_exact_stage2_when_the_proxy_is_exact():
+    # Grid weights and tau = 0: the proxy values are the exact s, so the A3
+    # output is the Prox output on the same mask.
+    rng = np.random.default_rng(11)
+    d, f = 256, 64
+    wg, _, _ = _grid_weights(rng, d, f)
+    wu, _, _ = _grid_weights(rng, d, f)
+    wd = rng.standard_normal((f, d)).astype(np.float32)
+    qg, sg = orc.quantize_proxy(wg)
+    qu, su = orc.quantize_proxy(wu)
+    x = rng.laplace(0, 1, d).astype(np.float32)
+    for act in ("silu", "gelu"):
+        ex = orc.prox_ffn(x, wg, wu, wd, qg, sg, qu, su, tau=0.0, k=20, act=act)
+        a3 = orc.prox_ffn(x, wg, wu, wd, qg, sg, qu, su, tau=0.0, k=20, act=act,
+                          proxy_values=True)
+        np.testing.assert_array_equal(a3["idx_s"], ex["idx_s"])
+        assert a3["s_sp"] is None
+        np.testing.assert_allclose(a3["y"], ex["y"], rtol=1e-11, atol=1e-11)
+
+
+def test_a3_is_the_masked_sum_of_proxy_values():
+    # With an input threshold the A3 output differs from Prox and is exactly
+    # the W_down rows of the selected channels weighted by s~.
+    lay = synth.make_layer(_small_cfg(256, 96), n_tokens=1)
+    qg, sg, qu, su = _packed(lay)
+    x = lay.x_eval[0]
+    tau = orc.calibrate_tau(lay.x_cal, 0.5)
+    a3 = orc.prox_ffn(x, lay.w_gate, lay.w_up, lay.w_down, qg, sg, qu, su, tau=tau, k=30,
+                      proxy_values=True)
+    ex = orc.prox_ffn(x, lay.w_gate, lay.w_up, lay.w_down, qg, sg, qu, su, tau=tau, k=30)
+    acc = np.zeros(lay.d_model)
+    for j in a3["idx_s"]:
+        acc += a3["s_tilde"][j] * lay.w_down[j].astype(np.float64)
+    np.testing.assert_allclose(a3["y"], acc, rtol=1e-12, atol=1e-15)
+    assert np.linalg.norm(a3["y"] - ex["y"]) > 1e-3 * np.linalg.norm(ex["y"])
