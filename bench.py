@@ -476,37 +476,54 @@ def run_ours(args, dist):
 
         # ---- alpha on B200 (Prox App. A.3): Stage 1 vs a bf16 GEMV over the same
         # kept input rows.  Stage 1 runs both proxy projections, so
-        # alpha = t_stage1 / (2 t_gemv); the GEMV is cuBLAS (torch.matmul).
+        # alpha = t_stage1 / (2 t_gemv).  The GEMV is cuBLAS (torch.matmul) on the
+        # kept rows stored input-major [n_x, F] (x @ W) and output-major [F, n_x]
+        # (W^T x); the faster one is the denominator.  alpha_roofline takes a GEMV
+        # that streams its 2 n_x F bytes at the measured HBM peak instead.
         n_x = max(1, int(round(mean_nx)))
         slice_bytes = 2 * n_x * f
         n_win = max(2, math.ceil(2 * l2 / slice_bytes) + 1)
         w_src = bf16_dev(lay.w_gate_bits)
-        wins = [w_src[:n_x].clone() for _ in range(n_win)]
-        del w_src
+
+        def time_gemv(wins, fn):
+            with torch.cuda.stream(stream):
+                for i in range(3 * n_win):
+                    fn(wins[i % n_win])
+                g0 = torch.cuda.Event(enable_timing=True)
+                g1 = torch.cuda.Event(enable_timing=True)
+                reps = 20 * n_win
+                g0.record(stream)
+                for i in range(reps):
+                    fn(wins[i % n_win])
+                g1.record(stream)
+            g1.synchronize()
+            return g0.elapsed_time(g1) * 1e3 / reps
+
         xs = torch.randn(1, n_x, device="cuda").to(torch.bfloat16)
+        xcol = xs.reshape(n_x, 1).contiguous()
         ys = torch.empty(1, f, device="cuda", dtype=torch.bfloat16)
-        with torch.cuda.stream(stream):
-            for i in range(3 * n_win):
-                torch.matmul(xs, wins[i % n_win], out=ys)
-            g0 = torch.cuda.Event(enable_timing=True)
-            g1 = torch.cuda.Event(enable_timing=True)
-            reps = 20 * n_win
-            g0.record(stream)
-            for i in range(reps):
-                torch.matmul(xs, wins[i % n_win], out=ys)
-            g1.record(stream)
-        g1.synchronize()
-        gemv_us = g0.elapsed_time(g1) * 1e3 / reps
-        del wins, xs, ys
+        ycol = torch.empty(f, 1, device="cuda", dtype=torch.bfloat16)
+        wins = [w_src[:n_x].clone() for _ in range(n_win)]
+        gemv_in_us = time_gemv(wins, lambda w: torch.matmul(xs, w, out=ys))
+        del wins
+        wins = [w_src[:n_x].t().contiguous() for _ in range(n_win)]
+        gemv_out_us = time_gemv(wins, lambda w: torch.matmul(w, xcol, out=ycol))
+        del wins, w_src, xs, xcol, ys, ycol
+        gemv_us = min(gemv_in_us, gemv_out_us)
+        gemv_roof_us = slice_bytes / (peaks["hbm_gbs"] * 1e9) * 1e6
         t1_us = result["kernel_us"]["stage1"]
         proxy_bytes = n_x * f // 2 + 2 * f * g  # one projection: codes of the kept rows + scales
         result["alpha"] = {
-            "n_x": n_x, "stage1_us": t1_us, "bf16_gemv_us": round(gemv_us, 2),
+            "n_x": n_x, "stage1_us": t1_us,
+            "bf16_gemv_us": {"input_major": round(gemv_in_us, 2),
+                             "output_major": round(gemv_out_us, 2),
+                             "at_hbm_peak": round(gemv_roof_us, 2)},
             "alpha_time": round(t1_us / (2 * gemv_us), 4),
-            "alpha_bytes": round(proxy_bytes / (2 * n_x * f), 4),
+            "alpha_roofline": round(t1_us / (2 * gemv_roof_us), 4),
+            "alpha_bytes": round(proxy_bytes / slice_bytes, 4),
             "bf16_gemv_gbs": round(slice_bytes / (gemv_us * 1e-6) / 1e9, 1),
-            "note": ("Stage 1 (both INT4 proxies + scores) over 2 x one cuBLAS bf16 GEMV "
-                     f"[1 x {n_x}] @ [{n_x} x {f}] of the same kept rows, "
+            "note": ("Stage 1 (both INT4 proxies + scores, event-timed alone) over 2 x the "
+                     f"faster cuBLAS bf16 GEMV of the same {n_x} kept rows x {f} channels, "
                      f"{n_win} rotating weight windows (> L2)")}
 
         # ---- end to end through the host-buffer entry point ----------------------
