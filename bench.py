@@ -23,6 +23,7 @@ import hashlib
 import json
 import math
 import os
+import platform
 import statistics
 import subprocess
 import sys
@@ -575,6 +576,17 @@ def _oracle_threads():
         return os.cpu_count() or 1
 
 
+def _cpu_model():
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for line in fh:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return platform.processor() or "unknown"
+
+
 def cpu_baseline(lay, tau, k, seconds):
     from oracle import prox_oracle as orc
     qg, sg = orc.quantize_proxy(lay.w_gate)
@@ -588,6 +600,7 @@ def cpu_baseline(lay, tau, k, seconds):
         if (el >= seconds and n >= 2) or n >= lay.x_eval.shape[0]:
             break
     return {"value": round(n / el, 3), "unit": UNIT, "cores": _oracle_threads(), "kind": "oracle",
+            "cpu": _cpu_model(), "nproc": os.cpu_count(),
             "sample": f"{n} tokens of the same workload through the fp64 numpy oracle "
                       f"({el:.1f} s; proxy packing done once beforehand, not timed)"}
 
@@ -631,6 +644,7 @@ def run_reference(args, dist):
         "config": {"workload": cfg.workload_name(s1, args.s2), "d_model": cfg.d_model,
                    "d_ff": cfg.d_ff, "k": k, "tokens_per_step": per_step, "batch": 1},
         "cpu_baseline": {"value": round(tok_s, 3), "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "cpu": _cpu_model(), "nproc": os.cpu_count(),
                          "sample": f"{per_step} token per step of the same workload through the "
                                    f"fp64 numpy oracle"},
         "e2e": {"value": round(tok_s, 3), "unit": UNIT, "h2d_bytes_per_step": 0,
