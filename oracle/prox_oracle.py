@@ -373,15 +373,17 @@ def calibrate_stack(layers, x_cal, s1, k, group=GROUP, eps=1e-6, s2=None):
     return taus, inputs
 
 
-def stack_forward(layers, taus, x, k, group=GROUP, eps=1e-6):
-    """One token through the stack: the Prox step of every layer, RMSNorm in
-    between.  Returns the per-layer inputs and the last layer's output."""
+def stack_forward(layers, taus, x, k, group=GROUP, eps=1e-6, taus_s=None):
+    """One token through the stack: the Prox step of every layer (top-k, or
+    the score threshold taus_s[l] when given), RMSNorm in between.  Returns
+    the per-layer inputs and the last layer's output."""
     xs = []
     x = np.asarray(x, dtype=np.float32)
     y = None
     for li, ((wg, wu, wd, qg, sg, qu, su), tau) in enumerate(zip(layers, taus)):
         xs.append(x)
-        y = prox_ffn(x, wg, wu, wd, qg, sg, qu, su, tau=tau, k=k, group=group)["y"]
+        tau_s = None if taus_s is None else taus_s[li]
+        y = prox_ffn(x, wg, wu, wd, qg, sg, qu, su, tau=tau, k=k, group=group, tau_s=tau_s)["y"]
         if li + 1 < len(layers):
             x = stack_next_input(y, eps)
     return xs, y

@@ -140,3 +140,57 @@ def test_stack_of_eight_small_layers(prox):
 def test_stack32_first_two_layers_full_size(prox):
     # the 32-layer workload's own seeds and shapes, first two layers
     _stack_case(prox, synth.get_config("stack32"), n_layers=2, n_cal=16, n_tok=1)
+
+
+def test_stack_threshold_rule_small(prox):
+    """Algorithm 1 with both thresholds: every layer's tau_x and then tau_s are
+    fixed on the inputs that layer receives from the finalised layers before
+    it.  Teacher-forced on the oracle's per-layer inputs the GPU's tau_x is
+    bit-exact and its tau_s (from its own proxy scores) within the score
+    tolerance; the free-running calibration tracks the oracle's."""
+    from activation_sparse_swiglu_b200.stack import Stack
+    cfg = synth.WorkloadConfig(name="stack_small", index=63, d_model=512, d_ff=1376, sigma=0.02,
+                               outlier_frac=0.01, outlier_scale=20.0, s1_percent=(50,),
+                               s2_percent=(70,), n_tokens=2, n_cal=32, n_layers=4)
+    lays = [synth.make_layer(cfg, li, draw_tokens=(li == 0), n_cal=32, n_tokens=2)
+            for li in range(4)]
+    x_cal, x_eval = lays[0].x_cal, lays[0].x_eval
+    olays = [OracleLayer(lay) for lay in lays]
+    layers = [(l.w_gate, l.w_up, l.w_down, o.qg, o.sg, o.qu, o.su) for l, o in zip(lays, olays)]
+    k = cfg.k()
+    taus, taus_s, cal_inputs = orc.calibrate_stack(layers, x_cal, 0.5, k, s2=0.7)
+    weights = [(bits_to_bf16(l.w_gate_bits), bits_to_bf16(l.w_up_bits), bits_to_bf16(l.w_down_bits))
+               for l in lays]
+    stack = Stack(weights, k, max_batch=32)
+    del weights
+    g_taus, g_taus_s, _ = stack.calibrate(torch.from_numpy(x_cal).cuda(), 0.5, s2=0.7)
+    for gt, ot in zip(g_taus, taus):
+        assert abs(gt - ot) <= 1e-4 * ot, (gt, ot)
+    for gt, ot in zip(g_taus_s, taus_s):
+        assert abs(gt - ot) <= 5e-3 * ot, (gt, ot)
+    for li, layer in enumerate(stack.layers):
+        assert layer.info()["mask_mode"] == prox.MASK_THRESHOLD
+        xin = torch.from_numpy(cal_inputs[li]).cuda()
+        assert np.float32(prox.calibrate_thresholds(xin, 0.5)) == taus[li]
+        layer.set_tau(taus[li])
+        tau_s_g = prox.calibrate_thresholds(layer.proxy_scores(xin), 0.7)
+        assert abs(tau_s_g - taus_s[li]) <= 1e-3 * taus_s[li]
+        layer.set_mask(prox.MASK_THRESHOLD, float(taus_s[li]))
+    # teacher-forced forward under the threshold rule
+    for t in range(2):
+        xs, y_ref = orc.stack_forward(layers, taus, x_eval[t], k, taus_s=taus_s)
+        for li, (layer, olay) in enumerate(zip(stack.layers, olays)):
+            ref = olay.step(xs[li], taus[li], k, tau_s=taus_s[li])
+            xd = torch.from_numpy(np.ascontiguousarray(xs[li], dtype=np.float32)).cuda()
+            gpu_idx = layer.debug_mask(xd).cpu().numpy().astype(np.int64)
+            diff = np.setxor1d(gpu_idx, ref["idx_s"])
+            assert np.all(np.abs(ref["scores"][diff] - taus_s[li]) <= 1e-3 * taus_s[li])
+            lay = lays[li]
+            want, _ = orc.stage2(xs[li], lay.w_gate, lay.w_up, lay.w_down, gpu_idx)
+            y_g = layer.forward(xd)
+            torch.cuda.synchronize()
+            assert rel_l2(y_g.cpu().numpy().reshape(-1), want) <= OUT_RTOL
+    for layer in stack.layers:
+        assert layer.error_word() == 0
+    stack.close()
+

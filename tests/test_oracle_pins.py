@@ -445,6 +445,17 @@ def test_stack_keep_all_is_the_dense_chain():
     np.testing.assert_allclose(y, h, rtol=1e-12, atol=1e-12)
 
 
+def test_stack_threshold_rule_keep_all_is_the_dense_chain():
+    # s1 = 0 and s2 = 0: every tau and tau_s is 0, the score threshold keeps
+    # every channel (scores are >= 0), and the stack is the dense chain
+    cfg, layers, x_cal, x_eval = _small_stack()
+    taus, taus_s, _ = orc.calibrate_stack(layers, x_cal, 0.0, 1, s2=0.0)
+    assert taus == [0.0] * len(layers) and taus_s == [0.0] * len(layers)
+    _, y = orc.stack_forward(layers, taus, x_eval[1], 1, taus_s=taus_s)
+    _, y_dense = orc.stack_forward(layers, taus, x_eval[1], cfg.d_ff)
+    np.testing.assert_allclose(y, y_dense, rtol=1e-12, atol=1e-12)
+
+
 def test_stack_every_layer_keeps_the_target_fraction_of_its_own_inputs():
     cfg, layers, x_cal, _ = _small_stack()
     taus, inputs = orc.calibrate_stack(layers, x_cal, 0.5, cfg.k())
