@@ -27,6 +27,14 @@ Readings taken where the paper is silent or differs from the workload spec
 * calibration: exact lower order statistic of |x| over all calibration values
   at rank floor(s1 * n) (0-based); s1 = 0 gives tau = 0.
 * Stage 2 uses the full input x, not the sparsified one (*Prox* §4.1, Stage 2).
+* GeGLU gate (*Prox* §5 names Gemma-3's GeGLU FFN, not the GELU form): both
+  GELU(z) = z Phi(z), evaluated through erfc, and the tanh form.
+* ablation A3 (*Prox* §5.2): the signed proxy values act(g~) u~ of the selected
+  channels (same selection rule as Prox) go into W_down.
+* allocation (*Prox* §4.2): a target whose re-solved s2 would leave [0, 1] has
+  no allocation and raises.
+* the Stage-2 score threshold tau_s: the same exact lower order statistic as
+  tau_x, over the calibration tokens' scores held as fp32.
 """
 
 from __future__ import annotations
