@@ -27,6 +27,28 @@ std::mutex g_calib_scratch_mu;
 
 thread_local std::string g_last_error;
 
+// Test-only fault injection: when positive, the allocation that brings the
+// count to zero fails as if the device were out of memory.
+std::atomic<int> g_alloc_countdown{0};
+
+cudaError_t dev_alloc(void** p, size_t bytes) {
+  int c = g_alloc_countdown.load();
+  while (c > 0 && !g_alloc_countdown.compare_exchange_weak(c, c - 1)) {
+  }
+  if (c == 1) {
+    *p = nullptr;
+    return cudaErrorMemoryAllocation;
+  }
+  return cudaMalloc(p, bytes);
+}
+template <typename T>
+cudaError_t dev_alloc(T** p, size_t bytes) {
+  void* v = nullptr;
+  const cudaError_t e = dev_alloc(&v, bytes);
+  *p = static_cast<T*>(v);
+  return e;
+}
+
 prox_status fail(prox_status st, const char* fmt, ...) {
   char buf[512];
   va_list ap;
@@ -114,7 +136,7 @@ prox_status alloc_workspace(prox_layer* L) {
   const size_t o_in = take((size_t)kHostChunkTokens * d * 4);
   const size_t o_out = take((size_t)kHostChunkTokens * d * 4);
   void* base = nullptr;
-  PROX_CUDA(cudaMalloc(&base, off), "cudaMalloc(workspace)");
+  PROX_CUDA(dev_alloc(&base, off), "cudaMalloc(workspace)");
   PROX_CUDA(cudaMemset(base, 0, off), "cudaMemset(workspace)");
   char* b = static_cast<char*>(base);
   prox::Workspace& w = L->ws;
@@ -316,14 +338,14 @@ prox_status prox_layer_create(const uint16_t* W_gate, const uint16_t* W_up, cons
   };
   step(prox::setup_stage1_kernels());
   step(prox::setup_stage2_kernels());
-  step(cudaMalloc(&L->wgu, 2 * F * d * 2));
-  step(cudaMalloc(&L->wd, F * d * 2));
-  step(cudaMalloc(&L->pq, d * F));
-  step(cudaMalloc(&L->ps, (size_t)L->G * F * 2 * 2));
-  step(cudaMalloc(&cg, d * F / 2));
-  step(cudaMalloc(&cu, d * F / 2));
-  step(cudaMalloc(&sg, (size_t)L->G * F * 2));
-  step(cudaMalloc(&su, (size_t)L->G * F * 2));
+  step(dev_alloc(&L->wgu, 2 * F * d * 2));
+  step(dev_alloc(&L->wd, F * d * 2));
+  step(dev_alloc(&L->pq, d * F));
+  step(dev_alloc(&L->ps, (size_t)L->G * F * 2 * 2));
+  step(dev_alloc(&cg, d * F / 2));
+  step(dev_alloc(&cu, d * F / 2));
+  step(dev_alloc(&sg, (size_t)L->G * F * 2));
+  step(dev_alloc(&su, (size_t)L->G * F * 2));
   if (e == cudaSuccess) {
     step(prox::launch_pack_proxy(W_gate, L->d, L->F, cg, sg, s));
     step(prox::launch_pack_proxy(W_up, L->d, L->F, cu, su, s));
@@ -347,6 +369,12 @@ prox_status prox_layer_create(const uint16_t* W_gate, const uint16_t* W_up, cons
     return st;
   }
   *out_host = L;
+  return PROX_OK;
+}
+
+prox_status prox_debug_fail_alloc(int nth) {
+  if (nth < 0) return fail(PROX_EINVAL, "nth=%d must be >= 0", nth);
+  g_alloc_countdown.store(nth);
   return PROX_OK;
 }
 

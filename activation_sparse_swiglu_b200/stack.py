@@ -8,9 +8,57 @@ scores of those same inputs.  Every step runs in the library's kernels
 
 from __future__ import annotations
 
+import json
+import math
+
 import torch
 
-from . import MASK_THRESHOLD, Layer, calibrate_thresholds, rmsnorm
+from . import MASK_THRESHOLD, MASK_TOPK, Layer, calibrate_thresholds, rmsnorm
+
+ARTEFACT_FORMAT = "prox-thresholds"
+ARTEFACT_VERSION = 1
+
+
+def thresholds_to_json(taus, taus_s=None, *, d_model: int, d_ff: int, k: int, s1: float,
+                       s2: float | None = None) -> str:
+    """The calibration artefact of a stack (Prox App. A.7: thresholds are
+    calibrated once and never re-estimated at inference): per layer tau_x and,
+    under the threshold rule, tau_s.  Floats are written so that they read back
+    bit for bit."""
+    if taus_s is not None and len(taus_s) != len(taus):
+        raise ValueError("taus and taus_s differ in length")
+    layers = [{"tau_x": float(t), "tau_s": None if taus_s is None else float(taus_s[i])}
+              for i, t in enumerate(taus)]
+    doc = {"format": ARTEFACT_FORMAT, "version": ARTEFACT_VERSION, "d_model": int(d_model),
+           "d_ff": int(d_ff), "k": int(k), "s1": float(s1),
+           "s2": None if s2 is None else float(s2), "layers": layers}
+    _check_artefact(doc)
+    return json.dumps(doc, indent=1)
+
+
+def _check_artefact(doc) -> None:
+    if doc.get("format") != ARTEFACT_FORMAT or doc.get("version") != ARTEFACT_VERSION:
+        raise ValueError("not a prox-thresholds artefact of a known version")
+    if not isinstance(doc.get("layers"), list) or not doc["layers"]:
+        raise ValueError("the artefact holds no layers")
+    if not 1 <= int(doc["k"]) <= int(doc["d_ff"]):
+        raise ValueError("k must lie in [1, d_ff]")
+    has_s = [ly.get("tau_s") is not None for ly in doc["layers"]]
+    if any(has_s) and not all(has_s):
+        raise ValueError("tau_s must be given for every layer or for none")
+    for ly in doc["layers"]:
+        for key in ("tau_x", "tau_s"):
+            v = ly.get(key)
+            if key == "tau_x" or v is not None:
+                if not isinstance(v, (int, float)) or not math.isfinite(v) or v < 0:
+                    raise ValueError(f"{key} must be a finite value >= 0, got {v!r}")
+
+
+def thresholds_from_json(text: str) -> dict:
+    """Parses and checks an artefact written by thresholds_to_json."""
+    doc = json.loads(text)
+    _check_artefact(doc)
+    return doc
 
 
 class Stack:
@@ -45,6 +93,41 @@ class Stack:
         if s2 is not None:
             return list(self.taus), taus_s, inputs
         return list(self.taus), inputs
+
+    def save_thresholds(self, path: str, s1: float, s2: float | None = None) -> None:
+        """Writes the current per-layer thresholds as a calibration artefact."""
+        infos = [layer.info() for layer in self.layers]
+        taus = [inf["tau_x"] for inf in infos]
+        taus_s = None
+        if any(inf["mask_mode"] == MASK_THRESHOLD for inf in infos):
+            taus_s = [inf["tau_s"] for inf in infos]
+        text = thresholds_to_json(taus, taus_s, d_model=infos[0]["d_model"],
+                                  d_ff=infos[0]["d_ff"], k=self.k, s1=s1, s2=s2)
+        with open(path, "w") as fh:
+            fh.write(text)
+
+    def load_thresholds(self, path: str) -> dict:
+        """Applies a calibration artefact: tau_x per layer and, when present,
+        the score-threshold rule with tau_s (otherwise top-k with the
+        artefact's k).  Shapes and layer count must match."""
+        with open(path) as fh:
+            doc = thresholds_from_json(fh.read())
+        if len(doc["layers"]) != len(self.layers):
+            raise ValueError("the artefact has a different number of layers")
+        for layer, ly in zip(self.layers, doc["layers"]):
+            inf = layer.info()
+            if (inf["d_model"], inf["d_ff"]) != (doc["d_model"], doc["d_ff"]):
+                raise ValueError("the artefact was calibrated for another layer shape")
+        self.k = int(doc["k"])
+        for li, (layer, ly) in enumerate(zip(self.layers, doc["layers"])):
+            layer.set_tau(ly["tau_x"])
+            layer.set_k(self.k)
+            if ly["tau_s"] is None:
+                layer.set_mask(MASK_TOPK)
+            else:
+                layer.set_mask(MASK_THRESHOLD, ly["tau_s"])
+            self.taus[li] = ly["tau_x"]
+        return doc
 
     def forward(self, x: torch.Tensor, stream=None):
         """Tokens [B, d] through every layer; returns the per-layer inputs and

@@ -300,6 +300,14 @@ PROX_API prox_status prox_debug_mask(const prox_layer* layer, const float* x, in
 PROX_API prox_status prox_forward_with_mask(prox_layer* layer, const float* x, const int32_t* idx_s,
                                    int k, float* out, float* s_sp, void* stream);
 
+/* Test-only fault injection on the host: the nth device allocation that
+ * prox_layer_create makes from now on (1 = the next one; a create makes nine:
+ * four weight buffers, four packing temporaries, the workspace) fails as if
+ * the device were out of memory, so the caller sees PROX_ENOMEM and the
+ * library frees whatever it had allocated; 0 cancels a pending injection.
+ * Process-wide; nothing fails on the device.  nth < 0 gives PROX_EINVAL. */
+PROX_API prox_status prox_debug_fail_alloc(int nth);
+
 /* ------------------------------------------------------------------------
  * Harness kernels
  * ------------------------------------------------------------------------ */

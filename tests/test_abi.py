@@ -115,3 +115,10 @@ def test_cost_model_host_functions_match_the_oracle(plib):
     assert lib.prox_effective_sparsity(1.2, 0.5, 1 / 3, ctypes.byref(c)) == plib.PROX_EINVAL
     assert lib.prox_runtime_sparsity(5000, 0, 4, 512, 1024, 1 / 3, None, None, None) == plib.PROX_EINVAL
     assert lib.prox_runtime_sparsity(0, 0, 0, 512, 1024, 1 / 3, None, None, None) == plib.PROX_EINVAL
+
+
+def test_fault_injection_arguments(plib):
+    lib = plib.lib
+    assert lib.prox_debug_fail_alloc(-1) == plib.PROX_EINVAL
+    assert lib.prox_debug_fail_alloc(3) == plib.PROX_OK
+    assert lib.prox_debug_fail_alloc(0) == plib.PROX_OK  # cancelled again

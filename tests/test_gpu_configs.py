@@ -8,6 +8,9 @@ layer gets the oracle's inputs for that layer; the free-running GPU stack is
 checked only loosely (its earlier layers round differently).
 """
 
+import os
+import tempfile
+
 import numpy as np
 import pytest
 import torch
@@ -190,6 +193,19 @@ def test_stack_threshold_rule_small(prox):
             y_g = layer.forward(xd)
             torch.cuda.synchronize()
             assert rel_l2(y_g.cpu().numpy().reshape(-1), want) <= OUT_RTOL
+    # the calibration artefact: saved, the layers reset, loaded back bit for bit
+    with tempfile.TemporaryDirectory() as td:
+        path = os.path.join(td, "thresholds.json")
+        stack.save_thresholds(path, 0.5, 0.7)
+        for layer in stack.layers:
+            layer.set_tau(0.0)
+            layer.set_mask(prox.MASK_TOPK)
+        stack.load_thresholds(path)
+    for li, layer in enumerate(stack.layers):
+        inf = layer.info()
+        assert inf["mask_mode"] == prox.MASK_THRESHOLD
+        assert np.float32(inf["tau_x"]) == np.float32(taus[li])
+        assert np.float32(inf["tau_s"]) == np.float32(taus_s[li])
     for layer in stack.layers:
         assert layer.error_word() == 0
     stack.close()
