@@ -23,7 +23,9 @@
 // per touched slice and written to global memory.  Each CTA then adds its row
 // count to the slice's counter; the CTA that completes a slice adds that
 // slice's partials in CTA order (deterministic), scores the channels,
-// score_j = |SiLU(g~_j) u~_j|, counts them in an 8192-bin histogram of their
+// score_j = |act(g~_j) u~_j| (act the layer's gate activation: SiLU, or GELU
+// for a GeGLU FFN; the signed value is kept too when Stage 2 runs the A3
+// ablation), counts them in an 8192-bin histogram of their
 // top bits -- the first level of the radix select -- and appends (key,
 // channel) to the bin's bucket at the slot the count returned.
 #include "prox_device.cuh"

@@ -21,7 +21,8 @@
 //            packed f32x2 FMAs, warp-shuffle reduction) and parks them in
 //            shared memory; after the last channel the partials are summed in
 //            a fixed order into g = x . W_gate[:, j], u = x . W_up[:, j] and
-//            s_j = SiLU(g) u;
+//            s_j = act(g) u (the A3 ablation skips the gate/up records
+//            and takes s_j = s~_j from Stage 1);
 //   phase B: all warps accumulate y_part += s_j W_down[j, :] for the CTA's
 //            channels, each thread owning 8-column groups of the output.
 // Each CTA writes its fp32 partial y; reduce_kernel sums the partials in a
