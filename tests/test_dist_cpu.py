@@ -49,3 +49,24 @@ def test_two_rank_max_and_value():
     for rank, t, value in res:
         assert t == pytest.approx(15.0)
         assert value == pytest.approx(512 / 0.015)
+
+
+def test_reference_arm_under_torchrun_prints_once():
+    """`bench.py --impl reference` launched like the multi-GPU runs: rank 0
+    times the oracle and prints the one JSON line, the other rank exits 0
+    without work."""
+    import json
+    import subprocess
+    port = _free_port()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), "bench.py", "--impl",
+           "reference", "--gpus", "2", "--steps", "2", "--warmup", "3", "--workload", "tiny"]
+    out = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=300)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, out.stdout
+    rec = json.loads(lines[0])
+    assert rec["impl"] == "reference" and rec["value"] > 0 and rec["steps"] == 2
+    assert rec["cpu_baseline"]["kind"] == "oracle"
+    assert rec["e2e"]["h2d_bytes_per_step"] == 0 and rec["e2e"]["value"] == rec["value"]
+    assert "tiny" in rec["config"]["workload"]
