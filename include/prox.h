@@ -22,6 +22,10 @@
  *  - Shape rules (else PROX_EINVAL, checked before any launch):
  *    d_model > 0 and d_model % 128 == 0; d_ff > 0 and d_ff % 32 == 0;
  *    d_model <= 16384; d_ff <= 32768; 1 <= k <= d_ff; pointers 16-byte aligned.
+ *    Stage 1 keeps its share of the kept input rows in shared memory, which
+ *    bounds ceil(d_ff/512) * d_model <= 5192 * (number of SMs): about 768 K on
+ *    a 148-SM B200, so every d_model at d_ff = 14336 but d_model <= 11904 at
+ *    d_ff = 32768.  prox_layer_create returns PROX_EUNSUPPORTED beyond it.
  *  - Errors: every call returns a prox_status; prox_last_error() copies a
  *    message for the calling thread's last failure.  No C++ exception crosses
  *    this boundary.  Device-side checks (an index out of range in a caller's
