@@ -690,3 +690,12 @@ def test_a3_is_the_masked_sum_of_proxy_values():
         acc += a3["s_tilde"][j] * lay.w_down[j].astype(np.float64)
     np.testing.assert_allclose(a3["y"], acc, rtol=1e-12, atol=1e-15)
     assert np.linalg.norm(a3["y"] - ex["y"]) > 1e-3 * np.linalg.norm(ex["y"])
+
+
+def test_mask_overlap_report_runs():
+    # the reporting script behind the quoted synthetic overlap (not a pin:
+    # the paper's figure is for trained weights)
+    from oracle import mask_overlap
+    k, ov = mask_overlap.overlap("tiny", 2, 0.5, 70)
+    assert k == 413 and ov.shape == (2,)
+    assert np.all((ov > 0.5) & (ov <= 1.0))
