@@ -588,21 +588,36 @@ def _cpu_model():
 
 
 def cpu_baseline(lay, tau, k, seconds):
+    """The fp64 oracle on the host: all cores for `seconds`, then a shorter
+    single-thread sample of the same workload."""
     from oracle import prox_oracle as orc
     qg, sg = orc.quantize_proxy(lay.w_gate)
     qu, su = orc.quantize_proxy(lay.w_up)
-    n, t0 = 0, time.perf_counter()
-    while True:
-        x = lay.x_eval[n % lay.x_eval.shape[0]]
-        orc.prox_ffn(x, lay.w_gate, lay.w_up, lay.w_down, qg, sg, qu, su, tau=tau, k=k)
-        n += 1
-        el = time.perf_counter() - t0
-        if (el >= seconds and n >= 2) or n >= lay.x_eval.shape[0]:
-            break
-    return {"value": round(n / el, 3), "unit": UNIT, "cores": _oracle_threads(), "kind": "oracle",
-            "cpu": _cpu_model(), "nproc": os.cpu_count(),
-            "sample": f"{n} tokens of the same workload through the fp64 numpy oracle "
-                      f"({el:.1f} s; proxy packing done once beforehand, not timed)"}
+
+    def timed(limit_s):
+        n, t0 = 0, time.perf_counter()
+        while True:
+            x = lay.x_eval[n % lay.x_eval.shape[0]]
+            orc.prox_ffn(x, lay.w_gate, lay.w_up, lay.w_down, qg, sg, qu, su, tau=tau, k=k)
+            n += 1
+            el = time.perf_counter() - t0
+            if (el >= limit_s and n >= 2) or n >= lay.x_eval.shape[0]:
+                return n, el
+
+    n, el = timed(seconds)
+    out = {"value": round(n / el, 3), "unit": UNIT, "cores": _oracle_threads(), "kind": "oracle",
+           "cpu": _cpu_model(), "nproc": os.cpu_count(),
+           "sample": f"{n} tokens of the same workload through the fp64 numpy oracle "
+                     f"({el:.1f} s; proxy packing done once beforehand, not timed)"}
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            n1, el1 = timed(seconds / 3)
+        out["single_thread"] = {"value": round(n1 / el1, 3), "unit": UNIT, "cores": 1,
+                                "sample": f"{n1} tokens ({el1:.1f} s), BLAS limited to one thread"}
+    except ImportError:
+        pass
+    return out
 
 
 # ---------------------------------------------------------------------------
