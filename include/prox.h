@@ -166,10 +166,15 @@ PROX_API prox_status prox_layer_create(const uint16_t* W_gate, const uint16_t* W
                               const uint16_t* W_down, int d_model, int d_ff, float tau_x,
                               int k, int max_batch, void* stream, prox_layer** out_host);
 
+/* Frees the layer's device buffers (on the layer's device, switching to it
+ * and back if another one is current) and the handle.  The frees are
+ * cudaFree calls, which wait for work still running on the device.  NULL is
+ * accepted (PROX_OK); the handle may not be used afterwards. */
 PROX_API prox_status prox_layer_destroy(prox_layer* layer);
 
 /* Change the threshold or k of an existing layer (host-side; affects calls
- * enqueued afterwards). */
+ * enqueued afterwards).  tau_x must be finite and >= 0, k in [1, d_ff], else
+ * PROX_EINVAL and the layer is unchanged. */
 PROX_API prox_status prox_layer_set_tau(prox_layer* layer, float tau_x);
 PROX_API prox_status prox_layer_set_k(prox_layer* layer, int k);
 
@@ -186,6 +191,9 @@ PROX_API prox_status prox_layer_set_activation(prox_layer* layer, int act);
  * prox_forward_with_mask and prox_dense_ffn always compute exact values. */
 PROX_API prox_status prox_layer_set_stage2(prox_layer* layer, int source);
 
+/* Copies the layer's shapes, current settings, launch geometry and byte
+ * counts into info_host (host memory, caller-owned).  Host only; NULL
+ * arguments give PROX_EINVAL. */
 PROX_API prox_status prox_layer_get_info(const prox_layer* layer, prox_layer_info* info_host);
 
 /* Reads (and clears) the layer's device error word; synchronises `stream`. */
