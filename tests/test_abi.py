@@ -122,3 +122,20 @@ def test_fault_injection_arguments(plib):
     assert lib.prox_debug_fail_alloc(-1) == plib.PROX_EINVAL
     assert lib.prox_debug_fail_alloc(3) == plib.PROX_OK
     assert lib.prox_debug_fail_alloc(0) == plib.PROX_OK  # cancelled again
+
+
+def test_every_entry_point_is_documented():
+    """Each PROX_API declaration in include/prox.h follows a comment block (a
+    declaration may share the comment of the one right above it)."""
+    lines = open(os.path.join(ROOT, "include", "prox.h")).read().splitlines()
+    undocumented = []
+    for i, line in enumerate(lines):
+        m = re.search(r"PROX_API\s+[\w\s\*]+?\b(prox_\w+)\s*\(", line)
+        if not m:
+            continue
+        j = i - 1
+        while j >= 0 and lines[j].strip().startswith("PROX_API"):
+            j -= 1  # grouped declarations share one comment
+        if j < 0 or not lines[j].strip().endswith("*/"):
+            undocumented.append(m.group(1))
+    assert not undocumented, undocumented
