@@ -57,6 +57,18 @@ def _dev(t: torch.Tensor, dtype: torch.dtype, name: str) -> torch.Tensor:
     return t
 
 
+def _need(t: torch.Tensor, numel: int, name: str) -> None:
+    """The library writes `numel` values through t's pointer: t must hold them."""
+    if t.numel() < numel:
+        raise ValueError(f"{name} holds {t.numel()} values, {numel} needed")
+
+
+def _one_token(x: torch.Tensor, d_model: int, name: str = "x") -> None:
+    if x.numel() != d_model:
+        raise ValueError(f"{name} must hold one token of d_model={d_model} values, "
+                         f"got {x.numel()}")
+
+
 def pack_proxy(w: torch.Tensor, group: int = GROUP, stream=None):
     """INT4 proxy of a bf16 [d_model, d_ff] weight: (codes uint8 [d, d_ff/2],
     scales fp16 [d/group, d_ff])."""
@@ -98,12 +110,18 @@ def rmsnorm(y: torch.Tensor, eps: float = 1e-6, out: torch.Tensor | None = None,
     y2 = y.reshape(-1, y.shape[-1])
     if out is None:
         out = torch.empty_like(y)
+    else:
+        _dev(out, torch.float32, "out")
+        _need(out, y2.numel(), "out")
     check(lib.prox_rmsnorm(_ptr(y2), _ptr(out), y2.shape[0], y2.shape[1], float(eps),
                            _stream(stream)))
     return out
 
 
 def copy(src: torch.Tensor, dst: torch.Tensor, stream=None) -> None:
+    for t, name in ((src, "src"), (dst, "dst")):
+        if not isinstance(t, torch.Tensor) or not t.is_cuda or not t.is_contiguous():
+            raise TypeError(f"{name} must be a contiguous CUDA tensor")
     nbytes = src.numel() * src.element_size()
     if dst.numel() * dst.element_size() < nbytes:
         raise ValueError("dst is smaller than src")
@@ -246,6 +264,7 @@ class Layer:
     def debug_mask(self, x: torch.Tensor, stream=None) -> torch.Tensor:
         """The Stage-2 channels one token selects under the current rule (int32, ascending)."""
         _dev(x, torch.float32, "x")
+        _one_token(x, self.d_model)
         idx = torch.empty(self.d_ff, dtype=torch.int32, device=x.device)
         n = torch.zeros(1, dtype=torch.int32, device=x.device)
         check(lib.prox_debug_mask(self.handle, _ptr(x), _ptr(idx), _ptr(n), _stream(stream)))
@@ -259,6 +278,7 @@ class Layer:
             out = torch.empty_like(x2)
         else:
             _dev(out, torch.float32, "out")
+            _need(out, x2.numel(), "out")
         return x2, out
 
     def forward(self, x: torch.Tensor, out: torch.Tensor | None = None, stream=None):
@@ -281,18 +301,30 @@ class Layer:
         x2 = x_host.reshape(-1, self.d_model)
         if out_host is None:
             out_host = torch.empty_like(x2)
+        elif (out_host.is_cuda or out_host.dtype != torch.float32
+              or not out_host.is_contiguous()):
+            raise TypeError("out_host must be a contiguous fp32 CPU tensor")
+        else:
+            _need(out_host, x2.numel(), "out_host")
         check(lib.prox_ffn_forward_host(self.handle, _ptr(x2), _ptr(out_host), x2.shape[0],
                                         _stream(stream)))
         return out_host
 
     def forward_profiled(self, x: torch.Tensor, out: torch.Tensor, events, stream=None):
         """One token, kernels serialised, with 4 torch.cuda.Event(enable_timing=True)."""
+        _dev(x, torch.float32, "x")
+        _dev(out, torch.float32, "out")
+        _one_token(x, self.d_model)
+        _need(out, self.d_model, "out")
+        if len(events) != 4:
+            raise ValueError("forward_profiled needs 4 events")
         arr = (ctypes.c_void_p * 4)(*[ctypes.c_void_p(e.cuda_event) for e in events])
         check(lib.prox_ffn_forward_profiled(self.handle, _ptr(x), _ptr(out), arr, _stream(stream)))
 
     def debug_stage1(self, x: torch.Tensor, stream=None) -> dict:
         """Stage 1 of one token: idx_x, n_x, g_tilde, u_tilde, idx_s (CUDA tensors)."""
         _dev(x, torch.float32, "x")
+        _one_token(x, self.d_model)
         dev = x.device
         k = self.k
         idx_x = torch.full((self.d_model,), -1, dtype=torch.int32, device=dev)
@@ -309,8 +341,12 @@ class Layer:
         """Stage 2 on a given channel list (int32 CUDA tensor)."""
         _dev(x, torch.float32, "x")
         _dev(idx_s, torch.int32, "idx_s")
+        _one_token(x, self.d_model)
         if out is None:
             out = torch.empty(self.d_model, dtype=torch.float32, device=x.device)
+        else:
+            _dev(out, torch.float32, "out")
+            _need(out, self.d_model, "out")
         s_sp = torch.empty(idx_s.numel(), dtype=torch.float32, device=x.device) if want_s else None
         check(lib.prox_forward_with_mask(self.handle, _ptr(x), _ptr(idx_s), idx_s.numel(), _ptr(out),
                                          _ptr(s_sp), _stream(stream)))

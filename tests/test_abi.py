@@ -139,3 +139,20 @@ def test_every_entry_point_is_documented():
         if j < 0 or not lines[j].strip().endswith("*/"):
             undocumented.append(m.group(1))
     assert not undocumented, undocumented
+
+
+def test_binding_refuses_short_or_host_buffers():
+    """The Python binding checks what the C ABI cannot see (tensor sizes and
+    memory spaces) before any library call."""
+    import torch
+    import activation_sparse_swiglu_b200 as prox
+    with pytest.raises(ValueError):
+        prox._need(torch.empty(10), 11, "out")
+    prox._need(torch.empty(10), 10, "out")
+    with pytest.raises(ValueError):
+        prox._one_token(torch.empty(2, 512), 512)
+    prox._one_token(torch.empty(512), 512)
+    with pytest.raises(TypeError):  # host tensors never reach the copy kernel
+        prox.copy(torch.empty(16), torch.empty(16))
+    with pytest.raises(TypeError):
+        prox.rmsnorm(torch.empty(4, 8))
