@@ -63,6 +63,15 @@ def _need(t: torch.Tensor, numel: int, name: str) -> None:
         raise ValueError(f"{name} holds {t.numel()} values, {numel} needed")
 
 
+def _on_current_device(**tensors) -> None:
+    """Every named tensor lives on the current CUDA device (the library
+    launches on that device and reads the pointers there)."""
+    cur = torch.cuda.current_device()
+    for name, t in tensors.items():
+        if t.device.type != "cuda" or t.device.index != cur:
+            raise ValueError(f"{name} is on {t.device}, not on the current CUDA device cuda:{cur}")
+
+
 def _one_token(x: torch.Tensor, d_model: int, name: str = "x") -> None:
     if x.numel() != d_model:
         raise ValueError(f"{name} must hold one token of d_model={d_model} values, "
@@ -93,12 +102,16 @@ def calibrate_thresholds(x_cal: torch.Tensor, s1: float, stream=None) -> float:
 def calibrate_thresholds_noalloc(x_cal: torch.Tensor, s1: float, tau: torch.Tensor,
                                  stream=None) -> torch.Tensor:
     """The same quantile written to the 1-element fp32 device tensor `tau` in
-    stream order, with no allocation (fixed static scratch; concurrent calls on
-    one device race)."""
+    stream order, with no device allocation, for callers that cannot allocate
+    at that point (their device memory belongs to another allocator, or the
+    implicit synchronisation of an allocation is not acceptable).  The scratch
+    is a fixed static array per device; concurrent calls on one device race.
+    x_cal and tau must live on the current CUDA device."""
     _dev(x_cal, torch.float32, "x_cal")
     _dev(tau, torch.float32, "tau")
     if tau.numel() < 1:
         raise ValueError("tau needs one element")
+    _on_current_device(x_cal=x_cal, tau=tau)
     n, d = x_cal.shape
     check(lib.prox_calibrate_thresholds_noalloc(_ptr(x_cal), n, d, float(s1), _ptr(tau),
                                                 _stream(stream)))
@@ -310,16 +323,24 @@ class Layer:
                                         _stream(stream)))
         return out_host
 
-    def forward_profiled(self, x: torch.Tensor, out: torch.Tensor, events, stream=None):
-        """One token, kernels serialised, with 4 torch.cuda.Event(enable_timing=True)."""
+    def forward_profiled(self, x: torch.Tensor, out: torch.Tensor, events,
+                         phase_ns: torch.Tensor | None = None, stream=None):
+        """One token with its kernel bracketed by 2 torch.cuda.Event(enable_timing=True)
+        (no programmatic overlap).  phase_ns: optional int64 CUDA tensor
+        [stage1_ctas, 16] receiving each CTA's phase stamps (GPU global timer, ns;
+        slot meanings in include/prox.h)."""
         _dev(x, torch.float32, "x")
         _dev(out, torch.float32, "out")
         _one_token(x, self.d_model)
         _need(out, self.d_model, "out")
-        if len(events) != 4:
-            raise ValueError("forward_profiled needs 4 events")
-        arr = (ctypes.c_void_p * 4)(*[ctypes.c_void_p(e.cuda_event) for e in events])
-        check(lib.prox_ffn_forward_profiled(self.handle, _ptr(x), _ptr(out), arr, _stream(stream)))
+        if len(events) != 2:
+            raise ValueError("forward_profiled needs 2 events")
+        if phase_ns is not None:
+            _dev(phase_ns, torch.int64, "phase_ns")
+            _need(phase_ns, self.info()["stage1_ctas"] * 16, "phase_ns")
+        arr = (ctypes.c_void_p * 2)(*[ctypes.c_void_p(e.cuda_event) for e in events])
+        check(lib.prox_ffn_forward_profiled(self.handle, _ptr(x), _ptr(out), arr, _ptr(phase_ns),
+                                            _stream(stream)))
 
     def debug_stage1(self, x: torch.Tensor, stream=None) -> dict:
         """Stage 1 of one token: idx_x, n_x, g_tilde, u_tilde, idx_s (CUDA tensors)."""

@@ -74,12 +74,13 @@ SIGNATURES = {
     "prox_ffn_forward": (_I, [_P, _P, _P, _I, _P]),
     "prox_dense_ffn": (_I, [_P, _P, _P, _I, _P]),
     "prox_ffn_forward_host": (_I, [_P, _P, _P, _I, _P]),
-    "prox_ffn_forward_profiled": (_I, [_P, _P, _P, ctypes.POINTER(_P), _P]),
+    "prox_ffn_forward_profiled": (_I, [_P, _P, _P, ctypes.POINTER(_P), _P, _P]),
     "prox_debug_stage1": (_I, [_P, _P, _P, _P, _P, _P, _P, _P]),
     "prox_layer_proxy_scores": (_I, [_P, _P, _I, _P, _P]),
     "prox_debug_mask": (_I, [_P, _P, _P, _P, _P]),
     "prox_forward_with_mask": (_I, [_P, _P, _P, _I, _P, _P, _P]),
     "prox_debug_fail_alloc": (_I, [_I]),
+    "prox_debug_wait_timeout": (_I, [_P, _P]),
     "prox_rmsnorm": (_I, [_P, _P, _I, _I, _F, _P]),
     "prox_copy": (_I, [_P, _P, _S, _P]),
     "prox_last_error": (_S, [ctypes.c_char_p, _S]),

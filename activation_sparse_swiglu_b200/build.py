@@ -18,9 +18,9 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libprox.so")
 
-SOURCES = ["prox_api.cu", "stage1.cu", "stage2.cu", "pack.cu", "calibrate.cu",
-           "misc.cu"]
-HEADERS = ["prox_device.cuh", "prox_internal.h", "select.cuh"]
+SOURCES = ["prox_api.cu", "token.cu", "pack.cu", "calibrate.cu", "misc.cu"]
+HEADERS = ["prox_device.cuh", "prox_internal.h", "select.cuh", "token_args.cuh", "stage1.cuh",
+           "stage2.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

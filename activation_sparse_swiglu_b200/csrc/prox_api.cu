@@ -13,17 +13,43 @@
 #include "prox_device.cuh"
 #include "prox_internal.h"
 
-namespace prox {
-cudaError_t setup_stage1_kernels();
-cudaError_t setup_stage2_kernels();
-}  // namespace prox
-
 namespace {
 
 constexpr int kMaxDevices = 64;
-// Device address of the static calibration scratch, per device, set once.
+// Device address of the static calibration scratch per device, and the CUDA
+// context it was looked up in (a device reset makes a new context, in which
+// the module and its static array are loaded anew).
 std::atomic<uint32_t*> g_calib_scratch_addr[kMaxDevices];
+std::atomic<void*> g_calib_scratch_ctx[kMaxDevices];
 std::mutex g_calib_scratch_mu;
+
+// The current driver context, read through the runtime's driver entry-point
+// table (no link-time dependency on the driver library).  nullptr if the
+// entry point is unavailable.
+void* current_context() {
+  using Fn = int (*)(void**);
+  static Fn fn = []() -> Fn {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<Fn>(p);
+  }();
+  void* ctx = nullptr;
+  if (fn && fn(&ctx) != 0) ctx = nullptr;
+  return ctx;
+}
+
+// Device memory of device `dev` (device-allocated or managed)?
+bool on_device(const void* p, int dev) {
+  cudaPointerAttributes at;
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return (at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged) && at.device == dev;
+}
 
 thread_local std::string g_last_error;
 
@@ -125,13 +151,12 @@ prox_status alloc_workspace(prox_layer* L) {
   const size_t o_g = take(F * 4);
   const size_t o_u = take(F * 4);
   const size_t o_hist = take(prox::kScoreBins * 4);
-  const size_t o_bucket = take((size_t)prox::kScoreBins * prox::kBucketCap * 8);
   const size_t o_mask = take(F * 4);
   const size_t o_idx = take(F * 4);
-  const size_t o_s1p = take(prox::stage1_part_floats(L->P1) * 4);
-  const size_t o_s1c = take((size_t)L->C * 4);
+  const size_t o_s1p = take(prox::stage1_part_floats(L->P) * 4);
   const size_t o_ypart = take((size_t)L->P * d * 4);
   const size_t o_stats = take(24);
+  const size_t o_gbar = take(8);
   const size_t o_err = take(4);
   const size_t o_in = take((size_t)kHostChunkTokens * d * 4);
   const size_t o_out = take((size_t)kHostChunkTokens * d * 4);
@@ -147,23 +172,25 @@ prox_status alloc_workspace(prox_layer* L) {
   w.g_dbg = reinterpret_cast<float*>(b + o_g);
   w.u_dbg = reinterpret_cast<float*>(b + o_u);
   w.hist = reinterpret_cast<uint32_t*>(b + o_hist);
-  w.bucket = reinterpret_cast<uint2*>(b + o_bucket);
   w.sel_mask = reinterpret_cast<int32_t*>(b + o_mask);
   w.idx_s = reinterpret_cast<int32_t*>(b + o_idx);
   w.s1_part = reinterpret_cast<float*>(b + o_s1p);
-  w.s1_cnt = reinterpret_cast<int*>(b + o_s1c);
   w.ypart = reinterpret_cast<float*>(b + o_ypart);
   w.stats = reinterpret_cast<unsigned long long*>(b + o_stats);
+  w.gbar = reinterpret_cast<unsigned long long*>(b + o_gbar);
   w.err = reinterpret_cast<int*>(b + o_err);
   w.stage_in = reinterpret_cast<float*>(b + o_in);
   w.stage_out = reinterpret_cast<float*>(b + o_out);
   return PROX_OK;
 }
 
-// The Stage-2 selection of the forward step: the layer's rule (top-k or the
-// score threshold).
-prox::Stage2Launch topk_launch(const prox_layer* L) {
-  prox::Stage2Launch m;
+// One token of the forward step under the layer's Stage-2 rule (top-k or the
+// score threshold) and value source.
+prox::TokenLaunch forward_launch(const prox_layer* L, const float* x, float* out) {
+  prox::TokenLaunch m;
+  m.x = x;
+  m.out = out;
+  m.stage1 = true;
   m.mode = L->mask_mode == PROX_MASK_THRESHOLD ? 3 : 1;
   m.k = L->k;
   m.tau_s = L->tau_s;
@@ -171,21 +198,18 @@ prox::Stage2Launch topk_launch(const prox_layer* L) {
   return m;
 }
 
-// Stage 1 -> select -> Stage 2 (gate/up + down) -> output reduction, one token.
 cudaError_t enqueue_token(const prox_layer* L, const float* x, float* out, cudaStream_t s) {
-  cudaError_t e;
-  if ((e = prox::launch_stage1(L, x, prox::Stage1Taps{}, s, true)) != cudaSuccess) return e;
-  if ((e = prox::launch_stage2(L, x, topk_launch(L), s, true, true)) != cudaSuccess) return e;
-  return prox::launch_reduce(L, out, s, true);
+  return prox::launch_token(L, forward_launch(L, x, out), s, true);
 }
 
 cudaError_t enqueue_dense(const prox_layer* L, const float* x, float* out, cudaStream_t s) {
-  prox::Stage2Launch m;
+  prox::TokenLaunch m;
+  m.x = x;
+  m.out = out;
+  m.stage1 = false;
   m.mode = 2;
   m.k = L->F;
-  cudaError_t e = prox::launch_stage2(L, x, m, s, false, true);
-  if (e != cudaSuccess) return e;
-  return prox::launch_reduce(L, out, s, true);
+  return prox::launch_token(L, m, s, true);
 }
 
 prox_status check_layer(const prox_layer* L) {
@@ -270,14 +294,18 @@ prox_status prox_calibrate_thresholds_noalloc(const float* X_cal, int n_tok, int
   prox_status st = check_device(&dev, &sms);
   if (st != PROX_OK) return st;
   if (dev < 0 || dev >= kMaxDevices) return fail(PROX_EUNSUPPORTED, "device ordinal %d out of range", dev);
-  // The scratch address is looked up once per device, with that device
-  // current (it is the caller's current device here).
+  if (!on_device(X_cal, dev) || !on_device(tau_dev, dev))
+    return fail(PROX_EINVAL, "X_cal and tau_dev must be device memory of the current device %d", dev);
+  // The scratch address is looked up once per device and context, with that
+  // device current (it is the caller's current device here).
+  void* ctx = current_context();
   uint32_t* scratch = g_calib_scratch_addr[dev].load(std::memory_order_acquire);
-  if (!scratch) {
+  if (!scratch || g_calib_scratch_ctx[dev].load(std::memory_order_acquire) != ctx) {
     std::lock_guard<std::mutex> lock(g_calib_scratch_mu);
     scratch = g_calib_scratch_addr[dev].load(std::memory_order_relaxed);
-    if (!scratch) {
+    if (!scratch || g_calib_scratch_ctx[dev].load(std::memory_order_relaxed) != ctx) {
       PROX_CUDA(prox::calibrate_static_scratch(&scratch), "cudaGetSymbolAddress(calibration scratch)");
+      g_calib_scratch_ctx[dev].store(ctx, std::memory_order_release);
       g_calib_scratch_addr[dev].store(scratch, std::memory_order_release);
     }
   }
@@ -318,14 +346,21 @@ prox_status prox_layer_create(const uint16_t* W_gate, const uint16_t* W_up, cons
   L->tau = tau_x;
   L->device = dev;
   L->num_sms = sms;
-  prox::choose_stage1_grid(L->d, L->F, sms, &L->C, &L->P1, &L->s1_lmax);
-  prox::choose_stage2(L->d, L->F, sms, &L->P, &L->ring_slots, &L->stage2_groups,
-                     &L->stage2_smem);
-  L->stage1_smem = prox::stage1_smem_bytes(L->s1_lmax);
-  if (L->stage1_smem > (size_t)prox::kMaxSmemPerBlock) {
-    const size_t need = L->stage1_smem;
+  if (sms > prox::kMaxCtas) {
     delete L;
-    return fail(PROX_EUNSUPPORTED, "Stage-1 shared memory %zu exceeds the per-CTA limit", need);
+    return fail(PROX_EUNSUPPORTED, "%d SMs exceed the %d CTAs the per-token kernel supports", sms,
+                prox::kMaxCtas);
+  }
+  L->P = sms;
+  prox::choose_stage1_grid(L->d, L->F, sms, &L->C, &L->s1_lmax, &L->s1_nb);
+  size_t s2_smem = 0;
+  prox::choose_stage2(L->d, L->F, sms, &L->ring_slots, &L->stage2_groups, &s2_smem);
+  const size_t s1_smem = prox::stage1_smem_bytes(L->s1_lmax, L->s1_nb);
+  L->token_smem = s1_smem > s2_smem ? s1_smem : s2_smem;
+  if (L->token_smem > (size_t)prox::kMaxSmemPerBlock) {
+    const size_t need = L->token_smem;
+    delete L;
+    return fail(PROX_EUNSUPPORTED, "per-token kernel shared memory %zu exceeds the per-CTA limit", need);
   }
 
   cudaStream_t s = as_stream(stream);
@@ -336,8 +371,7 @@ prox_status prox_layer_create(const uint16_t* W_gate, const uint16_t* W_up, cons
   auto step = [&](cudaError_t r) {
     if (e == cudaSuccess) e = r;
   };
-  step(prox::setup_stage1_kernels());
-  step(prox::setup_stage2_kernels());
+  step(prox::setup_token_kernels());
   step(dev_alloc(&L->wgu, 2 * F * d * 2));
   step(dev_alloc(&L->wd, F * d * 2));
   step(dev_alloc(&L->pq, d * F));
@@ -369,6 +403,13 @@ prox_status prox_layer_create(const uint16_t* W_gate, const uint16_t* W_up, cons
     return st;
   }
   *out_host = L;
+  return PROX_OK;
+}
+
+prox_status prox_debug_wait_timeout(prox_layer* L, void* stream) {
+  prox_status st = check_layer(L);
+  if (st != PROX_OK) return st;
+  PROX_CUDA(prox::launch_barrier_probe(L, as_stream(stream)), "barrier probe launch");
   return PROX_OK;
 }
 
@@ -439,7 +480,7 @@ prox_status prox_layer_get_info(const prox_layer* L, prox_layer_info* info) {
   info->max_batch = L->max_batch;
   info->tau_x = L->tau;
   info->stage1_col_slices = L->C;
-  info->stage1_ctas = L->P1;
+  info->stage1_ctas = L->P;
   info->stage2_ctas = L->P;
   info->stage2_ring_slots = L->ring_slots;
   info->weight_bytes = (size_t)3 * L->F * L->d * 2;
@@ -461,6 +502,13 @@ prox_status prox_layer_error(prox_layer* L, int32_t* word_host, void* stream) {
   PROX_CUDA(cudaMemcpyAsync(&v, L->ws.err, 4, cudaMemcpyDeviceToHost, s), "read error word");
   PROX_CUDA(cudaMemsetAsync(L->ws.err, 0, 4, s), "clear error word");
   PROX_CUDA(cudaStreamSynchronize(s), "cudaStreamSynchronize");
+  if (v & PROX_DEVERR_WAIT_TIMEOUT) {
+    // A token whose wait ran out may have left the grid-barrier counter and
+    // the histogram mid-way: start the next token clean.
+    PROX_CUDA(cudaMemsetAsync(L->ws.gbar, 0, 8, s), "reset grid barrier");
+    PROX_CUDA(cudaMemsetAsync(L->ws.hist, 0, prox::kScoreBins * 4, s), "reset histogram");
+    PROX_CUDA(cudaStreamSynchronize(s), "cudaStreamSynchronize");
+  }
   *word_host = v;
   return PROX_OK;
 }
@@ -586,19 +634,17 @@ prox_status prox_ffn_forward_host(prox_layer* L, const float* x_host, float* out
 }
 
 prox_status prox_ffn_forward_profiled(const prox_layer* L, const float* x, float* out,
-                                      void* const* events, void* stream) {
+                                      void* const* events, uint64_t* phase_ns, void* stream) {
   prox_status st = check_layer(L);
   if (st != PROX_OK) return st;
   if (!events || !x || !out) return fail(PROX_EINVAL, "NULL argument");
+  if (!aligned16(x) || !aligned16(out)) return fail(PROX_EINVAL, "x and out must be 16-byte aligned");
   cudaStream_t s = as_stream(stream);
-  auto ev = [&](int i) { return reinterpret_cast<cudaEvent_t>(events[i]); };
-  PROX_CUDA(cudaEventRecord(ev(0), s), "cudaEventRecord");
-  PROX_CUDA(prox::launch_stage1(L, x, prox::Stage1Taps{}, s, false), "stage1 launch");
-  PROX_CUDA(cudaEventRecord(ev(1), s), "cudaEventRecord");
-  PROX_CUDA(prox::launch_stage2(L, x, topk_launch(L), s, false, true), "stage2 launch");
-  PROX_CUDA(cudaEventRecord(ev(2), s), "cudaEventRecord");
-  PROX_CUDA(prox::launch_reduce(L, out, s, false), "reduce launch");
-  PROX_CUDA(cudaEventRecord(ev(3), s), "cudaEventRecord");
+  prox::TokenLaunch m = forward_launch(L, x, out);
+  m.phase_ns = reinterpret_cast<unsigned long long*>(phase_ns);
+  PROX_CUDA(cudaEventRecord(reinterpret_cast<cudaEvent_t>(events[0]), s), "cudaEventRecord");
+  PROX_CUDA(prox::launch_token(L, m, s, false), "token launch");
+  PROX_CUDA(cudaEventRecord(reinterpret_cast<cudaEvent_t>(events[1]), s), "cudaEventRecord");
   return PROX_OK;
 }
 
@@ -610,18 +656,15 @@ prox_status prox_debug_stage1(prox_layer* L, const float* x, int32_t* idx_x, int
   if (idx_s && L->mask_mode != PROX_MASK_TOPK)
     return fail(PROX_EINVAL, "idx_s holds k channels under top-k only; use prox_debug_mask");
   cudaStream_t s = as_stream(stream);
-  prox::Stage1Taps t1;
-  t1.g = g_tilde;
-  t1.u = u_tilde;
-  t1.idx_x = idx_x;
-  t1.n_x = n_x;
-  PROX_CUDA(prox::launch_stage1(L, x, t1, s, false), "stage1 launch");
-  // the selection step of the forward path, stopped before the weight streaming
-  prox::Stage2Launch m = topk_launch(L);
+  // the forward step of the token, stopped after the channel selection
+  prox::TokenLaunch m = forward_launch(L, x, nullptr);
+  m.taps.g = g_tilde;
+  m.taps.u = u_tilde;
+  m.taps.idx_x = idx_x;
+  m.taps.n_x = n_x;
   m.select_only = true;
   m.sel_mask = L->ws.sel_mask;
-  PROX_CUDA(prox::launch_stage2(L, x, m, s, false, true), "stage2 launch");
-  PROX_CUDA(cudaMemsetAsync(L->ws.hist, 0, prox::kScoreBins * 4, s), "clear histogram");
+  PROX_CUDA(prox::launch_token(L, m, s, false), "token launch");
   if (idx_s)
     PROX_CUDA(prox::launch_mask_to_list(L->ws.sel_mask, L->F, idx_s, nullptr, s),
               "mask compaction launch");
@@ -635,12 +678,10 @@ prox_status prox_debug_mask(const prox_layer* L, const float* x, int32_t* idx_s,
   if (!x || !aligned16(x) || !idx_s || !n_s)
     return fail(PROX_EINVAL, "x (16-byte aligned), idx_s and n_s must be non-NULL");
   cudaStream_t s = as_stream(stream);
-  PROX_CUDA(prox::launch_stage1(L, x, prox::Stage1Taps{}, s, false), "stage1 launch");
-  prox::Stage2Launch m = topk_launch(L);
+  prox::TokenLaunch m = forward_launch(L, x, nullptr);
   m.select_only = true;
   m.sel_mask = L->ws.sel_mask;
-  PROX_CUDA(prox::launch_stage2(L, x, m, s, false, true), "stage2 launch");
-  PROX_CUDA(cudaMemsetAsync(L->ws.hist, 0, prox::kScoreBins * 4, s), "clear histogram");
+  PROX_CUDA(prox::launch_token(L, m, s, false), "token launch");
   PROX_CUDA(prox::launch_mask_to_list(L->ws.sel_mask, L->F, idx_s, n_s, s), "mask compaction launch");
   return PROX_OK;
 }
@@ -653,11 +694,13 @@ prox_status prox_layer_proxy_scores(const prox_layer* L, const float* x, int B, 
   if (!x || !scores || !aligned16(x)) return fail(PROX_EINVAL, "x (16-byte aligned) and scores must be non-NULL");
   cudaStream_t s = as_stream(stream);
   for (int b = 0; b < B; ++b) {
-    PROX_CUDA(prox::launch_stage1(L, x + (size_t)b * L->d, prox::Stage1Taps{}, s, false),
-              "stage1 launch");
+    prox::TokenLaunch m;
+    m.x = x + (size_t)b * L->d;
+    m.stage1 = true;
+    m.mode = -1;
+    PROX_CUDA(prox::launch_token(L, m, s, false), "token launch");
     PROX_CUDA(cudaMemcpyAsync(scores + (size_t)b * L->F, L->ws.scores, (size_t)L->F * 4,
                               cudaMemcpyDeviceToDevice, s), "copy scores");
-    PROX_CUDA(cudaMemsetAsync(L->ws.hist, 0, prox::kScoreBins * 4, s), "clear histogram");
   }
   return PROX_OK;
 }
@@ -670,13 +713,15 @@ prox_status prox_forward_with_mask(prox_layer* L, const float* x, const int32_t*
   if (!x || !out || !idx_s || !aligned16(x) || !aligned16(out))
     return fail(PROX_EINVAL, "bad pointer");
   cudaStream_t s = as_stream(stream);
-  prox::Stage2Launch m;
+  prox::TokenLaunch m;
+  m.x = x;
+  m.out = out;
+  m.stage1 = false;
   m.mode = 0;
   m.idx = idx_s;
   m.k = k;
   m.s_sp = s_sp;
-  PROX_CUDA(prox::launch_stage2(L, x, m, s, false, true), "stage2 launch");
-  PROX_CUDA(prox::launch_reduce(L, out, s, true), "reduce launch");
+  PROX_CUDA(prox::launch_token(L, m, s, false), "token launch");
   return PROX_OK;
 }
 

@@ -58,14 +58,17 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar, uint32_t count) {
                "r"(count)
                : "memory");
 }
+// The waiting thread may be suspended until the phase completes, for at most
+// kWaitSuspendNs per try, so a wait costs few issue slots.
+constexpr uint32_t kWaitSuspendNs = 100000;
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "n"(kWaitSuspendNs)
       : "memory");
   return ok != 0;
 }

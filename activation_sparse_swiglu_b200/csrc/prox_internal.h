@@ -15,13 +15,15 @@ constexpr int kGroup = 128;          // proxy quantisation group (input rows)
 constexpr int kHistBins = 2048;      // calibration radix levels: 11 bits
 constexpr int kScoreShift = 18;      // top-k select, first radix level: score bits [30:18]
 constexpr int kScoreBins = 8192;
-constexpr int kBucketCap = 64;       // (key, channel) entries kept per histogram bin
 constexpr int kStage1Warps = 16;     // Stage-1 warps per CTA (one CTA per SM)
-constexpr int kSelectCand = 4096;    // candidate buffer of the select (level-1 bin)
+constexpr int kSelectCand = 2048;    // candidate buffer of the select (level-1 bin)
 constexpr int kSelectSlice = 256;    // channels per select CTA (and per rank-offset entry)
 constexpr int kMaxSlices = 160;      // >= d_ff / kSelectSlice + 1
 constexpr int kStage2Consumers = 16;  // Stage-2 consumer warps (+1 producer warp)
-constexpr int kReduceWarps = 16;     // output reduction: warps per 32 columns
+constexpr int kTokenThreads = (kStage2Consumers + 1) * 32;  // threads of the per-token kernel
+constexpr int kPhaseStamps = 16;     // phase stamp slots per CTA of the per-token kernel
+constexpr int kMaxCtas = 256;        // per-token kernel grid (one CTA per SM) at most
+constexpr size_t kStage2SmemBudget = 208 * 1024;  // Stage-2 ring and tables
 constexpr int kMaxDModel = 16384;
 constexpr int kMaxDff = 32768;       // bounds the select's slice table (kMaxSlices)
 constexpr int kSmemPerSm = 233472;   // shared memory per SM on sm_100 (228 KB)
@@ -35,13 +37,12 @@ struct Workspace {
   float* g_dbg = nullptr;         // debug g~ [F]
   float* u_dbg = nullptr;         // debug u~ [F]
   uint32_t* hist = nullptr;       // [kScoreBins] score bits 30..18, zero between tokens
-  uint2* bucket = nullptr;        // [kScoreBins][kBucketCap] (key, channel) per bin
   int32_t* sel_mask = nullptr;    // [F] debug: 1 where the channel is selected
   int32_t* idx_s = nullptr;       // [F] debug: selected channels (first k valid)
-  float* s1_part = nullptr;        // Stage-1 partial sums [P1][2][1024]
-  int* s1_cnt = nullptr;          // [C] Stage-1 row slices reported per slice, zero between tokens
-  float* ypart = nullptr;         // Stage-2 output partials [P][d]
+  float* s1_part = nullptr;       // Stage-1 partial sums [P][2][1024]
+  float* ypart = nullptr;         // Stage-2 partial output rows [P][d]
   unsigned long long* stats = nullptr;  // [3] sum n_x, tokens, sum of selected channels
+  unsigned long long* gbar = nullptr;  // grid-barrier arrival counter of the per-token kernel
   int* err = nullptr;             // device error word
   float* stage_in = nullptr;      // host-path staging [kHostChunkTokens][d]
   float* stage_out = nullptr;
@@ -59,11 +60,14 @@ struct prox_layer {
   int act = 0;           // PROX_ACT_*: gate activation of the GLU
   int stage2_source = 0; // PROX_STAGE2_EXACT or PROX_STAGE2_PROXY_VALUES
   int device = 0, num_sms = 0;
-  // Stage-1 geometry: C column slices, P1 CTAs, at most s1_lmax rows per CTA
-  int C = 0, P1 = 0, s1_lmax = 0;
+  // Per-token kernel: P CTAs (one per SM), token_smem bytes of shared memory.
+  int P = 0;
+  size_t token_smem = 0;
+  // Stage-1 geometry: C column slices, at most s1_lmax rows per CTA, s1_nb
+  // row batches in flight per warp
+  int C = 0, s1_lmax = 0, s1_nb = 4;
   // Stage-2 geometry
-  int P = 0, ring_slots = 0, stage2_groups = 1;
-  size_t stage2_smem = 0, stage1_smem = 0;
+  int ring_slots = 0, stage2_groups = 1;
   // library-owned weights
   uint16_t* wgu = nullptr;   // bf16 [F][2d]: gate column j | up column j
   uint16_t* wd = nullptr;    // bf16 [F][d]
@@ -82,23 +86,26 @@ struct Stage1Taps {
   int32_t* n_x = nullptr;   // their number
   float* s_tilde = nullptr; // signed proxy values act(g~) u~ [F]
 };
-// How Stage 2 obtains its channels.
-struct Stage2Launch {
-  int mode = 1;               // 0: given list `idx`, 1: top-k select, 2: dense, 3: score threshold
-  float tau_s = 0.f;          // mode 3: channels with score >= tau_s
+// One launch of the per-token kernel: which phases run and on what.
+struct TokenLaunch {
+  const float* x = nullptr;
+  float* out = nullptr;         // output row (Stage-2 modes, not select_only)
+  bool stage1 = true;           // Stage 1 runs (threshold, proxies, scores)
+  int mode = 1;                 // -1 Stage 1 only, 0 given list `idx`, 1 top-k, 2 dense, 3 threshold
+  float tau_s = 0.f;            // mode 3: channels with score >= tau_s
   const int32_t* idx = nullptr;
   int k = 0;
-  int32_t* sel_mask = nullptr;  // top-k: 1/0 per channel written here (debug)
-  float* s_sp = nullptr;       // optional act(g) u per listed channel
-  bool proxy_values = false;   // ablation: s~ of Stage 1 instead of the exact s
-  bool select_only = false;    // top-k: stop after selecting
+  int32_t* sel_mask = nullptr;  // top-k / threshold: 1/0 per channel written here (debug)
+  float* s_sp = nullptr;        // optional act(g) u per listed channel
+  bool proxy_values = false;    // ablation: s~ of Stage 1 instead of the exact s
+  bool select_only = false;     // stop after selecting
+  Stage1Taps taps;
+  unsigned long long* phase_ns = nullptr;  // optional phase stamps [P][kPhaseStamps]
 };
 
-cudaError_t launch_stage1(const prox_layer* L, const float* x, const Stage1Taps& taps,
-                          cudaStream_t s, bool pdl);
-cudaError_t launch_stage2(const prox_layer* L, const float* x, const Stage2Launch& m,
-                          cudaStream_t s, bool pdl, bool x_ready);
-cudaError_t launch_reduce(const prox_layer* L, float* out, cudaStream_t s, bool pdl);
+cudaError_t setup_token_kernels();
+cudaError_t launch_barrier_probe(const prox_layer* L, cudaStream_t s);
+cudaError_t launch_token(const prox_layer* L, const TokenLaunch& m, cudaStream_t s, bool pdl);
 
 cudaError_t launch_pack_proxy(const uint16_t* W, int d, int F, uint8_t* codes,
                               uint16_t* scales, cudaStream_t s);
@@ -122,11 +129,12 @@ cudaError_t launch_copy(const void* src, void* dst, size_t bytes, cudaStream_t s
 cudaError_t launch_mask_to_list(const int32_t* mask, int n, int32_t* list, int32_t* count,
                                 cudaStream_t s);
 
-// Stage-1 column slices, CTAs and per-CTA row capacity for a shape on `num_sms` SMs.
-void choose_stage1_grid(int d, int F, int num_sms, int* C, int* P1, int* lmax);
-size_t stage1_smem_bytes(int lmax);
-size_t stage1_part_floats(int P1);
-// Stage-2 ring depth and dynamic shared memory for d_model = d.
-void choose_stage2(int d, int F, int num_sms, int* P, int* slots, int* groups, size_t* smem);
+// Stage-1 column slices, per-CTA row capacity and ring depth for a shape on
+// `num_sms` SMs (one CTA each).
+void choose_stage1_grid(int d, int F, int num_sms, int* C, int* lmax, int* nb);
+size_t stage1_smem_bytes(int lmax, int nb);
+size_t stage1_part_floats(int P);
+// Stage-2 ring depth, consumer groups and shared memory for d_model = d.
+void choose_stage2(int d, int F, int num_sms, int* slots, int* groups, size_t* smem);
 
 }  // namespace prox

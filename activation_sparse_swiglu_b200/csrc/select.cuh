@@ -2,15 +2,13 @@
 // selection"): the k channels of largest proxy score |s~_j|, ties going to the
 // lower channel index.
 //
-// select_cut_cta -- the exact cut, computed by every Stage-2 CTA once all
-// scores of the token are written.  Stage 1 counts the scores in an 8192-bin
-// histogram of their bits 30..18 (the first radix level) and appends each
-// (key, channel) to its bin's bucket (the counter's old value is the slot).
-// The cut is then:
+// select_cut -- the exact cut, computed by every CTA of the per-token kernel
+// once all scores of the token are written, from the token's scores held in
+// the CTA's shared memory.  Stage 1 counts the scores in an 8192-bin histogram
+// of their bits 30..18 (the first radix level).  The cut is then:
 //   1. the boundary bin b1 holding the k-th largest key (a scan over the
 //      histogram, 32 bins per thread);
-//   2. the candidates -- the keys of bin b1 -- read from b1's bucket (or, when
-//      the bucket overflowed, gathered by a pass over all scores);
+//   2. the candidates -- the keys of bin b1 -- gathered from the shared keys;
 //   3. the candidates ordered by (key descending, index ascending) --
 //      directly when there are few, by radix select on the remaining key bits
 //      and then the index bits otherwise -- give the k-th largest key T and
@@ -27,32 +25,46 @@ constexpr int kSelectDirect = 768;   // candidates ranked directly (O(n^2))
 constexpr int kSelectWorkers = 256;  // threads that scan
 static_assert(kScoreBins == kSelectWorkers * 32, "32 histogram bins per worker");
 
-// Shared scratch of select_cut_cta (16-byte aligned).
-struct SelectScratch {
-  uint32_t h[kScoreBins];          // the histogram, then the finer radix levels
+// Shared scratch of select_cut; the keys of all channels follow it.
+struct alignas(16) SelectScratch {
+  uint32_t h[1024];                // the finer radix levels
   uint32_t ck[kSelectCand];        // candidate keys
   int32_t ci[kSelectCand];         // candidate channels
   unsigned long long c64[kSelectDirect];
-  int scan[33];
+  int scan[36];
   int misc[16];
 };
+
+// Bytes of the selection's shared memory for d_ff = F: the scratch, then the
+// keys [F].
+__host__ __device__ constexpr size_t select_smem_bytes(int F) {
+  return ((sizeof(SelectScratch) + 15) & ~(size_t)15) + (size_t)F * 4;
+}
+__device__ __forceinline__ uint32_t* select_keys(SelectScratch& sc) {
+  return reinterpret_cast<uint32_t*>(reinterpret_cast<unsigned char*>(&sc) +
+                                     ((sizeof(SelectScratch) + 15) & ~(size_t)15));
+}
 
 struct TopkCut {
   uint32_t T;   // key of the k-th largest score
   int tie_cut;  // keys equal to T are selected up to this channel
 };
 
+__device__ __forceinline__ bool selected(uint32_t key, int e, const TopkCut& cut) {
+  return key > cut.T || (key == cut.T && e <= cut.tie_cut);
+}
+
 // Over the candidate keys (bin b1): the gathered list, or -- when it
-// overflowed -- every key of the scores in bin b1 (worker threads).
+// overflowed -- every key of bin b1 in the shared keys (worker threads).
 template <typename Fn>
-__device__ __forceinline__ void for_each_cand(const float* scores, int F, bool listed, int n,
+__device__ __forceinline__ void for_each_cand(const uint32_t* sk, int F, bool listed, int n,
                                               const SelectScratch& sc, uint32_t b1, Fn fn) {
   if (threadIdx.x >= kSelectWorkers) return;
   if (listed) {
     for (int i = threadIdx.x; i < n; i += kSelectWorkers) fn(sc.ck[i], sc.ci[i]);
   } else {
     for (int e = threadIdx.x; e < F; e += kSelectWorkers) {
-      const uint32_t key = __float_as_uint(__ldcg(scores + e));
+      const uint32_t key = sk[e];
       if ((key >> kScoreShift) == b1) fn(key, e);
     }
   }
@@ -63,40 +75,29 @@ __device__ __forceinline__ uint32_t key_of(const uint4 (&kb)[8], int j) {
   return (j & 3) == 0 ? v.x : (j & 3) == 1 ? v.y : (j & 3) == 2 ? v.z : v.w;
 }
 
-// Every thread of the CTA calls it (blockDim.x >= 256).
-__device__ TopkCut select_cut_cta(const float* scores, const uint32_t* hist, const uint2* bucket,
-                                  int F, int k, SelectScratch& sc) {
+// Every thread of the CTA calls it (blockDim.x >= 256); sk holds the keys of
+// all F channels.
+__device__ TopkCut select_cut(const uint32_t* hist, const uint32_t* sk, int F, int k,
+                              SelectScratch& sc) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const bool worker = tid < kSelectWorkers;
 
-  // the histogram, coalesced, into shared memory; 16-byte chunk i stored at
-  // i ^ (i >> 3) & 7 so that a thread reading eight consecutive chunks meets
-  // no bank conflicts with its neighbours
-  if (worker) {
-#pragma unroll
-    for (int j = 0; j < kScoreBins / 4 / kSelectWorkers; ++j) {
-      const int i = (warp * (kScoreBins / 4 / kSelectWorkers) + j) * 32 + lane;
-      reinterpret_cast<uint4*>(sc.h)[i ^ ((i >> 3) & 7)] =
-          __ldcg(reinterpret_cast<const uint4*>(hist) + i);
-    }
-  }
-  __syncthreads();
-
-  // 1. boundary bin: worker t holds bins [32q, 32q+32), q = 255 - t, so an
-  // exclusive scan over threads counts the keys in higher bins
+  // 1. boundary bin: worker t holds bins [32q, 32q+32), q = 255 - t, read
+  // straight from the histogram in global memory; an exclusive scan over
+  // threads counts the keys in higher bins
   {
     const int q = kSelectWorkers - 1 - tid;
     uint4 hv[8];
     int own = 0;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      hv[j] = worker ? reinterpret_cast<const uint4*>(sc.h)[(8 * q + j) ^ (q & 7)]
+      hv[j] = worker ? __ldcg(reinterpret_cast<const uint4*>(hist) + 8 * q + j)
                      : make_uint4(0u, 0u, 0u, 0u);
       own += (int)(hv[j].x + hv[j].y + hv[j].z + hv[j].w);
     }
     int total;
     const int above = block_exclusive_scan(own, sc.scan, &total);
-    if (tid == 0) sc.misc[3] = 0;  // candidates gathered (pass over the scores)
+    if (tid == 0) sc.misc[3] = 0;  // candidates gathered
     if (worker && above < k && above + own >= k) {
       int run = above;
 #pragma unroll
@@ -118,19 +119,15 @@ __device__ TopkCut select_cut_cta(const float* scores, const uint32_t* hist, con
 
   // 2. the candidates
   const bool listed = n1 <= kSelectCand;
-  if (n1 <= kBucketCap) {
-    for (int i = tid; i < n1; i += blockDim.x) {
-      const uint2 kc = __ldcg(bucket + (size_t)b1 * kBucketCap + i);
-      sc.ck[i] = kc.x;
-      sc.ci[i] = (int)kc.y;
-    }
-  } else if (listed) {
-    for (int e = tid; e < F && worker; e += kSelectWorkers) {
-      const uint32_t key = __float_as_uint(__ldcg(scores + e));
+  if (listed) {
+    for (int e = tid; e < F; e += blockDim.x) {
+      const uint32_t key = sk[e];
       if ((key >> kScoreShift) == b1) {
         const int slot = atomicAdd(&sc.misc[3], 1);
-        sc.ck[slot] = key;
-        sc.ci[slot] = e;
+        if (slot < kSelectCand) {
+          sc.ck[slot] = key;
+          sc.ci[slot] = e;
+        }
       }
     }
   }
@@ -171,7 +168,7 @@ __device__ TopkCut select_cut_cta(const float* scores, const uint32_t* hist, con
     for (int i = tid; i < 1024; i += blockDim.x) h[i] = 0u;
     __syncthreads();
     // level 2: key bits 17..8
-    for_each_cand(scores, F, listed, n1, sc, b1,
+    for_each_cand(sk, F, listed, n1, sc, b1,
                   [&](uint32_t kk, int) { atomicAdd(&h[(kk >> 8) & 0x3FFu], 1u); });
     __syncthreads();
     if (warp == 0) {
@@ -187,7 +184,7 @@ __device__ TopkCut select_cut_cta(const float* scores, const uint32_t* hist, con
     for (int i = tid; i < 1024; i += blockDim.x) h[i] = 0u;
     __syncthreads();
     // level 3: key bits 7..0
-    for_each_cand(scores, F, listed, n1, sc, b1, [&](uint32_t kk, int) {
+    for_each_cand(sk, F, listed, n1, sc, b1, [&](uint32_t kk, int) {
       if ((kk >> 8) == p2) atomicAdd(&h[kk & 0xFFu], 1u);
     });
     __syncthreads();
@@ -209,7 +206,7 @@ __device__ TopkCut select_cut_cta(const float* scores, const uint32_t* hist, con
     if (k_eq < n_eq) {
       for (int i = tid; i < 1024; i += blockDim.x) h[i] = 0u;
       __syncthreads();
-      for_each_cand(scores, F, listed, n1, sc, b1, [&](uint32_t kk, int ix) {
+      for_each_cand(sk, F, listed, n1, sc, b1, [&](uint32_t kk, int ix) {
         if (kk == T) atomicAdd(&h[(ix >> 7) & 0xFFu], 1u);
       });
       __syncthreads();
@@ -225,7 +222,7 @@ __device__ TopkCut select_cut_cta(const float* scores, const uint32_t* hist, con
       const int hi7 = sc.misc[10];
       for (int i = tid; i < 1024; i += blockDim.x) h[i] = 0u;
       __syncthreads();
-      for_each_cand(scores, F, listed, n1, sc, b1, [&](uint32_t kk, int ix) {
+      for_each_cand(sk, F, listed, n1, sc, b1, [&](uint32_t kk, int ix) {
         if (kk == T && (ix >> 7) == hi7) atomicAdd(&h[ix & 0x7F], 1u);
       });
       __syncthreads();
@@ -243,10 +240,6 @@ __device__ TopkCut select_cut_cta(const float* scores, const uint32_t* hist, con
   cut.tie_cut = sc.misc[12];
   __syncthreads();  // the scratch may be reused after return
   return cut;
-}
-
-__device__ __forceinline__ bool selected(uint32_t key, int e, const TopkCut& cut) {
-  return key > cut.T || (key == cut.T && e <= cut.tie_cut);
 }
 
 }  // namespace prox

@@ -1,0 +1,353 @@
+// Stage 2 of the Prox decode step (Prox §4.1 "Stage 2: exact sparse
+// computation"; §4.3 fused output-sparse gate/up kernel and input-sparse
+// down GEMV), and the dense SwiGLU baseline (Prox §2.1), which is the same
+// phase with every channel kept.  Second phase of the fused per-token kernel
+// (token.cu).
+//
+// Every CTA loads the token's scores into shared memory, finds the exact top-k
+// cut of the token (select.cuh: T and the tie cut) or applies the score
+// threshold, ranks the selected channels in ascending channel order and takes
+// the ranks [n_sel c / P, n_sel (c + 1) / P): every CTA streams the same
+// number of channels (to one), whatever the mask looks like.  A given list is
+// split by list position the same way, and the dense baseline splits all
+// channels.  Producer lanes stream, with 1-D bulk async copies (TMA engine)
+// into a ring of slots, first the gate/up channel records of the CTA's
+// channels (gate column then up column, d_model bf16 each: one copy per
+// channel), then their W_down rows (two rows per slot).  The consumer warps
+// take every ring item in order (so each mbarrier wait is for the phase right
+// after one the waiting thread has already seen complete):
+//   phase A: for each channel every warp of the owning group forms partial
+//            dot products of its share of the column with the full x (x kept
+//            in registers; fp32, packed f32x2 FMAs, warp-shuffle reduction)
+//            and parks them in shared memory; after the last channel the
+//            partials are summed in a fixed order into g = x . W_gate[:, j],
+//            u = x . W_up[:, j] and s_j = act(g) u (the A3 ablation skips the
+//            gate/up records and takes s_j = s~_j from Stage 1);
+//   phase B: the warps accumulate y_part += s_j W_down[j, :] for the CTA's
+//            channels, each thread owning 8-column groups of the output.
+// The CTA's fp32 partial row goes to global memory; the kernel adds the
+// partial rows in a fixed order after a grid barrier.
+#pragma once
+#include "select.cuh"
+#include "token_args.cuh"
+
+namespace prox {
+namespace s2 {
+
+constexpr int NCW = kStage2Consumers;
+
+// Layout of Stage 2's shared memory (bytes from the start): full and empty
+// barriers [slots], s_val, s_idx [max_rec], s_pg, s_pu [max_rec][NCW], then
+// the ring, 128-byte aligned (the selection's scratch and keys use the ring's
+// bytes before the ring starts).
+__host__ __device__ constexpr size_t ring_offset(int slots, int max_rec) {
+  return ((size_t)slots * 16 + (size_t)max_rec * (8 + 8 * NCW) + 127) & ~(size_t)127;
+}
+
+// Selects the CTA's channels, streams them and writes the CTA's partial output
+// row to a.ypart (not in select_only mode).  Every thread calls it.  MAXM =
+// ceil(d_model / (8 * 32 * warps per group)): 8-element chunks per lane and
+// column.
+template <int MAXM>
+__device__ void run(const TokenArgs& a, unsigned char* smem, bool* dead) {
+  const int d = a.d, slots = a.slots;
+  const uint32_t col_bytes = 2u * (uint32_t)d;     // one bf16 column / row
+  const uint32_t slot_bytes = 2u * col_bytes;      // a gate/up record, or two W_down rows
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int P = gridDim.x, cta = blockIdx.x;
+
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+  uint64_t* empty = full + slots;
+  float* s_val = reinterpret_cast<float*>(empty + slots);        // [max_rec]
+  int* s_idx = reinterpret_cast<int*>(s_val + a.max_rec);        // [max_rec]
+  float* s_pg = reinterpret_cast<float*>(s_idx + a.max_rec);     // [max_rec][NCW]
+  float* s_pu = s_pg + (size_t)a.max_rec * NCW;                  // [max_rec][NCW]
+  unsigned char* ring = smem + ring_offset(slots, a.max_rec);
+
+  // Consumer warps form NG groups of WPG; a group takes whole ring items, warp
+  // wi of a group the elements [wi*qd, (wi+1)*qd) of each column / row
+  // (qd = d / WPG), lane chunks e8 = m*32 + lane of 8 elements.
+  const int NG = a.groups, WPG = NCW / NG, qd = d / WPG;
+  const int grp = warp / WPG, wi = warp % WPG;
+  auto elem = [&](int m) { return wi * qd + (m * 32 + lane) * 8; };
+  auto elem_ok = [&](int m) { return (m * 32 + lane) * 8 < qd; };
+
+  // The CTA's channels: ranks [r0, r0 + n) of the selection (ascending channel
+  // order), of the list (list order) or of all channels (dense).
+  int r0 = 0, n = 0;
+  if (a.mode == kModeTopK || a.mode == kModeThreshold) {
+    SelectScratch& sc = *reinterpret_cast<SelectScratch*>(ring);
+    uint32_t* sk = select_keys(sc);
+    {
+      // every load in flight before the first store (F <= 32768: at most two rounds)
+      constexpr int LU = 8;
+      const int n4 = a.F >> 2;
+      for (int e0 = tid; e0 < n4; e0 += LU * (int)blockDim.x) {
+        uint4 v[LU];
+#pragma unroll
+        for (int u = 0; u < LU; ++u) {
+          const int e = e0 + u * (int)blockDim.x;
+          v[u] = e < n4 ? __ldcg(reinterpret_cast<const uint4*>(a.scores) + e) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < LU; ++u) {
+          const int e = e0 + u * (int)blockDim.x;
+          if (e < n4) reinterpret_cast<uint4*>(sk)[e] = v[u];
+        }
+      }
+    }
+    __syncthreads();
+    TopkCut cut;
+    if (a.mode == kModeTopK) {
+      cut = select_cut(a.hist, sk, a.F, a.k, sc);
+    } else {
+      // Prox §4.1: score >= tau_s, i.e. key >= bits(tau_s) with every tie kept
+      cut.T = __float_as_uint(a.tau_s);
+      cut.tie_cut = a.F;
+    }
+    // thread t ranks the channels [t*per, (t+1)*per)
+    const int per = (a.F + blockDim.x - 1) / blockDim.x;
+    const int j0 = min(tid * per, a.F), j1 = min(j0 + per, a.F);
+    int cnt = 0;
+    for (int j = j0; j < j1; ++j) cnt += selected(sk[j], j, cut) ? 1 : 0;
+    int total;
+    int r = block_exclusive_scan(cnt, sc.scan, &total);
+    r0 = (int)(((long long)total * cta) / P);
+    n = (int)(((long long)total * (cta + 1)) / P) - r0;
+    for (int j = j0; j < j1; ++j) {
+      if (selected(sk[j], j, cut)) {
+        if (r >= r0 && r < r0 + n) s_idx[r - r0] = j;
+        ++r;
+      }
+    }
+    if (a.sel_mask) {
+      const int m0 = (int)(((long long)a.F * cta) / P), m1 = (int)(((long long)a.F * (cta + 1)) / P);
+      for (int j = m0 + tid; j < m1; j += blockDim.x) a.sel_mask[j] = selected(sk[j], j, cut) ? 1 : 0;
+    }
+    if (tid == 0 && cta == 0 && a.stats && !a.select_only) {
+      atomicAdd(a.stats + 1, 1ull);
+      atomicAdd(a.stats + 2, (unsigned long long)total);
+    }
+  } else {
+    // list positions, or channels, [k c / P, k (c + 1) / P)
+    const int k = a.mode == kModeDense ? a.F : a.k;
+    r0 = (int)(((long long)k * cta) / P);
+    n = (int)(((long long)k * (cta + 1)) / P) - r0;
+    for (int i = tid; i < n; i += blockDim.x) {
+      if (a.mode == kModeList) {
+        int j = __ldcg(a.idx + r0 + i);
+        if (j < 0 || j >= a.F) {
+          atomicOr(a.err, PROX_DEVERR_MASK_INDEX);
+          j = 0;
+        }
+        s_idx[i] = j;
+      } else {
+        s_idx[i] = r0 + i;
+      }
+    }
+  }
+  stamp(a.ts, 4);
+  if (a.select_only) return;
+
+  // The ring and barriers take over bytes that the select (and Stage 1) wrote
+  // through the generic proxy: order those writes before the bulk copies.
+  fence_proxy_async_smem();
+  __syncthreads();
+  if (tid == 0) {
+    for (int s = 0; s < slots; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], NCW / NG);
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+  stamp(a.ts, 11);
+  if (a.ts && tid == 0) a.ts[(size_t)cta * kPhaseStamps + 13] = (unsigned long long)n;
+
+  // Ring items: channel records q < n (gate column | up column), then W_down
+  // row pairs (rows 2p, 2p+1).  Group g takes records g, g+NG, ... and pairs
+  // g, g+NG, ...; its items, records first, use the group's own SPG slots
+  // [g*SPG, (g+1)*SPG) round robin, so every slot's waiter is one group that
+  // takes its uses in order.  Producer lane g fills group g's slots.
+  const int nB = (n + 1) >> 1;
+  const int SPG = slots / NG;
+  auto group_items = [&](int g, int cnt) { return cnt > g ? (cnt - g + NG - 1) / NG : 0; };
+  float* out_row = a.ypart + (size_t)cta * d;
+  if (warp == NCW) {
+    // ---------------- producer lanes 0..NG-1 ----------------
+    if (lane < NG) {
+      const int g = lane;
+      bool pdead = *dead;
+      const uint64_t pol = l2_policy_evict_first();
+      const int nA_g = a.proxy_values ? 0 : group_items(g, n), nB_g = group_items(g, nB);
+      const int tot_g = nA_g + nB_g;
+      for (int li = 0; li < tot_g; ++li) {
+        const int slot = g * SPG + li % SPG, use = li / SPG;
+        if (use > 0) mbar_wait(&empty[slot], (uint32_t)((use - 1) & 1), a.err, &pdead);
+        unsigned char* dst = ring + (size_t)slot * slot_bytes;
+        if (li < nA_g) {
+          const int r = g + li * NG;
+          mbar_arrive_expect_tx(&full[slot], slot_bytes);
+          bulk_copy_g2s(dst, a.wgu + (size_t)s_idx[r] * 2 * (size_t)d, slot_bytes, &full[slot], pol);
+        } else {
+          const int r0 = 2 * (g + (li - nA_g) * NG);
+          const int nr = r0 + 1 < n ? 2 : 1;
+          mbar_arrive_expect_tx(&full[slot], (uint32_t)nr * col_bytes);
+          bulk_copy_g2s(dst, a.wd + (size_t)s_idx[r0] * (size_t)d, col_bytes, &full[slot], pol);
+          if (nr == 2)
+            bulk_copy_g2s(dst + col_bytes, a.wd + (size_t)s_idx[r0 + 1] * (size_t)d, col_bytes,
+                          &full[slot], pol);
+        }
+      }
+      // Every issued copy must land before this CTA's shared memory is reused:
+      // wait for the last use of each slot of the group.
+      bool fdead = false;
+      for (int j = 0; j < SPG && j < tot_g; ++j) {
+        const int last = j + ((tot_g - 1 - j) / SPG) * SPG;  // last li with li % SPG == j
+        mbar_wait(&full[g * SPG + j], (uint32_t)((last / SPG) & 1), a.err, &fdead);
+      }
+    }
+  } else {
+    // this thread's x elements, kept in registers
+    float4 xr[MAXM][2];
+#pragma unroll
+    for (int m = 0; m < MAXM; ++m) {
+      const int e = elem(m);
+      xr[m][0] = elem_ok(m) ? __ldg(reinterpret_cast<const float4*>(a.x + e)) : make_float4(0, 0, 0, 0);
+      xr[m][1] = elem_ok(m) ? __ldg(reinterpret_cast<const float4*>(a.x + e + 4)) : make_float4(0, 0, 0, 0);
+    }
+    bool cdead = *dead;
+    // ---------------- phase A: gate/up partial dot products ----------------
+    // The warp's share of an item goes into registers, the slot goes back to the
+    // producer, then the FMAs.
+    const int nA_g = a.proxy_values ? 0 : group_items(grp, n);
+    for (int li = 0; li < nA_g; ++li) {
+      const int r = grp + li * NG;
+      const int slot = grp * SPG + li % SPG;
+      mbar_wait(&full[slot], (uint32_t)((li / SPG) & 1), a.err, &cdead);
+      const unsigned char* wg = ring + (size_t)slot * slot_bytes;
+      const unsigned char* wu = wg + col_bytes;
+      uint4 gv[MAXM], uv[MAXM];
+#pragma unroll
+      for (int m = 0; m < MAXM; ++m) {
+        const int e = elem(m);
+        gv[m] = elem_ok(m) ? *reinterpret_cast<const uint4*>(wg + (size_t)e * 2) : make_uint4(0u, 0u, 0u, 0u);
+        uv[m] = elem_ok(m) ? *reinterpret_cast<const uint4*>(wu + (size_t)e * 2) : make_uint4(0u, 0u, 0u, 0u);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[slot], 1);
+      float2 ag0 = make_float2(0.f, 0.f), ag1 = ag0, au0 = ag0, au1 = ag0;
+#pragma unroll
+      for (int m = 0; m < MAXM; ++m) {
+        const float4 xa = xr[m][0], xb = xr[m][1];
+        ag0 = __ffma2_rn(bf16x2_to_f2(gv[m].x), make_float2(xa.x, xa.y), ag0);
+        au0 = __ffma2_rn(bf16x2_to_f2(uv[m].x), make_float2(xa.x, xa.y), au0);
+        ag1 = __ffma2_rn(bf16x2_to_f2(gv[m].y), make_float2(xa.z, xa.w), ag1);
+        au1 = __ffma2_rn(bf16x2_to_f2(uv[m].y), make_float2(xa.z, xa.w), au1);
+        ag0 = __ffma2_rn(bf16x2_to_f2(gv[m].z), make_float2(xb.x, xb.y), ag0);
+        au0 = __ffma2_rn(bf16x2_to_f2(uv[m].z), make_float2(xb.x, xb.y), au0);
+        ag1 = __ffma2_rn(bf16x2_to_f2(gv[m].w), make_float2(xb.z, xb.w), ag1);
+        au1 = __ffma2_rn(bf16x2_to_f2(uv[m].w), make_float2(xb.z, xb.w), au1);
+      }
+      float g = (ag0.x + ag0.y) + (ag1.x + ag1.y);
+      float u = (au0.x + au0.y) + (au1.x + au1.y);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        g += __shfl_xor_sync(0xffffffffu, g, o);
+        u += __shfl_xor_sync(0xffffffffu, u, o);
+      }
+      if (lane == 0) {
+        s_pg[r * NCW + wi] = g;
+        s_pu[r * NCW + wi] = u;
+      }
+    }
+    asm volatile("bar.sync 1, %0;" ::"r"(NCW * 32) : "memory");
+    for (int r = tid; r < n; r += NCW * 32) {
+      float sv;
+      if (a.proxy_values) {
+        sv = __ldcg(a.s_tilde_src + s_idx[r]);
+      } else {
+        float g = 0.f, u = 0.f;
+        for (int w = 0; w < WPG; ++w) {
+          g += s_pg[r * NCW + w];
+          u += s_pu[r * NCW + w];
+        }
+        sv = act_f32(g, a.act) * u;
+      }
+      s_val[r] = sv;
+      if (a.s_sp) a.s_sp[r0 + r] = sv;
+    }
+    asm volatile("bar.sync 1, %0;" ::"r"(NCW * 32) : "memory");
+    stamp(a.ts, 12);
+
+    // ---------------- phase B: y_part = sum_t s_t W_down[j_t, :] ----------------
+    // The group's row pairs; warp wi accumulates its columns [wi*qd, (wi+1)*qd).
+    float2 acc[MAXM * 4];
+#pragma unroll
+    for (int i = 0; i < MAXM * 4; ++i) acc[i] = make_float2(0.f, 0.f);
+    const int nB_g = group_items(grp, nB);
+    for (int lb = 0; lb < nB_g; ++lb) {
+      const int li = nA_g + lb;
+      const int p = grp + lb * NG;  // row pair
+      const int slot = grp * SPG + li % SPG;
+      mbar_wait(&full[slot], (uint32_t)((li / SPG) & 1), a.err, &cdead);
+      const unsigned char* w = ring + (size_t)slot * slot_bytes;
+      const bool two = 2 * p + 1 < n;
+      uint4 wv[2][MAXM];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+#pragma unroll
+        for (int m = 0; m < MAXM; ++m) {
+          const int e = elem(m);
+          wv[h][m] = (elem_ok(m) && (h == 0 || two))
+                         ? *reinterpret_cast<const uint4*>(w + h * col_bytes + (size_t)e * 2)
+                         : make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[slot], 1);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const float sv = (h == 0 || two) ? s_val[2 * p + h] : 0.f;
+        const float2 s2 = make_float2(sv, sv);
+#pragma unroll
+        for (int m = 0; m < MAXM; ++m) {
+          const uint4 w4 = wv[h][m];
+          acc[4 * m + 0] = __ffma2_rn(bf16x2_to_f2(w4.x), s2, acc[4 * m + 0]);
+          acc[4 * m + 1] = __ffma2_rn(bf16x2_to_f2(w4.y), s2, acc[4 * m + 1]);
+          acc[4 * m + 2] = __ffma2_rn(bf16x2_to_f2(w4.z), s2, acc[4 * m + 2]);
+          acc[4 * m + 3] = __ffma2_rn(bf16x2_to_f2(w4.w), s2, acc[4 * m + 3]);
+        }
+      }
+    }
+    // The groups' partial rows are added in group order (deterministic).  Every
+    // copy has landed (each item was waited for), so the ring holds them.
+    asm volatile("bar.sync 1, %0;" ::"r"(NCW * 32) : "memory");
+    float* s_y = reinterpret_cast<float*>(ring);  // [NG][d]
+#pragma unroll
+    for (int m = 0; m < MAXM; ++m) {
+      if (elem_ok(m)) {
+        float* dst = s_y + (size_t)grp * d + elem(m);
+        *reinterpret_cast<float4*>(dst) =
+            make_float4(acc[4 * m].x, acc[4 * m].y, acc[4 * m + 1].x, acc[4 * m + 1].y);
+        *reinterpret_cast<float4*>(dst + 4) =
+            make_float4(acc[4 * m + 2].x, acc[4 * m + 2].y, acc[4 * m + 3].x, acc[4 * m + 3].y);
+      }
+    }
+    asm volatile("bar.sync 1, %0;" ::"r"(NCW * 32) : "memory");
+    for (int e = tid * 4; e < d; e += NCW * 32 * 4) {
+      float4 v = *reinterpret_cast<const float4*>(s_y + e);
+      for (int g = 1; g < NG; ++g) {
+        const float4 t = *reinterpret_cast<const float4*>(s_y + (size_t)g * d + e);
+        v.x += t.x;
+        v.y += t.y;
+        v.z += t.z;
+        v.w += t.w;
+      }
+      *reinterpret_cast<float4*>(out_row + e) = v;
+    }
+  }
+}
+
+}  // namespace s2
+}  // namespace prox

@@ -134,19 +134,29 @@ PROX_API prox_status prox_pack_proxy(const uint16_t* W, int d_model, int d_ff, i
 PROX_API prox_status prox_calibrate_thresholds(const float* X_cal, int n_tok, int d_model, float s1,
                                       float* tau_host, void* stream);
 
-/* The calibration above without any allocation (the Prox pages have no
- * counterpart: this is an engineering variant for allocation-free hosts and
- * CUDA graphs).  Same quantile, same exactness.  Its scratch is a fixed
- * static __device__ array of 2056 uint32 (8 KB) per device, found with
- * cudaGetSymbolAddress on the first call made on that device (with it
- * current): make that first call before any stream capture.  Every call
- * zeroes the histogram it needs before counting, so nothing has to start at
- * zero.  Calls that overlap on one device (other streams, other threads)
- * share that scratch and race: serialise them.  X_cal: fp32 [n_tok, d_model]
- * on the current device, 16-byte aligned; n_tok * d_model must stay below
- * 2^31 (the counters are 32-bit), else PROX_EINVAL with a message.  tau_dev:
- * one float on the device, written in stream order (nothing synchronises).
- * Allocates nothing: no cudaMalloc, cudaMallocAsync or cudaFree. */
+/* The calibration above without any allocation.  The Prox pages have no
+ * counterpart: this entry point exists for callers that cannot allocate
+ * device memory at the moment they calibrate -- a host process whose device
+ * memory belongs to another allocator (a serving framework that has reserved
+ * it all for its own pool), or a latency-critical path where cudaMalloc's
+ * implicit device-wide synchronisation and cudaMallocAsync's pool growth are
+ * not acceptable.  Same quantile, same exactness as
+ * prox_calibrate_thresholds.  Its scratch is a fixed static __device__ array
+ * of 2056 uint32 (8 KB) per device, which every device that loads the
+ * library holds until the process exits.  Set-up: the first call made on a
+ * device (with that device current) looks up the array's device address with
+ * cudaGetSymbolAddress and caches it per device and CUDA context; make that
+ * first call before any stream capture.  A device reset (cudaDeviceReset) or
+ * a new primary context makes the next call look the address up again.
+ * Every call zeroes the histogram it needs before counting, so nothing has to
+ * start at zero.  Calls that overlap on one device (other streams, other
+ * threads) share that scratch and race: serialise them.  X_cal: fp32
+ * [n_tok, d_model] in device memory of the current device, 16-byte aligned;
+ * n_tok * d_model must stay below 2^31 (the counters are 32-bit), else
+ * PROX_EINVAL with a message.  tau_dev: one float in device memory of the
+ * current device, written in stream order (nothing synchronises).  A pointer
+ * to host memory or to another device gives PROX_EINVAL.  Allocates nothing:
+ * no cudaMalloc, cudaMallocAsync or cudaFree. */
 PROX_API prox_status prox_calibrate_thresholds_noalloc(const float* X_cal, int n_tok, int d_model,
                                                        float s1, float* tau_dev, void* stream);
 
@@ -259,7 +269,9 @@ PROX_API prox_status prox_runtime_sparsity(int64_t sum_nx, int64_t sum_sel, int6
  *            full x (or s~_j in PROX_STAGE2_PROXY_VALUES mode);
  *            out = sum_j s_j W_down[j, :].
  * x, out: fp32 [B, d_model] (out may not alias x).  B <= max_batch.
- * Three kernels per token, chained with programmatic dependent launch. */
+ * One cooperative kernel per token on every SM (Stage 1, grid barrier, the
+ * cut and Stage 2, grid barrier, the output sum), each launch
+ * programmatically dependent on the previous one in the stream. */
 PROX_API prox_status prox_ffn_forward(const prox_layer* layer, const float* x, float* out, int B,
                              void* stream);
 
@@ -275,12 +287,19 @@ PROX_API prox_status prox_dense_ffn(const prox_layer* layer, const float* x, flo
 PROX_API prox_status prox_ffn_forward_host(prox_layer* layer, const float* x_host, float* out_host,
                                   int n_tok, void* stream);
 
-/* prox_ffn_forward for one token with cudaEvent_t events[4] (passed as void*)
- * recorded before Stage 1, between Stage 1 and Stage 2, between Stage 2 and
- * the output reduction, and after it; the kernels are then serialised
- * (no programmatic overlap) so each interval is one kernel's duration. */
+/* prox_ffn_forward for one token with cudaEvent_t events_host[2] (passed as
+ * void*) recorded right before and right after the token's kernel, which is
+ * launched without programmatic overlap so the interval is its duration.
+ * phase_ns (device, may be NULL): uint64 [stage1_ctas][16] receiving, per CTA,
+ * the GPU global timer (ns) at: 0 kernel entry, 1 the previous kernel of the
+ * stream complete, 2 Stage 1 done, 3 all scores visible (first grid barrier),
+ * 4 channels selected, 5 partial output row written, 6 second grid barrier,
+ * 7 output written, 8 kept rows compacted, 9 Stage-1 row loop done, 10 Stage-1
+ * partials written, 11 Stage-2 ring set up, 12 gate/up phase done; slot 13
+ * holds the CTA's number of selected channels; 14 and 15 are unused. */
 PROX_API prox_status prox_ffn_forward_profiled(const prox_layer* layer, const float* x, float* out,
-                                      void* const* events_host, void* stream);
+                                               void* const* events_host, uint64_t* phase_ns,
+                                               void* stream);
 
 /* ------------------------------------------------------------------------
  * Test taps: the same kernels, exposing intermediate results
@@ -319,6 +338,15 @@ PROX_API prox_status prox_forward_with_mask(prox_layer* layer, const float* x, c
  * library frees whatever it had allocated; 0 cancels a pending injection.
  * Process-wide; nothing fails on the device.  nth < 0 gives PROX_EINVAL. */
 PROX_API prox_status prox_debug_fail_alloc(int nth);
+
+/* Test-only exercise of the bounded device waits, with no fault: launches one
+ * CTA that arrives at the layer's grid barrier and waits for an arrival that
+ * never comes.  The wait runs out after its bound (2e8 SM cycles, about 0.1 s),
+ * sets PROX_DEVERR_WAIT_TIMEOUT in the layer's error word and the kernel
+ * returns.  prox_layer_error then reports the bit and, as after any timeout,
+ * resets the barrier, the Stage-1 counters and the histogram so that the next
+ * token runs clean.  Stream-ordered. */
+PROX_API prox_status prox_debug_wait_timeout(prox_layer* layer, void* stream);
 
 /* ------------------------------------------------------------------------
  * Harness kernels

@@ -156,3 +156,24 @@ def test_binding_refuses_short_or_host_buffers():
         prox.copy(torch.empty(16), torch.empty(16))
     with pytest.raises(TypeError):
         prox.rmsnorm(torch.empty(4, 8))
+
+
+def test_noalloc_binding_checks_the_device(monkeypatch):
+    """The binding refuses tensors that are not on the current CUDA device
+    before the allocation-free calibration runs (checked with stand-ins for
+    tensors, no GPU needed)."""
+    import types
+
+    import torch
+
+    import activation_sparse_swiglu_b200 as prox
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
+    here = types.SimpleNamespace(device=torch.device("cuda", 0))
+    other = types.SimpleNamespace(device=torch.device("cuda", 1))
+    host = types.SimpleNamespace(device=torch.device("cpu"))
+    prox._on_current_device(x_cal=here, tau=here)
+    for bad in (other, host):
+        with pytest.raises(ValueError, match="current CUDA device"):
+            prox._on_current_device(x_cal=here, tau=bad)
+        with pytest.raises(ValueError, match="current CUDA device"):
+            prox._on_current_device(x_cal=bad, tau=here)

@@ -1,6 +1,8 @@
 """Failure paths on a GPU without any GPU fault: an injected out-of-memory at
 each of the nine device allocations of layer creation comes back as
-PROX_ENOMEM, leaks nothing, and leaves the library usable."""
+PROX_ENOMEM, leaks nothing, and leaves the library usable; a device wait that
+can never complete runs out after its bound, is reported in the layer's error
+word, and the layer recovers."""
 
 import gc
 
@@ -58,6 +60,27 @@ def test_injected_allocation_failure_at_every_site(prox):
         layer = prox.Layer(wg, wu, wd, tau=0.5, k=k)
     finally:
         prox.lib.prox_debug_fail_alloc(0)
+    y = layer.forward(x)
+    torch.cuda.synchronize()
+    assert torch.equal(y, y_ref)
+    assert layer.error_word() == 0
+    layer.close()
+
+
+def test_bounded_wait_runs_out_and_recovers(prox):
+    """A grid-barrier wait that can never complete (the probe expects one more
+    CTA than it launches) runs out after its bound, reports
+    PROX_DEVERR_WAIT_TIMEOUT in the error word, and the layer computes the
+    same output as before once the error word has been read."""
+    lay = synth.make_layer("tiny", n_tokens=2, n_cal=8)
+    wg, wu, wd = (bits_to_bf16(b) for b in (lay.w_gate_bits, lay.w_up_bits, lay.w_down_bits))
+    layer = prox.Layer(wg, wu, wd, tau=0.5, k=lay.config.k())
+    x = torch.from_numpy(lay.x_eval[0]).cuda()
+    y_ref = layer.forward(x).clone()
+    assert layer.error_word() == 0
+    prox.check(prox.lib.prox_debug_wait_timeout(layer.handle, None))
+    torch.cuda.synchronize()
+    assert layer.error_word() & prox.DEVERR_WAIT_TIMEOUT
     y = layer.forward(x)
     torch.cuda.synchronize()
     assert torch.equal(y, y_ref)
