@@ -327,7 +327,7 @@ class Layer:
                          phase_ns: torch.Tensor | None = None, stream=None):
         """One token with its kernel bracketed by 2 torch.cuda.Event(enable_timing=True)
         (no programmatic overlap).  phase_ns: optional int64 CUDA tensor
-        [stage1_ctas, 16] receiving each CTA's phase stamps (GPU global timer, ns;
+        [stage1_ctas, 24] receiving each CTA's phase stamps (GPU global timer, ns;
         slot meanings in include/prox.h)."""
         _dev(x, torch.float32, "x")
         _dev(out, torch.float32, "out")
@@ -337,7 +337,7 @@ class Layer:
             raise ValueError("forward_profiled needs 2 events")
         if phase_ns is not None:
             _dev(phase_ns, torch.int64, "phase_ns")
-            _need(phase_ns, self.info()["stage1_ctas"] * 16, "phase_ns")
+            _need(phase_ns, self.info()["stage1_ctas"] * 24, "phase_ns")
         arr = (ctypes.c_void_p * 2)(*[ctypes.c_void_p(e.cuda_event) for e in events])
         check(lib.prox_ffn_forward_profiled(self.handle, _ptr(x), _ptr(out), arr, _ptr(phase_ns),
                                             _stream(stream)))

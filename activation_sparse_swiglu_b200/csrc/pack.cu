@@ -2,7 +2,10 @@
 //  * pack_proxy_kernel: symmetric INT4 proxy of one [d_model, d_ff] bf16
 //    matrix, groups of 128 input rows per channel, fp16 scales;
 //  * interleave_proxy_kernel: gate and up codes (and scales) interleaved per
-//    32-channel block so one input row of both proxies is one contiguous run;
+//    32-channel block, stored slice-major: the 512-byte column slice s of
+//    input row i (16 blocks: 512 channels of both proxies) sits at
+//    (s * d_model + i) * 512, so the kept rows of one slice are read in
+//    ascending address order;
 //  * gateup_records_kernel: channel-contiguous gate/up records for Stage 2.
 #include "prox_device.cuh"
 #include "prox_internal.h"
@@ -43,8 +46,10 @@ __global__ void pack_proxy_kernel(const uint32_t* __restrict__ W, int F, uint8_t
   }
 }
 
-// pq row i = for each 32-channel block: 16 B gate codes, 16 B up codes.
-// ps[g] = for each block: 32 gate scales, 32 up scales.
+// pq: slice s of row i = for each of its 16 blocks of 32 channels: 16 B gate
+// codes, 16 B up codes, at byte (s * d + i) * 512 (the last slice of a d_ff
+// that is not a multiple of 512 is padded).  ps[g] = for each block: 32 gate
+// scales, 32 up scales.
 __global__ void interleave_proxy_kernel(const uint4* __restrict__ cg, const uint4* __restrict__ cu,
                                         const uint4* __restrict__ sg, const uint4* __restrict__ su,
                                         int d, int F, uint4* __restrict__ pq, uint4* __restrict__ ps) {
@@ -54,9 +59,11 @@ __global__ void interleave_proxy_kernel(const uint4* __restrict__ cg, const uint
   const size_t stride = (size_t)gridDim.x * blockDim.x;
   for (size_t t = (size_t)blockIdx.x * blockDim.x + threadIdx.x; t < n_code + n_scale; t += stride) {
     if (t < n_code) {
-      // block t of the flattened [d][nblk] grid: 16 bytes from each proxy
-      pq[2 * t] = cg[t];
-      pq[2 * t + 1] = cu[t];
+      // block b of row i (t = i * nblk + b): 16 bytes from each proxy
+      const size_t i = t / nblk, b = t % nblk;
+      const size_t o = (((b >> 4) * (size_t)d + i) * 16 + (b & 15)) * 2;
+      pq[o] = cg[t];
+      pq[o + 1] = cu[t];
     } else {
       const size_t u = t - n_code;  // (group, block): 32 halves = 4 uint4 per proxy
       for (int q = 0; q < 4; ++q) {

@@ -151,6 +151,10 @@ prox_status alloc_workspace(prox_layer* L) {
   const size_t o_g = take(F * 4);
   const size_t o_u = take(F * 4);
   const size_t o_hist = take(prox::kScoreBins * 4);
+  const size_t o_chist = take(128 * 4);
+  const size_t o_bucket = take((size_t)prox::kScoreBins * prox::kBucketCap * 8);
+  const size_t o_slist = take(F * 4);
+  const size_t o_scnt = take((size_t)prox::kMaxCtas * 4);
   const size_t o_mask = take(F * 4);
   const size_t o_idx = take(F * 4);
   const size_t o_s1p = take(prox::stage1_part_floats(L->P) * 4);
@@ -172,6 +176,10 @@ prox_status alloc_workspace(prox_layer* L) {
   w.g_dbg = reinterpret_cast<float*>(b + o_g);
   w.u_dbg = reinterpret_cast<float*>(b + o_u);
   w.hist = reinterpret_cast<uint32_t*>(b + o_hist);
+  w.chist = reinterpret_cast<uint32_t*>(b + o_chist);
+  w.bucket = reinterpret_cast<uint2*>(b + o_bucket);
+  w.sel_list = reinterpret_cast<int32_t*>(b + o_slist);
+  w.sel_cnt = reinterpret_cast<int32_t*>(b + o_scnt);
   w.sel_mask = reinterpret_cast<int32_t*>(b + o_mask);
   w.idx_s = reinterpret_cast<int32_t*>(b + o_idx);
   w.s1_part = reinterpret_cast<float*>(b + o_s1p);
@@ -351,6 +359,10 @@ prox_status prox_layer_create(const uint16_t* W_gate, const uint16_t* W_up, cons
     return fail(PROX_EUNSUPPORTED, "%d SMs exceed the %d CTAs the per-token kernel supports", sms,
                 prox::kMaxCtas);
   }
+  if ((d_ff + sms - 1) / sms > 512) {
+    delete L;
+    return fail(PROX_EUNSUPPORTED, "d_ff=%d over %d SMs exceeds 512 channels per CTA", d_ff, sms);
+  }
   L->P = sms;
   prox::choose_stage1_grid(L->d, L->F, sms, &L->C, &L->s1_lmax, &L->s1_nb);
   size_t s2_smem = 0;
@@ -374,7 +386,7 @@ prox_status prox_layer_create(const uint16_t* W_gate, const uint16_t* W_up, cons
   step(prox::setup_token_kernels());
   step(dev_alloc(&L->wgu, 2 * F * d * 2));
   step(dev_alloc(&L->wd, F * d * 2));
-  step(dev_alloc(&L->pq, d * F));
+  step(dev_alloc(&L->pq, (size_t)L->C * d * 512));  // slice-major, last slice padded
   step(dev_alloc(&L->ps, (size_t)L->G * F * 2 * 2));
   step(dev_alloc(&cg, d * F / 2));
   step(dev_alloc(&cu, d * F / 2));
@@ -504,9 +516,10 @@ prox_status prox_layer_error(prox_layer* L, int32_t* word_host, void* stream) {
   PROX_CUDA(cudaStreamSynchronize(s), "cudaStreamSynchronize");
   if (v & PROX_DEVERR_WAIT_TIMEOUT) {
     // A token whose wait ran out may have left the grid-barrier counter and
-    // the histogram mid-way: start the next token clean.
+    // the histograms mid-way: start the next token clean.
     PROX_CUDA(cudaMemsetAsync(L->ws.gbar, 0, 8, s), "reset grid barrier");
     PROX_CUDA(cudaMemsetAsync(L->ws.hist, 0, prox::kScoreBins * 4, s), "reset histogram");
+    PROX_CUDA(cudaMemsetAsync(L->ws.chist, 0, 128 * 4, s), "reset coarse histogram");
     PROX_CUDA(cudaStreamSynchronize(s), "cudaStreamSynchronize");
   }
   *word_host = v;

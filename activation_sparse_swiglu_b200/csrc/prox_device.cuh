@@ -72,6 +72,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// Non-blocking test of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 // Wait for the phase with the given parity to complete, for at most
 // kWaitLimitCycles.  Returns false (after flagging `err` and setting *dead)
 // if it ran out; with *dead already set it returns false at once.
@@ -186,57 +198,6 @@ __device__ __forceinline__ T block_exclusive_scan(T v, T* scratch, T* total) {
   *total = scratch[32];
   __syncthreads();
   return out;
-}
-
-// One warp: among the 32*PER bins of h (counts per bin, larger bin = larger
-// key; lane L covers bins [L*PER, (L+1)*PER), read 4 at a time) find the bin
-// holding the krem-th largest key (1-based).  Returns the bin, the remaining
-// rank inside it and the bin's count.  Works on global (GLOBAL = true, read
-// through L2) or shared memory.
-template <int PER, bool GLOBAL>
-__device__ __forceinline__ void warp_find_bin(const uint32_t* h, int krem, int* bin, int* rem,
-                                              int* count) {
-  const int lane = threadIdx.x & 31;
-  const uint4* hv = reinterpret_cast<const uint4*>(h + lane * PER);
-  auto ld = [&](int q) -> uint4 { return GLOBAL ? __ldcg(hv + q) : hv[q]; };
-  int v = 0;
-#pragma unroll
-  for (int q = 0; q < PER / 4; ++q) {
-    const uint4 t = ld(q);
-    v += (int)(t.x + t.y + t.z + t.w);
-  }
-  int incl = v;  // keys in this lane's bins and in the bins of the lanes above
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int nb = __shfl_down_sync(0xffffffffu, incl, o);
-    if (lane + o < 32) incl += nb;
-  }
-  const int above = incl - v;
-  const bool mine = above < krem && incl >= krem;
-  const int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
-  int my_bin = 0, my_rem = 0, my_cnt = 0;
-  if (mine) {
-    int running = above;
-    bool found = false;
-    for (int q = PER / 4 - 1; q >= 0 && !found; --q) {
-      const uint4 t = ld(q);
-      const uint32_t c4[4] = {t.x, t.y, t.z, t.w};
-#pragma unroll
-      for (int j = 3; j >= 0; --j) {
-        const int hb = (int)c4[j];
-        if (!found && running + hb >= krem) {
-          my_bin = lane * PER + 4 * q + j;
-          my_rem = krem - running;
-          my_cnt = hb;
-          found = true;
-        }
-        running += hb;
-      }
-    }
-  }
-  *bin = __shfl_sync(0xffffffffu, my_bin, src);
-  *rem = __shfl_sync(0xffffffffu, my_rem, src);
-  *count = __shfl_sync(0xffffffffu, my_cnt, src);
 }
 
 }  // namespace prox

@@ -15,13 +15,13 @@ constexpr int kGroup = 128;          // proxy quantisation group (input rows)
 constexpr int kHistBins = 2048;      // calibration radix levels: 11 bits
 constexpr int kScoreShift = 18;      // top-k select, first radix level: score bits [30:18]
 constexpr int kScoreBins = 8192;
+constexpr int kBucketCap = 128;      // (key, channel) entries kept per fine histogram bin
 constexpr int kStage1Warps = 16;     // Stage-1 warps per CTA (one CTA per SM)
-constexpr int kSelectCand = 2048;    // candidate buffer of the select (level-1 bin)
 constexpr int kSelectSlice = 256;    // channels per select CTA (and per rank-offset entry)
 constexpr int kMaxSlices = 160;      // >= d_ff / kSelectSlice + 1
 constexpr int kStage2Consumers = 16;  // Stage-2 consumer warps (+1 producer warp)
 constexpr int kTokenThreads = (kStage2Consumers + 1) * 32;  // threads of the per-token kernel
-constexpr int kPhaseStamps = 16;     // phase stamp slots per CTA of the per-token kernel
+constexpr int kPhaseStamps = 24;     // phase stamp slots per CTA of the per-token kernel
 constexpr int kMaxCtas = 256;        // per-token kernel grid (one CTA per SM) at most
 constexpr size_t kStage2SmemBudget = 208 * 1024;  // Stage-2 ring and tables
 constexpr int kMaxDModel = 16384;
@@ -36,7 +36,11 @@ struct Workspace {
   float* s_tilde = nullptr;       // act(g~) u~ [F], signed (proxy-values Stage 2 only)
   float* g_dbg = nullptr;         // debug g~ [F]
   float* u_dbg = nullptr;         // debug u~ [F]
-  uint32_t* hist = nullptr;       // [kScoreBins] score bits 30..18, zero between tokens
+  uint32_t* hist = nullptr;       // [kScoreBins] scores' bits 30..18, zero between tokens
+  uint32_t* chist = nullptr;      // [128] scores' bits 30..24, zero between tokens
+  uint2* bucket = nullptr;        // [kScoreBins][kBucketCap] (key, channel) per fine bin
+  int32_t* sel_list = nullptr;    // [F] each CTA's selected channels, at its range's start
+  int32_t* sel_cnt = nullptr;     // [kMaxCtas] each CTA's selected count
   int32_t* sel_mask = nullptr;    // [F] debug: 1 where the channel is selected
   int32_t* idx_s = nullptr;       // [F] debug: selected channels (first k valid)
   float* s1_part = nullptr;       // Stage-1 partial sums [P][2][1024]
@@ -71,7 +75,7 @@ struct prox_layer {
   // library-owned weights
   uint16_t* wgu = nullptr;   // bf16 [F][2d]: gate column j | up column j
   uint16_t* wd = nullptr;    // bf16 [F][d]
-  uint8_t* pq = nullptr;     // INT4 codes [d][F], gate/up interleaved per 16 B
+  uint8_t* pq = nullptr;     // INT4 codes [C][d][512 B], gate/up interleaved per 16 B
   uint16_t* ps = nullptr;    // fp16 scales [G][F/32][2][32]
   prox::Workspace ws;
 };

@@ -2,43 +2,52 @@
 // selection"): the k channels of largest proxy score |s~_j|, ties going to the
 // lower channel index.
 //
-// select_cut -- the exact cut, computed by every CTA of the per-token kernel
-// once all scores of the token are written, from the token's scores held in
-// the CTA's shared memory.  Stage 1 counts the scores in an 8192-bin histogram
-// of their bits 30..18 (the first radix level).  The cut is then:
-//   1. the boundary bin b1 holding the k-th largest key (a scan over the
-//      histogram, 32 bins per thread);
-//   2. the candidates -- the keys of bin b1 -- gathered from the shared keys;
-//   3. the candidates ordered by (key descending, index ascending) --
-//      directly when there are few, by radix select on the remaining key bits
-//      and then the index bits otherwise -- give the k-th largest key T and
-//      the tie cut: channel j is selected iff key_j > T, or key_j == T and
-//      j <= tie cut.
-// Scores are non-negative floats, so their bit patterns order like the values.
+// While scoring, every CTA of the per-token kernel counts its channels' keys
+// (the fp32 bit patterns of the scores, which order like the values) in two
+// global histograms, a fine one over bits 30..18 (8192 bins) and a coarse one
+// over bits 30..24 (128 bins, each the sum of 64 fine bins), adding per bin
+// the counts it first gathered in shared memory; the fine bin's old count
+// places the CTA's (key, channel) pairs of that bin in the bin's bucket.  After a grid barrier every CTA finds the exact cut itself,
+// reading only small pieces:
+//   1. the coarse histogram (512 bytes): the coarse bin holding the k-th
+//      largest key;
+//   2. that coarse bin's 64 fine bins: the fine bin b1 holding it and the
+//      rank wanted inside b1;
+//   3. b1's bucket: the candidates, ranked by (key descending, index
+//      ascending), which gives the k-th largest key T and the tie cut:
+//      channel j is selected iff key_j > T, or key_j == T and j <= tie cut.
+// When b1 holds more keys than its bucket (many equal scores) the CTA loads
+// every score and runs a radix select over them instead: a most-significant-
+// digit-first select, 4 bits per level, with per-thread digit counts packed
+// four to a 64-bit word (16 bits each) and summed over the CTA.
 #pragma once
 #include "prox_device.cuh"
 #include "prox_internal.h"
 
 namespace prox {
 
-constexpr int kSelectDirect = 768;   // candidates ranked directly (O(n^2))
-constexpr int kSelectWorkers = 256;  // threads that scan
-static_assert(kScoreBins == kSelectWorkers * 32, "32 histogram bins per worker");
+constexpr int kCoarseShift = 24;     // coarse histogram: key bits 30..24
+constexpr int kCoarseBins = 128;
+static_assert((kScoreBins >> (kCoarseShift - kScoreShift)) == kCoarseBins, "64 fine bins per coarse bin");
+constexpr int kFinePerCoarse = kScoreBins / kCoarseBins;
+constexpr int kOwnMax = 512;         // channels a CTA scores, at most
 
-// Shared scratch of select_cut; the keys of all channels follow it.
+// Shared scratch of the selection.
 struct alignas(16) SelectScratch {
-  uint32_t h[1024];                // the finer radix levels
-  uint32_t ck[kSelectCand];        // candidate keys
-  int32_t ci[kSelectCand];         // candidate channels
-  unsigned long long c64[kSelectDirect];
+  uint32_t own[kOwnMax];           // the keys of the CTA's own channels
+  uint32_t coarse[kCoarseBins];    // the CTA's coarse counts while scoring
+  uint32_t ck[kBucketCap];         // candidate keys
+  int32_t ci[kBucketCap];          // candidate channels
+  unsigned long long wsum[32][4];  // per-warp packed digit counts
   int scan[36];
   int misc[16];
 };
 
-// Bytes of the selection's shared memory for d_ff = F: the scratch, then the
-// keys [F].
+// Bytes of the selection's shared memory for d_ff = F: the scratch, then
+// room for every key (used only when the boundary bin overflows its bucket)
+// or, while scoring, for the CTA's fine histogram.
 __host__ __device__ constexpr size_t select_smem_bytes(int F) {
-  return ((sizeof(SelectScratch) + 15) & ~(size_t)15) + (size_t)F * 4;
+  return ((sizeof(SelectScratch) + 15) & ~(size_t)15) + (size_t)(F > kScoreBins ? F : kScoreBins) * 4;
 }
 __device__ __forceinline__ uint32_t* select_keys(SelectScratch& sc) {
   return reinterpret_cast<uint32_t*>(reinterpret_cast<unsigned char*>(&sc) +
@@ -54,191 +63,176 @@ __device__ __forceinline__ bool selected(uint32_t key, int e, const TopkCut& cut
   return key > cut.T || (key == cut.T && e <= cut.tie_cut);
 }
 
-// Over the candidate keys (bin b1): the gathered list, or -- when it
-// overflowed -- every key of bin b1 in the shared keys (worker threads).
-template <typename Fn>
-__device__ __forceinline__ void for_each_cand(const uint32_t* sk, int F, bool listed, int n,
-                                              const SelectScratch& sc, uint32_t b1, Fn fn) {
-  if (threadIdx.x >= kSelectWorkers) return;
-  if (listed) {
-    for (int i = threadIdx.x; i < n; i += kSelectWorkers) fn(sc.ck[i], sc.ci[i]);
-  } else {
-    for (int e = threadIdx.x; e < F; e += kSelectWorkers) {
-      const uint32_t key = sk[e];
-      if ((key >> kScoreShift) == b1) fn(key, e);
-    }
-  }
+// Digit counts over the CTA: thread t's values come from its packed words
+// c[4] (digit d at bits 16 (d % 4) of c[d / 4]).  Returns the 16 totals in
+// tot[16] (every thread).  Totals stay below 2^16.
+__device__ __forceinline__ void block_digit_counts(const unsigned long long (&c)[4],
+                                                   SelectScratch& sc, int (&tot)[16]) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  unsigned long long w[4] = {c[0], c[1], c[2], c[3]};
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) w[q] += __shfl_xor_sync(0xffffffffu, w[q], o);
+  if (lane == 0)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) sc.wsum[warp][q] = w[q];
+  __syncthreads();
+  unsigned long long s[4] = {0ull, 0ull, 0ull, 0ull};
+  for (int i = 0; i < nw; ++i)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) s[q] += sc.wsum[i][q];
+#pragma unroll
+  for (int dgt = 0; dgt < 16; ++dgt) tot[dgt] = (int)((s[dgt >> 2] >> (16 * (dgt & 3))) & 0xFFFFull);
+  __syncthreads();  // wsum may be rewritten after return
 }
 
-__device__ __forceinline__ uint32_t key_of(const uint4 (&kb)[8], int j) {
-  const uint4 v = kb[j >> 2];
-  return (j & 3) == 0 ? v.x : (j & 3) == 1 ? v.y : (j & 3) == 2 ? v.z : v.w;
+__device__ __forceinline__ void add_digit(unsigned long long (&c)[4], uint32_t dgt) {
+  const unsigned long long inc = 1ull << (16 * (dgt & 3u));
+  c[0] += (dgt >> 2) == 0 ? inc : 0ull;
+  c[1] += (dgt >> 2) == 1 ? inc : 0ull;
+  c[2] += (dgt >> 2) == 2 ? inc : 0ull;
+  c[3] += (dgt >> 2) == 3 ? inc : 0ull;
 }
 
-// Every thread of the CTA calls it (blockDim.x >= 256); sk holds the keys of
-// all F channels.
-__device__ TopkCut select_cut(const uint32_t* hist, const uint32_t* sk, int F, int k,
-                              SelectScratch& sc) {
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const bool worker = tid < kSelectWorkers;
-
-  // 1. boundary bin: worker t holds bins [32q, 32q+32), q = 255 - t, read
-  // straight from the histogram in global memory; an exclusive scan over
-  // threads counts the keys in higher bins
-  {
-    const int q = kSelectWorkers - 1 - tid;
-    uint4 hv[8];
-    int own = 0;
+// Radix select over keys spread over the threads: `items(fn)` calls
+// fn(key, channel) for each of this thread's keys.  Returns the krem-th
+// largest key (1-based) in *T, how many keys equal it in *n_eq, and the rank
+// wanted among those in *k_eq.  Every thread calls it.
+template <typename Items>
+__device__ void radix_kth(Items items, int krem, SelectScratch& sc, uint32_t* T, int* n_eq,
+                          int* k_eq) {
+  uint32_t prefix = 0u, pmask = 0u;
+  int neq = 0;
+  for (int shift = 28; shift >= 0; shift -= 4) {
+    unsigned long long c[4] = {0ull, 0ull, 0ull, 0ull};
+    items([&](uint32_t key, int) {
+      if ((key & pmask) == prefix) add_digit(c, (key >> shift) & 15u);
+    });
+    int tot[16];
+    block_digit_counts(c, sc, tot);
+    int above = 0, dsel = 0, cnt = 0;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      hv[j] = worker ? __ldcg(reinterpret_cast<const uint4*>(hist) + 8 * q + j)
-                     : make_uint4(0u, 0u, 0u, 0u);
-      own += (int)(hv[j].x + hv[j].y + hv[j].z + hv[j].w);
-    }
-    int total;
-    const int above = block_exclusive_scan(own, sc.scan, &total);
-    if (tid == 0) sc.misc[3] = 0;  // candidates gathered
-    if (worker && above < k && above + own >= k) {
-      int run = above;
-#pragma unroll
-      for (int j = 31; j >= 0; --j) {
-        const int c = (int)key_of(hv, j);
-        if (run < k && run + c >= k) {
-          sc.misc[0] = 32 * q + j;  // b1
-          sc.misc[1] = k - run;     // rank wanted inside b1 (1-based)
-          sc.misc[2] = c;           // keys in b1
-        }
-        run += c;
+    for (int dgt = 15; dgt >= 0; --dgt) {  // the digit holding the krem-th largest
+      if (cnt == 0 && above + tot[dgt] >= krem) {
+        dsel = dgt;
+        cnt = tot[dgt];
+      } else if (cnt == 0) {
+        above += tot[dgt];
       }
     }
+    krem -= above;
+    neq = cnt;
+    prefix |= (uint32_t)dsel << shift;
+    pmask |= 15u << shift;
+  }
+  *T = prefix;
+  *n_eq = neq;
+  *k_eq = krem;
+}
+
+// The want-th smallest channel (1-based) among the keys equal to T.
+template <typename Items>
+__device__ int radix_tie(Items items, uint32_t T, int want, SelectScratch& sc) {
+  uint32_t ip = 0u, im = 0u;
+  for (int shift = 12; shift >= 0; shift -= 4) {  // channels < 2^16
+    unsigned long long c[4] = {0ull, 0ull, 0ull, 0ull};
+    items([&](uint32_t key, int ch) {
+      if (key == T && ((uint32_t)ch & im) == ip) add_digit(c, ((uint32_t)ch >> shift) & 15u);
+    });
+    int tot[16];
+    block_digit_counts(c, sc, tot);
+    int below = 0, dsel = 0;
+    bool found = false;
+#pragma unroll
+    for (int dgt = 0; dgt < 16; ++dgt) {
+      if (!found && below + tot[dgt] >= want) {
+        dsel = dgt;
+        found = true;
+      } else if (!found) {
+        below += tot[dgt];
+      }
+    }
+    want -= below;
+    ip |= (uint32_t)dsel << shift;
+    im |= 15u << shift;
+  }
+  return (int)ip;
+}
+
+// Among bins read in descending bin order (thread t holds the count of the
+// t-th largest bin, 0 past the last), the one holding the krem-th largest
+// key: writes its position t and the rank wanted inside it to misc[0],
+// misc[1] and its count to misc[2].  Every thread calls it.
+__device__ __forceinline__ void find_bin_desc(int count, int krem, SelectScratch& sc) {
+  int total;
+  const int above = block_exclusive_scan(count, sc.scan, &total);
+  if (count > 0 && above < krem && above + count >= krem) {
+    sc.misc[0] = (int)threadIdx.x;
+    sc.misc[1] = krem - above;
+    sc.misc[2] = count;
   }
   __syncthreads();
-  const uint32_t b1 = (uint32_t)sc.misc[0];
+}
+
+// The exact cut of the token; every CTA calls it once the histograms and
+// buckets are complete (blockDim.x >= kCoarseBins).  1 <= k <= F.
+__device__ TopkCut select_cut(const uint32_t* hist, const uint32_t* chist, const uint2* bucket,
+                              const float* scores, int F, int k, SelectScratch& sc) {
+  const int tid = threadIdx.x;
+  // 1. the coarse bin (bins read from the top)
+  find_bin_desc(tid < kCoarseBins ? (int)__ldcg(chist + (kCoarseBins - 1 - tid)) : 0, k, sc);
+  const int cb = kCoarseBins - 1 - sc.misc[0];
+  const int k1 = sc.misc[1];
+  __syncthreads();
+  // 2. its fine bins
+  const int fb0 = cb * kFinePerCoarse;
+  find_bin_desc(tid < kFinePerCoarse ? (int)__ldcg(hist + fb0 + (kFinePerCoarse - 1 - tid)) : 0, k1,
+                sc);
+  const uint32_t b1 = (uint32_t)(fb0 + kFinePerCoarse - 1 - sc.misc[0]);
   const int krem = sc.misc[1];
   const int n1 = sc.misc[2];
-
-  // 2. the candidates
-  const bool listed = n1 <= kSelectCand;
-  if (listed) {
-    for (int e = tid; e < F; e += blockDim.x) {
-      const uint32_t key = sk[e];
-      if ((key >> kScoreShift) == b1) {
-        const int slot = atomicAdd(&sc.misc[3], 1);
-        if (slot < kSelectCand) {
-          sc.ck[slot] = key;
-          sc.ci[slot] = e;
-        }
-      }
-    }
-  }
-  __syncthreads();
-
-  // 3. the exact cut among the candidates: T and the tie cut into misc[7],
-  // misc[12]
-  if (listed && n1 <= kSelectDirect) {
-    // The order is that of the composite key << 32 | (~index) descending, so a
-    // candidate's rank is the number of larger composites.  Padding with 0
-    // (below every real composite) lets the comparison loop run in blocks of
-    // 8; TPC adjacent threads share a candidate.
-    const int n8 = (n1 + 7) & ~7;
-    for (int i = tid; i < n8; i += blockDim.x)
-      sc.c64[i] = i < n1 ? ((unsigned long long)sc.ck[i] << 32) | (uint32_t)~(uint32_t)sc.ci[i] : 0ull;
-    __syncthreads();
-    if (worker) {
-      int TPC = 1;
-      while (TPC < 32 && n1 * TPC * 2 <= kSelectWorkers) TPC *= 2;
-      const int per_pass = kSelectWorkers / TPC;
-      for (int i0 = 0; i0 < n1; i0 += per_pass) {
-        const int i = i0 + tid / TPC, sub = tid % TPC;
-        const unsigned long long c = i < n1 ? sc.c64[i] : ~0ull;
-        int rank = 0;
-        for (int j = sub * 8; j < n8; j += TPC * 8) {
-#pragma unroll
-          for (int u = 0; u < 8; ++u) rank += sc.c64[j + u] > c;
-        }
-        for (int o = 1; o < TPC; o <<= 1) rank += __shfl_xor_sync(0xffffffffu, rank, o);
-        if (i < n1 && sub == 0 && rank == krem - 1) {
-          sc.misc[7] = (int)sc.ck[i];
-          sc.misc[12] = sc.ci[i];
-        }
-      }
-    }
-  } else {
-    uint32_t* h = sc.h;
-    for (int i = tid; i < 1024; i += blockDim.x) h[i] = 0u;
-    __syncthreads();
-    // level 2: key bits 17..8
-    for_each_cand(sk, F, listed, n1, sc, b1,
-                  [&](uint32_t kk, int) { atomicAdd(&h[(kk >> 8) & 0x3FFu], 1u); });
-    __syncthreads();
-    if (warp == 0) {
-      int b2, k2, c2;
-      warp_find_bin<32, false>(h, krem, &b2, &k2, &c2);
-      if (lane == 0) {
-        sc.misc[5] = b2;
-        sc.misc[6] = k2;
-      }
-    }
-    __syncthreads();
-    const uint32_t p2 = (b1 << 10) | (uint32_t)sc.misc[5];  // key bits 30..8
-    for (int i = tid; i < 1024; i += blockDim.x) h[i] = 0u;
-    __syncthreads();
-    // level 3: key bits 7..0
-    for_each_cand(sk, F, listed, n1, sc, b1, [&](uint32_t kk, int) {
-      if ((kk >> 8) == p2) atomicAdd(&h[kk & 0xFFu], 1u);
-    });
-    __syncthreads();
-    if (warp == 0) {
-      int b3, k3, c3;
-      warp_find_bin<8, false>(h, sc.misc[6], &b3, &k3, &c3);
-      if (lane == 0) {
-        sc.misc[7] = (int)((p2 << 8) | (uint32_t)b3);
-        sc.misc[8] = k3;  // keys equal to T that are taken
-        sc.misc[9] = c3;  // keys equal to T
-        sc.misc[12] = F;  // every key equal to T taken, unless cut below
-      }
-    }
-    __syncthreads();
-    const uint32_t T = (uint32_t)sc.misc[7];
-    const int k_eq = sc.misc[8], n_eq = sc.misc[9];
-    // tie cut: the k_eq-th smallest index among keys equal to T (radix on the
-    // index: bits 14..7, then 6..0), i.e. the (n_eq - k_eq + 1)-th largest.
-    if (k_eq < n_eq) {
-      for (int i = tid; i < 1024; i += blockDim.x) h[i] = 0u;
-      __syncthreads();
-      for_each_cand(sk, F, listed, n1, sc, b1, [&](uint32_t kk, int ix) {
-        if (kk == T) atomicAdd(&h[(ix >> 7) & 0xFFu], 1u);
-      });
-      __syncthreads();
-      if (warp == 0) {
-        int bi, ki, ci;
-        warp_find_bin<8, false>(h, n_eq - k_eq + 1, &bi, &ki, &ci);
-        if (lane == 0) {
-          sc.misc[10] = bi;
-          sc.misc[11] = ki;
-        }
-      }
-      __syncthreads();
-      const int hi7 = sc.misc[10];
-      for (int i = tid; i < 1024; i += blockDim.x) h[i] = 0u;
-      __syncthreads();
-      for_each_cand(sk, F, listed, n1, sc, b1, [&](uint32_t kk, int ix) {
-        if (kk == T && (ix >> 7) == hi7) atomicAdd(&h[ix & 0x7F], 1u);
-      });
-      __syncthreads();
-      if (warp == 0) {
-        int bl, kl, cl;
-        warp_find_bin<4, false>(h, sc.misc[11], &bl, &kl, &cl);
-        if (lane == 0) sc.misc[12] = (hi7 << 7) | bl;
-      }
-      __syncthreads();
-    }
-  }
   __syncthreads();
   TopkCut cut;
-  cut.T = (uint32_t)sc.misc[7];
-  cut.tie_cut = sc.misc[12];
-  __syncthreads();  // the scratch may be reused after return
+  if (n1 <= kBucketCap) {
+    // 3. the candidates, ranked: the one with krem - 1 larger (key, ~channel)
+    // composites is the cut
+    if (tid < n1) {
+      const uint2 kc = __ldcg(bucket + (size_t)b1 * kBucketCap + tid);
+      sc.ck[tid] = kc.x;
+      sc.ci[tid] = (int)kc.y;
+    }
+    __syncthreads();
+    if (tid < n1) {
+      const unsigned long long c = ((unsigned long long)sc.ck[tid] << 32) | (uint32_t)~(uint32_t)sc.ci[tid];
+      int rank = 0;
+      for (int j = 0; j < n1; ++j)
+        rank += (((unsigned long long)sc.ck[j] << 32) | (uint32_t)~(uint32_t)sc.ci[j]) > c;
+      if (rank == krem - 1) {
+        sc.misc[7] = (int)sc.ck[tid];
+        sc.misc[12] = sc.ci[tid];
+      }
+    }
+    __syncthreads();
+    cut.T = (uint32_t)sc.misc[7];
+    cut.tie_cut = sc.misc[12];
+    __syncthreads();
+    return cut;
+  }
+  // 3'. b1 overflowed its bucket (many equal scores): radix select over every
+  // key, loaded into shared memory
+  uint32_t* sk = select_keys(sc);
+  for (int e = tid; e < (F >> 2); e += blockDim.x)
+    reinterpret_cast<uint4*>(sk)[e] = __ldcg(reinterpret_cast<const uint4*>(scores) + e);
+  __syncthreads();
+  const int per = (F + (int)blockDim.x - 1) / (int)blockDim.x;
+  const int j0 = min(tid * per, F), j1 = min(j0 + per, F);
+  auto all = [&](auto fn) {
+    for (int j = j0; j < j1; ++j) fn(sk[j], j);
+  };
+  int n_eq, k_eq;
+  radix_kth(all, k, sc, &cut.T, &n_eq, &k_eq);
+  cut.tie_cut = k_eq < n_eq ? radix_tie(all, cut.T, k_eq, sc) : F;
   return cut;
 }
 

@@ -5,11 +5,13 @@
 // Work: the set of (column slice, kept input row) pairs.  A column slice is
 // 512 bytes of an interleaved proxy row (16 blocks of 32 channels, each block
 // 16 B of gate codes then 16 B of up codes), i.e. 512 channels of both
-// proxies.  Every CTA thresholds all of x (|x_i| >= tau) and compacts the kept
-// rows in ascending order; the C * n_x pairs, slice-major, are then split into
-// equal contiguous ranges, one per CTA and, inside it, one per warp, so every
-// warp streams the same number of 512-byte row slices whatever the mask looks
-// like.  A CTA's range lies in at most two adjacent slices.
+// proxies; the proxy is stored slice-major, so a slice's kept rows are read in
+// ascending address order.  The C * d_model (slice, row) pairs, slice-major,
+// are split into equal contiguous ranges, one per CTA (a static split: a CTA's
+// range lies in at most two adjacent slices); each CTA thresholds the rows of
+// its range (|x_i| >= tau), compacts its kept pairs in order and splits them
+// into equal contiguous ranges, one per warp, so every warp streams the same
+// number of 512-byte row slices whatever the mask looks like.
 //
 // A warp streams its rows through a shared-memory ring with asynchronous
 // 16-byte copies (cp.async, L2 only; each lane copies and later reads back its
@@ -25,10 +27,11 @@
 // the partials of the CTAs that hold its slice in CTA order (deterministic),
 // scores it, score_j = |act(g~_j) u~_j| (act the layer's gate activation:
 // SiLU, or GELU for a GeGLU FFN; the signed value is kept too when Stage 2
-// runs the A3 ablation), and -- for the top-k rule -- counts it in an
-// 8192-bin histogram of the score's top bits, the first level of the radix
-// select (score_channels).
+// runs the A3 ablation), keeps its key in shared memory for the selection
+// and, for the top-k rule, counts it in the histograms and buckets of
+// select.cuh (score_channels).
 #pragma once
+#include "select.cuh"
 #include "token_args.cuh"
 
 namespace prox {
@@ -41,6 +44,7 @@ constexpr int SLICE = 512;   // bytes (= channels of both proxies) per column sl
 constexpr int PART = 1024;   // partial values per slice: 32 chunks x 32 channels
 constexpr int U = 4;         // rows per batch
 constexpr int BATCH = U * SLICE;
+static_assert(kOwnMax <= kTokenThreads, "scoring takes one channel per thread");
 
 // (w & M) | e in one instruction; e is a register (the exponents come from
 // kernel parameters, so they are not folded into a second immediate).
@@ -94,44 +98,56 @@ __device__ __forceinline__ int cta_of(int t, int T, int P) {
   return (int)(((unsigned)(t + 1) * (unsigned)P + (unsigned)T - 1u) / (unsigned)T) - 1;
 }
 
-// Scores the channels [F c / P, F (c + 1) / P) of CTA c once every CTA's
-// partials are visible: thread t < the CTA's channel count takes one channel
-// and adds its gate and up partials over the CTAs holding its slice, in CTA
-// order.  n_x == 0: every score is 0.  Every thread of the CTA calls it.
-__device__ void score_channels(const TokenArgs& a, int n_x, bool histogram) {
-  const int P = gridDim.x, cta = blockIdx.x;
+// Scores the channels [F c / P, F (c + 1) / P) of CTA c (at most kOwnMax,
+// so one per thread) once every CTA's partials are visible: thread t adds the
+// gate and up partials of channel c0 + t over the CTAs whose pair ranges
+// cover its slice, in CTA order.  For the top-k rule the CTA first counts its
+// keys in shared-memory histograms; one thread per non-empty fine bin then
+// adds the CTA's count to the global bin, whose old value places the CTA's
+// keys of that bin in the bin's bucket, and the coarse counts are added the
+// same way, so a global bin sees one atomic per CTA, not one per channel.
+// Every thread of the CTA calls it.
+__device__ void score_channels(const TokenArgs& a, bool histogram, SelectScratch& sel) {
+  const int P = gridDim.x, cta = blockIdx.x, tid = threadIdx.x;
   const int c0 = (int)(((long long)a.F * cta) / P);
   const int c1 = (int)(((long long)a.F * (cta + 1)) / P);
-  for (int ch = c0 + (int)threadIdx.x; ch < c1; ch += blockDim.x) {
+  const int T = a.C * a.d;
+  uint32_t* fine = select_keys(sel);  // [kScoreBins]: the CTA's counts, then its bucket offsets
+  if (histogram) {
+    for (int i = tid; i < kCoarseBins; i += blockDim.x) sel.coarse[i] = 0u;
+    for (int i = tid; i < kScoreBins; i += blockDim.x) fine[i] = 0u;
+    __syncthreads();
+  }
+  const int ch = c0 + tid;
+  const bool mine = ch < c1;
+  uint32_t key = 0u, fb = 0u, rank = 0u;
+  if (mine) {
     const int c = ch / SLICE, m = ch % SLICE;
     // channel m of the slice is block blk = m / 32, channel j = m % 32 of it:
     // its gate and up sums are the partial elements j*32 + 2*blk and + 1
     const int e = (m & 31) * 32 + 2 * (m >> 5);
+    const int i_lo = cta_of(c * a.d, T, P);
+    const int i_hi = cta_of((c + 1) * a.d - 1, T, P);
     float g = 0.f, u = 0.f;
-    if (n_x > 0) {
-      const int T = a.C * n_x;
-      const int i_lo = cta_of(c * n_x, T, P);
-      const int i_hi = cta_of((c + 1) * n_x - 1, T, P);
-      for (int i0 = i_lo; i0 <= i_hi; i0 += 8) {
-        float2 v[8];
+    for (int i0 = i_lo; i0 <= i_hi; i0 += 8) {
+      float2 v[8];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const int i = i0 + q;
-          v[q] = make_float2(0.f, 0.f);
-          if (i <= i_hi) {
-            const unsigned tlo = (unsigned)T * (unsigned)i / (unsigned)P;
-            const unsigned thi = (unsigned)T * (unsigned)(i + 1) / (unsigned)P;
-            if (thi > tlo) {  // CTA i holds pairs; slice c is its first or second
-              const int off = (i * 2 + (c - (int)(tlo / (unsigned)n_x))) * PART;
-              v[q] = __ldcg(reinterpret_cast<const float2*>(a.part + off + e));
-            }
+      for (int q = 0; q < 8; ++q) {
+        const int i = i0 + q;
+        v[q] = make_float2(0.f, 0.f);
+        if (i <= i_hi) {
+          const unsigned tlo = (unsigned)T * (unsigned)i / (unsigned)P;
+          const unsigned thi = (unsigned)T * (unsigned)(i + 1) / (unsigned)P;
+          if (thi > tlo) {  // CTA i holds pairs; slice c is its first or second
+            const int off = (i * 2 + (c - (int)(tlo / (unsigned)a.d))) * PART;
+            v[q] = __ldcg(reinterpret_cast<const float2*>(a.part + off + e));
           }
         }
+      }
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          g += v[q].x;
-          u += v[q].y;
-        }
+      for (int q = 0; q < 8; ++q) {
+        g += v[q].x;
+        u += v[q].y;
       }
     }
     const float sv = act_f32(g, a.act) * u;
@@ -140,7 +156,23 @@ __device__ void score_channels(const TokenArgs& a, int n_x, bool histogram) {
     if (a.s_tilde) a.s_tilde[ch] = sv;
     if (a.g_dbg) a.g_dbg[ch] = g;
     if (a.u_dbg) a.u_dbg[ch] = u;
-    if (histogram) atomicAdd(a.hist + (__float_as_uint(sc) >> kScoreShift), 1u);
+    key = __float_as_uint(sc);
+    sel.own[tid] = key;
+    if (histogram) {
+      fb = key >> kScoreShift;
+      rank = atomicAdd(&fine[fb], 1u);
+      atomicAdd(&sel.coarse[key >> kCoarseShift], 1u);
+    }
+  }
+  if (!histogram) return;
+  __syncthreads();
+  if (mine && rank == 0u) fine[fb] = atomicAdd(a.hist + fb, fine[fb]);
+  for (int i = tid; i < kCoarseBins; i += blockDim.x)
+    if (sel.coarse[i]) atomicAdd(a.chist + i, sel.coarse[i]);
+  __syncthreads();
+  if (mine) {
+    const uint32_t slot = fine[fb] + rank;
+    if (slot < (uint32_t)kBucketCap) a.bucket[fb * kBucketCap + slot] = make_uint2(key, (uint32_t)ch);
   }
 }
 
@@ -152,11 +184,11 @@ constexpr size_t smem_bytes(int lmax) {
          (size_t)PART * 4 + (37 + kTokenThreads) * 4;
 }
 
-// The row loop of Stage 1: the CTA's partial sums of the slices it touches
-// go to a.part.  Returns n_x (the kept rows of the token).  Every thread of
-// the CTA calls it; warps NW and above take no rows.
+// The row loop of Stage 1: the CTA's partial sums of the slices its pair
+// range touches go to a.part.  Every thread of the CTA calls it; warps NW and
+// above take no rows.
 template <int NB>
-__device__ int run(const TokenArgs& a, unsigned char* smem) {
+__device__ void run(const TokenArgs& a, unsigned char* smem) {
   constexpr int RING = NB * BATCH;  // ring bytes per warp
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int P = gridDim.x, cta = blockIdx.x;
@@ -172,65 +204,70 @@ __device__ int run(const TokenArgs& a, unsigned char* smem) {
   int* s_m = s_scan + 33;                                            // [4]
   int* s_src = s_m + 4;                                              // [kTokenThreads]
 
-  // ---- kept rows of x, ascending: thread t < NT owns rows [t*rpt, (t+1)*rpt) ----
-  const int rpt = (a.d + NT - 1) / NT;
-  const int r0 = tid < NT ? tid * rpt : a.d;
-  const int r1 = min(r0 + rpt, a.d);
-  const bool vec = (rpt & 3) == 0;  // rows r0.. are 16-byte aligned
-  auto x_at = [&](int row) -> float4 {  // rows row..row+3 (those < r1)
-    if (vec) return __ldg(reinterpret_cast<const float4*>(a.x + row));
-    float4 v;
-    v.x = __ldg(a.x + row);
-    v.y = row + 1 < r1 ? __ldg(a.x + row + 1) : 0.f;
-    v.z = row + 2 < r1 ? __ldg(a.x + row + 2) : 0.f;
-    v.w = row + 3 < r1 ? __ldg(a.x + row + 3) : 0.f;
-    return v;
-  };
-  int cnt = 0;
-  for (int row = r0; row < r1; row += 4) {
-    const float4 v = x_at(row);
-    cnt += (fabsf(v.x) >= a.tau) + (row + 1 < r1 && fabsf(v.y) >= a.tau) +
-           (row + 2 < r1 && fabsf(v.z) >= a.tau) + (row + 3 < r1 && fabsf(v.w) >= a.tau);
-  }
-  int n_x;
-  int pos = block_exclusive_scan(cnt, s_scan, &n_x);
-  if (n_x == 0) {
-    // nothing kept: g~ = u~ = 0 everywhere (score_channels needs no partials)
-    if (cta == 0 && tid == 0) {
-      if (a.n_x) *a.n_x = 0;
-    }
-    return 0;
-  }
-  const unsigned T = (unsigned)a.C * (unsigned)n_x;   // T * P < 2^31
+  // ---- this CTA's pairs: [tlo, thi) of the C * d (slice, row) pairs,
+  // slice-major; pair p of the range is slice cA + (rA + p >= d), row
+  // (rA + p) mod d.  The split is static: it does not depend on the token. ----
+  const int d = a.d;
+  const unsigned T = (unsigned)a.C * (unsigned)d;  // T * P < 2^31
   const unsigned tlo = T * (unsigned)cta / (unsigned)P, thi = T * (unsigned)(cta + 1) / (unsigned)P;
-  const int len = (int)(thi - tlo);      // <= n_x, since C < P
-  const int cA = (int)(tlo / (unsigned)n_x), pA = (int)(tlo % (unsigned)n_x);
-  const int l_split = n_x - pA;          // local rows l >= l_split lie in slice cA + 1
-  // local row l of this CTA is compacted position (pA + l) mod n_x
-  for (int row0 = r0; row0 < r1; row0 += 4) {
-    const float4 v4 = x_at(row0);
-    const float vv[4] = {v4.x, v4.y, v4.z, v4.w};
+  const int span = (int)(thi - tlo);               // <= d, since C < P
+  const int cA = (int)(tlo / (unsigned)d), rA = (int)(tlo % (unsigned)d);
+  const int first = min(span, d - rA);             // pairs of the range in slice cA
+  // ---- its kept pairs (|x_row| >= tau), in pair order: thread t owns pairs
+  // [t*per, (t+1)*per); the two slices' counts are packed in one word ----
+  const int per = (span + (int)blockDim.x - 1) / (int)blockDim.x;
+  const int p0 = min(tid * per, span), p1 = min(p0 + per, span);
+  float xv[4];
+  unsigned cnt = 0;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int row = row0 + q;
-      if (row < r1 && fabsf(vv[q]) >= a.tau) {
-        int l = pos - pA;
-        if (l < 0) l += n_x;
-        if (l < len) {
-          // the row slice's byte offset in the proxy, and its segment key
-          // (slice, quantisation group), nondecreasing over the CTA's rows
-          const int sl = l >= l_split ? 1 : 0;
-          s_rx[l] = make_int2(row * a.F + (cA + sl) * SLICE, __float_as_int(vv[q]));
-          s_key[l] = sl * 128 + (row >> 7);
-        }
-        if (cta == 0 && a.idx_x) a.idx_x[pos] = row;
-        ++pos;
-      }
+  for (int q = 0; q < 4; ++q) {  // the first four pairs (all of them while span <= 4 * blockDim.x)
+    const int p = p0 + q;
+    xv[q] = 0.f;
+    if (p < p1) {
+      const int row = rA + p < d ? rA + p : rA + p - d;
+      xv[q] = __ldg(a.x + row);
+      if (fabsf(xv[q]) >= a.tau) cnt += p < first ? 1u : 0x10000u;
     }
   }
-  if (cta == 0 && tid == 0) {
-    atomicAdd(a.stats, (unsigned long long)n_x);
-    if (a.n_x) *a.n_x = n_x;
+  for (int p = p0 + 4; p < p1; ++p) {  // longer ranges (d > 4 * blockDim.x)
+    const int row = rA + p < d ? rA + p : rA + p - d;
+    if (fabsf(__ldg(a.x + row)) >= a.tau) cnt += p < first ? 1u : 0x10000u;
+  }
+  unsigned tot;
+  const unsigned pre = block_exclusive_scan(cnt, reinterpret_cast<unsigned*>(s_scan), &tot);
+  const int l_split = (int)(tot & 0xFFFFu);        // kept pairs in slice cA
+  const int len = l_split + (int)(tot >> 16);      // kept pairs of the CTA
+  {
+    int l0 = (int)(pre & 0xFFFFu), l1 = l_split + (int)(pre >> 16);
+    // the row slice's byte offset in the proxy, and its segment key (slice,
+    // quantisation group), nondecreasing over the CTA's rows
+    auto place = [&](int p, float v) {
+      if (fabsf(v) >= a.tau) {
+        const int row = rA + p < d ? rA + p : rA + p - d;
+        const int sl = p < first ? 0 : 1;
+        const int l = sl ? l1++ : l0++;
+        s_rx[l] = make_int2(((cA + sl) * d + row) * SLICE, __float_as_int(v));
+        s_key[l] = sl * 128 + (row >> 7);
+      }
+    };
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (p0 + q < p1) place(p0 + q, xv[q]);
+    for (int p = p0 + 4; p < p1; ++p) place(p, __ldg(a.x + (rA + p < d ? rA + p : rA + p - d)));
+  }
+  // realised input sparsity: the kept rows counted once, in slice 0
+  if (tid == 0 && cA == 0 && l_split > 0) atomicAdd(a.stats, (unsigned long long)l_split);
+  if (cta == 0 && (a.idx_x || a.n_x)) {
+    // test taps: the token's kept rows, ascending, and their number
+    const int rpt = (d + (int)blockDim.x - 1) / (int)blockDim.x;
+    const int q0 = min(tid * rpt, d), q1 = min(q0 + rpt, d);
+    int c = 0;
+    for (int row = q0; row < q1; ++row) c += fabsf(__ldg(a.x + row)) >= a.tau;
+    int n_all;
+    int pos = block_exclusive_scan(c, s_scan, &n_all);
+    for (int row = q0; row < q1; ++row)
+      if (fabsf(__ldg(a.x + row)) >= a.tau && a.idx_x) a.idx_x[pos++] = row;
+    if (tid == 0 && a.n_x) *a.n_x = n_all;
   }
   __syncthreads();
   stamp(a.ts, 8);
@@ -353,7 +390,7 @@ __device__ int run(const TokenArgs& a, unsigned char* smem) {
     s_src[tid] = l1 <= l0 ? 0 : (l1 <= l_split ? 1 : (l0 >= l_split ? 2 : 3));
   }
   __syncthreads();
-  const int nsl = len > l_split ? 2 : 1;
+  const int nsl = span > first ? 2 : 1;  // slices the CTA's pair range touches
   for (int e = tid; e < PART; e += blockDim.x) {
     float p0 = 0.f, p1 = 0.f;
 #pragma unroll
@@ -370,7 +407,6 @@ __device__ int run(const TokenArgs& a, unsigned char* smem) {
     a.part[((size_t)cta * 2) * PART + e] = p0;
     if (nsl == 2) a.part[((size_t)cta * 2 + 1) * PART + e] = p1;
   }
-  return n_x;
 }
 
 }  // namespace s1

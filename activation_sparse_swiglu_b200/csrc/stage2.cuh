@@ -4,11 +4,15 @@
 // phase with every channel kept.  Second phase of the fused per-token kernel
 // (token.cu).
 //
-// Every CTA loads the token's scores into shared memory, finds the exact top-k
-// cut of the token (select.cuh: T and the tie cut) or applies the score
-// threshold, ranks the selected channels in ascending channel order and takes
-// the ranks [n_sel c / P, n_sel (c + 1) / P): every CTA streams the same
-// number of channels (to one), whatever the mask looks like.  A given list is
+// Every CTA finds the token's exact top-k cut (select.cuh: key T and the tie
+// cut) or applies the score threshold, lists the channels of its own range
+// [F c / P, F (c + 1) / P) -- the channels it scored -- past it, ascending, at
+// the range's start in a.sel_list and writes their count; after a grid
+// barrier CTA c takes the ranks
+// [S c / P, S (c + 1) / P) of the whole selection (S channels, ascending), so
+// every CTA streams the same number of channels (to one) whatever the mask
+// looks like; a given list is split the same way by list position, and the
+// dense baseline splits all channels.  A given list is
 // split by list position the same way, and the dense baseline splits all
 // channels.  Producer lanes stream, with 1-D bulk async copies (TMA engine)
 // into a ring of slots, first the gate/up channel records of the CTA's
@@ -49,7 +53,7 @@ __host__ __device__ constexpr size_t ring_offset(int slots, int max_rec) {
 // ceil(d_model / (8 * 32 * warps per group)): 8-element chunks per lane and
 // column.
 template <int MAXM>
-__device__ void run(const TokenArgs& a, unsigned char* smem, bool* dead) {
+__device__ void run(const TokenArgs& a, unsigned char* smem, GridSync& gs) {
   const int d = a.d, slots = a.slots;
   const uint32_t col_bytes = 2u * (uint32_t)d;     // one bf16 column / row
   const uint32_t slot_bytes = 2u * col_bytes;      // a gate/up record, or two W_down rows
@@ -76,57 +80,51 @@ __device__ void run(const TokenArgs& a, unsigned char* smem, bool* dead) {
   // order), of the list (list order) or of all channels (dense).
   int r0 = 0, n = 0;
   if (a.mode == kModeTopK || a.mode == kModeThreshold) {
+    // this CTA's own channels (those it scored; their keys are in sc.own) past
+    // the token's cut: the exact top-k cut, or the score threshold of Prox §4.1
+    // (key >= bits(tau_s), every tie kept)
     SelectScratch& sc = *reinterpret_cast<SelectScratch*>(ring);
-    uint32_t* sk = select_keys(sc);
-    {
-      // every load in flight before the first store (F <= 32768: at most two rounds)
-      constexpr int LU = 8;
-      const int n4 = a.F >> 2;
-      for (int e0 = tid; e0 < n4; e0 += LU * (int)blockDim.x) {
-        uint4 v[LU];
-#pragma unroll
-        for (int u = 0; u < LU; ++u) {
-          const int e = e0 + u * (int)blockDim.x;
-          v[u] = e < n4 ? __ldcg(reinterpret_cast<const uint4*>(a.scores) + e) : make_uint4(0u, 0u, 0u, 0u);
-        }
-#pragma unroll
-        for (int u = 0; u < LU; ++u) {
-          const int e = e0 + u * (int)blockDim.x;
-          if (e < n4) reinterpret_cast<uint4*>(sk)[e] = v[u];
-        }
-      }
-    }
-    __syncthreads();
     TopkCut cut;
     if (a.mode == kModeTopK) {
-      cut = select_cut(a.hist, sk, a.F, a.k, sc);
+      cut = select_cut(a.hist, a.chist, a.bucket, a.scores, a.F, a.k, sc);
+      stamp(a.ts, 15);
     } else {
-      // Prox §4.1: score >= tau_s, i.e. key >= bits(tau_s) with every tie kept
       cut.T = __float_as_uint(a.tau_s);
       cut.tie_cut = a.F;
     }
-    // thread t ranks the channels [t*per, (t+1)*per)
-    const int per = (a.F + blockDim.x - 1) / blockDim.x;
-    const int j0 = min(tid * per, a.F), j1 = min(j0 + per, a.F);
-    int cnt = 0;
-    for (int j = j0; j < j1; ++j) cnt += selected(sk[j], j, cut) ? 1 : 0;
-    int total;
-    int r = block_exclusive_scan(cnt, sc.scan, &total);
-    r0 = (int)(((long long)total * cta) / P);
-    n = (int)(((long long)total * (cta + 1)) / P) - r0;
-    for (int j = j0; j < j1; ++j) {
-      if (selected(sk[j], j, cut)) {
-        if (r >= r0 && r < r0 + n) s_idx[r - r0] = j;
-        ++r;
+    const int c0 = (int)(((long long)a.F * cta) / P);
+    const int m = (int)(((long long)a.F * (cta + 1)) / P) - c0;
+    const bool sel = tid < m && selected(sc.own[tid], c0 + tid, cut);
+    int own_n;
+    const int pos = block_exclusive_scan(sel ? 1 : 0, sc.scan, &own_n);
+    if (sel) a.sel_list[c0 + pos] = c0 + tid;
+    if (a.sel_mask && tid < m) a.sel_mask[c0 + tid] = sel ? 1 : 0;
+    if (tid == 0) {
+      a.sel_cnt[cta] = own_n;
+      if (a.stats && !a.select_only) {
+        if (cta == 0) atomicAdd(a.stats + 1, 1ull);
+        atomicAdd(a.stats + 2, (unsigned long long)own_n);
       }
     }
-    if (a.sel_mask) {
-      const int m0 = (int)(((long long)a.F * cta) / P), m1 = (int)(((long long)a.F * (cta + 1)) / P);
-      for (int j = m0 + tid; j < m1; j += blockDim.x) a.sel_mask[j] = selected(sk[j], j, cut) ? 1 : 0;
-    }
-    if (tid == 0 && cta == 0 && a.stats && !a.select_only) {
-      atomicAdd(a.stats + 1, 1ull);
-      atomicAdd(a.stats + 2, (unsigned long long)total);
+    grid_barrier(gs, P, a.err);  // every range's list and count is written
+    const int cnt = tid < P ? __ldcg(a.sel_cnt + tid) : 0;
+    int total;
+    const int first = block_exclusive_scan(cnt, sc.scan, &total);
+    if (tid < P) sc.own[tid] = (uint32_t)first;  // rank of range tid's first channel
+    __syncthreads();
+    // ranks [total c / P, total (c + 1) / P) of the selection, ascending:
+    // rank q lives in the last range whose first rank is <= q
+    r0 = (int)(((long long)total * cta) / P);
+    n = (int)(((long long)total * (cta + 1)) / P) - r0;
+    for (int i = tid; i < n; i += blockDim.x) {
+      const int q = r0 + i;
+      int lo = 0, hi = P - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if ((int)sc.own[mid] <= q) lo = mid;
+        else hi = mid - 1;
+      }
+      s_idx[i] = __ldcg(a.sel_list + (int)(((long long)a.F * lo) / P) + (q - (int)sc.own[lo]));
     }
   } else {
     // list positions, or channels, [k c / P, k (c + 1) / P)
@@ -174,37 +172,66 @@ __device__ void run(const TokenArgs& a, unsigned char* smem, bool* dead) {
   auto group_items = [&](int g, int cnt) { return cnt > g ? (cnt - g + NG - 1) / NG : 0; };
   float* out_row = a.ypart + (size_t)cta * d;
   if (warp == NCW) {
-    // ---------------- producer lanes 0..NG-1 ----------------
-    if (lane < NG) {
-      const int g = lane;
-      bool pdead = *dead;
+    // ---------------- producer: one thread fills every group's slots ----------------
+    // It polls the groups in turn with non-blocking tests, so a group that is
+    // slow to free a slot never holds up the copies of another.
+    if (lane == 0) {
       const uint64_t pol = l2_policy_evict_first();
-      const int nA_g = a.proxy_values ? 0 : group_items(g, n), nB_g = group_items(g, nB);
-      const int tot_g = nA_g + nB_g;
-      for (int li = 0; li < tot_g; ++li) {
-        const int slot = g * SPG + li % SPG, use = li / SPG;
-        if (use > 0) mbar_wait(&empty[slot], (uint32_t)((use - 1) & 1), a.err, &pdead);
-        unsigned char* dst = ring + (size_t)slot * slot_bytes;
-        if (li < nA_g) {
-          const int r = g + li * NG;
-          mbar_arrive_expect_tx(&full[slot], slot_bytes);
-          bulk_copy_g2s(dst, a.wgu + (size_t)s_idx[r] * 2 * (size_t)d, slot_bytes, &full[slot], pol);
-        } else {
-          const int r0 = 2 * (g + (li - nA_g) * NG);
-          const int nr = r0 + 1 < n ? 2 : 1;
-          mbar_arrive_expect_tx(&full[slot], (uint32_t)nr * col_bytes);
-          bulk_copy_g2s(dst, a.wd + (size_t)s_idx[r0] * (size_t)d, col_bytes, &full[slot], pol);
-          if (nr == 2)
-            bulk_copy_g2s(dst + col_bytes, a.wd + (size_t)s_idx[r0 + 1] * (size_t)d, col_bytes,
-                          &full[slot], pol);
+      int next[4] = {0, 0, 0, 0}, nA[4] = {0, 0, 0, 0}, tot[4] = {0, 0, 0, 0};
+      int remaining = 0;
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        if (g >= NG) continue;
+        nA[g] = a.proxy_values ? 0 : group_items(g, n);
+        tot[g] = nA[g] + group_items(g, nB);
+        remaining += tot[g];
+      }
+      long long t_idle = clock64();
+      bool pdead = gs.dead;
+      while (remaining > 0 && !pdead) {
+        bool progress = false;
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          if (g >= NG) continue;
+          const int li = next[g];
+          if (li >= tot[g]) continue;
+          const int slot = g * SPG + li % SPG, use = li / SPG;
+          if (use > 0 && !mbar_test_wait(&empty[slot], (uint32_t)((use - 1) & 1))) continue;
+          unsigned char* dst = ring + (size_t)slot * slot_bytes;
+          if (li < nA[g]) {
+            const int r = g + li * NG;
+            mbar_arrive_expect_tx(&full[slot], slot_bytes);
+            bulk_copy_g2s(dst, a.wgu + (size_t)s_idx[r] * 2 * (size_t)d, slot_bytes, &full[slot], pol);
+          } else {
+            const int r0 = 2 * (g + (li - nA[g]) * NG);
+            const int nr = r0 + 1 < n ? 2 : 1;
+            mbar_arrive_expect_tx(&full[slot], (uint32_t)nr * col_bytes);
+            bulk_copy_g2s(dst, a.wd + (size_t)s_idx[r0] * (size_t)d, col_bytes, &full[slot], pol);
+            if (nr == 2)
+              bulk_copy_g2s(dst + col_bytes, a.wd + (size_t)s_idx[r0 + 1] * (size_t)d, col_bytes,
+                            &full[slot], pol);
+          }
+          next[g] = li + 1;
+          --remaining;
+          progress = true;
+        }
+        if (progress) {
+          t_idle = clock64();
+        } else if (clock64() - t_idle > kWaitLimitCycles) {
+          atomicOr(a.err, PROX_DEVERR_WAIT_TIMEOUT);
+          pdead = true;
         }
       }
       // Every issued copy must land before this CTA's shared memory is reused:
-      // wait for the last use of each slot of the group.
+      // wait for the last issued use of each slot (bounded).
       bool fdead = false;
-      for (int j = 0; j < SPG && j < tot_g; ++j) {
-        const int last = j + ((tot_g - 1 - j) / SPG) * SPG;  // last li with li % SPG == j
-        mbar_wait(&full[g * SPG + j], (uint32_t)((last / SPG) & 1), a.err, &fdead);
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        if (g >= NG) continue;
+        for (int j = 0; j < SPG && j < next[g]; ++j) {
+          const int last = j + ((next[g] - 1 - j) / SPG) * SPG;  // last li < next[g], li % SPG == j
+          mbar_wait(&full[g * SPG + j], (uint32_t)((last / SPG) & 1), a.err, &fdead);
+        }
       }
     }
   } else {
@@ -216,7 +243,7 @@ __device__ void run(const TokenArgs& a, unsigned char* smem, bool* dead) {
       xr[m][0] = elem_ok(m) ? __ldg(reinterpret_cast<const float4*>(a.x + e)) : make_float4(0, 0, 0, 0);
       xr[m][1] = elem_ok(m) ? __ldg(reinterpret_cast<const float4*>(a.x + e + 4)) : make_float4(0, 0, 0, 0);
     }
-    bool cdead = *dead;
+    bool cdead = gs.dead;
     // ---------------- phase A: gate/up partial dot products ----------------
     // The warp's share of an item goes into registers, the slot goes back to the
     // producer, then the FMAs.

@@ -5,18 +5,20 @@
 //   Stage 1 (stage1.cuh): threshold x, INT4 proxy GEMV over the kept rows
 //            into per-CTA partial sums;
 //   barrier: every partial sum is written;
-//   scores:  each CTA adds up the partials of its share of the channels and
-//            scores them, |act(g~) u~| (with the level-1 histogram of their
-//            bits for the top-k rule);
-//   barrier: every score and the histogram are complete;
-//   Stage 2 (stage2.cuh): each CTA finds the exact top-k cut (or applies the
-//            score threshold, a given list, or keeps every channel for the
-//            dense baseline), streams its selected channel records and W_down
-//            rows and writes a partial output row;
+//   scores:  each CTA adds up the partials of its own share of the channels
+//            and scores them, |act(g~) u~| (for the top-k rule counting them
+//            in the histograms of select.cuh);
+//   barrier: (top-k) the histograms are complete;
+//   Stage 2 (stage2.cuh): each CTA finds the token's exact top-k cut (or
+//            applies the score threshold) and lists its own channels past it;
+//   barrier: (top-k, threshold) every CTA's list and count is written;
+//            each CTA then takes an even share of the token's ranked
+//            selection (or of a given list, or of every channel for the
+//            dense baseline), streams those channel records and W_down rows
+//            and writes a partial output row;
 //   barrier: every partial row is complete;
 //   output:  CTA c adds the partial rows of its share of the columns in a
-//            fixed order (deterministic) and clears the histogram for the
-//            next token.
+//            fixed order (deterministic).
 //
 // The launch is cooperative (all CTAs resident, which the barriers need) and
 // programmatically dependent on the previous kernel in the stream: it waits
@@ -41,23 +43,28 @@ __global__ void __launch_bounds__(kTokenThreads, 1) token_kernel(TokenArgs a) {
   stamp(a.ts, 1);
   const bool topk = a.mode == kModeTopK;
   if (a.stage1) {
-    const int n_x = s1::run<NB>(a, smem);
+    s1::run<NB>(a, smem);
     stamp(a.ts, 2);
     grid_barrier(gs, gridDim.x, a.err);  // every CTA's Stage-1 partials are written
     stamp(a.ts, 3);
-    s1::score_channels(a, n_x, topk);
+    SelectScratch& sc = *reinterpret_cast<SelectScratch*>(smem + s2::ring_offset(a.slots, a.max_rec));
+    s1::score_channels(a, topk, sc);
     stamp(a.ts, 10);
     if (a.mode == kModeNone) return;
-    grid_barrier(gs, gridDim.x, a.err);  // every score (and the histogram) is written
-    stamp(a.ts, 14);
+    if (topk) {
+      grid_barrier(gs, gridDim.x, a.err);  // the histograms and buckets are complete
+      stamp(a.ts, 14);
+    }
   }
   if (a.mode == kModeNone) return;
-  s2::run<MAXM>(a, smem, &gs.dead);
+  s2::run<MAXM>(a, smem, gs);
   stamp(a.ts, 5);
   grid_barrier(gs, gridDim.x, a.err);  // every partial row is written; every CTA is past the cut
   stamp(a.ts, 6);
-  if (a.stage1 && topk && blockIdx.x == gridDim.x - 1)
+  if (a.stage1 && topk && blockIdx.x == gridDim.x - 1) {  // ready for the next token
     for (int i = threadIdx.x; i < kScoreBins; i += blockDim.x) a.hist[i] = 0u;
+    if (threadIdx.x < kCoarseBins) a.chist[threadIdx.x] = 0u;
+  }
   if (a.select_only) return;
 
   // out[4q .. 4q+3] for the float4 columns q of this CTA: warp w sums column
@@ -170,7 +177,7 @@ void choose_stage2(int d, int F, int num_sms, int* slots, int* groups, size_t* s
   *groups = ng;
   *slots = s;
   size_t region = (size_t)s * slot_bytes;
-  if (region < select_smem_bytes(F)) region = select_smem_bytes(F);  // the select's scratch and keys
+  if (region < select_smem_bytes(F)) region = select_smem_bytes(F);  // the selection's scratch and keys
   if (region < (size_t)ng * d * 4) region = (size_t)ng * d * 4;       // the groups' partial rows
   *smem = s2::ring_offset(s, max_rec) + region;
 }
@@ -220,6 +227,10 @@ cudaError_t launch_token(const prox_layer* L, const TokenLaunch& m, cudaStream_t
   a.s_tilde = m.taps.s_tilde ? m.taps.s_tilde : (m.proxy_values ? L->ws.s_tilde : nullptr);
   a.s_tilde_src = L->ws.s_tilde;
   a.hist = L->ws.hist;
+  a.chist = L->ws.chist;
+  a.bucket = L->ws.bucket;
+  a.sel_list = L->ws.sel_list;
+  a.sel_cnt = L->ws.sel_cnt;
   a.stats = L->ws.stats;
   a.part = L->ws.s1_part;
   a.ypart = L->ws.ypart;

@@ -26,7 +26,7 @@ struct TokenArgs {
   const float* x;        // [d] this token's input
   float* out;            // [d] this token's output (Stage 2 modes)
   // library-owned weights
-  const uint8_t* pq;     // INT4 proxy codes [d][F], gate/up interleaved per 16 B
+  const uint8_t* pq;     // INT4 proxy codes [C][d][512 B], gate/up interleaved per 16 B
   const __half* ps;      // fp16 scales [G][F/32][2][32]
   const uint16_t* wgu;   // bf16 channel records [F][2d]
   const uint16_t* wd;    // bf16 W_down rows [F][d]
@@ -50,7 +50,11 @@ struct TokenArgs {
   float* scores;         // |act(g~) u~| [F]
   float* s_tilde;        // Stage 1 writes act(g~) u~ here when non-null [F]
   const float* s_tilde_src;  // A3 Stage 2 reads it here
-  uint32_t* hist;        // [kScoreBins] level-1 histogram of the scores' bits 30..18
+  uint32_t* hist;        // [kScoreBins] fine histogram of the scores' bits 30..18
+  uint32_t* chist;       // [128] coarse histogram of the scores' bits 30..24
+  uint2* bucket;         // [kScoreBins][kBucketCap] (key, channel) per fine bin
+  int32_t* sel_list;     // [F] CTA c's selected channels from its range's first channel on
+  int32_t* sel_cnt;      // [P] CTA c's selected count
   unsigned long long* stats;
   float* part;           // Stage-1 partial sums [P][2][1024]
   float* ypart;          // Stage-2 partial output rows [P][d]
@@ -72,8 +76,8 @@ struct TokenArgs {
 // 3 partials visible (barrier), 4 channels selected, 5 partial output row
 // written, 6 partial rows visible (barrier), 7 output written; 8 kept rows
 // compacted, 9 Stage-1 row loop done, 10 scores of the CTA's channels written,
-// 14 all scores visible (barrier); 11 Stage-2 ring set up, 12 gate/up phase
-// done; slot 13 holds the CTA's channel count, not a time.
+// 14 the histograms complete (barrier); 11 Stage-2 ring set up, 12 gate/up
+// phase done; slot 13 holds the CTA's channel count, not a time.
 __device__ __forceinline__ void stamp(unsigned long long* ts, int i) {
   if (ts && threadIdx.x == 0) {
     unsigned long long t;
@@ -87,6 +91,9 @@ __device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long
   asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
   return v;
 }
+__device__ __forceinline__ void st_relaxed_u64(unsigned long long* p, unsigned long long v) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
 __device__ __forceinline__ void red_add_u64(unsigned long long* p, unsigned long long v) {
   asm volatile("red.relaxed.gpu.global.add.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
@@ -96,10 +103,12 @@ __device__ __forceinline__ void fence_acq_rel_gpu() {
 
 // Grid-wide barriers of one launch whose CTAs are all resident (cooperative
 // launch, one CTA per SM).  The layer's 64-bit arrival counter only grows:
-// thread 0 of every CTA reads it once when the launch starts (the previous
-// launch on the layer is complete by then, so every CTA reads the same value,
-// base), and barrier i of the launch is complete once the counter reaches
-// base + i * expected.  A CTA's thread 0, after a bar.sync, releases the CTA's
+// thread 0 of every CTA reads it once when the launch starts; the previous
+// launch on the layer is complete by then and every barrier adds exactly
+// gridDim.x arrivals, so rounding the value read down to a multiple of
+// gridDim.x gives every CTA the same base even when faster CTAs have already
+// arrived at the first barrier.  Barrier i of the launch is complete once the
+// counter reaches base + i * expected.  A CTA's thread 0, after a bar.sync, releases the CTA's
 // writes (fence) and arrives with a reduction (no round trip); it then polls
 // the counter and acquires (fence) once the target is reached.  So every
 // write made before the barrier by any thread of any CTA is visible to every
@@ -117,7 +126,12 @@ struct GridSync {
 __device__ __forceinline__ GridSync grid_sync_begin(unsigned long long* ctr) {
   GridSync g;
   g.ctr = ctr;
-  g.base = threadIdx.x == 0 ? ld_relaxed_u64(ctr) : 0ull;
+  if (threadIdx.x == 0) {
+    const unsigned long long v = ld_relaxed_u64(ctr);
+    g.base = v - v % gridDim.x;
+  } else {
+    g.base = 0ull;
+  }
   g.n = 0;
   g.dead = false;
   return g;
@@ -134,6 +148,7 @@ __device__ __forceinline__ void grid_barrier(GridSync& g, unsigned expected, int
     if (!g.dead) {
       const long long t0 = clock64();
       while (ld_relaxed_u64(g.ctr) < target) {
+        __nanosleep(64);
         if (clock64() - t0 > kWaitLimitCycles) {
           atomicOr(err, PROX_DEVERR_WAIT_TIMEOUT);
           g.dead = true;

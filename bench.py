@@ -329,7 +329,7 @@ def phase_breakdown(layers, xs, outs, n, stream):
     CTA reaches the stamp; times are from the first CTA's entry."""
     import torch
     P = layers[0].info()["stage1_ctas"]
-    ph = torch.zeros((P, 16), dtype=torch.int64, device="cuda")
+    ph = torch.zeros((P, 24), dtype=torch.int64, device="cuda")
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
     for e in evs:
         e.record(stream)
@@ -337,6 +337,7 @@ def phase_breakdown(layers, xs, outs, n, stream):
     # slot -> name (include/prox.h, prox_ffn_forward_profiled); 13 is a count
     names = {0: "entry", 1: "prev_done", 8: "stage1_compact", 9: "stage1_loop",
              2: "stage1_partials", 3: "barrier_a", 10: "scored", 14: "barrier_b",
+             15: "topk_cut",
              4: "selected", 11: "stage2_ring", 12: "stage2_gate_up", 5: "stage2",
              6: "barrier_c", 7: "out"}
     per, kt = [], []
@@ -349,6 +350,9 @@ def phase_breakdown(layers, xs, outs, n, stream):
             if t >= 4:
                 a = ph.cpu().numpy().astype(np.int64)
                 a[:, 13] = a[:, 0].min()
+                for col in (15, 16, 17, 18):  # written by one CTA only
+                    nz = a[:, col] > 0
+                    a[~nz, col] = a[nz, col].max() if nz.any() else a[:, 0].min()
                 per.append((a.max(0) - a[:, 0].min()) / 1e3)
                 kt.append(evs[0].elapsed_time(evs[1]) * 1e3)
     per = np.stack(per)

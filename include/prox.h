@@ -290,13 +290,15 @@ PROX_API prox_status prox_ffn_forward_host(prox_layer* layer, const float* x_hos
 /* prox_ffn_forward for one token with cudaEvent_t events_host[2] (passed as
  * void*) recorded right before and right after the token's kernel, which is
  * launched without programmatic overlap so the interval is its duration.
- * phase_ns (device, may be NULL): uint64 [stage1_ctas][16] receiving, per CTA,
+ * phase_ns (device, may be NULL): uint64 [stage1_ctas][24] receiving, per CTA,
  * the GPU global timer (ns) at: 0 kernel entry, 1 the previous kernel of the
  * stream complete, 2 Stage 1 done, 3 all scores visible (first grid barrier),
  * 4 channels selected, 5 partial output row written, 6 second grid barrier,
- * 7 output written, 8 kept rows compacted, 9 Stage-1 row loop done, 10 Stage-1
- * partials written, 11 Stage-2 ring set up, 12 gate/up phase done; slot 13
- * holds the CTA's number of selected channels; 14 and 15 are unused. */
+ * 7 output written, 8 kept rows compacted, 9 Stage-1 row loop done, 10 the
+ * CTA's scores written, 11 Stage-2 ring set up, 12 gate/up phase done, 14 the
+ * score histograms complete (top-k rule: second grid barrier), 15 the top-k
+ * cut found; slot 13 holds the CTA's number of selected channels; the other
+ * slots are 0. */
 PROX_API prox_status prox_ffn_forward_profiled(const prox_layer* layer, const float* x, float* out,
                                                void* const* events_host, uint64_t* phase_ns,
                                                void* stream);
