@@ -20,7 +20,7 @@ from ._lib import (ACT_GELU_ERF, ACT_GELU_TANH, ACT_SILU, DEVERR_MASK_INDEX, DEV
                    MASK_THRESHOLD, MASK_TOPK, STAGE2_EXACT, STAGE2_PROXY_VALUES, LayerInfo,
                    ProxError, check, last_error, lib)
 
-__all__ = ["Layer", "pack_proxy", "calibrate_thresholds", "rmsnorm", "copy", "version",
+__all__ = ["Layer", "phase_times_us", "pack_proxy", "calibrate_thresholds", "rmsnorm", "copy", "version",
            "effective_sparsity", "allocate_sparsity", "runtime_sparsity", "ALPHA",
            "ACT_SILU", "ACT_GELU_TANH", "ACT_GELU_ERF", "STAGE2_EXACT", "STAGE2_PROXY_VALUES",
            "ProxError", "DEVERR_MASK_INDEX", "DEVERR_WAIT_TIMEOUT", "MASK_TOPK", "MASK_THRESHOLD",
@@ -142,6 +142,24 @@ def copy(src: torch.Tensor, dst: torch.Tensor, stream=None) -> None:
 
 
 ALPHA = 1.0 / 3.0  # proxy-projection cost the paper allocates with (Prox §4.2)
+
+
+def phase_times_us(stamps) -> "np.ndarray":
+    """Raw stamps of Layer.forward_profiled ([P, 24] int64, host or device) as
+    float64 microseconds from the earliest CTA entry, NaN where a CTA wrote no
+    stamp; slot 13 (a channel count) is passed through.  Each CTA's cycle
+    counts are placed on the global-timer line by its entry and exit readings
+    (slots 0 / 22 and 21 / 23)."""
+    import numpy as np
+    a = np.asarray(stamps.cpu() if hasattr(stamps, "cpu") else stamps).astype(np.float64)
+    clk0, clk1, gt0, gt1 = a[:, 0:1], a[:, 21:22], a[:, 22:23], a[:, 23:24]
+    ns_per_clk = (gt1 - gt0) / np.maximum(clk1 - clk0, 1.0)
+    t = gt0 + (a - clk0) * ns_per_clk
+    t[a == 0] = np.nan
+    t[:, 22], t[:, 23] = a[:, 22], a[:, 23]
+    out = (t - np.nanmin(gt0)) / 1e3
+    out[:, 13] = a[:, 13]
+    return out
 
 
 def effective_sparsity(s1: float, s2: float, alpha: float = ALPHA) -> float:
@@ -327,8 +345,9 @@ class Layer:
                          phase_ns: torch.Tensor | None = None, stream=None):
         """One token with its kernel bracketed by 2 torch.cuda.Event(enable_timing=True)
         (no programmatic overlap).  phase_ns: optional int64 CUDA tensor
-        [stage1_ctas, 24] receiving each CTA's phase stamps (GPU global timer, ns;
-        slot meanings in include/prox.h)."""
+        [stage1_ctas, 24] receiving each CTA's raw phase stamps (SM cycle counts
+        plus the global timer at entry and exit; slot meanings in
+        include/prox.h); phase_times_us turns them into one time line."""
         _dev(x, torch.float32, "x")
         _dev(out, torch.float32, "out")
         _one_token(x, self.d_model)

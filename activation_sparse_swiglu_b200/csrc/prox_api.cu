@@ -150,18 +150,21 @@ prox_status alloc_workspace(prox_layer* L) {
   const size_t o_st = take(F * 4);
   const size_t o_g = take(F * 4);
   const size_t o_u = take(F * 4);
-  const size_t o_hist = take(prox::kScoreBins * 4);
-  const size_t o_chist = take(128 * 4);
-  const size_t o_bucket = take((size_t)prox::kScoreBins * prox::kBucketCap * 8);
-  const size_t o_slist = take(F * 4);
-  const size_t o_scnt = take((size_t)prox::kMaxCtas * 4);
   const size_t o_mask = take(F * 4);
   const size_t o_idx = take(F * 4);
-  const size_t o_s1p = take(prox::stage1_part_floats(L->P) * 4);
-  const size_t o_ypart = take((size_t)L->P * d * 4);
   const size_t o_stats = take(24);
-  const size_t o_gbar = take(8);
   const size_t o_err = take(4);
+  const size_t o_xchg = off;
+  const size_t o_hist = take(2 * prox::kScoreBins * 4);
+  const size_t o_chist = take(2 * 128 * 4);
+  const size_t o_bucket = take((size_t)prox::kScoreBins * prox::kBucketCap * 16);
+  const size_t o_st64 = take(F * 8);
+  const size_t o_slist = take(F * 8);
+  const size_t o_scnt = take((size_t)prox::kMaxCtas * 8);
+  const size_t o_s1p = take(prox::stage1_part_floats(L->P) * 8);
+  const size_t o_ypart = take((size_t)L->P * d * 8);
+  const size_t o_gbar = take(8);
+  const size_t xchg_bytes = off - o_xchg;
   const size_t o_in = take((size_t)kHostChunkTokens * d * 4);
   const size_t o_out = take((size_t)kHostChunkTokens * d * 4);
   void* base = nullptr;
@@ -177,13 +180,16 @@ prox_status alloc_workspace(prox_layer* L) {
   w.u_dbg = reinterpret_cast<float*>(b + o_u);
   w.hist = reinterpret_cast<uint32_t*>(b + o_hist);
   w.chist = reinterpret_cast<uint32_t*>(b + o_chist);
-  w.bucket = reinterpret_cast<uint2*>(b + o_bucket);
-  w.sel_list = reinterpret_cast<int32_t*>(b + o_slist);
-  w.sel_cnt = reinterpret_cast<int32_t*>(b + o_scnt);
+  w.bucket = reinterpret_cast<unsigned long long*>(b + o_bucket);
+  w.st64 = reinterpret_cast<unsigned long long*>(b + o_st64);
+  w.sel_list = reinterpret_cast<unsigned long long*>(b + o_slist);
+  w.sel_cnt = reinterpret_cast<unsigned long long*>(b + o_scnt);
+  w.xchg = b + o_xchg;
+  w.xchg_bytes = xchg_bytes;
   w.sel_mask = reinterpret_cast<int32_t*>(b + o_mask);
   w.idx_s = reinterpret_cast<int32_t*>(b + o_idx);
-  w.s1_part = reinterpret_cast<float*>(b + o_s1p);
-  w.ypart = reinterpret_cast<float*>(b + o_ypart);
+  w.s1_part = reinterpret_cast<unsigned long long*>(b + o_s1p);
+  w.ypart = reinterpret_cast<unsigned long long*>(b + o_ypart);
   w.stats = reinterpret_cast<unsigned long long*>(b + o_stats);
   w.gbar = reinterpret_cast<unsigned long long*>(b + o_gbar);
   w.err = reinterpret_cast<int*>(b + o_err);
@@ -515,11 +521,11 @@ prox_status prox_layer_error(prox_layer* L, int32_t* word_host, void* stream) {
   PROX_CUDA(cudaMemsetAsync(L->ws.err, 0, 4, s), "clear error word");
   PROX_CUDA(cudaStreamSynchronize(s), "cudaStreamSynchronize");
   if (v & PROX_DEVERR_WAIT_TIMEOUT) {
-    // A token whose wait ran out may have left the grid-barrier counter and
-    // the histograms mid-way: start the next token clean.
-    PROX_CUDA(cudaMemsetAsync(L->ws.gbar, 0, 8, s), "reset grid barrier");
-    PROX_CUDA(cudaMemsetAsync(L->ws.hist, 0, prox::kScoreBins * 4, s), "reset histogram");
-    PROX_CUDA(cudaMemsetAsync(L->ws.chist, 0, 128 * 4, s), "reset coarse histogram");
+    // A token whose wait ran out may have left the launch counter, the
+    // histograms and the tagged exchange words mid-way: start the next token
+    // clean (a counter back at 0 repeats earlier tags, so every tagged word
+    // is cleared with it).
+    PROX_CUDA(cudaMemsetAsync(L->ws.xchg, 0, L->ws.xchg_bytes, s), "reset exchange words");
     PROX_CUDA(cudaStreamSynchronize(s), "cudaStreamSynchronize");
   }
   *word_host = v;

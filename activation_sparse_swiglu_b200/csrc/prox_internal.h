@@ -36,17 +36,22 @@ struct Workspace {
   float* s_tilde = nullptr;       // act(g~) u~ [F], signed (proxy-values Stage 2 only)
   float* g_dbg = nullptr;         // debug g~ [F]
   float* u_dbg = nullptr;         // debug u~ [F]
-  uint32_t* hist = nullptr;       // [kScoreBins] scores' bits 30..18, zero between tokens
-  uint32_t* chist = nullptr;      // [128] scores' bits 30..24, zero between tokens
-  uint2* bucket = nullptr;        // [kScoreBins][kBucketCap] (key, channel) per fine bin
-  int32_t* sel_list = nullptr;    // [F] each CTA's selected channels, at its range's start
-  int32_t* sel_cnt = nullptr;     // [kMaxCtas] each CTA's selected count
   int32_t* sel_mask = nullptr;    // [F] debug: 1 where the channel is selected
   int32_t* idx_s = nullptr;       // [F] debug: selected channels (first k valid)
-  float* s1_part = nullptr;       // Stage-1 partial sums [P][2][1024]
-  float* ypart = nullptr;         // Stage-2 partial output rows [P][d]
   unsigned long long* stats = nullptr;  // [3] sum n_x, tokens, sum of selected channels
-  unsigned long long* gbar = nullptr;  // grid-barrier arrival counter of the per-token kernel
+  // What the CTAs of one per-token launch exchange (one contiguous range,
+  // cleared after a wait ran out).  Tagged words: payload | launch tag << 32.
+  uint32_t* hist = nullptr;       // [2][kScoreBins] scores' bits 30..18, by launch parity
+  uint32_t* chist = nullptr;      // [2][kCoarseBins] scores' bits 30..24, by launch parity
+  unsigned long long* bucket = nullptr;  // [kScoreBins][kBucketCap][2] tagged (key, channel)
+  unsigned long long* st64 = nullptr;    // [F] tagged bits of act(g~) u~
+  unsigned long long* sel_list = nullptr;  // [F] tagged selected channels, at each CTA's range start
+  unsigned long long* sel_cnt = nullptr;   // [kMaxCtas] tagged selected count per CTA
+  unsigned long long* s1_part = nullptr;   // [P][2][1024] tagged Stage-1 partial sums
+  unsigned long long* ypart = nullptr;     // [P][d] tagged Stage-2 partial output rows
+  unsigned long long* gbar = nullptr;  // launch counter: every CTA adds 1 when it ends
+  void* xchg = nullptr;           // the exchange range, for clearing
+  size_t xchg_bytes = 0;
   int* err = nullptr;             // device error word
   float* stage_in = nullptr;      // host-path staging [kHostChunkTokens][d]
   float* stage_out = nullptr;

@@ -7,10 +7,10 @@
 // global histograms, a fine one over bits 30..18 (8192 bins) and a coarse one
 // over bits 30..24 (128 bins, each the sum of 64 fine bins), adding per bin
 // the counts it first gathered in shared memory; the fine bin's old count
-// places the CTA's (key, channel) pairs of that bin in the bin's bucket.  After a grid barrier every CTA finds the exact cut itself,
-// reading only small pieces:
-//   1. the coarse histogram (512 bytes): the coarse bin holding the k-th
-//      largest key;
+// places the CTA's (key, channel) pairs of that bin in the bin's bucket.
+// Every CTA then finds the exact cut itself, reading only small pieces:
+//   1. the coarse histogram (512 bytes), once complete: the coarse bin
+//      holding the k-th largest key;
 //   2. that coarse bin's 64 fine bins: the fine bin b1 holding it and the
 //      rank wanted inside b1;
 //   3. b1's bucket: the candidates, ranked by (key descending, index
@@ -23,6 +23,7 @@
 #pragma once
 #include "prox_device.cuh"
 #include "prox_internal.h"
+#include "token_args.cuh"
 
 namespace prox {
 
@@ -163,8 +164,15 @@ __device__ int radix_tie(Items items, uint32_t T, int want, SelectScratch& sc) {
 // Among bins read in descending bin order (thread t holds the count of the
 // t-th largest bin, 0 past the last), the one holding the krem-th largest
 // key: writes its position t and the rank wanted inside it to misc[0],
-// misc[1] and its count to misc[2].  Every thread calls it.
-__device__ __forceinline__ void find_bin_desc(int count, int krem, SelectScratch& sc) {
+// misc[1] and its count to misc[2] (position 0, rank 1, count 0 when the
+// counts hold fewer than krem keys).  Returns the sum of the counts.  Every
+// thread calls it.
+__device__ __forceinline__ int find_bin_desc(int count, int krem, SelectScratch& sc) {
+  if (threadIdx.x == 0) {
+    sc.misc[0] = 0;
+    sc.misc[1] = 1;
+    sc.misc[2] = 0;
+  }
   int total;
   const int above = block_exclusive_scan(count, sc.scan, &total);
   if (count > 0 && above < krem && above + count >= krem) {
@@ -173,22 +181,38 @@ __device__ __forceinline__ void find_bin_desc(int count, int krem, SelectScratch
     sc.misc[2] = count;
   }
   __syncthreads();
+  return total;
 }
 
-// The exact cut of the token; every CTA calls it once the histograms and
-// buckets are complete (blockDim.x >= kCoarseBins).  1 <= k <= F.
-__device__ TopkCut select_cut(const uint32_t* hist, const uint32_t* chist, const uint2* bucket,
-                              const float* scores, int F, int k, SelectScratch& sc) {
+// The exact cut of the launch; every CTA calls it once it has added its own
+// counts (blockDim.x >= kCoarseBins).  1 <= k <= F.  The histograms are
+// complete when the coarse counts add up to F and the fine counts under a
+// coarse bin add up to its count (every count only grows), so the CTA polls
+// them until they do; bucket entries and keys are tagged words.  A wait that
+// runs out sets PROX_DEVERR_WAIT_TIMEOUT and goes on with what it has.
+__device__ TopkCut select_cut(const uint32_t* hist, const uint32_t* chist,
+                              const unsigned long long* bucket, const unsigned long long* st64, int F,
+                              int k, SelectScratch& sc, uint32_t tag, int* err,
+                              unsigned long long* ts) {
   const int tid = threadIdx.x;
   // 1. the coarse bin (bins read from the top)
-  find_bin_desc(tid < kCoarseBins ? (int)__ldcg(chist + (kCoarseBins - 1 - tid)) : 0, k, sc);
+  long long t0 = clock64();
+  for (;;) {
+    const int cnt = tid < kCoarseBins ? (int)ld_relaxed_u32(chist + (kCoarseBins - 1 - tid)) : 0;
+    if (find_bin_desc(cnt, k, sc) == F || !wait_more(t0, err)) break;
+  }
+  stamp(ts, 14);
   const int cb = kCoarseBins - 1 - sc.misc[0];
   const int k1 = sc.misc[1];
+  const int ncb = sc.misc[2];
   __syncthreads();
   // 2. its fine bins
   const int fb0 = cb * kFinePerCoarse;
-  find_bin_desc(tid < kFinePerCoarse ? (int)__ldcg(hist + fb0 + (kFinePerCoarse - 1 - tid)) : 0, k1,
-                sc);
+  t0 = clock64();
+  for (;;) {
+    const int cnt = tid < kFinePerCoarse ? (int)ld_relaxed_u32(hist + fb0 + (kFinePerCoarse - 1 - tid)) : 0;
+    if (find_bin_desc(cnt, k1, sc) == ncb || !wait_more(t0, err)) break;
+  }
   const uint32_t b1 = (uint32_t)(fb0 + kFinePerCoarse - 1 - sc.misc[0]);
   const int krem = sc.misc[1];
   const int n1 = sc.misc[2];
@@ -198,9 +222,16 @@ __device__ TopkCut select_cut(const uint32_t* hist, const uint32_t* chist, const
     // 3. the candidates, ranked: the one with krem - 1 larger (key, ~channel)
     // composites is the cut
     if (tid < n1) {
-      const uint2 kc = __ldcg(bucket + (size_t)b1 * kBucketCap + tid);
-      sc.ck[tid] = kc.x;
-      sc.ci[tid] = (int)kc.y;
+      const unsigned long long* src = bucket + ((size_t)b1 * kBucketCap + tid) * 2;
+      ulonglong2 kc = ld_tag2(src);
+      t0 = clock64();
+      while (!(tag_ok(kc.x, tag) && tag_ok(kc.y, tag)) && wait_more(t0, err)) kc = ld_tag2(src);
+      sc.ck[tid] = (uint32_t)kc.x;
+      sc.ci[tid] = (int)(uint32_t)kc.y;
+    }
+    if (tid == 0) {
+      sc.misc[7] = 0;
+      sc.misc[12] = F;
     }
     __syncthreads();
     if (tid < n1) {
@@ -220,10 +251,15 @@ __device__ TopkCut select_cut(const uint32_t* hist, const uint32_t* chist, const
     return cut;
   }
   // 3'. b1 overflowed its bucket (many equal scores): radix select over every
-  // key, loaded into shared memory
+  // key (the magnitude bits of the tagged act(g~) u~), loaded into shared
+  // memory
   uint32_t* sk = select_keys(sc);
-  for (int e = tid; e < (F >> 2); e += blockDim.x)
-    reinterpret_cast<uint4*>(sk)[e] = __ldcg(reinterpret_cast<const uint4*>(scores) + e);
+  for (int e = tid; e < F; e += blockDim.x) {
+    unsigned long long w = ld_tag(st64 + e);
+    t0 = clock64();
+    while (!tag_ok(w, tag) && wait_more(t0, err)) w = ld_tag(st64 + e);
+    sk[e] = (uint32_t)w & 0x7FFFFFFFu;
+  }
   __syncthreads();
   const int per = (F + (int)blockDim.x - 1) / (int)blockDim.x;
   const int j0 = min(tid * per, F), j1 = min(j0 + per, F);

@@ -42,6 +42,7 @@ constexpr int NT = NW * 32;
 static_assert(kMaxDModel % NT == 0, "rows per thread");
 constexpr int SLICE = 512;   // bytes (= channels of both proxies) per column slice
 constexpr int PART = 1024;   // partial values per slice: 32 chunks x 32 channels
+constexpr int PARTP = 32 * 33;  // the same in shared memory, rows of 32 padded to 33
 constexpr int U = 4;         // rows per batch
 constexpr int BATCH = U * SLICE;
 static_assert(kOwnMax <= kTokenThreads, "scoring takes one channel per thread");
@@ -99,15 +100,18 @@ __device__ __forceinline__ int cta_of(int t, int T, int P) {
 }
 
 // Scores the channels [F c / P, F (c + 1) / P) of CTA c (at most kOwnMax,
-// so one per thread) once every CTA's partials are visible: thread t adds the
-// gate and up partials of channel c0 + t over the CTAs whose pair ranges
-// cover its slice, in CTA order.  For the top-k rule the CTA first counts its
-// keys in shared-memory histograms; one thread per non-empty fine bin then
+// so one per thread): thread t adds the gate and up partials of channel
+// c0 + t over the CTAs whose pair ranges cover its slice, in CTA order,
+// polling each tagged partial until this launch's has arrived.  It writes the
+// score, keeps its key (the score's bits) in shared memory and publishes the
+// signed act(g~) u~ as a tagged word.  For the top-k rule the CTA first counts
+// its keys in shared-memory histograms; one thread per non-empty fine bin then
 // adds the CTA's count to the global bin, whose old value places the CTA's
-// keys of that bin in the bin's bucket, and the coarse counts are added the
-// same way, so a global bin sees one atomic per CTA, not one per channel.
-// Every thread of the CTA calls it.
-__device__ void score_channels(const TokenArgs& a, bool histogram, SelectScratch& sel) {
+// keys of that bin in the bin's bucket (tagged), and the coarse counts are
+// added the same way, so a global bin sees one atomic per CTA, not one per
+// channel.  Every thread of the CTA calls it.
+__device__ void score_channels(const TokenArgs& a, bool histogram, SelectScratch& sel, uint32_t tag,
+                               uint32_t* hist, uint32_t* chist) {
   const int P = gridDim.x, cta = blockIdx.x, tid = threadIdx.x;
   const int c0 = (int)(((long long)a.F * cta) / P);
   const int c1 = (int)(((long long)a.F * (cta + 1)) / P);
@@ -123,41 +127,54 @@ __device__ void score_channels(const TokenArgs& a, bool histogram, SelectScratch
   uint32_t key = 0u, fb = 0u, rank = 0u;
   if (mine) {
     const int c = ch / SLICE, m = ch % SLICE;
-    // channel m of the slice is block blk = m / 32, channel j = m % 32 of it:
-    // its gate and up sums are the partial elements j*32 + 2*blk and + 1
-    const int e = (m & 31) * 32 + 2 * (m >> 5);
+    const int e = 2 * m;  // channel m's gate and up sums in a CTA's partial row
     const int i_lo = cta_of(c * a.d, T, P);
     const int i_hi = cta_of((c + 1) * a.d - 1, T, P);
     float g = 0.f, u = 0.f;
     for (int i0 = i_lo; i0 <= i_hi; i0 += 8) {
-      float2 v[8];
+      ulonglong2 v[8];
+      int off[8];  // element offset of CTA i0 + q's partial pair, or -1
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
         const int i = i0 + q;
-        v[q] = make_float2(0.f, 0.f);
+        off[q] = -1;
+        v[q] = make_ulonglong2(tag_word(0u, tag), tag_word(0u, tag));
         if (i <= i_hi) {
           const unsigned tlo = (unsigned)T * (unsigned)i / (unsigned)P;
           const unsigned thi = (unsigned)T * (unsigned)(i + 1) / (unsigned)P;
           if (thi > tlo) {  // CTA i holds pairs; slice c is its first or second
-            const int off = (i * 2 + (c - (int)(tlo / (unsigned)a.d))) * PART;
-            v[q] = __ldcg(reinterpret_cast<const float2*>(a.part + off + e));
+            off[q] = (i * 2 + (c - (int)(tlo / (unsigned)a.d))) * PART + e;
+            v[q] = ld_tag2(a.part + off[q]);
           }
         }
       }
+      const long long t0 = clock64();
+      for (;;) {
+        bool all = true;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) all = all && tag_ok(v[q].x, tag) && tag_ok(v[q].y, tag);
+        if (all || !wait_more(t0, a.err)) break;
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          if (off[q] >= 0 && !(tag_ok(v[q].x, tag) && tag_ok(v[q].y, tag))) v[q] = ld_tag2(a.part + off[q]);
+      }
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
-        g += v[q].x;
-        u += v[q].y;
+        g += __uint_as_float((uint32_t)v[q].x);
+        u += __uint_as_float((uint32_t)v[q].y);
       }
     }
+    stamp(a.ts, 3);
     const float sv = act_f32(g, a.act) * u;
     const float sc = fabsf(sv);
     a.scores[ch] = sc;
+    st_tag(a.st64 + ch, tag_word(__float_as_uint(sv), tag));
     if (a.s_tilde) a.s_tilde[ch] = sv;
     if (a.g_dbg) a.g_dbg[ch] = g;
     if (a.u_dbg) a.u_dbg[ch] = u;
     key = __float_as_uint(sc);
     sel.own[tid] = key;
+
     if (histogram) {
       fb = key >> kScoreShift;
       rank = atomicAdd(&fine[fb], 1u);
@@ -166,13 +183,14 @@ __device__ void score_channels(const TokenArgs& a, bool histogram, SelectScratch
   }
   if (!histogram) return;
   __syncthreads();
-  if (mine && rank == 0u) fine[fb] = atomicAdd(a.hist + fb, fine[fb]);
+  if (mine && rank == 0u) fine[fb] = atomicAdd(hist + fb, fine[fb]);
   for (int i = tid; i < kCoarseBins; i += blockDim.x)
-    if (sel.coarse[i]) atomicAdd(a.chist + i, sel.coarse[i]);
+    if (sel.coarse[i]) atomicAdd(chist + i, sel.coarse[i]);
   __syncthreads();
   if (mine) {
     const uint32_t slot = fine[fb] + rank;
-    if (slot < (uint32_t)kBucketCap) a.bucket[fb * kBucketCap + slot] = make_uint2(key, (uint32_t)ch);
+    if (slot < (uint32_t)kBucketCap)
+      st_tag2(a.bucket + ((size_t)fb * kBucketCap + slot) * 2, tag_word(key, tag), tag_word((uint32_t)ch, tag));
   }
 }
 
@@ -180,15 +198,16 @@ __device__ void score_channels(const TokenArgs& a, bool histogram, SelectScratch
 // the CTA's kept rows, the stash of the warp that crosses a slice boundary.
 template <int NB>
 constexpr size_t smem_bytes(int lmax) {
-  return (size_t)NW * NB * BATCH + (size_t)NW * PART * 4 + (size_t)lmax * 12 +
-         (size_t)PART * 4 + (37 + kTokenThreads) * 4;
+  return (size_t)NW * NB * BATCH + (size_t)NW * PARTP * 4 + (size_t)lmax * 12 +
+         (size_t)PARTP * 4 + (37 + kTokenThreads) * 4;
 }
 
 // The row loop of Stage 1: the CTA's partial sums of the slices its pair
-// range touches go to a.part.  Every thread of the CTA calls it; warps NW and
-// above take no rows.
+// range touches go to a.part as tagged words (the tag from the launch
+// counter read at the kernel's start).  Every thread of the CTA calls it;
+// warps NW and above take no rows.
 template <int NB>
-__device__ void run(const TokenArgs& a, unsigned char* smem) {
+__device__ void run(const TokenArgs& a, unsigned char* smem, unsigned long long counter) {
   constexpr int RING = NB * BATCH;  // ring bytes per warp
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int P = gridDim.x, cta = blockIdx.x;
@@ -196,11 +215,11 @@ __device__ void run(const TokenArgs& a, unsigned char* smem) {
   const Magic mg = a.mg;
 
   unsigned char* ring = smem;                                        // [NW][RING]
-  float* s_tot = reinterpret_cast<float*>(smem + NW * RING);         // [NW][PART]
-  int2* s_rx = reinterpret_cast<int2*>(s_tot + NW * PART);           // [lmax] (offset, x)
+  float* s_tot = reinterpret_cast<float*>(smem + NW * RING);         // [NW][PARTP]
+  int2* s_rx = reinterpret_cast<int2*>(s_tot + NW * PARTP);          // [lmax] (offset, x)
   int* s_key = reinterpret_cast<int*>(s_rx + a.lmax);                // [lmax] segment key
-  float* s_stash = reinterpret_cast<float*>(s_key + a.lmax);         // [PART]
-  int* s_scan = reinterpret_cast<int*>(s_stash + PART);              // [33]
+  float* s_stash = reinterpret_cast<float*>(s_key + a.lmax);         // [PARTP]
+  int* s_scan = reinterpret_cast<int*>(s_stash + PARTP);             // [33]
   int* s_m = s_scan + 33;                                            // [4]
   int* s_src = s_m + 4;                                              // [kTokenThreads]
 
@@ -279,9 +298,9 @@ __device__ void run(const TokenArgs& a, unsigned char* smem) {
     const int nbw = (wl1 - wl0 + U - 1) / U;
     unsigned char* wring = ring + warp * RING + lane * 16;
     const uint8_t* pq_lane = a.pq + lane * 16;
-    float* wtot = s_tot + warp * PART + lane;  // element j*32 + lane: channel j of the chunk
+    float* wtot = s_tot + warp * PARTP + lane;  // element j*32 + lane (at j*33 + lane): channel j of the chunk
 #pragma unroll
-    for (int j = 0; j < 32; ++j) wtot[j * 32] = 0.f;
+    for (int j = 0; j < 32; ++j) wtot[j * 33] = 0.f;
     // Only the last slice can be narrower than 512 bytes; a warp with rows there
     // checks each lane's chunk before copying it.
     const bool checked = (a.F % SLICE) != 0 && wl1 > wl0 &&
@@ -319,8 +338,8 @@ __device__ void run(const TokenArgs& a, unsigned char* smem) {
         for (int m = 0; m < 4; ++m) {
           const int h = qd * 4 + m;
           const float2 s2 = __half22float2(*reinterpret_cast<const __half2*>(&sw[m]));
-          wtot[(2 * h) * 32] = fmaf(s2.x, acc[h].x, wtot[(2 * h) * 32]);
-          wtot[(2 * h + 1) * 32] = fmaf(s2.y, acc[h].y, wtot[(2 * h + 1) * 32]);
+          wtot[(2 * h) * 33] = fmaf(s2.x, acc[h].x, wtot[(2 * h) * 33]);
+          wtot[(2 * h + 1) * 33] = fmaf(s2.y, acc[h].y, wtot[(2 * h + 1) * 33]);
           acc[h] = make_float2(0.f, 0.f);
         }
       }
@@ -355,8 +374,8 @@ __device__ void run(const TokenArgs& a, unsigned char* smem) {
               // the warp crosses into the next slice: park the first slice's sums
 #pragma unroll
               for (int j2 = 0; j2 < 32; ++j2) {
-                s_stash[j2 * 32 + lane] = wtot[j2 * 32];
-                wtot[j2 * 32] = 0.f;
+                s_stash[j2 * 33 + lane] = wtot[j2 * 33];
+                wtot[j2 * 33] = 0.f;
               }
             }
             cur_key = key;
@@ -391,21 +410,29 @@ __device__ void run(const TokenArgs& a, unsigned char* smem) {
   }
   __syncthreads();
   const int nsl = span > first ? 2 : 1;  // slices the CTA's pair range touches
-  for (int e = tid; e < PART; e += blockDim.x) {
+  const uint32_t tag = launch_tag(counter);  // (the counter was loaded at the kernel's start)
+  // Element e = j*32 + 2*blk + h of the sums is the gate (h = 0) or up
+  // (h = 1) sum of channel m = blk*32 + j of the slice; it is stored at
+  // 2m + h, so the scoring threads (one per channel, consecutive channels)
+  // read consecutive 16-byte pairs, and each warp's stores cover whole
+  // sectors.
+  for (int pos = tid; pos < PART; pos += blockDim.x) {
+    const int m = pos >> 1;
+    const int ep = (m & 31) * 33 + 2 * (m >> 5) + (pos & 1);  // e in the padded layout
     float p0 = 0.f, p1 = 0.f;
 #pragma unroll
     for (int w = 0; w < NW; ++w) {
       const int kind = s_src[w];
-      const float v = s_tot[w * PART + e];
+      const float v = s_tot[w * PARTP + ep];
       if (kind == 1) p0 += v;
       if (kind == 2) p1 += v;
       if (kind == 3) {
-        p0 += s_stash[e];
+        p0 += s_stash[ep];
         p1 += v;
       }
     }
-    a.part[((size_t)cta * 2) * PART + e] = p0;
-    if (nsl == 2) a.part[((size_t)cta * 2 + 1) * PART + e] = p1;
+    st_tag(a.part + ((size_t)cta * 2) * PART + pos, tag_word(__float_as_uint(p0), tag));
+    if (nsl == 2) st_tag(a.part + ((size_t)cta * 2 + 1) * PART + pos, tag_word(__float_as_uint(p1), tag));
   }
 }
 

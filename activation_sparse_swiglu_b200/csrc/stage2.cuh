@@ -49,11 +49,13 @@ __host__ __device__ constexpr size_t ring_offset(int slots, int max_rec) {
 }
 
 // Selects the CTA's channels, streams them and writes the CTA's partial output
-// row to a.ypart (not in select_only mode).  Every thread calls it.  MAXM =
+// row to a.ypart as tagged words (not in select_only mode; returns whether it
+// did).  Every thread calls it.  MAXM =
 // ceil(d_model / (8 * 32 * warps per group)): 8-element chunks per lane and
 // column.
 template <int MAXM>
-__device__ void run(const TokenArgs& a, unsigned char* smem, GridSync& gs) {
+__device__ bool run(const TokenArgs& a, unsigned char* smem, uint32_t tag, const uint32_t* hist,
+                    const uint32_t* chist, const Phases& ph) {
   const int d = a.d, slots = a.slots;
   const uint32_t col_bytes = 2u * (uint32_t)d;     // one bf16 column / row
   const uint32_t slot_bytes = 2u * col_bytes;      // a gate/up record, or two W_down rows
@@ -86,7 +88,9 @@ __device__ void run(const TokenArgs& a, unsigned char* smem, GridSync& gs) {
     SelectScratch& sc = *reinterpret_cast<SelectScratch*>(ring);
     TopkCut cut;
     if (a.mode == kModeTopK) {
-      cut = select_cut(a.hist, a.chist, a.bucket, a.scores, a.F, a.k, sc);
+      phase_wait(ph, 1);  // every CTA has counted its scores
+      stamp(a.ts, 17);
+      cut = select_cut(hist, chist, a.bucket, a.st64, a.F, a.k, sc, tag, a.err, a.ts);
       stamp(a.ts, 15);
     } else {
       cut.T = __float_as_uint(a.tau_s);
@@ -95,19 +99,29 @@ __device__ void run(const TokenArgs& a, unsigned char* smem, GridSync& gs) {
     const int c0 = (int)(((long long)a.F * cta) / P);
     const int m = (int)(((long long)a.F * (cta + 1)) / P) - c0;
     const bool sel = tid < m && selected(sc.own[tid], c0 + tid, cut);
+
     int own_n;
     const int pos = block_exclusive_scan(sel ? 1 : 0, sc.scan, &own_n);
-    if (sel) a.sel_list[c0 + pos] = c0 + tid;
+    if (sel) st_tag(a.sel_list + c0 + pos, tag_word((uint32_t)(c0 + tid), tag));
     if (a.sel_mask && tid < m) a.sel_mask[c0 + tid] = sel ? 1 : 0;
     if (tid == 0) {
-      a.sel_cnt[cta] = own_n;
+      st_tag(a.sel_cnt + cta, tag_word((uint32_t)own_n, tag));
       if (a.stats && !a.select_only) {
         if (cta == 0) atomicAdd(a.stats + 1, 1ull);
         atomicAdd(a.stats + 2, (unsigned long long)own_n);
       }
     }
-    grid_barrier(gs, P, a.err);  // every range's list and count is written
-    const int cnt = tid < P ? __ldcg(a.sel_cnt + tid) : 0;
+    phase_arrive(ph);  // 2: counts written
+    phase_wait(ph, 2);
+    stamp(a.ts, 18);
+    // every range's count
+    int cnt = 0;
+    if (tid < P) {
+      unsigned long long w = ld_tag(a.sel_cnt + tid);
+      const long long t0 = clock64();
+      while (!tag_ok(w, tag) && wait_more(t0, a.err)) w = ld_tag(a.sel_cnt + tid);
+      cnt = tag_ok(w, tag) ? (int)(uint32_t)w : 0;
+    }
     int total;
     const int first = block_exclusive_scan(cnt, sc.scan, &total);
     if (tid < P) sc.own[tid] = (uint32_t)first;  // rank of range tid's first channel
@@ -124,9 +138,14 @@ __device__ void run(const TokenArgs& a, unsigned char* smem, GridSync& gs) {
         if ((int)sc.own[mid] <= q) lo = mid;
         else hi = mid - 1;
       }
-      s_idx[i] = __ldcg(a.sel_list + (int)(((long long)a.F * lo) / P) + (q - (int)sc.own[lo]));
+      const unsigned long long* src = a.sel_list + (int)(((long long)a.F * lo) / P) + (q - (int)sc.own[lo]);
+      unsigned long long w = ld_tag(src);
+      const long long t0 = clock64();
+      while (!tag_ok(w, tag) && wait_more(t0, a.err)) w = ld_tag(src);
+      s_idx[i] = tag_ok(w, tag) ? (int)(uint32_t)w : 0;
     }
   } else {
+    phase_arrive(ph);  // 2 (no counts to exchange)
     // list positions, or channels, [k c / P, k (c + 1) / P)
     const int k = a.mode == kModeDense ? a.F : a.k;
     r0 = (int)(((long long)k * cta) / P);
@@ -145,7 +164,7 @@ __device__ void run(const TokenArgs& a, unsigned char* smem, GridSync& gs) {
     }
   }
   stamp(a.ts, 4);
-  if (a.select_only) return;
+  if (a.select_only) return false;
 
   // The ring and barriers take over bytes that the select (and Stage 1) wrote
   // through the generic proxy: order those writes before the bulk copies.
@@ -170,7 +189,7 @@ __device__ void run(const TokenArgs& a, unsigned char* smem, GridSync& gs) {
   const int nB = (n + 1) >> 1;
   const int SPG = slots / NG;
   auto group_items = [&](int g, int cnt) { return cnt > g ? (cnt - g + NG - 1) / NG : 0; };
-  float* out_row = a.ypart + (size_t)cta * d;
+  unsigned long long* out_row = a.ypart + (size_t)cta * d;
   if (warp == NCW) {
     // ---------------- producer: one thread fills every group's slots ----------------
     // It polls the groups in turn with non-blocking tests, so a group that is
@@ -187,7 +206,7 @@ __device__ void run(const TokenArgs& a, unsigned char* smem, GridSync& gs) {
         remaining += tot[g];
       }
       long long t_idle = clock64();
-      bool pdead = gs.dead;
+      bool pdead = false;
       while (remaining > 0 && !pdead) {
         bool progress = false;
 #pragma unroll
@@ -243,7 +262,7 @@ __device__ void run(const TokenArgs& a, unsigned char* smem, GridSync& gs) {
       xr[m][0] = elem_ok(m) ? __ldg(reinterpret_cast<const float4*>(a.x + e)) : make_float4(0, 0, 0, 0);
       xr[m][1] = elem_ok(m) ? __ldg(reinterpret_cast<const float4*>(a.x + e + 4)) : make_float4(0, 0, 0, 0);
     }
-    bool cdead = gs.dead;
+    bool cdead = false;
     // ---------------- phase A: gate/up partial dot products ----------------
     // The warp's share of an item goes into registers, the slot goes back to the
     // producer, then the FMAs.
@@ -292,7 +311,10 @@ __device__ void run(const TokenArgs& a, unsigned char* smem, GridSync& gs) {
     for (int r = tid; r < n; r += NCW * 32) {
       float sv;
       if (a.proxy_values) {
-        sv = __ldcg(a.s_tilde_src + s_idx[r]);
+        unsigned long long w = ld_tag(a.st64 + s_idx[r]);
+        const long long t0 = clock64();
+        while (!tag_ok(w, tag) && wait_more(t0, a.err)) w = ld_tag(a.st64 + s_idx[r]);
+        sv = __uint_as_float((uint32_t)w);
       } else {
         float g = 0.f, u = 0.f;
         for (int w = 0; w < WPG; ++w) {
@@ -362,18 +384,19 @@ __device__ void run(const TokenArgs& a, unsigned char* smem, GridSync& gs) {
       }
     }
     asm volatile("bar.sync 1, %0;" ::"r"(NCW * 32) : "memory");
-    for (int e = tid * 4; e < d; e += NCW * 32 * 4) {
-      float4 v = *reinterpret_cast<const float4*>(s_y + e);
+    // one 16-byte tagged pair per lane and store: each warp store covers
+    // whole sectors
+    for (int e = tid * 2; e < d; e += NCW * 32 * 2) {
+      float2 v = *reinterpret_cast<const float2*>(s_y + e);
       for (int g = 1; g < NG; ++g) {
-        const float4 t = *reinterpret_cast<const float4*>(s_y + (size_t)g * d + e);
+        const float2 t = *reinterpret_cast<const float2*>(s_y + (size_t)g * d + e);
         v.x += t.x;
         v.y += t.y;
-        v.z += t.z;
-        v.w += t.w;
       }
-      *reinterpret_cast<float4*>(out_row + e) = v;
+      st_tag2(out_row + e, tag_word(__float_as_uint(v.x), tag), tag_word(__float_as_uint(v.y), tag));
     }
   }
+  return true;
 }
 
 }  // namespace s2

@@ -1,30 +1,31 @@
 // The fused per-token kernel of the Prox decode step: one launch runs the
-// whole step of one token (Prox §4.1) on all SMs, one CTA per SM, with
-// grid-wide barriers between the phases instead of kernel boundaries:
+// whole step of one token (Prox §4.1) on all SMs, one CTA per SM:
 //
 //   Stage 1 (stage1.cuh): threshold x, INT4 proxy GEMV over the kept rows
-//            into per-CTA partial sums;
-//   barrier: every partial sum is written;
+//            into per-CTA partial sums, written as tagged words;
 //   scores:  each CTA adds up the partials of its own share of the channels
-//            and scores them, |act(g~) u~| (for the top-k rule counting them
-//            in the histograms of select.cuh);
-//   barrier: (top-k) the histograms are complete;
-//   Stage 2 (stage2.cuh): each CTA finds the token's exact top-k cut (or
-//            applies the score threshold) and lists its own channels past it;
-//   barrier: (top-k, threshold) every CTA's list and count is written;
-//            each CTA then takes an even share of the token's ranked
-//            selection (or of a given list, or of every channel for the
-//            dense baseline), streams those channel records and W_down rows
-//            and writes a partial output row;
-//   barrier: every partial row is complete;
+//            (polling until each has arrived) and scores them,
+//            |act(g~) u~|, counting them for the top-k rule in the
+//            histograms of select.cuh;
+//   Stage 2 (stage2.cuh): each CTA finds the token's exact top-k cut once
+//            the histograms are complete (or applies the score threshold),
+//            lists its own channels past it with their count, then takes an
+//            even share of the token's ranked selection (or of a given list,
+//            or of every channel for the dense baseline), streams those
+//            channel records and W_down rows and writes a tagged partial
+//            output row;
 //   output:  CTA c adds the partial rows of its share of the columns in a
 //            fixed order (deterministic).
 //
-// The launch is cooperative (all CTAs resident, which the barriers need) and
-// programmatically dependent on the previous kernel in the stream: it waits
-// for it before touching x or the workspace, then lets the next one launch.
-// Every wait (barrier, mbarrier) is bounded and reports a timeout in the
-// layer's error word.
+// The CTAs never wait at a grid-wide barrier: whatever one CTA hands to
+// another is a tagged word (token_args.cuh) that the reader polls for, and
+// counts are complete when they add up to a known total.  The launch is
+// cooperative (every CTA resident, so every wait ends) and programmatically
+// dependent on the previous kernel in the stream: it waits for it before
+// touching x or the workspace, then lets the next one launch.  Every wait is
+// bounded and reports a timeout in the layer's error word; every CTA adds one
+// to the layer's launch counter as it ends, which gives the next launch its
+// tag and its histogram parity.
 #include "prox_device.cuh"
 #include "prox_internal.h"
 #include "stage1.cuh"
@@ -33,80 +34,130 @@
 namespace prox {
 namespace {
 
+// The CTA's share of the output: the column pairs [q0, q1) of out.  Warp w
+// takes the partial rows p = w, w + W, ... (W warps), lane l the pairs
+// q0 + l, q0 + l + 32, ...: a warp's loads of one row are one contiguous
+// stretch, all of them in flight at once (kRowChunk rows per round) and
+// polled until every tag is this launch's.  Each lane adds its rows in
+// order; the warps' sums are then added in warp order (deterministic).
+constexpr int kRowChunk = 9;
+__device__ void reduce_output(const TokenArgs& a, uint32_t tag, unsigned char* smem) {
+  const int P = gridDim.x, nq = a.d >> 1, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int NW = kTokenThreads / 32;
+  const int q0 = (int)(((long long)nq * blockIdx.x) / P);
+  const int q1 = (int)(((long long)nq * (blockIdx.x + 1)) / P);
+  const int nqc = q1 - q0;
+  float2* s_sum = reinterpret_cast<float2*>(smem);  // [NW][nqc]
+  for (int l = lane; l < ((nqc + 31) & ~31); l += 32) {
+    const bool col = l < nqc;
+    float2 acc = make_float2(0.f, 0.f);
+    for (int p0 = warp; p0 < P; p0 += NW * kRowChunk) {
+      ulonglong2 v[kRowChunk];
+      const unsigned long long zero = tag_word(0u, tag);  // rows past P add 0
+#pragma unroll
+      for (int i = 0; i < kRowChunk; ++i) {
+        const int p = p0 + i * NW;
+        v[i] = col && p < P ? ld_tag2(a.ypart + (size_t)p * a.d + 2 * (q0 + l)) : make_ulonglong2(zero, zero);
+      }
+      const long long t0 = clock64();
+      for (;;) {
+        bool all = true;
+#pragma unroll
+        for (int i = 0; i < kRowChunk; ++i) all = all && tag_ok(v[i].x, tag) && tag_ok(v[i].y, tag);
+        if (all || !wait_more(t0, a.err)) break;
+#pragma unroll
+        for (int i = 0; i < kRowChunk; ++i) {
+          const int p = p0 + i * NW;
+          if (col && p < P && !(tag_ok(v[i].x, tag) && tag_ok(v[i].y, tag)))
+            v[i] = ld_tag2(a.ypart + (size_t)p * a.d + 2 * (q0 + l));
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < kRowChunk; ++i) {
+        acc.x += __uint_as_float((uint32_t)v[i].x);
+        acc.y += __uint_as_float((uint32_t)v[i].y);
+      }
+    }
+    if (col) s_sum[warp * nqc + l] = acc;
+  }
+  __syncthreads();
+  stamp(a.ts, 6);
+  for (int l = threadIdx.x; l < nqc; l += blockDim.x) {
+    float2 t = s_sum[l];
+    for (int w = 1; w < NW; ++w) {
+      t.x += s_sum[w * nqc + l].x;
+      t.y += s_sum[w * nqc + l].y;
+    }
+    reinterpret_cast<float2*>(a.out)[q0 + l] = t;
+  }
+}
+
 template <int NB, int MAXM>
 __global__ void __launch_bounds__(kTokenThreads, 1) token_kernel(TokenArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
-  stamp(a.ts, 0);
+  stamp_timer(a.ts, 0, 22);
   pdl_wait();     // the previous kernel of the stream is complete: x and the workspace are ours
   pdl_trigger();  // the next kernel may launch (it waits for this one before touching anything)
-  GridSync gs = grid_sync_begin(a.gbar);
+  // The launch counter (every thread reads it: the dynamic shared memory
+  // belongs to the phases).  Its value is first needed when Stage 1 writes
+  // its partials, so the load overlaps Stage 1's start.
+  const unsigned long long gv = ld_relaxed_u64(a.gbar);
   stamp(a.ts, 1);
   const bool topk = a.mode == kModeTopK;
+  if (a.stage1) s1::run<NB>(a, smem, gv);
+  // the launch index e: every earlier launch added kPhases * gridDim.x to the
+  // counter, and fewer than that many of this launch's additions can be in it
+  const unsigned long long e = gv / ((unsigned long long)kPhases * gridDim.x);
+  const uint32_t tag = launch_tag(gv);
+  const int par = (int)(e & 1ull);
+  const Phases ph{a.gbar, e * kPhases * gridDim.x, a.err};
+  {
+    // clear the histograms of the other parity for the next launch
+    uint32_t* nh = a.hist + (size_t)(par ^ 1) * kScoreBins;
+    const int b0 = (int)(((long long)kScoreBins * blockIdx.x) / gridDim.x);
+    const int b1 = (int)(((long long)kScoreBins * (blockIdx.x + 1)) / gridDim.x);
+    for (int i = b0 + threadIdx.x; i < b1; i += blockDim.x) nh[i] = 0u;
+    if (blockIdx.x == 0 && threadIdx.x < kCoarseBins) a.chist[(par ^ 1) * kCoarseBins + threadIdx.x] = 0u;
+  }
+  uint32_t* hist = a.hist + (size_t)par * kScoreBins;
+  uint32_t* chist = a.chist + par * kCoarseBins;
   if (a.stage1) {
-    s1::run<NB>(a, smem);
+    phase_arrive(ph);  // 0: partials written
     stamp(a.ts, 2);
-    grid_barrier(gs, gridDim.x, a.err);  // every CTA's Stage-1 partials are written
-    stamp(a.ts, 3);
+    phase_wait(ph, 0);
+    stamp(a.ts, 16);
     SelectScratch& sc = *reinterpret_cast<SelectScratch*>(smem + s2::ring_offset(a.slots, a.max_rec));
-    s1::score_channels(a, topk, sc);
+    s1::score_channels(a, topk, sc, tag, hist, chist);
+    phase_arrive(ph);  // 1: scores counted
     stamp(a.ts, 10);
-    if (a.mode == kModeNone) return;
-    if (topk) {
-      grid_barrier(gs, gridDim.x, a.err);  // the histograms and buckets are complete
-      stamp(a.ts, 14);
-    }
+  } else {
+    phase_arrive(ph);
+    phase_arrive(ph);
   }
-  if (a.mode == kModeNone) return;
-  s2::run<MAXM>(a, smem, gs);
-  stamp(a.ts, 5);
-  grid_barrier(gs, gridDim.x, a.err);  // every partial row is written; every CTA is past the cut
-  stamp(a.ts, 6);
-  if (a.stage1 && topk && blockIdx.x == gridDim.x - 1) {  // ready for the next token
-    for (int i = threadIdx.x; i < kScoreBins; i += blockDim.x) a.hist[i] = 0u;
-    if (threadIdx.x < kCoarseBins) a.chist[threadIdx.x] = 0u;
+  bool rows = false;
+  if (a.mode != kModeNone) {
+    rows = s2::run<MAXM>(a, smem, tag, hist, chist, ph);  // arrives at phase 2
+    stamp(a.ts, 5);
+  } else {
+    phase_arrive(ph);
   }
-  if (a.select_only) return;
-
-  // out[4q .. 4q+3] for the float4 columns q of this CTA: warp w sums column
-  // q over the partial rows p = lane, lane + 32, ... in order (all loads in
-  // flight at once), then across lanes by a fixed shuffle tree.
-  const int P = gridDim.x, nq = a.d >> 2, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int q0 = (int)(((long long)nq * blockIdx.x) / P);
-  const int q1 = (int)(((long long)nq * (blockIdx.x + 1)) / P);
-  const float4* yp = reinterpret_cast<const float4*>(a.ypart);
-  for (int q = q0 + warp; q < q1; q += kTokenThreads / 32) {
-    float4 v[kMaxCtas / 32];
-#pragma unroll
-    for (int u = 0; u < kMaxCtas / 32; ++u) {
-      const int p = lane + 32 * u;
-      v[u] = p < P ? __ldcg(yp + (size_t)p * nq + q) : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    float4 s = v[0];
-#pragma unroll
-    for (int u = 1; u < kMaxCtas / 32; ++u) {
-      s.x += v[u].x;
-      s.y += v[u].y;
-      s.z += v[u].z;
-      s.w += v[u].w;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      s.x += __shfl_xor_sync(0xffffffffu, s.x, o);
-      s.y += __shfl_xor_sync(0xffffffffu, s.y, o);
-      s.z += __shfl_xor_sync(0xffffffffu, s.z, o);
-      s.w += __shfl_xor_sync(0xffffffffu, s.w, o);
-    }
-    if (lane == 0) reinterpret_cast<float4*>(a.out)[q] = s;
+  phase_arrive(ph);  // 3: partial output rows written
+  if (rows) {
+    phase_wait(ph, 3);
+    stamp(a.ts, 19);
+    reduce_output(a, tag, smem);
+    stamp(a.ts, 7);
   }
-  stamp(a.ts, 7);
+  stamp_timer(a.ts, 21, 23);
 }
 
-// Test probe of the bounded waits: one CTA arrives at the layer's grid
-// barrier expecting one more arrival that never comes, so its wait runs out,
-// sets PROX_DEVERR_WAIT_TIMEOUT and returns.  Nothing faults.
+// Test probe of the bounded waits: one CTA adds 1 to the layer's launch
+// counter and waits for a second addition that never comes.
 __global__ void barrier_probe_kernel(unsigned long long* gbar, int* err) {
-  GridSync gs = grid_sync_begin(gbar);
-  grid_barrier(gs, gridDim.x + 1, err);
+  const unsigned long long v = ld_relaxed_u64(gbar);
+  const Phases ph{gbar, v, err};
+  phase_arrive(ph);
+  phase_wait(ph, 1);
 }
 
 template <int NB>
@@ -225,12 +276,12 @@ cudaError_t launch_token(const prox_layer* L, const TokenLaunch& m, cudaStream_t
   a.idx = m.idx;
   a.scores = L->ws.scores;
   a.s_tilde = m.taps.s_tilde ? m.taps.s_tilde : (m.proxy_values ? L->ws.s_tilde : nullptr);
-  a.s_tilde_src = L->ws.s_tilde;
   a.hist = L->ws.hist;
   a.chist = L->ws.chist;
   a.bucket = L->ws.bucket;
   a.sel_list = L->ws.sel_list;
   a.sel_cnt = L->ws.sel_cnt;
+  a.st64 = L->ws.st64;
   a.stats = L->ws.stats;
   a.part = L->ws.s1_part;
   a.ypart = L->ws.ypart;

@@ -1,6 +1,6 @@
 // Arguments of the fused per-token kernel (token.cu) and the small device
-// primitives its phases share: the grid-wide barrier and the exponent words of
-// the INT4 decode.
+// primitives its phases share: the tagged exchange words and the exponent
+// words of the INT4 decode.
 #pragma once
 
 #include "prox_device.cuh"
@@ -49,16 +49,17 @@ struct TokenArgs {
   // workspace
   float* scores;         // |act(g~) u~| [F]
   float* s_tilde;        // Stage 1 writes act(g~) u~ here when non-null [F]
-  const float* s_tilde_src;  // A3 Stage 2 reads it here
-  uint32_t* hist;        // [kScoreBins] fine histogram of the scores' bits 30..18
-  uint32_t* chist;       // [128] coarse histogram of the scores' bits 30..24
-  uint2* bucket;         // [kScoreBins][kBucketCap] (key, channel) per fine bin
-  int32_t* sel_list;     // [F] CTA c's selected channels from its range's first channel on
-  int32_t* sel_cnt;      // [P] CTA c's selected count
   unsigned long long* stats;
-  float* part;           // Stage-1 partial sums [P][2][1024]
-  float* ypart;          // Stage-2 partial output rows [P][d]
-  unsigned long long* gbar;  // grid-barrier arrival counter
+  // exchanged between the CTAs of the launch (tagged words: payload | tag << 32)
+  uint32_t* hist;        // [2][kScoreBins] fine histograms of the scores' bits 30..18
+  uint32_t* chist;       // [2][kCoarseBins] coarse histograms of the scores' bits 30..24
+  unsigned long long* bucket;  // [kScoreBins][kBucketCap][2] tagged (key, channel) per fine bin
+  unsigned long long* st64;    // [F] tagged bits of act(g~) u~
+  unsigned long long* sel_list;  // [F] tagged: CTA c's selected channels from its range's start
+  unsigned long long* sel_cnt;   // [P] tagged: CTA c's selected count
+  unsigned long long* part;    // [P][2][1024] tagged Stage-1 partial sums
+  unsigned long long* ypart;   // [P][d] tagged Stage-2 partial output rows
+  unsigned long long* gbar;    // launch counter: every CTA adds 1 when it ends
   int* err;              // device error word
   // taps (each may be null)
   float* g_dbg;
@@ -71,18 +72,26 @@ struct TokenArgs {
   Magic mg;
 };
 
-// Phase stamp i of this CTA (globaltimer, ns) when stamps were asked for:
-// 0 kernel entry, 1 previous kernel complete, 2 Stage-1 partials written,
-// 3 partials visible (barrier), 4 channels selected, 5 partial output row
-// written, 6 partial rows visible (barrier), 7 output written; 8 kept rows
-// compacted, 9 Stage-1 row loop done, 10 scores of the CTA's channels written,
-// 14 the histograms complete (barrier); 11 Stage-2 ring set up, 12 gate/up
-// phase done; slot 13 holds the CTA's channel count, not a time.
+// Phase stamp i of this CTA (the SM's clock64 cycle count) when stamps were
+// asked for (a cycle count costs next to nothing; the global timer is read
+// only at entry, slot 22, and exit, slot 23, with the exit cycle count in
+// slot 21, to place the cycle counts on one ns time line):
+// 0 kernel entry, 1 previous kernel complete, 8 kept rows compacted, 9 Stage-1
+// row loop done, 2 Stage-1 partials written, 3 the partials of thread 0's
+// channel received, 10 the CTA's channels scored and counted, 14 the coarse
+// histogram complete, 15 the top-k cut found, 4 the CTA's Stage-2 channels
+// known, 11 Stage-2 ring set up, 12 gate/up phase done, 5 partial output row
+// written, 6 the partial rows of the CTA's columns received, 7 output
+// written; slot 13 holds the CTA's Stage-2 channel count, not a time.
 __device__ __forceinline__ void stamp(unsigned long long* ts, int i) {
+  if (ts && threadIdx.x == 0) ts[(size_t)blockIdx.x * kPhaseStamps + i] = (unsigned long long)clock64();
+}
+__device__ __forceinline__ void stamp_timer(unsigned long long* ts, int clock_slot, int timer_slot) {
   if (ts && threadIdx.x == 0) {
     unsigned long long t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    ts[(size_t)blockIdx.x * kPhaseStamps + i] = t;
+    ts[(size_t)blockIdx.x * kPhaseStamps + clock_slot] = (unsigned long long)clock64();
+    ts[(size_t)blockIdx.x * kPhaseStamps + timer_slot] = t;
   }
 }
 
@@ -116,47 +125,94 @@ __device__ __forceinline__ void fence_acq_rel_gpu() {
 // PROX_DEVERR_WAIT_TIMEOUT, marks itself dead (later barriers do not wait)
 // and carries on, so a CTA that never arrives cannot hang the GPU; the host
 // resets the counter in prox_layer_error.
-struct GridSync {
-  unsigned long long* ctr;
-  unsigned long long base;  // thread 0: the counter when the launch started
-  unsigned n;               // barriers passed so far
-  bool dead;                // thread 0: a wait of this CTA ran out
-};
-
-__device__ __forceinline__ GridSync grid_sync_begin(unsigned long long* ctr) {
-  GridSync g;
-  g.ctr = ctr;
-  if (threadIdx.x == 0) {
-    const unsigned long long v = ld_relaxed_u64(ctr);
-    g.base = v - v % gridDim.x;
-  } else {
-    g.base = 0ull;
-  }
-  g.n = 0;
-  g.dead = false;
-  return g;
+// Tagged words.  Everything one CTA of a launch writes for others to read is
+// a 64-bit word holding a 32-bit payload and, in its high half, the launch's
+// tag, stored and loaded with single 64-bit relaxed accesses (single-copy
+// atomic at gpu scope).  A reader polls until the tag is the launch's: the
+// payload it then holds is the one written in this launch, with no fence and
+// no barrier between writer and reader.  The tag is the launch's index (the
+// launch counter over the grid size, which every launch advances by exactly
+// one) with the top bit set, so it is never that of zeroed memory and never
+// that of the launch before.
+__device__ __forceinline__ unsigned long long tag_word(uint32_t payload, uint32_t tag) {
+  return ((unsigned long long)tag << 32) | payload;
+}
+__device__ __forceinline__ bool tag_ok(unsigned long long w, uint32_t tag) {
+  return (uint32_t)(w >> 32) == tag;
+}
+__device__ __forceinline__ void st_tag(unsigned long long* p, unsigned long long w) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(w) : "memory");
+}
+__device__ __forceinline__ void st_tag2(unsigned long long* p, unsigned long long w0,
+                                        unsigned long long w1) {
+  asm volatile("st.relaxed.gpu.global.v2.u64 [%0], {%1, %2};" ::"l"(p), "l"(w0), "l"(w1) : "memory");
+}
+__device__ __forceinline__ unsigned long long ld_tag(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ ulonglong2 ld_tag2(const unsigned long long* p) {
+  ulonglong2 v;
+  asm volatile("ld.relaxed.gpu.global.v2.u64 {%0, %1}, [%2];" : "=l"(v.x), "=l"(v.y) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint32_t ld_relaxed_u32(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
 }
 
-// Every thread of the CTA calls it.
-__device__ __forceinline__ void grid_barrier(GridSync& g, unsigned expected, int* err) {
+// Bounded waiting: a poll loop calls wait_more(t0, err) after each miss; it
+// sleeps briefly (the pollers must not crowd out the CTAs still streaming)
+// and returns false once kWaitLimitCycles have passed since t0, after setting
+// PROX_DEVERR_WAIT_TIMEOUT.  The caller then carries on with what it has.
+__device__ __forceinline__ bool wait_more(long long t0, int* err) {
+  __nanosleep(64);
+  if (clock64() - t0 > kWaitLimitCycles) {
+    atomicOr(err, PROX_DEVERR_WAIT_TIMEOUT);
+    return false;
+  }
+  return true;
+}
+
+// Phase hints.  Each CTA adds 1 to the layer's launch counter at each of the
+// kPhases phase points of every launch, whether or not the launch runs that
+// phase: 0 Stage-1 partials written, 1 scores counted, 2 selection counts
+// written, 3 partial output rows written.  So a launch starts with the
+// counter at a multiple of kPhases * gridDim.x, its index is the counter over
+// that (a CTA reading it late still sees fewer than kPhases * gridDim.x of
+// this launch's additions), and phase j of the launch has been passed by
+// every CTA once the counter reaches base + (j + 1) * gridDim.x.  A reader
+// waits for that (one polling thread per CTA, on one word) before it reads
+// what the phase wrote; the data itself is tagged, so an add that overtakes
+// the writes it follows costs a re-poll, never a wrong value.  No fence.
+constexpr int kPhases = 4;
+
+// The launch's tag from the launch counter read at its start.
+__device__ __forceinline__ uint32_t launch_tag(unsigned long long counter) {
+  return (uint32_t)(counter / ((unsigned long long)kPhases * gridDim.x)) | 0x80000000u;
+}
+
+struct Phases {
+  unsigned long long* ctr;
+  unsigned long long base;  // kPhases * gridDim.x * launch index
+  int* err;
+};
+
+// Every thread of the CTA calls it, after its writes of the phase.
+__device__ __forceinline__ void phase_arrive(const Phases& ph) {
   __syncthreads();
-  ++g.n;
+  if (threadIdx.x == 0) red_add_u64(ph.ctr, 1ull);
+}
+
+// Every thread of the CTA calls it; bounded (wait_more).
+__device__ __forceinline__ void phase_wait(const Phases& ph, int j) {
   if (threadIdx.x == 0) {
-    const unsigned long long target = g.base + (unsigned long long)g.n * expected;
-    fence_acq_rel_gpu();
-    red_add_u64(g.ctr, 1ull);
-    if (!g.dead) {
-      const long long t0 = clock64();
-      while (ld_relaxed_u64(g.ctr) < target) {
-        __nanosleep(64);
-        if (clock64() - t0 > kWaitLimitCycles) {
-          atomicOr(err, PROX_DEVERR_WAIT_TIMEOUT);
-          g.dead = true;
-          break;
-        }
-      }
+    const unsigned long long target = ph.base + (unsigned long long)(j + 1) * gridDim.x;
+    const long long t0 = clock64();
+    while (ld_relaxed_u64(ph.ctr) < target && wait_more(t0, ph.err)) {
     }
-    fence_acq_rel_gpu();
   }
   __syncthreads();
 }
