@@ -324,6 +324,33 @@ class Layer:
         check(lib.prox_dense_ffn(self.handle, _ptr(x2), _ptr(out), x2.shape[0], _stream(stream)))
         return out
 
+    def forward_batch(self, x: torch.Tensor, out: torch.Tensor | None = None, stream=None):
+        """B <= 16 tokens in one batched step (union loads; needs max_batch > 1)."""
+        x2, out = self._io(x, out)
+        check(lib.prox_ffn_forward_batch(self.handle, _ptr(x2), _ptr(out), x2.shape[0],
+                                         _stream(stream)))
+        return out
+
+    def dense_batch(self, x: torch.Tensor, out: torch.Tensor | None = None, stream=None):
+        """Dense baseline for B <= 16 tokens reading every weight once."""
+        x2, out = self._io(x, out)
+        check(lib.prox_dense_ffn_batch(self.handle, _ptr(x2), _ptr(out), x2.shape[0],
+                                       _stream(stream)))
+        return out
+
+    def batch_union_sizes(self, stream=None) -> tuple[int, int]:
+        """(union input rows, union channels) of the last forward_batch."""
+        rows, chans = ctypes.c_int32(0), ctypes.c_int32(0)
+        check(lib.prox_batch_union_sizes(self.handle, ctypes.byref(rows), ctypes.byref(chans),
+                                         _stream(stream)))
+        return rows.value, chans.value
+
+    def debug_batch_masks(self, B: int, stream=None) -> torch.Tensor:
+        """uint8 [B, d_ff] per-token masks of the last forward_batch (CUDA)."""
+        m = torch.empty((B, self.d_ff), dtype=torch.uint8, device="cuda")
+        check(lib.prox_debug_batch_masks(self.handle, _ptr(m), B, _stream(stream)))
+        return m
+
     def forward_host(self, x_host: torch.Tensor, out_host: torch.Tensor | None = None,
                      stream=None):
         """Tokens whose inputs/outputs live in host memory (pinned for async copies)."""

@@ -73,6 +73,10 @@ SIGNATURES = {
                                    ctypes.POINTER(_D)]),
     "prox_ffn_forward": (_I, [_P, _P, _P, _I, _P]),
     "prox_dense_ffn": (_I, [_P, _P, _P, _I, _P]),
+    "prox_ffn_forward_batch": (_I, [_P, _P, _P, _I, _P]),
+    "prox_dense_ffn_batch": (_I, [_P, _P, _P, _I, _P]),
+    "prox_batch_union_sizes": (_I, [_P, _P, _P, _P]),
+    "prox_debug_batch_masks": (_I, [_P, _P, _I, _P]),
     "prox_ffn_forward_host": (_I, [_P, _P, _P, _I, _P]),
     "prox_ffn_forward_profiled": (_I, [_P, _P, _P, ctypes.POINTER(_P), _P, _P]),
     "prox_debug_stage1": (_I, [_P, _P, _P, _P, _P, _P, _P, _P]),

@@ -18,7 +18,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libprox.so")
 
-SOURCES = ["prox_api.cu", "token.cu", "pack.cu", "calibrate.cu", "misc.cu"]
+SOURCES = ["prox_api.cu", "token.cu", "batch.cu", "pack.cu", "calibrate.cu", "misc.cu"]
 HEADERS = ["prox_device.cuh", "prox_internal.h", "select.cuh", "token_args.cuh", "stage1.cuh",
            "stage2.cuh"]
 

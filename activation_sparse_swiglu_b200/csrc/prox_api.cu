@@ -165,6 +165,12 @@ prox_status alloc_workspace(prox_layer* L) {
   const size_t o_ypart = take((size_t)L->P * d * 8);
   const size_t o_gbar = take(8);
   const size_t xchg_bytes = off - o_xchg;
+  // the batched step's scratch (max_batch > 1), in the same allocation
+  size_t o_batch = 0;
+  if (L->max_batch > 1) {
+    prox::choose_batch_splits(L->d, L->F, L->num_sms, &L->b_s1, &L->b_s5);
+    o_batch = take(prox::batch_ws_bytes(L->d, L->F, L->b_s1, L->b_s5));
+  }
   const size_t o_in = take((size_t)kHostChunkTokens * d * 4);
   const size_t o_out = take((size_t)kHostChunkTokens * d * 4);
   void* base = nullptr;
@@ -194,6 +200,10 @@ prox_status alloc_workspace(prox_layer* L) {
   w.gbar = reinterpret_cast<unsigned long long*>(b + o_gbar);
   w.err = reinterpret_cast<int*>(b + o_err);
   w.stage_in = reinterpret_cast<float*>(b + o_in);
+  if (L->max_batch > 1) {
+    L->bws_base = b + o_batch;
+    prox::carve_batch_ws(L->bws_base, L->d, L->F, L->b_s1, L->b_s5, &L->bws);
+  }
   w.stage_out = reinterpret_cast<float*>(b + o_out);
   return PROX_OK;
 }
@@ -390,6 +400,7 @@ prox_status prox_layer_create(const uint16_t* W_gate, const uint16_t* W_up, cons
     if (e == cudaSuccess) e = r;
   };
   step(prox::setup_token_kernels());
+  step(prox::setup_batch_kernels());
   step(dev_alloc(&L->wgu, 2 * F * d * 2));
   step(dev_alloc(&L->wd, F * d * 2));
   step(dev_alloc(&L->pq, (size_t)L->C * d * 512));  // slice-major, last slice padded
@@ -625,6 +636,58 @@ prox_status prox_dense_ffn(const prox_layer* L, const float* x, float* out, int 
     cudaError_t e = enqueue_dense(L, x + (size_t)b * L->d, out + (size_t)b * L->d, s);
     if (e != cudaSuccess) return cuda_fail(e, "prox_dense_ffn launch");
   }
+  return PROX_OK;
+}
+
+namespace {
+prox_status batch_call(const prox_layer* L, const float* x, float* out, int B, bool dense, void* stream,
+                       const char* what) {
+  prox_status st = check_layer(L);
+  if (st != PROX_OK) return st;
+  if (!L->bws_base) return fail(PROX_EINVAL, "%s needs a layer created with max_batch > 1", what);
+  const int bmax = L->max_batch < prox::kBatchMax ? L->max_batch : prox::kBatchMax;
+  if (B < 1 || B > bmax) return fail(PROX_EINVAL, "B=%d must be in [1, %d]", B, bmax);
+  if (!x || !out || !aligned16(x) || !aligned16(out))
+    return fail(PROX_EINVAL, "x and out must be non-NULL 16-byte aligned pointers");
+  if (x == out) return fail(PROX_EINVAL, "out may not alias x");
+  if (!dense && L->stage2_source != PROX_STAGE2_EXACT)
+    return fail(PROX_EUNSUPPORTED, "%s computes the exact Stage 2 only", what);
+  PROX_CUDA(prox::launch_batch(L, x, out, B, dense, as_stream(stream)), what);
+  return PROX_OK;
+}
+}  // namespace
+
+prox_status prox_ffn_forward_batch(const prox_layer* L, const float* x, float* out, int B, void* stream) {
+  return batch_call(L, x, out, B, false, stream, "prox_ffn_forward_batch");
+}
+
+prox_status prox_dense_ffn_batch(const prox_layer* L, const float* x, float* out, int B, void* stream) {
+  return batch_call(L, x, out, B, true, stream, "prox_dense_ffn_batch");
+}
+
+prox_status prox_batch_union_sizes(const prox_layer* L, int32_t* rows_host, int32_t* channels_host,
+                                   void* stream) {
+  prox_status st = check_layer(L);
+  if (st != PROX_OK) return st;
+  if (!L->bws_base) return fail(PROX_EINVAL, "the layer has no batched step (max_batch == 1)");
+  if (!rows_host || !channels_host) return fail(PROX_EINVAL, "NULL output");
+  int32_t v[2] = {0, 0};
+  cudaStream_t s = as_stream(stream);
+  PROX_CUDA(cudaMemcpyAsync(v, L->bws.cnt, 8, cudaMemcpyDeviceToHost, s), "read union sizes");
+  PROX_CUDA(cudaStreamSynchronize(s), "cudaStreamSynchronize");
+  *rows_host = v[0];
+  *channels_host = v[1];
+  return PROX_OK;
+}
+
+prox_status prox_debug_batch_masks(const prox_layer* L, uint8_t* masks, int B, void* stream) {
+  prox_status st = check_layer(L);
+  if (st != PROX_OK) return st;
+  if (!L->bws_base) return fail(PROX_EINVAL, "the layer has no batched step (max_batch == 1)");
+  if (!masks || B < 1 || B > prox::kBatchMax) return fail(PROX_EINVAL, "masks NULL or B out of [1, 16]");
+  PROX_CUDA(cudaMemcpyAsync(masks, L->bws.smask, (size_t)B * L->F, cudaMemcpyDeviceToDevice,
+                            as_stream(stream)),
+            "copy batch masks");
   return PROX_OK;
 }
 

@@ -5,6 +5,7 @@
 #include <algorithm>
 #include <cstddef>
 #include <cstdint>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include "prox.h"
@@ -29,6 +30,7 @@ constexpr int kMaxDff = 32768;       // bounds the select's slice table (kMaxSli
 constexpr int kSmemPerSm = 233472;   // shared memory per SM on sm_100 (228 KB)
 constexpr int kMaxSmemPerBlock = 232448;  // opt-in dynamic shared memory per CTA (227 KB)
 constexpr int kHostChunkTokens = 64; // staging chunk of prox_ffn_forward_host
+constexpr int kBatchMax = 16;        // tokens of one batched (union) step
 
 // Per-token scratch of one layer (device memory owned by the handle).
 struct Workspace {
@@ -59,6 +61,27 @@ struct Workspace {
   size_t bytes = 0;
 };
 
+// Scratch of the batched step (batch.cu), allocated when max_batch > 1.
+// Token-major arrays have kBatchMax rows; Fp = d_ff rounded up to 64.
+struct BatchWs {
+  __nv_bfloat16* xu_hi = nullptr;  // [16][d] x^ of the union rows (kept or 0), bf16 hi part
+  __nv_bfloat16* xu_lo = nullptr;  //          ... and the rest
+  __nv_bfloat16* xf_hi = nullptr;  // [16][d] x split the same way
+  __nv_bfloat16* xf_lo = nullptr;
+  int* urow = nullptr;             // [d] the union rows, ascending
+  int* gstart = nullptr;           // [G] first union entry of each quantisation group
+  int* gcount = nullptr;           // [G] union rows in each group
+  int* cnt = nullptr;              // [4] union rows, union channels
+  float* part1 = nullptr;          // [S1][16][2][F] Stage-1 sums per row split
+  float* scores = nullptr;         // [16][F]
+  uint8_t* smask = nullptr;        // [16][F] per-token channel masks
+  int* ulist = nullptr;            // [F] the union channels, ascending
+  uint32_t* utok = nullptr;        // [F] the tokens that selected each
+  __nv_bfloat16* hh = nullptr;     // [16][Fp] h per token and union entry, hi part
+  __nv_bfloat16* hl = nullptr;     //                                      ... lo part
+  float* yp = nullptr;             // [S5][16][d] down partials per entry split
+};
+
 }  // namespace prox
 
 struct prox_layer {
@@ -83,6 +106,10 @@ struct prox_layer {
   uint8_t* pq = nullptr;     // INT4 codes [C][d][512 B], gate/up interleaved per 16 B
   uint16_t* ps = nullptr;    // fp16 scales [G][F/32][2][32]
   prox::Workspace ws;
+  // batched step: row splits of its Stage 1, entry splits of its down product
+  int b_s1 = 0, b_s5 = 0;
+  void* bws_base = nullptr;
+  prox::BatchWs bws;
 };
 
 namespace prox {
@@ -113,6 +140,14 @@ struct TokenLaunch {
 };
 
 cudaError_t setup_token_kernels();
+// The batched step (batch.cu): B <= kBatchMax tokens, union loads; dense =
+// every channel for every token (the batched dense baseline).
+cudaError_t setup_batch_kernels();
+void choose_batch_splits(int d, int F, int num_sms, int* s1, int* s5);
+size_t batch_ws_bytes(int d, int F, int s1, int s5);
+void carve_batch_ws(void* base, int d, int F, int s1, int s5, BatchWs* w);
+cudaError_t launch_batch(const prox_layer* L, const float* X, float* Y, int B, bool dense,
+                         cudaStream_t s);
 cudaError_t launch_barrier_probe(const prox_layer* L, cudaStream_t s);
 cudaError_t launch_token(const prox_layer* L, const TokenLaunch& m, cudaStream_t s, bool pdl);
 

@@ -190,7 +190,7 @@ __device__ __forceinline__ int find_bin_desc(int count, int krem, SelectScratch&
 // coarse bin add up to its count (every count only grows), so the CTA polls
 // them until they do; bucket entries and keys are tagged words.  A wait that
 // runs out sets PROX_DEVERR_WAIT_TIMEOUT and goes on with what it has.
-__device__ TopkCut select_cut(const uint32_t* hist, const uint32_t* chist,
+__device__ inline TopkCut select_cut(const uint32_t* hist, const uint32_t* chist,
                               const unsigned long long* bucket, const unsigned long long* st64, int F,
                               int k, SelectScratch& sc, uint32_t tag, int* err,
                               unsigned long long* ts) {

@@ -6,8 +6,8 @@ python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 One step = the workload's 256 decode tokens, one at a time (batch 1), each a
 full pass of the hot path in one kernel launch: Stage-1 threshold + INT4 proxy
-GEMV + scores, grid barrier, exact top-k cut, Stage-2 gate/up + W_down over the
-selected channels, grid barrier, output sum.  The layer is a seeded synthetic
+GEMV + scores, exact top-k cut, Stage-2 gate/up + W_down over the selected
+channels, output sum (the CTAs exchange tagged words, no grid barrier).  The layer is a seeded synthetic
 Llama-3-8B-shaped FFN (d_model 4096, d_ff 14336, bf16 weights N(0, 0.02^2),
 Laplace inputs with 0.5% outlier channels x30), s1 = 50% (tau calibrated on 256
 draws), s2 = 70% (k = 4301).  Consecutive tokens rotate over enough identical
@@ -328,6 +328,7 @@ def phase_breakdown(layers, xs, outs, n, stream):
     launched alone (no programmatic overlap): each phase ends when its last
     CTA reaches the stamp; times are from the first CTA's entry."""
     import torch
+    import activation_sparse_swiglu_b200 as prox
     P = layers[0].info()["stage1_ctas"]
     ph = torch.zeros((P, 24), dtype=torch.int64, device="cuda")
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
@@ -335,11 +336,11 @@ def phase_breakdown(layers, xs, outs, n, stream):
         e.record(stream)
     stream.synchronize()
     # slot -> name (include/prox.h, prox_ffn_forward_profiled); 13 is a count
-    names = {0: "entry", 1: "prev_done", 8: "stage1_compact", 9: "stage1_loop",
-             2: "stage1_partials", 3: "barrier_a", 10: "scored", 14: "barrier_b",
-             15: "topk_cut",
-             4: "selected", 11: "stage2_ring", 12: "stage2_gate_up", 5: "stage2",
-             6: "barrier_c", 7: "out"}
+    names = {8: "stage1_compact", 9: "stage1_loop", 2: "stage1_partials",
+             16: "partials_phase", 3: "partials_in", 10: "scored", 17: "scores_phase",
+             14: "histogram_complete", 15: "topk_cut", 18: "counts_phase", 4: "selected",
+             11: "stage2_ring", 12: "stage2_gate_up", 5: "stage2", 19: "rows_phase",
+             6: "rows_in", 7: "out"}
     per, kt = [], []
     with torch.cuda.stream(stream):
         for t in range(n + 4):
@@ -348,15 +349,10 @@ def phase_breakdown(layers, xs, outs, n, stream):
                                                      evs, phase_ns=ph, stream=stream)
             evs[1].synchronize()
             if t >= 4:
-                a = ph.cpu().numpy().astype(np.int64)
-                a[:, 13] = a[:, 0].min()
-                for col in (15, 16, 17, 18):  # written by one CTA only
-                    nz = a[:, col] > 0
-                    a[~nz, col] = a[nz, col].max() if nz.any() else a[:, 0].min()
-                per.append((a.max(0) - a[:, 0].min()) / 1e3)
+                per.append(np.nanmax(prox.phase_times_us(ph), axis=0))
                 kt.append(evs[0].elapsed_time(evs[1]) * 1e3)
     per = np.stack(per)
-    out = {nm: round(float(np.median(per[:, i])), 2) for i, nm in names.items()}
+    out = {nm: round(float(np.nanmedian(per[:, i])), 2) for i, nm in names.items()}
     out["kernel_event_us"] = round(statistics.median(kt), 2)
     return out
 
@@ -469,8 +465,8 @@ class Bench:
             "device_error_words": err_words,
         })
         r["roofline"] = {
-            "kernel": "token_kernel (Stage 1, grid barrier, exact top-k cut, Stage 2 gate/up + "
-                      "W_down, grid barrier, output sum: the whole step of one token)",
+            "kernel": "token_kernel (Stage 1, exact top-k cut, Stage 2 gate/up + W_down, "
+                      "output sum: the whole step of one token)",
             "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
             "frac": round(achieved / peak, 4),
             "frac_of_spec_8tbs": round(achieved / SPEC_HBM_GBS, 4),
@@ -666,7 +662,7 @@ class Bench:
             "alpha_bytes": round(proxy_bytes / slice_bytes, 4),
             "bf16_gemv_gbs": round(slice_bytes / (gemv_us * 1e-6) / 1e9, 1),
             "note": ("Stage-1 part of the token kernel (entry to the last CTA's scores: both INT4 "
-                     "proxies, partials, a grid barrier and the scores; launched alone) over 2 x "
+                     "proxies, the partial exchange and the scores; launched alone) over 2 x "
                      f"the faster cuBLAS bf16 GEMV of the same {n_x} kept rows x "
                      f"{f} channels, {n_win} rotating weight windows (> L2)")}
         # The paper's allocation at the alpha measured here (Prox §4.2).

@@ -269,9 +269,10 @@ PROX_API prox_status prox_runtime_sparsity(int64_t sum_nx, int64_t sum_sel, int6
  *            full x (or s~_j in PROX_STAGE2_PROXY_VALUES mode);
  *            out = sum_j s_j W_down[j, :].
  * x, out: fp32 [B, d_model] (out may not alias x).  B <= max_batch.
- * One cooperative kernel per token on every SM (Stage 1, grid barrier, the
- * cut and Stage 2, grid barrier, the output sum), each launch
- * programmatically dependent on the previous one in the stream. */
+ * One cooperative kernel per token on every SM (Stage 1, the cut, Stage 2 and
+ * the output sum; the CTAs hand each other tagged words, no grid barrier),
+ * each launch programmatically dependent on the previous one in the stream.
+ * Token b's result does not depend on the other tokens of the call. */
 PROX_API prox_status prox_ffn_forward(const prox_layer* layer, const float* x, float* out, int B,
                              void* stream);
 
@@ -279,6 +280,42 @@ PROX_API prox_status prox_ffn_forward(const prox_layer* layer, const float* x, f
  * on the same bf16 buffers (Stage 2 with every channel kept). */
 PROX_API prox_status prox_dense_ffn(const prox_layer* layer, const float* x, float* out, int B,
                            void* stream);
+
+/* The same step for B tokens at once, reading every weight byte the batch
+ * needs once (the pages' kernels are batch 1 only, Prox §5.3 "Discussion";
+ * the masks are still per token, Prox §4.1 and App. A.6):
+ *   the union of the tokens' kept input rows is read once from the INT4
+ *   proxies, each token contributing only its own kept rows; each token then
+ *   takes its own top-k (or threshold) channel mask; the union of the
+ *   selected channels' gate/up records and W_down rows is read once, each
+ *   token contributing only through the channels it selected.
+ * The products run on the tensor cores (bf16 operands, fp32 accumulation,
+ * x and the intermediate values split into two bf16 parts so that they carry
+ * 16 significant bits); the sums are taken in another order than
+ * prox_ffn_forward's, so scores and outputs agree with it to rounding and the
+ * masks wherever no two scores are that close.  Exact Stage 2 only
+ * (PROX_STAGE2_PROXY_VALUES gives PROX_EUNSUPPORTED).  x, out: fp32
+ * [B, d_model], out not aliasing x; 1 <= B <= min(max_batch, 16); the layer
+ * must have been created with max_batch > 1 (else PROX_EINVAL).  The scratch
+ * is the layer's: calls on one layer must be stream-ordered.  No library
+ * counterpart in the pages: this is the batched serving path they leave
+ * open. */
+PROX_API prox_status prox_ffn_forward_batch(const prox_layer* layer, const float* x, float* out, int B,
+                                            void* stream);
+
+/* Dense GLU baseline for B tokens reading every weight once: the batched
+ * step's gate/up and down products over every channel with every token
+ * keeping it (Prox §2.1).  Same arguments and limits as
+ * prox_ffn_forward_batch. */
+PROX_API prox_status prox_dense_ffn_batch(const prox_layer* layer, const float* x, float* out, int B,
+                                          void* stream);
+
+/* The union sizes of the layer's last prox_ffn_forward_batch: rows_host =
+ * input rows some token kept, channels_host = channels some token selected
+ * (the bytes that call streamed follow from them).  Synchronises `stream`;
+ * PROX_EINVAL on a layer without the batched step or NULL outputs. */
+PROX_API prox_status prox_batch_union_sizes(const prox_layer* layer, int32_t* rows_host,
+                                            int32_t* channels_host, void* stream);
 
 /* Same as prox_ffn_forward for n_tok tokens whose inputs and outputs live in
  * HOST memory (pinned memory makes the copies asynchronous): copies each
@@ -332,6 +369,12 @@ PROX_API prox_status prox_debug_mask(const prox_layer* layer, const float* x, in
  * act(g) u for each listed channel.  Always the exact Stage 2. */
 PROX_API prox_status prox_forward_with_mask(prox_layer* layer, const float* x, const int32_t* idx_s,
                                    int k, float* out, float* s_sp, void* stream);
+
+/* Test-only: the per-token channel masks of the layer's last
+ * prox_ffn_forward_batch, uint8 [B][d_ff] (1 = selected) into the device
+ * buffer masks (caller-owned).  Stream-ordered; PROX_EINVAL on a layer
+ * without the batched step, NULL masks or B outside [1, 16]. */
+PROX_API prox_status prox_debug_batch_masks(const prox_layer* layer, uint8_t* masks, int B, void* stream);
 
 /* Test-only fault injection on the host: the nth device allocation that
  * prox_layer_create makes from now on (1 = the next one; a create makes nine:
