@@ -106,65 +106,93 @@ __device__ __forceinline__ void split_bf16(float v, __nv_bfloat16* hi, __nv_bflo
 // prepare: the union of kept rows, x^ (union-compacted) and x, split hi / lo
 // ---------------------------------------------------------------------------
 
-// One CTA of 1024 threads.  Rows in rounds of 1024 (one per thread, coalesced);
-// the union rows are compacted in ascending order with a running offset.
-// Writes urow[n_u], xu_hi/lo[16][d] (columns < n_u), xf_hi/lo[16][d],
-// gstart/gcount per quantisation group and cnt[0] = n_u; adds the kept rows
-// and the tokens to the layer's statistics.
-__global__ void __launch_bounds__(1024) batch_prepare_kernel(const float* __restrict__ X, int B, int d,
-                                                             float tau, BatchWs w,
-                                                             unsigned long long* stats) {
-  __shared__ int s_scan[40];
-  const int tid = threadIdx.x;
-  const int G = d / kGroup;
-  for (int g = tid; g < G; g += blockDim.x) w.gcount[g] = 0;
-  __syncthreads();
-  int base = 0;
-  unsigned kept_total = 0;
-  for (int r0 = 0; r0 < d; r0 += blockDim.x) {
-    const int r = r0 + tid;
-    float xv[NB];
-    bool any = false;
+// Two kernels over blocks of 256 rows (two quantisation groups each).
+// prepare_count: x split into xf_hi / xf_lo for the 16 token slots (0 past
+// B), and each block's number of union rows in rcount[block]; adds the kept
+// (token, row) pairs and the tokens to the layer's statistics.
+__global__ void __launch_bounds__(256) batch_prepare_count_kernel(const float* __restrict__ X, int B, int d,
+                                                                  float tau, BatchWs w,
+                                                                  unsigned long long* stats) {
+  __shared__ int s_red[8];
+  const int r = blockIdx.x * 256 + threadIdx.x;
+  bool any = false;
+  int kept = 0;
+  if (r < d) {
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
-      xv[b] = (r < d && b < B) ? __ldg(X + (size_t)b * d + r) : 0.f;
-      const bool keep = fabsf(xv[b]) >= tau && r < d && b < B;
-      kept_total += keep ? 1u : 0u;
+      const float v = b < B ? __ldg(X + (size_t)b * d + r) : 0.f;
+      const bool keep = b < B && fabsf(v) >= tau;
+      kept += keep ? 1 : 0;
       any = any || keep;
+      split_bf16(v, w.xf_hi + (size_t)b * d + r, w.xf_lo + (size_t)b * d + r);
     }
-    if (r < d)
+  }
+  const int n_any = __syncthreads_count(any);
+  // the block's kept pairs: warp sums, then warp 0
+  int kw = kept;
 #pragma unroll
-      for (int b = 0; b < NB; ++b) split_bf16(xv[b], w.xf_hi + (size_t)b * d + r, w.xf_lo + (size_t)b * d + r);
-    int total;
-    const int pos = base + block_exclusive_scan(any ? 1 : 0, s_scan, &total);
-    if (any) {
-      w.urow[pos] = r;
-#pragma unroll
-      for (int b = 0; b < NB; ++b) {
-        const float v = fabsf(xv[b]) >= tau ? xv[b] : 0.f;
-        split_bf16(v, w.xu_hi + (size_t)b * d + pos, w.xu_lo + (size_t)b * d + pos);
-      }
-      atomicAdd(w.gcount + r / kGroup, 1);
+  for (int o = 16; o > 0; o >>= 1) kw += __shfl_xor_sync(0xffffffffu, kw, o);
+  if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = kw;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    w.rcount[blockIdx.x] = n_any;
+    int kt = 0;
+    for (int i = 0; i < 8; ++i) kt += s_red[i];
+    if (stats) {
+      atomicAdd(stats, (unsigned long long)kt);
+      if (blockIdx.x == 0) atomicAdd(stats + 1, (unsigned long long)B);
     }
-    base += total;
+  }
+}
+
+// prepare_place: block j's union rows go to [sum of rcount[< j], ...) in
+// ascending order: urow, xu_hi / xu_lo (x where the token keeps the row, else
+// 0), gstart / gcount of its two groups; the last block writes cnt[0].
+__global__ void __launch_bounds__(256) batch_prepare_place_kernel(const float* __restrict__ X, int B, int d,
+                                                                  float tau, BatchWs w) {
+  __shared__ int s_scan[40];
+  const int blk = blockIdx.x, tid = threadIdx.x, r = blk * 256 + tid;
+  int off = 0;
+  if (tid < 32) {
+    for (int j = tid; j < blk; j += 32) off += w.rcount[j];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) off += __shfl_xor_sync(0xffffffffu, off, o);
+    if (tid == 0) s_scan[36] = off;
+  }
+  float xv[NB];
+  bool any = false;
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+    xv[b] = (r < d && b < B) ? __ldg(X + (size_t)b * d + r) : 0.f;
+    any = any || (r < d && b < B && fabsf(xv[b]) >= tau);
   }
   __syncthreads();
-  // group starts: the union rows are ascending, so group g's rows are
-  // [gstart[g], gstart[g] + gcount[g]) with gstart the prefix of the counts
-  if (tid == 0) {
-    int acc = 0;
-    for (int g = 0; g < G; ++g) {
-      w.gstart[g] = acc;
-      acc += w.gcount[g];
+  off = s_scan[36];
+  int total;
+  const int pre = block_exclusive_scan(any ? 1 : 0, s_scan, &total);
+  if (any) {
+    const int pos = off + pre;
+    w.urow[pos] = r;
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      const float v = (b < B && fabsf(xv[b]) >= tau) ? xv[b] : 0.f;
+      split_bf16(v, w.xu_hi + (size_t)b * d + pos, w.xu_lo + (size_t)b * d + pos);
     }
-    w.cnt[0] = base;
   }
-  // block total of the kept rows
-  unsigned tk;
-  block_exclusive_scan(kept_total, reinterpret_cast<unsigned*>(s_scan), &tk);
-  if (tid == 0 && stats) {
-    atomicAdd(stats, (unsigned long long)tk);
-    atomicAdd(stats + 1, (unsigned long long)B);
+  // the first group's count is the exclusive prefix at thread 128
+  __shared__ int s_half;
+  if (tid == 128) s_half = pre;
+  __syncthreads();
+  const int G = d / kGroup;
+  if (tid == 0) {
+    const int h0 = d - blk * 256 >= 256 ? s_half : total;  // a last block of 128 rows: one group
+    w.gstart[2 * blk] = off;
+    w.gcount[2 * blk] = h0;
+    if (2 * blk + 1 < G) {
+      w.gstart[2 * blk + 1] = off + h0;
+      w.gcount[2 * blk + 1] = total - h0;
+    }
+    if (blk == gridDim.x - 1) w.cnt[0] = off + total;
   }
 }
 
@@ -187,13 +215,14 @@ struct S1Smem {
   int t_i0[S1_MAX_TILES];
   short t_len[S1_MAX_TILES];
   short t_grp[S1_MAX_TILES];
+  int scan[40];
   int ntiles;
 };
 
 // Grid (2 C, S1 splits): CTA (hs, s) takes the outputs of half slice hs and
 // the quantisation groups [G s / S1, G (s + 1) / S1); writes
 // part1[s][token][gate|up][channel] (the group-scaled sums of its groups).
-__global__ void __launch_bounds__(S1_THREADS) batch_stage1_kernel(const uint8_t* __restrict__ pq,
+__global__ void __launch_bounds__(S1_THREADS, 2) batch_stage1_kernel(const uint8_t* __restrict__ pq,
                                                                   const __half* __restrict__ ps, int d,
                                                                   int F, BatchWs w) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
@@ -203,38 +232,67 @@ __global__ void __launch_bounds__(S1_THREADS) batch_stage1_kernel(const uint8_t*
   const int S1 = gridDim.y, s = blockIdx.y;
   const int G = d / kGroup;
   const int g0 = (int)((long long)G * s / S1), g1 = (int)((long long)G * (s + 1) / S1);
-  // the CTA's tiles: each group's union rows in runs of at most S1_KT
-  if (tid == 0) {
-    int n = 0;
-    for (int g = g0; g < g1; ++g) {
-      const int c = w.gcount[g], st = w.gstart[g];
-      for (int j = 0; j < c; j += S1_KT) {
-        sm.t_i0[n] = st + j;
-        sm.t_len[n] = (short)min(S1_KT, c - j);
-        sm.t_grp[n] = (short)g;
-        ++n;
-      }
+  // the CTA's tiles: each group's union rows in runs of at most S1_KT, listed
+  // in parallel (thread j takes group g0 + j)
+  {
+    const int j = tid, g = g0 + j;
+    const int c = g < g1 ? w.gcount[g] : 0, st = g < g1 ? w.gstart[g] : 0;
+    const int n = (c + S1_KT - 1) / S1_KT;
+    int tot;
+    const int at = block_exclusive_scan(n, reinterpret_cast<int*>(sm.scan), &tot);
+    for (int q = 0; q < n; ++q) {
+      sm.t_i0[at + q] = st + q * S1_KT;
+      sm.t_len[at + q] = (short)min(S1_KT, c - q * S1_KT);
+      sm.t_grp[at + q] = (short)g;
     }
-    sm.ntiles = n;
+    if (tid == 0) sm.ntiles = tot;
   }
   for (int i = tid; i < S1_KT * S1_LDS; i += S1_THREADS) (&sm.S[0][0])[i] = __float2bfloat16_rn(0.f);
   __syncthreads();
   const int nt = sm.ntiles;
   const uint8_t* slice_base = pq + (size_t)slice * d * 512 + half * 256;
 
-  // tile t's codes: row k of the tile (k < len) into raw[t % STAGES][k]
-  auto issue = [&](int t) {
-    if (t < nt) {
+  // tile t's codes: row k = tid / 16 of the tile (k < len) into
+  // raw[t % STAGES][k]; the row index is loaded a tile ahead (row_of)
+  auto row_of = [&](int t) {
+    const int k = tid >> 4;
+    return (t < nt && k < sm.t_len[t]) ? __ldg(w.urow + sm.t_i0[t] + k) : -1;
+  };
+  auto issue = [&](int t, int row) {
+    if (row >= 0) {
       const int k = tid >> 4, c16 = tid & 15;  // 32 rows x 16 chunks of 16 B
-      if (k < sm.t_len[t]) {
-        const int row = __ldg(w.urow + sm.t_i0[t] + k);
-        cp16(&sm.raw[t % S1_STAGES][k][c16 * 16], slice_base + (size_t)row * 512 + c16 * 16);
-      }
+      cp16(&sm.raw[t % S1_STAGES][k][c16 * 16], slice_base + (size_t)row * 512 + c16 * 16);
     }
     cp_commit();
   };
+  // tile t's x^ (token tid / 32, row tid % 32), fetched a tile ahead
+  auto fetch_x = [&](int t, __nv_bfloat16& hi, __nv_bfloat16& lo) {
+    const int n = tid >> 5, k = tid & 31;
+    hi = lo = __float2bfloat16_rn(0.f);
+    if (t < nt && k < sm.t_len[t]) {
+      hi = w.xu_hi[(size_t)n * d + sm.t_i0[t] + k];
+      lo = w.xu_lo[(size_t)n * d + sm.t_i0[t] + k];
+    }
+  };
+  // the fp16 scales of this lane's four outputs in group grp
+  const int g = lane >> 2;
+  auto fetch_scales = [&](int grp, float (&sc)[2][2]) {
 #pragma unroll
-  for (int t = 0; t < S1_STAGES - 1; ++t) issue(t);
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int m = warp * 32 + i * 16 + g + 8 * r;
+        const int blk = (slice * 512 + half * 256) / 32 + (m >> 6);  // < F / 32 for real channels
+        sc[i][r] = blk < F / 32 ? __half2float(__ldg(ps + ((size_t)grp * (F / 32) + blk) * 64 + (m & 63))) : 0.f;
+      }
+  };
+#pragma unroll
+  for (int t = 0; t < S1_STAGES - 1; ++t) issue(t, row_of(t));
+  int row_next = row_of(S1_STAGES - 1);
+  __nv_bfloat16 xh, xl;
+  fetch_x(0, xh, xl);
+  float scl[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+  if (nt > 0) fetch_scales(sm.t_grp[0], scl);
 
   float acc[2][2][4], tot[2][2][4];
 #pragma unroll
@@ -244,12 +302,15 @@ __global__ void __launch_bounds__(S1_THREADS) batch_stage1_kernel(const uint8_t*
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[i][h][e] = tot[i][h][e] = 0.f;
 
-  const int g = lane >> 2;
   for (int t = 0; t < nt; ++t) {
-    issue(t + S1_STAGES - 1);
+    issue(t + S1_STAGES - 1, row_next);
+    row_next = row_of(t + S1_STAGES);
     cp_wait<S1_STAGES - 1>();
     __syncthreads();  // tile t's codes are in; the previous tile's products are done
-    const int len = sm.t_len[t], i0 = sm.t_i0[t];
+    const int len = sm.t_len[t];
+    sm.bhi[tid >> 5][tid & 31] = xh;
+    sm.blo[tid >> 5][tid & 31] = xl;
+    fetch_x(t + 1, xh, xl);
     // decode: 32 rows x 64 words, 4 words per thread; word wd of row k holds
     // outputs 8 wd .. 8 wd + 7 (nibble p is output 8 wd + p); the code is q + 8
     for (int j = tid; j < S1_KT * 64; j += S1_THREADS) {
@@ -270,12 +331,6 @@ __global__ void __launch_bounds__(S1_THREADS) batch_stage1_kernel(const uint8_t*
         *reinterpret_cast<uint4*>(&sm.S[k][wd * 8]) = make_uint4(0u, 0u, 0u, 0u);
       }
     }
-    {
-      const int n = tid >> 5, k = tid & 31;  // 16 tokens x 32 rows
-      const bool ok = k < len;
-      sm.bhi[n][k] = ok ? w.xu_hi[(size_t)n * d + i0 + k] : __float2bfloat16_rn(0.f);
-      sm.blo[n][k] = ok ? w.xu_lo[(size_t)n * d + i0 + k] : __float2bfloat16_rn(0.f);
-    }
     __syncthreads();
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
@@ -289,25 +344,20 @@ __global__ void __launch_bounds__(S1_THREADS) batch_stage1_kernel(const uint8_t*
         }
       }
     }
-    // the group's last tile: scale its sums per (group, output) and add them
+    // the group's last tile: scale its sums per (group, output) and add them;
+    // the next group's scales are fetched right away
     if (t + 1 == nt || sm.t_grp[t + 1] != sm.t_grp[t]) {
-      const int grp = sm.t_grp[t];
 #pragma unroll
-      for (int i = 0; i < 2; ++i) {
+      for (int i = 0; i < 2; ++i)
 #pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          const int m = warp * 32 + i * 16 + g + 8 * r;  // output of the half slice
-          const int blk = (slice * 512 + half * 256) / 32 + (m >> 6);  // < F / 32 for real channels
-          const float sc = blk < F / 32 ? __half2float(__ldg(ps + ((size_t)grp * (F / 32) + blk) * 64 + (m & 63)))
-                                        : 0.f;
+        for (int r = 0; r < 2; ++r)
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            tot[i][h][2 * r] = fmaf(sc, acc[i][h][2 * r], tot[i][h][2 * r]);
-            tot[i][h][2 * r + 1] = fmaf(sc, acc[i][h][2 * r + 1], tot[i][h][2 * r + 1]);
+            tot[i][h][2 * r] = fmaf(scl[i][r], acc[i][h][2 * r], tot[i][h][2 * r]);
+            tot[i][h][2 * r + 1] = fmaf(scl[i][r], acc[i][h][2 * r + 1], tot[i][h][2 * r + 1]);
             acc[i][h][2 * r] = acc[i][h][2 * r + 1] = 0.f;
           }
-        }
-      }
+      if (t + 1 < nt) fetch_scales(sm.t_grp[t + 1], scl);
     }
   }
   cp_wait<0>();
@@ -352,170 +402,300 @@ __global__ void batch_score_kernel(BatchWs w, int F, int S1, int act, int thresh
 }
 
 // One CTA per token: the exact top-k of its F scores (ties to the lower
-// channel), by the radix select of select.cuh over keys held in shared memory.
-__global__ void __launch_bounds__(1024) batch_topk_kernel(BatchWs w, int F, int k) {
+// channel).  A most-significant-digit-first radix select over the keys (the
+// scores' bits), 8 bits per level, each level a shared-memory histogram of
+// the keys that match the digits fixed so far; then, among the keys equal to
+// the k-th largest, the lowest-indexed ones up to the rank still wanted.
+constexpr int TK_THREADS = 1024;
+__global__ void __launch_bounds__(TK_THREADS) batch_topk_kernel(BatchWs w, int F, int k) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
-  SelectScratch& sc = *reinterpret_cast<SelectScratch*>(smem_raw);
-  uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + ((sizeof(SelectScratch) + 15) & ~(size_t)15));
-  const int b = blockIdx.x, tid = threadIdx.x;
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw);  // [F]
+  __shared__ int hist[256];
+  __shared__ int s_pick[4];
+  __shared__ int s_scan[40];
+  const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const float* src = w.scores + (size_t)b * F;
-  for (int j = tid; j < F; j += blockDim.x) keys[j] = __float_as_uint(src[j]);
-  __syncthreads();
-  const int per = (F + (int)blockDim.x - 1) / (int)blockDim.x;
-  const int j0 = min(tid * per, F), j1 = min(j0 + per, F);
-  auto all = [&](auto fn) {
-    for (int j = j0; j < j1; ++j) fn(keys[j], j);
-  };
+  for (int j = tid; j < F; j += TK_THREADS) keys[j] = __float_as_uint(src[j]);
+  uint32_t prefix = 0u, pmask = 0u;
+  int krem = k, n_eq = 0;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    if (tid < 256) hist[tid] = 0;
+    __syncthreads();
+    for (int j = tid; j < F; j += TK_THREADS) {
+      const uint32_t key = keys[j];
+      if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
+    }
+    __syncthreads();
+    if (warp == 0) {
+      // lane l holds digits 255 - 8 l .. 248 - 8 l (descending)
+      int c[8], sum = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        c[i] = hist[255 - 8 * lane - i];
+        sum += c[i];
+      }
+      int incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      int above = incl - sum;
+      if (above < krem && incl >= krem) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          if (above < krem && above + c[i] >= krem) {
+            s_pick[0] = 255 - 8 * lane - i;
+            s_pick[1] = krem - above;
+            s_pick[2] = c[i];
+            above = krem;  // done
+          } else {
+            above += c[i];
+          }
+        }
+      }
+    }
+    __syncthreads();
+    prefix |= (uint32_t)s_pick[0] << shift;
+    pmask |= 255u << shift;
+    krem = s_pick[1];
+    n_eq = s_pick[2];
+    __syncthreads();
+  }
+  // ties: the krem lowest channels among the n_eq keys equal to prefix
+  int tie_cut = F;
+  if (krem < n_eq) {
+    const int per = (F + TK_THREADS - 1) / TK_THREADS;
+    const int j0 = min(tid * per, F), j1 = min(j0 + per, F);
+    int c = 0;
+    for (int j = j0; j < j1; ++j) c += keys[j] == prefix;
+    int tot;
+    const int before = block_exclusive_scan(c, s_scan, &tot);
+    if (before < krem && before + c >= krem) {
+      int seen = before;
+      for (int j = j0; j < j1; ++j)
+        if (keys[j] == prefix && ++seen == krem) s_pick[3] = j;
+    }
+    __syncthreads();
+    tie_cut = s_pick[3];
+  }
   TopkCut cut;
-  int n_eq, k_eq;
-  radix_kth(all, k, sc, &cut.T, &n_eq, &k_eq);
-  cut.tie_cut = k_eq < n_eq ? radix_tie(all, cut.T, k_eq, sc) : F;
-  for (int j = tid; j < F; j += blockDim.x) w.smask[(size_t)b * F + j] = selected(keys[j], j, cut) ? 1 : 0;
+  cut.T = prefix;
+  cut.tie_cut = tie_cut;
+  for (int j = tid; j < F; j += TK_THREADS) w.smask[(size_t)b * F + j] = selected(keys[j], j, cut) ? 1 : 0;
 }
 
-// One CTA of 1024 threads: the channels some token selected, ascending, with
-// the bit set of the tokens that did; cnt[1] = their number.  Adds the
-// selected (token, channel) pairs to the layer's statistics.
-__global__ void __launch_bounds__(1024) batch_union_kernel(BatchWs w, int F, int B,
-                                                           unsigned long long* stats) {
-  __shared__ int s_scan[40];
-  const int tid = threadIdx.x;
-  int base = 0;
-  unsigned nsel = 0;
-  for (int c0 = 0; c0 < F; c0 += blockDim.x) {
-    const int ch = c0 + tid;
-    uint32_t bits = 0u;
-    if (ch < F)
-      for (int b = 0; b < B; ++b) bits |= w.smask[(size_t)b * F + ch] ? (1u << b) : 0u;
-    nsel += __popc(bits);
-    int total;
-    const int pos = base + block_exclusive_scan(bits ? 1 : 0, s_scan, &total);
-    if (bits) {
-      w.ulist[pos] = ch;
-      w.utok[pos] = bits;
-    }
-    base += total;
+// The channels some token selected, ascending, with the bit set of the
+// tokens that did, in two kernels over blocks of 256 channels like prepare:
+// union_count writes each block's count to ccount and adds the selected
+// (token, channel) pairs to the layer's statistics; union_place writes
+// ulist / utok and, in the last block, cnt[1].
+__device__ __forceinline__ uint32_t token_bits(const BatchWs& w, int F, int B, int ch) {
+  uint32_t bits = 0u;
+  if (ch < F)
+    for (int b = 0; b < B; ++b) bits |= w.smask[(size_t)b * F + ch] ? (1u << b) : 0u;
+  return bits;
+}
+
+__global__ void __launch_bounds__(256) batch_union_count_kernel(BatchWs w, int F, int B,
+                                                                unsigned long long* stats) {
+  __shared__ int s_red[8];
+  const int ch = blockIdx.x * 256 + threadIdx.x;
+  const uint32_t bits = token_bits(w, F, B, ch);
+  const int n = __syncthreads_count(bits != 0u);
+  int sel = __popc(bits);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sel += __shfl_xor_sync(0xffffffffu, sel, o);
+  if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = sel;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    w.ccount[blockIdx.x] = n;
+    int t = 0;
+    for (int i = 0; i < 8; ++i) t += s_red[i];
+    if (stats) atomicAdd(stats + 2, (unsigned long long)t);
   }
-  if (tid == 0) w.cnt[1] = base;
-  unsigned ts;
-  block_exclusive_scan(nsel, reinterpret_cast<unsigned*>(s_scan), &ts);
-  if (tid == 0 && stats) atomicAdd(stats + 2, (unsigned long long)ts);
+}
+
+__global__ void __launch_bounds__(256) batch_union_place_kernel(BatchWs w, int F, int B) {
+  __shared__ int s_scan[40];
+  const int blk = blockIdx.x, tid = threadIdx.x, ch = blk * 256 + tid;
+  if (tid < 32) {
+    int off = 0;
+    for (int j = tid; j < blk; j += 32) off += w.ccount[j];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) off += __shfl_xor_sync(0xffffffffu, off, o);
+    if (tid == 0) s_scan[36] = off;
+  }
+  const uint32_t bits = token_bits(w, F, B, ch);
+  __syncthreads();
+  const int off = s_scan[36];
+  int total;
+  const int pre = block_exclusive_scan(bits ? 1 : 0, s_scan, &total);
+  if (bits) {
+    w.ulist[off + pre] = ch;
+    w.utok[off + pre] = bits;
+  }
+  if (tid == 0 && blk == gridDim.x - 1) w.cnt[1] = off + total;
 }
 
 // ---------------------------------------------------------------------------
 // gate/up over the union channels (or every channel: dense)
 // ---------------------------------------------------------------------------
 
-constexpr int GU_THREADS = 256;  // 8 warps: gate / up x four 16-channel tiles
-constexpr int GU_M = 64;         // channels per CTA
-constexpr int GU_KT = 64;        // d_model elements per stage
+constexpr int GU_THREADS = 256;  // 8 warps: gate / up x four quarters of the k tile
+constexpr int GU_M = 16;         // channels per work tile
+constexpr int GU_KT = 256;       // d_model elements per stage: 512 contiguous bytes per column
 constexpr int GU_STAGES = 3;
 constexpr int GU_LDA = GU_KT + 8;
+constexpr int GU_MAXE = 256;     // union entries a CTA's run may touch (checked by the host)
 
 struct GuSmem {
   __nv_bfloat16 a[GU_STAGES][2][GU_M][GU_LDA];     // gate, up column slices [channel][k]
   __nv_bfloat16 bhi[GU_STAGES][NB][GU_LDA], blo[GU_STAGES][NB][GU_LDA];  // x [token][k]
+  float red[4][2][GU_M][NB];                       // the k quarters' sums of an item
+  int ch[GU_MAXE];                                 // channels of the run's union entries
 };
 
-// CTA c: union entries [64 c, 64 c + 64) (dense: channels).  Writes
-// hh / hl[token][entry] = h split hi / lo, h = act(g) u for the tokens that
-// selected the channel and 0 for the others (and for entries past the union).
+// Work items (tile, ks): union entries [16 tile, 16 tile + 16) (dense:
+// channels) over the d_model range ks of KS equal ranges of k tiles; the
+// T KS items (T = ceil(n / 16)) are split into equal contiguous runs, one per
+// CTA, and a CTA streams the k tiles of its run through one cp.async ring.
+// Each stage holds 512 contiguous bytes of each of the 32 gate / up columns.
+// Warp w adds kind w % 2 over the quarter w / 2 of the stage; at an item's
+// end the quarters are added in order and the item's sums written to
+// gup[item][entry][token][gate|up].
 __global__ void __launch_bounds__(GU_THREADS) batch_gateup_kernel(const __nv_bfloat16* __restrict__ wgu, int d,
-                                                                  int F, int B, int act, int dense,
-                                                                  BatchWs w) {
+                                                                  int F, int KS, int dense, BatchWs w) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   GuSmem& sm = *reinterpret_cast<GuSmem*>(smem_raw);
   const int n_s = dense ? F : w.cnt[1];
-  const int e0 = blockIdx.x * GU_M, Fp = (F + 63) & ~63;
-  if (e0 >= n_s) return;
+  const int T = (n_s + GU_M - 1) / GU_M, I = T * KS;
+  const int it0 = (int)((long long)I * blockIdx.x / gridDim.x);
+  const int it1 = (int)((long long)I * (blockIdx.x + 1) / gridDim.x);
+  const int nkt = (d + GU_KT - 1) / GU_KT, kper = nkt / KS;  // k tiles per item
+  const int nsteps = (it1 - it0) * kper;
+  if (nsteps <= 0) return;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int kind = warp >> 2, m0 = (warp & 3) * 16;
-  const int nkt = d / GU_KT;
+  const int kind = warp & 1, kq = warp >> 1;
+  // the run's channels, from its first tile's first entry
+  const int e_base = (it0 / KS) * GU_M;
+  for (int i = tid; i < GU_MAXE; i += GU_THREADS) {
+    const int e = e_base + i;
+    sm.ch[i] = dense ? min(e, F - 1) : __ldg(w.ulist + min(e, n_s - 1));
+  }
+  __syncthreads();
 
-  auto channel = [&](int e) { return dense ? min(e, F - 1) : __ldg(w.ulist + min(e, n_s - 1)); };
-  auto issue = [&](int kt) {
-    if (kt < nkt) {
-      const int st = kt % GU_STAGES, k0 = kt * GU_KT;
-      // 2 x 64 channels x 8 chunks, then 2 x 16 tokens x 8 chunks: 1280 copies
-      for (int j = tid; j < 1280; j += GU_THREADS) {
+  auto issue = [&](int step) {
+    if (step < nsteps) {
+      const int st = step % GU_STAGES, item = it0 + step / kper;
+      const int el = (item / KS) * GU_M - e_base;  // first entry of the item, in the run
+      const int k0 = ((item % KS) * kper + step % kper) * GU_KT;
+      // 32 columns x 32 chunks, then 2 x 16 tokens x 32 chunks: 2048 copies
+      for (int j = tid; j < 2048; j += GU_THREADS) {
+        const int c = j & 31, kk = k0 + c * 8;
+        __nv_bfloat16* dst;
+        const __nv_bfloat16* src;
         if (j < 1024) {
-          const int kd = j >> 9, m = (j >> 3) & 63, c = j & 7;
-          const size_t col = (size_t)channel(e0 + m) * 2 * d + (size_t)kd * d + k0 + c * 8;
-          cp16(&sm.a[st][kd][m][c * 8], wgu + col);
+          const int kd = j >> 9, m = (j >> 5) & 15;
+          dst = &sm.a[st][kd][m][c * 8];
+          src = wgu + (size_t)sm.ch[el + m] * 2 * d + (size_t)kd * d + kk;
         } else {
-          const int jj = j - 1024, lo = jj >> 7, n = (jj >> 3) & 15, c = jj & 7;
-          const __nv_bfloat16* src = (lo ? w.xf_lo : w.xf_hi) + (size_t)n * d + k0 + c * 8;
-          cp16(lo ? &sm.blo[st][n][c * 8] : &sm.bhi[st][n][c * 8], src);
+          const int lo = (j >> 9) & 1, n = (j >> 5) & 15;
+          dst = lo ? &sm.blo[st][n][c * 8] : &sm.bhi[st][n][c * 8];
+          src = (lo ? w.xf_lo : w.xf_hi) + (size_t)n * d + kk;
         }
+        if (kk < d) cp16(dst, src);
+        else *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
       }
     }
     cp_commit();
   };
 #pragma unroll
-  for (int kt = 0; kt < GU_STAGES - 1; ++kt) issue(kt);
+  for (int q = 0; q < GU_STAGES - 1; ++q) issue(q);
   float acc[2][4];
 #pragma unroll
   for (int h = 0; h < 2; ++h)
 #pragma unroll
     for (int e = 0; e < 4; ++e) acc[h][e] = 0.f;
-  for (int kt = 0; kt < nkt; ++kt) {
-    issue(kt + GU_STAGES - 1);
+  const int g = lane >> 2, t = lane & 3;
+  for (int step = 0; step < nsteps; ++step) {
+    issue(step + GU_STAGES - 1);
     cp_wait<GU_STAGES - 1>();
     __syncthreads();
-    const int st = kt % GU_STAGES;
+    const int st = step % GU_STAGES;
 #pragma unroll
-    for (int k0 = 0; k0 < GU_KT; k0 += 16) {
+    for (int k0 = kq * 64; k0 < kq * 64 + 64; k0 += 16) {
       uint32_t a[4];
-      ldsm_a(a, a_row_mk(&sm.a[st][kind][0][0], GU_LDA, m0, k0));
+      ldsm_a(a, a_row_mk(&sm.a[st][kind][0][0], GU_LDA, 0, k0));
       mma_tokens(acc, a, &sm.bhi[st][0][0], &sm.blo[st][0][0], GU_LDA, k0);
+    }
+    if (step % kper == kper - 1) {
+      // the item's sums: the quarters through shared memory, added in order
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int r = 0; r < 2; ++r)
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            sm.red[kq][kind][g + 8 * r][8 * h + 2 * t + c] = acc[h][2 * r + c];
+            acc[h][2 * r + c] = 0.f;
+          }
+      __syncthreads();
+      const int item = it0 + step / kper;
+      float* dst = w.gup + (size_t)item * GU_M * NB * 2;
+      for (int j = tid; j < GU_M * NB * 2; j += GU_THREADS) {
+        const int kd = j & 1, n = (j >> 1) & 15, m = j >> 5;
+        dst[j] = ((sm.red[0][kd][m][n] + sm.red[1][kd][m][n]) + sm.red[2][kd][m][n]) + sm.red[3][kd][m][n];
+      }
     }
     __syncthreads();
   }
   cp_wait<0>();
-  __syncthreads();
-  // g and u through shared memory: gu[kind][channel][token]
-  float* gu = reinterpret_cast<float*>(smem_raw);
-  {
-    const int g = lane >> 2, t = lane & 3;
-#pragma unroll
-    for (int h = 0; h < 2; ++h)
-#pragma unroll
-      for (int r = 0; r < 2; ++r)
-#pragma unroll
-        for (int c = 0; c < 2; ++c)
-          gu[(kind * GU_M + m0 + g + 8 * r) * NB + 8 * h + 2 * t + c] = acc[h][2 * r + c];
-  }
-  __syncthreads();
-  for (int j = tid; j < GU_M * NB; j += GU_THREADS) {
-    const int m = j / NB, n = j % NB, e = e0 + m;
-    float h = 0.f;
-    if (e < n_s && n < B) {
-      const bool sel = dense || ((__ldg(w.utok + e) >> n) & 1u);
-      if (sel) h = act_f32(gu[m * NB + n], act) * gu[(GU_M + m) * NB + n];
+}
+
+// One thread per (union entry < roundup(n, 64), token): g and u summed over
+// the KS items in order, h = act(g) u for the tokens that selected the
+// channel (every token < B when dense), 0 otherwise; split into hh / hl.
+__global__ void batch_gateup_finish_kernel(BatchWs w, int F, int B, int KS, int act, int dense) {
+  const int n_s = dense ? F : w.cnt[1];
+  const int e = blockIdx.x * (blockDim.x / NB) + threadIdx.x / NB, n = threadIdx.x % NB;
+  const int Fp = (F + 63) & ~63;
+  if (e >= ((n_s + 63) / 64) * 64) return;
+  float h = 0.f;
+  if (e < n_s && n < B && (dense || ((__ldg(w.utok + e) >> n) & 1u))) {
+    const int tile = e / GU_M, m = e % GU_M;
+    float gs = 0.f, us = 0.f;
+    for (int ks = 0; ks < KS; ++ks) {
+      const float2 v = *reinterpret_cast<const float2*>(
+          w.gup + (((size_t)(tile * KS + ks) * GU_M + m) * NB + n) * 2);
+      gs += v.x;
+      us += v.y;
     }
-    if (e < ((n_s + GU_M - 1) / GU_M) * GU_M)
-      split_bf16(h, w.hh + (size_t)n * Fp + e, w.hl + (size_t)n * Fp + e);
+    h = act_f32(gs, act) * us;
   }
+  split_bf16(h, w.hh + (size_t)n * Fp + e, w.hl + (size_t)n * Fp + e);
 }
 
 // ---------------------------------------------------------------------------
 // down over the union channels, then the split sum
 // ---------------------------------------------------------------------------
 
-constexpr int DN_THREADS = 256;  // 8 warps, one 16-column tile each
-constexpr int DN_M = 128;        // output columns per CTA
-constexpr int DN_KT = 64;        // union entries per stage
-constexpr int DN_STAGES = 3;
+constexpr int DN_THREADS = 256;  // 8 warps, two 16-column tiles each
+constexpr int DN_M = 256;        // output columns per CTA: 512 contiguous bytes per W_down row
+constexpr int DN_KT = 32;        // union entries per stage
+constexpr int DN_STAGES = 4;
 constexpr int DN_LDA = DN_M + 8;
 constexpr int DN_LDB = DN_KT + 8;
+constexpr int DN_MAXE = 4096;    // union entries a CTA's split may touch (checked by the host)
 
 struct DnSmem {
   __nv_bfloat16 a[DN_STAGES][DN_KT][DN_LDA];        // W_down rows' column slices [entry][column]
   __nv_bfloat16 bhi[DN_STAGES][NB][DN_LDB], blo[DN_STAGES][NB][DN_LDB];  // h [token][entry]
+  int ch[DN_MAXE];                                  // the split's channels
 };
 
-// Grid (d / 128, S5): CTA (cb, s) takes columns [128 cb, 128 cb + 128) and the
-// entry tiles [T s / S5, T (s + 1) / S5) of the T = ceil(n / 64) tiles;
+// Grid (d / 256, S5): CTA (cb, s) takes columns [256 cb, 256 cb + 256) and the
+// entry tiles [T s / S5, T (s + 1) / S5) of the T = ceil(n / 32) tiles;
 // writes yp[s][token][column].
 __global__ void __launch_bounds__(DN_THREADS) batch_down_kernel(const __nv_bfloat16* __restrict__ wd, int d,
                                                                 int F, int dense, BatchWs w) {
@@ -527,17 +707,24 @@ __global__ void __launch_bounds__(DN_THREADS) batch_down_kernel(const __nv_bfloa
   const int T = (n_s + DN_KT - 1) / DN_KT;
   const int t0 = (int)((long long)T * s / S5), t1 = (int)((long long)T * (s + 1) / S5);
   const int nt = t1 - t0;
-  auto channel = [&](int e) { return dense ? min(e, F - 1) : __ldg(w.ulist + min(e, n_s - 1)); };
+  for (int i = tid; i < nt * DN_KT; i += DN_THREADS) {
+    const int e = t0 * DN_KT + i;
+    sm.ch[i] = dense ? min(e, F - 1) : __ldg(w.ulist + min(e, n_s - 1));
+  }
+  __syncthreads();
   auto issue = [&](int it) {
     if (it < nt) {
       const int st = it % DN_STAGES, e0 = (t0 + it) * DN_KT;
-      // 64 entries x 16 chunks, then 2 x 16 tokens x 8 chunks: 1280 copies
-      for (int j = tid; j < 1280; j += DN_THREADS) {
+      // 32 entries x 32 chunks, then 2 x 16 tokens x 4 chunks: 1152 copies
+      for (int j = tid; j < 1152; j += DN_THREADS) {
         if (j < 1024) {
-          const int k = j >> 4, c = j & 15;
-          cp16(&sm.a[st][k][c * 8], wd + (size_t)channel(e0 + k) * d + col0 + c * 8);
+          const int k = j >> 5, c = j & 31;
+          if (col0 + c * 8 < d)
+            cp16(&sm.a[st][k][c * 8], wd + (size_t)sm.ch[it * DN_KT + k] * d + col0 + c * 8);
+          else  // past the last column (d_model not a multiple of 256)
+            *reinterpret_cast<uint4*>(&sm.a[st][k][c * 8]) = make_uint4(0u, 0u, 0u, 0u);
         } else {
-          const int jj = j - 1024, lo = jj >> 7, n = (jj >> 3) & 15, c = jj & 7;
+          const int jj = j - 1024, lo = jj >> 6, n = (jj >> 2) & 15, c = jj & 3;
           const __nv_bfloat16* src = (lo ? w.hl : w.hh) + (size_t)n * Fp + e0 + c * 8;
           cp16(lo ? &sm.blo[st][n][c * 8] : &sm.bhi[st][n][c * 8], src);
         }
@@ -547,34 +734,41 @@ __global__ void __launch_bounds__(DN_THREADS) batch_down_kernel(const __nv_bfloa
   };
 #pragma unroll
   for (int it = 0; it < DN_STAGES - 1; ++it) issue(it);
-  float acc[2][4];
+  float acc[2][2][4];
 #pragma unroll
-  for (int h = 0; h < 2; ++h)
+  for (int i = 0; i < 2; ++i)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) acc[h][e] = 0.f;
-  const int m0 = warp * 16;
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[i][h][e] = 0.f;
   for (int it = 0; it < nt; ++it) {
     issue(it + DN_STAGES - 1);
     cp_wait<DN_STAGES - 1>();
     __syncthreads();
     const int st = it % DN_STAGES;
 #pragma unroll
-    for (int k0 = 0; k0 < DN_KT; k0 += 16) {
-      uint32_t a[4];
-      ldsm_a_trans(a, a_row_km(&sm.a[st][0][0], DN_LDA, m0, k0));
-      mma_tokens(acc, a, &sm.bhi[st][0][0], &sm.blo[st][0][0], DN_LDB, k0);
-    }
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int k0 = 0; k0 < DN_KT; k0 += 16) {
+        uint32_t a[4];
+        ldsm_a_trans(a, a_row_km(&sm.a[st][0][0], DN_LDA, warp * 32 + i * 16, k0));
+        mma_tokens(acc[i], a, &sm.bhi[st][0][0], &sm.blo[st][0][0], DN_LDB, k0);
+      }
     __syncthreads();
   }
   cp_wait<0>();
   const int g = lane >> 2, t = lane & 3;
 #pragma unroll
-  for (int h = 0; h < 2; ++h)
+  for (int i = 0; i < 2; ++i)
 #pragma unroll
-    for (int r = 0; r < 2; ++r)
+    for (int h = 0; h < 2; ++h)
 #pragma unroll
-      for (int c = 0; c < 2; ++c)
-        w.yp[((size_t)s * NB + 8 * h + 2 * t + c) * d + col0 + m0 + g + 8 * r] = acc[h][2 * r + c];
+      for (int r = 0; r < 2; ++r)
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const int col = col0 + warp * 32 + i * 16 + g + 8 * r;
+          if (col < d) w.yp[((size_t)s * NB + 8 * h + 2 * t + c) * d + col] = acc[i][h][2 * r + c];
+        }
 }
 
 // y[b][col] = the split partials added in split order.
@@ -596,26 +790,39 @@ __global__ void batch_reduce_kernel(BatchWs w, int d, int B, int S5, float* __re
 namespace prox {
 
 namespace {
-size_t topk_smem(int F) { return ((sizeof(SelectScratch) + 15) & ~(size_t)15) + (size_t)F * 4; }
+size_t topk_smem(int F) { return (size_t)F * 4; }
 size_t al256(size_t b) { return (b + 255) & ~(size_t)255; }
 }  // namespace
 
-void choose_batch_splits(int d, int F, int num_sms, int* s1, int* s5) {
+void choose_batch_splits(int d, int F, int num_sms, int* s1, int* s5, int* ks) {
   const int hs = 2 * ((F + 511) / 512);  // half slices
   const int G = d / kGroup;
   *s1 = std::max(1, std::min(G, (2 * num_sms + hs - 1) / hs));
-  const int cb = d / DN_M;
-  *s5 = std::max(1, (2 * num_sms + cb - 1) / cb);
+  *s5 = std::max(1, 2 * num_sms / ((d + DN_M - 1) / DN_M));
+  // a split's entries must fit its channel table: at most DN_MAXE
+  while ((size_t)((F + DN_KT - 1) / DN_KT + *s5 - 1) / *s5 * DN_KT > (size_t)DN_MAXE) ++*s5;
+  const int nkt = (d + GU_KT - 1) / GU_KT;
+  int k = std::min(8, nkt);
+  while (nkt % k) --k;
+  *ks = k;
 }
 
-size_t batch_ws_bytes(int d, int F, int s1, int s5) {
+bool batch_fits(int F, int num_sms, int ks) {
+  // a gate/up run (2 num_sms CTAs) touches at most this many union entries
+  const long long T = (F + GU_M - 1) / GU_M, I = T * ks, grid = 2LL * num_sms;
+  return ((I + grid - 1) / grid / ks + 2) * GU_M <= GU_MAXE;
+}
+
+size_t batch_ws_bytes(int d, int F, int s1, int s5, int ks) {
   const size_t Fp = (size_t)((F + 63) & ~63), G = (size_t)d / kGroup;
   return 4 * al256((size_t)NB * d * 2) + al256((size_t)d * 4) + 2 * al256(G * 4) + al256(16) +
+         al256((size_t)(d + 255) / 256 * 4) + al256((size_t)(F + 255) / 256 * 4) +
          al256((size_t)s1 * NB * 2 * F * 4) + al256((size_t)NB * F * 4) + al256((size_t)NB * F) +
-         2 * al256((size_t)F * 4) + 2 * al256((size_t)NB * Fp * 2) + al256((size_t)s5 * NB * d * 4);
+         2 * al256((size_t)F * 4) + al256(Fp / GU_M * ks * GU_M * NB * 2 * 4) +
+         2 * al256((size_t)NB * Fp * 2) + al256((size_t)s5 * NB * d * 4);
 }
 
-void carve_batch_ws(void* base, int d, int F, int s1, int s5, BatchWs* w) {
+void carve_batch_ws(void* base, int d, int F, int s1, int s5, int ks, BatchWs* w) {
   const size_t Fp = (size_t)((F + 63) & ~63), G = (size_t)d / kGroup;
   char* p = static_cast<char*>(base);
   auto take = [&](size_t bytes) {
@@ -631,11 +838,14 @@ void carve_batch_ws(void* base, int d, int F, int s1, int s5, BatchWs* w) {
   w->gstart = reinterpret_cast<int*>(take(G * 4));
   w->gcount = reinterpret_cast<int*>(take(G * 4));
   w->cnt = reinterpret_cast<int*>(take(16));
+  w->rcount = reinterpret_cast<int*>(take((size_t)(d + 255) / 256 * 4));
+  w->ccount = reinterpret_cast<int*>(take((size_t)(F + 255) / 256 * 4));
   w->part1 = reinterpret_cast<float*>(take((size_t)s1 * NB * 2 * F * 4));
   w->scores = reinterpret_cast<float*>(take((size_t)NB * F * 4));
   w->smask = reinterpret_cast<uint8_t*>(take((size_t)NB * F));
   w->ulist = reinterpret_cast<int*>(take((size_t)F * 4));
   w->utok = reinterpret_cast<uint32_t*>(take((size_t)F * 4));
+  w->gup = reinterpret_cast<float*>(take(Fp / GU_M * ks * GU_M * NB * 2 * 4));  // Fp / 16 tiles
   w->hh = reinterpret_cast<__nv_bfloat16*>(take((size_t)NB * Fp * 2));
   w->hl = reinterpret_cast<__nv_bfloat16*>(take((size_t)NB * Fp * 2));
   w->yp = reinterpret_cast<float*>(take((size_t)s5 * NB * d * 4));
@@ -662,19 +872,25 @@ cudaError_t launch_batch(const prox_layer* L, const float* X, float* Y, int B, b
   const int d = L->d, F = L->F;
   const __nv_bfloat16* wgu = reinterpret_cast<const __nv_bfloat16*>(L->wgu);
   const __nv_bfloat16* wd = reinterpret_cast<const __nv_bfloat16*>(L->wd);
-  batch_prepare_kernel<<<1, 1024, 0, s>>>(X, B, d, L->tau, w, dense ? nullptr : L->ws.stats);
+  const int rb = (d + 255) / 256, cb = (F + 255) / 256;
+  batch_prepare_count_kernel<<<rb, 256, 0, s>>>(X, B, d, L->tau, w, dense ? nullptr : L->ws.stats);
+  batch_prepare_place_kernel<<<rb, 256, 0, s>>>(X, B, d, L->tau, w);
   if (!dense) {
     batch_stage1_kernel<<<dim3(2 * ((F + 511) / 512), L->b_s1), S1_THREADS, sizeof(S1Smem), s>>>(
         L->pq, reinterpret_cast<const __half*>(L->ps), d, F, w);
     const bool thr = L->mask_mode == PROX_MASK_THRESHOLD;
     batch_score_kernel<<<dim3((F + 255) / 256, B), 256, 0, s>>>(w, F, L->b_s1, L->act, thr ? 1 : 0,
                                                                 L->tau_s);
-    if (!thr) batch_topk_kernel<<<B, 1024, topk_smem(F), s>>>(w, F, L->k);
-    batch_union_kernel<<<1, 1024, 0, s>>>(w, F, B, L->ws.stats);
+    if (!thr) batch_topk_kernel<<<B, TK_THREADS, topk_smem(F), s>>>(w, F, L->k);
+    batch_union_count_kernel<<<cb, 256, 0, s>>>(w, F, B, L->ws.stats);
+    batch_union_place_kernel<<<cb, 256, 0, s>>>(w, F, B);
   }
-  batch_gateup_kernel<<<(F + GU_M - 1) / GU_M, GU_THREADS, sizeof(GuSmem), s>>>(wgu, d, F, B, L->act,
-                                                                                dense ? 1 : 0, w);
-  batch_down_kernel<<<dim3(d / DN_M, L->b_s5), DN_THREADS, sizeof(DnSmem), s>>>(wd, d, F, dense ? 1 : 0, w);
+  batch_gateup_kernel<<<2 * L->num_sms, GU_THREADS, sizeof(GuSmem), s>>>(wgu, d, F, L->b_ks,
+                                                                          dense ? 1 : 0, w);
+  const int Fp = (F + 63) & ~63;
+  batch_gateup_finish_kernel<<<Fp * NB / 256, 256, 0, s>>>(w, F, B, L->b_ks, L->act, dense ? 1 : 0);
+  batch_down_kernel<<<dim3((d + DN_M - 1) / DN_M, L->b_s5), DN_THREADS, sizeof(DnSmem), s>>>(
+      wd, d, F, dense ? 1 : 0, w);
   batch_reduce_kernel<<<dim3((d + 255) / 256, B), 256, 0, s>>>(w, d, B, L->b_s5, Y);
   return cudaGetLastError();
 }

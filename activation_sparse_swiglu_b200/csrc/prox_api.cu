@@ -168,8 +168,11 @@ prox_status alloc_workspace(prox_layer* L) {
   // the batched step's scratch (max_batch > 1), in the same allocation
   size_t o_batch = 0;
   if (L->max_batch > 1) {
-    prox::choose_batch_splits(L->d, L->F, L->num_sms, &L->b_s1, &L->b_s5);
-    o_batch = take(prox::batch_ws_bytes(L->d, L->F, L->b_s1, L->b_s5));
+    prox::choose_batch_splits(L->d, L->F, L->num_sms, &L->b_s1, &L->b_s5, &L->b_ks);
+    if (!prox::batch_fits(L->F, L->num_sms, L->b_ks))
+      return fail(PROX_EUNSUPPORTED, "d_ff=%d on %d SMs exceeds the batched step's channel table",
+                  L->F, L->num_sms);
+    o_batch = take(prox::batch_ws_bytes(L->d, L->F, L->b_s1, L->b_s5, L->b_ks));
   }
   const size_t o_in = take((size_t)kHostChunkTokens * d * 4);
   const size_t o_out = take((size_t)kHostChunkTokens * d * 4);
@@ -202,7 +205,7 @@ prox_status alloc_workspace(prox_layer* L) {
   w.stage_in = reinterpret_cast<float*>(b + o_in);
   if (L->max_batch > 1) {
     L->bws_base = b + o_batch;
-    prox::carve_batch_ws(L->bws_base, L->d, L->F, L->b_s1, L->b_s5, &L->bws);
+    prox::carve_batch_ws(L->bws_base, L->d, L->F, L->b_s1, L->b_s5, L->b_ks, &L->bws);
   }
   w.stage_out = reinterpret_cast<float*>(b + o_out);
   return PROX_OK;
@@ -772,7 +775,7 @@ prox_status prox_layer_proxy_scores(const prox_layer* L, const float* x, int B, 
                                     void* stream) {
   prox_status st = check_layer(L);
   if (st != PROX_OK) return st;
-  if (B < 1 || B > L->max_batch) return fail(PROX_EINVAL, "B=%d must be in [1, %d]", B, L->max_batch);
+  if (B < 1) return fail(PROX_EINVAL, "B=%d must be >= 1", B);
   if (!x || !scores || !aligned16(x)) return fail(PROX_EINVAL, "x (16-byte aligned) and scores must be non-NULL");
   cudaStream_t s = as_stream(stream);
   for (int b = 0; b < B; ++b) {

@@ -72,11 +72,14 @@ struct BatchWs {
   int* gstart = nullptr;           // [G] first union entry of each quantisation group
   int* gcount = nullptr;           // [G] union rows in each group
   int* cnt = nullptr;              // [4] union rows, union channels
+  int* rcount = nullptr;           // [d / 256] union rows per block of 256 rows
+  int* ccount = nullptr;           // [d_ff / 256] union channels per block of 256
   float* part1 = nullptr;          // [S1][16][2][F] Stage-1 sums per row split
   float* scores = nullptr;         // [16][F]
   uint8_t* smask = nullptr;        // [16][F] per-token channel masks
   int* ulist = nullptr;            // [F] the union channels, ascending
   uint32_t* utok = nullptr;        // [F] the tokens that selected each
+  float* gup = nullptr;            // [Fp / 64 * KS][64][16][2] gate / up sums per work item
   __nv_bfloat16* hh = nullptr;     // [16][Fp] h per token and union entry, hi part
   __nv_bfloat16* hl = nullptr;     //                                      ... lo part
   float* yp = nullptr;             // [S5][16][d] down partials per entry split
@@ -107,7 +110,7 @@ struct prox_layer {
   uint16_t* ps = nullptr;    // fp16 scales [G][F/32][2][32]
   prox::Workspace ws;
   // batched step: row splits of its Stage 1, entry splits of its down product
-  int b_s1 = 0, b_s5 = 0;
+  int b_s1 = 0, b_s5 = 0, b_ks = 1;
   void* bws_base = nullptr;
   prox::BatchWs bws;
 };
@@ -143,9 +146,10 @@ cudaError_t setup_token_kernels();
 // The batched step (batch.cu): B <= kBatchMax tokens, union loads; dense =
 // every channel for every token (the batched dense baseline).
 cudaError_t setup_batch_kernels();
-void choose_batch_splits(int d, int F, int num_sms, int* s1, int* s5);
-size_t batch_ws_bytes(int d, int F, int s1, int s5);
-void carve_batch_ws(void* base, int d, int F, int s1, int s5, BatchWs* w);
+void choose_batch_splits(int d, int F, int num_sms, int* s1, int* s5, int* ks);
+bool batch_fits(int F, int num_sms, int ks);
+size_t batch_ws_bytes(int d, int F, int s1, int s5, int ks);
+void carve_batch_ws(void* base, int d, int F, int s1, int s5, int ks, BatchWs* w);
 cudaError_t launch_batch(const prox_layer* L, const float* X, float* Y, int B, bool dense,
                          cudaStream_t s);
 cudaError_t launch_barrier_probe(const prox_layer* L, cudaStream_t s);

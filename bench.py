@@ -891,25 +891,57 @@ class Bench:
         s = self.stream
         rows = []
         steps = max(2, self.args.steps // 10)
+        C = (f + 511) // 512
         for B in cfg.batch_sizes:
             nb = 64 // B  # batches per step
 
-            def body(B=B, nb=nb):
+            def chain(B=B, nb=nb):  # B single-token launches per batch
                 for i in range(nb):
                     layers[i % nc].forward(x[i * B:(i + 1) * B], out[i * B:(i + 1) * B], stream=s)
 
-            def dbody(B=B, nb=nb):
+            def union(B=B, nb=nb):  # one batched step per batch: union loads
                 for i in range(nb):
-                    layers[i % nc].dense(x[i * B:(i + 1) * B], out[i * B:(i + 1) * B], stream=s)
-            tok, _ = self.timer.tokens_per_s(body, nb * B, steps)
-            dtok, _ = self.timer.tokens_per_s(dbody, nb * B, steps)
-            rows.append({"batch": B, "tokens_per_s": round(tok, 1),
-                         "dense_tokens_per_s": round(dtok, 1),
-                         "speedup_vs_dense": round(tok / dtok, 3),
-                         "us_per_batch": round(B * 1e6 / tok, 1)})
+                    layers[i % nc].forward_batch(x[i * B:(i + 1) * B], out[i * B:(i + 1) * B], stream=s)
+
+            def dense(B=B, nb=nb):  # batched dense, every weight read once
+                for i in range(nb):
+                    layers[i % nc].dense_batch(x[i * B:(i + 1) * B], out[i * B:(i + 1) * B], stream=s)
+            # the union sizes of this step's batches (bytes the union path reads)
+            n_rows, n_ch = [], []
+            for i in range(nb):
+                layers[i % nc].forward_batch(x[i * B:(i + 1) * B], out[i * B:(i + 1) * B], stream=s)
+                r_, c_ = layers[i % nc].batch_union_sizes(stream=s)
+                n_rows.append(r_)
+                n_ch.append(c_)
+            mean_rows, mean_ch = float(np.mean(n_rows)), float(np.mean(n_ch))
+            union_bytes = mean_rows * C * 512 + mean_ch * 6 * d + 8 * B * d
+            dense_bytes = 6.0 * d * f + 8 * B * d
+            tok_c, _ = self.timer.tokens_per_s(chain, nb * B, steps)
+            tok_u, _ = self.timer.tokens_per_s(union, nb * B, steps)
+            tok_d, _ = self.timer.tokens_per_s(dense, nb * B, steps)
+            rows.append({
+                "batch": B,
+                "union_tokens_per_s": round(tok_u, 1),
+                "chain_tokens_per_s": round(tok_c, 1),
+                "dense_tokens_per_s": round(tok_d, 1),
+                "speedup_vs_dense": round(tok_u / tok_d, 3),
+                "chain_speedup_vs_dense": round(tok_c / tok_d, 3),
+                "union_rows_frac": round(mean_rows / d, 4),
+                "union_channels_frac": round(mean_ch / f, 4),
+                "union_bytes_per_batch": int(union_bytes),
+                "union_hbm_gbs": round(union_bytes * tok_u / B / 1e9, 1),
+                "dense_hbm_gbs": round(dense_bytes * tok_d / B / 1e9, 1),
+                "us_per_batch": round(B * 1e6 / tok_u, 1)})
+        best = [r["batch"] for r in rows if r["speedup_vs_dense"] > 1.0]
+        crossover = {"last_batch_union_beats_dense": max(best) if best else None}
         self.result["llama3_70b"] = {
             "workload": f"llama3_70b ffn layer d_model={d} d_ff={f} s1=50% s2=70% k={k}, "
-                        "per-token masks", "rows": rows, "layer_copies": nc}
+                        "per-token masks",
+            "paths": "union = prox_ffn_forward_batch (one batched step, union loads); chain = "
+                     "prox_ffn_forward (B batch-1 launches); dense = prox_dense_ffn_batch (every "
+                     "weight read once); bytes: union rows x proxy row + union channels x 6 d "
+                     "(gate/up record + W_down row) + x/out; dense 6 d d_ff + x/out",
+            "rows": rows, "crossover": crossover, "layer_copies": nc}
         for L in layers:
             L.close()
         torch.cuda.empty_cache()

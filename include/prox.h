@@ -354,7 +354,7 @@ PROX_API prox_status prox_debug_stage1(prox_layer* layer, const float* x, int32_
  * into scores [B, d_ff] (fp32, device), with the layer's tau_x.  The input to
  * calibrating tau_s (Prox App. A.7, Algorithm 1: the s2-quantile of these
  * scores over the calibration tokens, e.g. with prox_calibrate_thresholds).
- * Stream-ordered; B <= max_batch. */
+ * Stream-ordered; any B >= 1 (the tokens run one after another). */
 PROX_API prox_status prox_layer_proxy_scores(const prox_layer* layer, const float* x, int B,
                                              float* scores, void* stream);
 
