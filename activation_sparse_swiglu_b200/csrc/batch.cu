@@ -542,28 +542,25 @@ __global__ void __launch_bounds__(256) batch_union_place_kernel(BatchWs w, int F
 // gate/up over the union channels (or every channel: dense)
 // ---------------------------------------------------------------------------
 
-constexpr int GU_THREADS = 256;  // 8 warps: gate / up x four quarters of the k tile
-constexpr int GU_M = 16;         // channels per work tile
-constexpr int GU_KT = 256;       // d_model elements per stage: 512 contiguous bytes per column
+constexpr int GU_THREADS = 256;  // 8 warps: gate / up x four 16-channel tiles
+constexpr int GU_M = 64;         // channels per work tile
+constexpr int GU_KT = 64;        // d_model elements per stage
 constexpr int GU_STAGES = 3;
 constexpr int GU_LDA = GU_KT + 8;
-constexpr int GU_MAXE = 256;     // union entries a CTA's run may touch (checked by the host)
+constexpr int GU_MAXE = 1024;    // union entries a CTA's run may touch (checked by the host)
 
 struct GuSmem {
   __nv_bfloat16 a[GU_STAGES][2][GU_M][GU_LDA];     // gate, up column slices [channel][k]
   __nv_bfloat16 bhi[GU_STAGES][NB][GU_LDA], blo[GU_STAGES][NB][GU_LDA];  // x [token][k]
-  float red[4][2][GU_M][NB];                       // the k quarters' sums of an item
   int ch[GU_MAXE];                                 // channels of the run's union entries
 };
 
-// Work items (tile, ks): union entries [16 tile, 16 tile + 16) (dense:
+// Work items (tile, ks): union entries [64 tile, 64 tile + 64) (dense:
 // channels) over the d_model range ks of KS equal ranges of k tiles; the
-// T KS items (T = ceil(n / 16)) are split into equal contiguous runs, one per
-// CTA, and a CTA streams the k tiles of its run through one cp.async ring.
-// Each stage holds 512 contiguous bytes of each of the 32 gate / up columns.
-// Warp w adds kind w % 2 over the quarter w / 2 of the stage; at an item's
-// end the quarters are added in order and the item's sums written to
-// gup[item][entry][token][gate|up].
+// T KS items (T = ceil(n / 64)) are split into equal contiguous runs, one per
+// CTA, and a CTA streams the k tiles of its run through one cp.async ring
+// (the run's channel indices staged in shared memory first), writing each
+// item's gate and up sums to gup[item][entry][token][gate|up].
 __global__ void __launch_bounds__(GU_THREADS) batch_gateup_kernel(const __nv_bfloat16* __restrict__ wgu, int d,
                                                                   int F, int KS, int dense, BatchWs w) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
@@ -572,14 +569,14 @@ __global__ void __launch_bounds__(GU_THREADS) batch_gateup_kernel(const __nv_bfl
   const int T = (n_s + GU_M - 1) / GU_M, I = T * KS;
   const int it0 = (int)((long long)I * blockIdx.x / gridDim.x);
   const int it1 = (int)((long long)I * (blockIdx.x + 1) / gridDim.x);
-  const int nkt = (d + GU_KT - 1) / GU_KT, kper = nkt / KS;  // k tiles per item
+  const int kper = d / GU_KT / KS;        // k tiles per item
   const int nsteps = (it1 - it0) * kper;
   if (nsteps <= 0) return;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int kind = warp & 1, kq = warp >> 1;
-  // the run's channels, from its first tile's first entry
+  const int kind = warp >> 2, m0 = (warp & 3) * 16;
   const int e_base = (it0 / KS) * GU_M;
-  for (int i = tid; i < GU_MAXE; i += GU_THREADS) {
+  const int ne = min(GU_MAXE, ((it1 - 1) / KS + 1) * GU_M - e_base);
+  for (int i = tid; i < ne; i += GU_THREADS) {
     const int e = e_base + i;
     sm.ch[i] = dense ? min(e, F - 1) : __ldg(w.ulist + min(e, n_s - 1));
   }
@@ -588,24 +585,19 @@ __global__ void __launch_bounds__(GU_THREADS) batch_gateup_kernel(const __nv_bfl
   auto issue = [&](int step) {
     if (step < nsteps) {
       const int st = step % GU_STAGES, item = it0 + step / kper;
-      const int el = (item / KS) * GU_M - e_base;  // first entry of the item, in the run
+      const int el = (item / KS) * GU_M - e_base;
       const int k0 = ((item % KS) * kper + step % kper) * GU_KT;
-      // 32 columns x 32 chunks, then 2 x 16 tokens x 32 chunks: 2048 copies
-      for (int j = tid; j < 2048; j += GU_THREADS) {
-        const int c = j & 31, kk = k0 + c * 8;
-        __nv_bfloat16* dst;
-        const __nv_bfloat16* src;
+      // 2 x 64 channels x 8 chunks, then 2 x 16 tokens x 8 chunks: 1280 copies
+      for (int j = tid; j < 1280; j += GU_THREADS) {
         if (j < 1024) {
-          const int kd = j >> 9, m = (j >> 5) & 15;
-          dst = &sm.a[st][kd][m][c * 8];
-          src = wgu + (size_t)sm.ch[el + m] * 2 * d + (size_t)kd * d + kk;
+          const int kd = j >> 9, m = (j >> 3) & 63, c = j & 7;
+          const size_t col = (size_t)sm.ch[el + m] * 2 * d + (size_t)kd * d + k0 + c * 8;
+          cp16(&sm.a[st][kd][m][c * 8], wgu + col);
         } else {
-          const int lo = (j >> 9) & 1, n = (j >> 5) & 15;
-          dst = lo ? &sm.blo[st][n][c * 8] : &sm.bhi[st][n][c * 8];
-          src = (lo ? w.xf_lo : w.xf_hi) + (size_t)n * d + kk;
+          const int jj = j - 1024, lo = jj >> 7, n = (jj >> 3) & 15, c = jj & 7;
+          const __nv_bfloat16* src = (lo ? w.xf_lo : w.xf_hi) + (size_t)n * d + k0 + c * 8;
+          cp16(lo ? &sm.blo[st][n][c * 8] : &sm.bhi[st][n][c * 8], src);
         }
-        if (kk < d) cp16(dst, src);
-        else *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
       }
     }
     cp_commit();
@@ -624,29 +616,23 @@ __global__ void __launch_bounds__(GU_THREADS) batch_gateup_kernel(const __nv_bfl
     __syncthreads();
     const int st = step % GU_STAGES;
 #pragma unroll
-    for (int k0 = kq * 64; k0 < kq * 64 + 64; k0 += 16) {
+    for (int k0 = 0; k0 < GU_KT; k0 += 16) {
       uint32_t a[4];
-      ldsm_a(a, a_row_mk(&sm.a[st][kind][0][0], GU_LDA, 0, k0));
+      ldsm_a(a, a_row_mk(&sm.a[st][kind][0][0], GU_LDA, m0, k0));
       mma_tokens(acc, a, &sm.bhi[st][0][0], &sm.blo[st][0][0], GU_LDA, k0);
     }
     if (step % kper == kper - 1) {
-      // the item's sums: the quarters through shared memory, added in order
+      const int item = it0 + step / kper;
+      float* dst = w.gup + (size_t)item * GU_M * NB * 2;
 #pragma unroll
       for (int h = 0; h < 2; ++h)
 #pragma unroll
         for (int r = 0; r < 2; ++r)
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
-            sm.red[kq][kind][g + 8 * r][8 * h + 2 * t + c] = acc[h][2 * r + c];
+            dst[((m0 + g + 8 * r) * NB + 8 * h + 2 * t + c) * 2 + kind] = acc[h][2 * r + c];
             acc[h][2 * r + c] = 0.f;
           }
-      __syncthreads();
-      const int item = it0 + step / kper;
-      float* dst = w.gup + (size_t)item * GU_M * NB * 2;
-      for (int j = tid; j < GU_M * NB * 2; j += GU_THREADS) {
-        const int kd = j & 1, n = (j >> 1) & 15, m = j >> 5;
-        dst[j] = ((sm.red[0][kd][m][n] + sm.red[1][kd][m][n]) + sm.red[2][kd][m][n]) + sm.red[3][kd][m][n];
-      }
     }
     __syncthreads();
   }
@@ -808,8 +794,8 @@ void choose_batch_splits(int d, int F, int num_sms, int* s1, int* s5, int* ks) {
 }
 
 bool batch_fits(int F, int num_sms, int ks) {
-  // a gate/up run (2 num_sms CTAs) touches at most this many union entries
-  const long long T = (F + GU_M - 1) / GU_M, I = T * ks, grid = 2LL * num_sms;
+  // a gate/up run (3 num_sms CTAs) touches at most this many union entries
+  const long long T = (F + GU_M - 1) / GU_M, I = T * ks, grid = 3LL * num_sms;
   return ((I + grid - 1) / grid / ks + 2) * GU_M <= GU_MAXE;
 }
 
@@ -885,7 +871,7 @@ cudaError_t launch_batch(const prox_layer* L, const float* X, float* Y, int B, b
     batch_union_count_kernel<<<cb, 256, 0, s>>>(w, F, B, L->ws.stats);
     batch_union_place_kernel<<<cb, 256, 0, s>>>(w, F, B);
   }
-  batch_gateup_kernel<<<2 * L->num_sms, GU_THREADS, sizeof(GuSmem), s>>>(wgu, d, F, L->b_ks,
+  batch_gateup_kernel<<<3 * L->num_sms, GU_THREADS, sizeof(GuSmem), s>>>(wgu, d, F, L->b_ks,
                                                                           dense ? 1 : 0, w);
   const int Fp = (F + 63) & ~63;
   batch_gateup_finish_kernel<<<Fp * NB / 256, 256, 0, s>>>(w, F, B, L->b_ks, L->act, dense ? 1 : 0);

@@ -140,6 +140,33 @@ def test_stack_of_eight_small_layers(prox):
     _stack_case(prox, cfg, n_layers=8, n_cal=32, n_tok=2)
 
 
+def test_stack32_all_layers_teacher_forced(prox):
+    """All 32 full-size layers of the stack workload, one token, teacher-forced:
+    each layer is built, checked on the oracle's own input to it (its tau_x
+    from Algorithm 1 on the oracle's calibration inputs, bit-exact on the GPU;
+    mask and output as in every step check) and freed before the next, so
+    only one layer's weights are held at a time."""
+    cfg = synth.get_config("stack32")
+    k = cfg.k()
+    x_cal = x = None
+    for li in range(cfg.n_layers):
+        lay = synth.make_layer(cfg, li, draw_tokens=(li == 0), n_cal=2, n_tokens=1)
+        if li == 0:
+            x_cal, x = lay.x_cal, lay.x_eval[0]
+        olay = OracleLayer(lay)
+        tau = orc.calibrate_tau(x_cal, 0.5)
+        assert np.float32(prox.calibrate_thresholds(torch.from_numpy(x_cal).cuda(), 0.5)) == tau
+        layer = device_layer(lay, tau, k)
+        ref = _step_checks(layer, olay, x, tau, k)
+        assert layer.error_word() == 0
+        layer.close()
+        if li + 1 < cfg.n_layers:
+            x_cal = np.stack([orc.stack_next_input(olay.step(xt, tau, k)["y"]) for xt in x_cal])
+            x = orc.stack_next_input(ref["y"])
+        del lay, olay
+        torch.cuda.empty_cache()
+
+
 def test_stack32_first_two_layers_full_size(prox):
     # the 32-layer workload's own seeds and shapes, first two layers
     _stack_case(prox, synth.get_config("stack32"), n_layers=2, n_cal=16, n_tok=1)

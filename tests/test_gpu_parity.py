@@ -125,6 +125,10 @@ def _stage1_case(prox, lay, olay, tau, k, tokens):
                           taps["u_tilde"].cpu().numpy().astype(np.float64))
         ok, nbad = close_with_floor(scores_g, scores_o)
         assert ok, f"scores off at {nbad} channels"
+        # the scores the kernel itself ranks (device buffer, SiLU path)
+        scores_dev = layer.proxy_scores(torch.from_numpy(x).cuda().reshape(1, -1))
+        ok, nbad = close_with_floor(scores_dev.cpu().numpy().reshape(-1), scores_o)
+        assert ok, f"device scores off at {nbad} channels"
         n_diff += check_mask(taps["idx_s"].cpu().numpy(), orc.topk_channels(scores_o, k),
                              scores_o, k)
     assert layer.error_word() == 0

@@ -76,6 +76,11 @@ def test_geglu_llama3_8b_sampled(prox):
     _geglu_case(prox, "llama3_8b", prox.ACT_GELU_TANH, tokens=[0])
 
 
+def test_geglu_erf_llama3_8b_sampled(prox):
+    # GELU as z Phi(z) (erf form) at full size
+    _geglu_case(prox, "llama3_8b", prox.ACT_GELU_ERF, tokens=[0])
+
+
 def _a3_case(prox, name, tokens, threshold=False, act=0):
     lay = synth.make_layer(name, n_tokens=max(tokens) + 1, n_cal=16)
     olay = OracleLayer(lay)
