@@ -196,11 +196,15 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}, "fallback"
 
 
+TOKEN_KERNEL_SOURCES = ("token.cu", "token_args.cuh", "stage1.cuh", "stage2.cuh", "select.cuh",
+                        "prox_device.cuh")
+
+
 def kernel_source_hash() -> str:
-    """Hash of every kernel source file; a traffic record counts only while
-    the sources hash the same as when it was taken."""
+    """Hash of the per-token kernel's source files; a traffic record counts
+    only while they hash the same as when it was taken."""
     h = hashlib.sha256()
-    for name in sorted(os.listdir(CSRC)):
+    for name in TOKEN_KERNEL_SOURCES:
         with open(os.path.join(CSRC, name), "rb") as fh:
             h.update(name.encode())
             h.update(fh.read())

@@ -22,10 +22,13 @@
  *  - Shape rules (else PROX_EINVAL, checked before any launch):
  *    d_model > 0 and d_model % 128 == 0; d_ff > 0 and d_ff % 32 == 0;
  *    d_model <= 16384; d_ff <= 32768; 1 <= k <= d_ff; pointers 16-byte aligned.
- *    Stage 1 keeps its share of the kept input rows in shared memory, which
- *    bounds ceil(d_ff/512) * d_model <= 5192 * (number of SMs): about 768 K on
- *    a 148-SM B200, so every d_model at d_ff = 14336 but d_model <= 11904 at
- *    d_ff = 32768.  prox_layer_create returns PROX_EUNSUPPORTED beyond it.
+ *    Stage 1 keeps its share of the kept input rows in shared memory beside a
+ *    ring of at least two row batches, which bounds ceil(d_ff/512) * d_model
+ *    <= 7730 * (number of SMs), and the scoring takes one channel per thread,
+ *    which bounds d_ff <= 512 * (number of SMs): on a 148-SM B200 every shape
+ *    the rules above admit (at most 64 * 16384 = 1.05 M <= 1.14 M).  On a
+ *    device with fewer SMs prox_layer_create returns PROX_EUNSUPPORTED beyond
+ *    them.
  *  - Errors: every call returns a prox_status; prox_last_error() copies a
  *    message for the calling thread's last failure.  No C++ exception crosses
  *    this boundary.  Device-side checks (an index out of range in a caller's
@@ -328,14 +331,18 @@ PROX_API prox_status prox_ffn_forward_host(prox_layer* layer, const float* x_hos
  * void*) recorded right before and right after the token's kernel, which is
  * launched without programmatic overlap so the interval is its duration.
  * phase_ns (device, may be NULL): uint64 [stage1_ctas][24] receiving, per CTA,
- * the GPU global timer (ns) at: 0 kernel entry, 1 the previous kernel of the
- * stream complete, 2 Stage 1 done, 3 all scores visible (first grid barrier),
- * 4 channels selected, 5 partial output row written, 6 second grid barrier,
- * 7 output written, 8 kept rows compacted, 9 Stage-1 row loop done, 10 the
- * CTA's scores written, 11 Stage-2 ring set up, 12 gate/up phase done, 14 the
- * score histograms complete (top-k rule: second grid barrier), 15 the top-k
- * cut found; slot 13 holds the CTA's number of selected channels; the other
- * slots are 0. */
+ * the SM's cycle count (clock64) at: 0 kernel entry, 1 the previous kernel of
+ * the stream complete, 8 kept rows compacted, 9 Stage-1 row loop done,
+ * 2 Stage-1 partials written, 16 every CTA's partials written (phase 0),
+ * 3 the partials of thread 0's channel received, 10 the CTA's channels scored
+ * and counted, 17 every CTA's scores counted (phase 1), 14 the coarse
+ * histogram complete, 15 the top-k cut found, 18 every CTA's count written
+ * (phase 2), 4 the CTA's Stage-2 channels known, 11 Stage-2 ring set up,
+ * 12 gate/up phase done, 5 partial output row written, 19 every partial row
+ * written (phase 3), 6 the partial rows of the CTA's columns received,
+ * 7 output written, 21 exit; slots 22 and 23 hold the GPU global timer (ns)
+ * at entry and exit, which place the cycle counts on one time line; slot 13
+ * holds the CTA's number of Stage-2 channels; slots not reached are 0. */
 PROX_API prox_status prox_ffn_forward_profiled(const prox_layer* layer, const float* x, float* out,
                                                void* const* events_host, uint64_t* phase_ns,
                                                void* stream);
@@ -385,12 +392,12 @@ PROX_API prox_status prox_debug_batch_masks(const prox_layer* layer, uint8_t* ma
 PROX_API prox_status prox_debug_fail_alloc(int nth);
 
 /* Test-only exercise of the bounded device waits, with no fault: launches one
- * CTA that arrives at the layer's grid barrier and waits for an arrival that
- * never comes.  The wait runs out after its bound (2e8 SM cycles, about 0.1 s),
- * sets PROX_DEVERR_WAIT_TIMEOUT in the layer's error word and the kernel
- * returns.  prox_layer_error then reports the bit and, as after any timeout,
- * resets the barrier, the Stage-1 counters and the histogram so that the next
- * token runs clean.  Stream-ordered. */
+ * CTA that adds one to the layer's launch counter and waits for a second
+ * addition that never comes.  The wait runs out after its bound (2e8 SM
+ * cycles, about 0.1 s), sets PROX_DEVERR_WAIT_TIMEOUT in the layer's error
+ * word and the kernel returns.  prox_layer_error then reports the bit and, as
+ * after any timeout, clears the launch counter, the histograms and the tagged
+ * exchange words so that the next token runs clean.  Stream-ordered. */
 PROX_API prox_status prox_debug_wait_timeout(prox_layer* layer, void* stream);
 
 /* ------------------------------------------------------------------------

@@ -237,3 +237,35 @@ def test_stack_threshold_rule_small(prox):
         assert layer.error_word() == 0
     stack.close()
 
+
+
+# ---------------------------------------------------------------------------
+# The largest shape the header admits
+# ---------------------------------------------------------------------------
+
+def test_largest_shape_runs(prox):
+    """d_model 16384, d_ff 32768 (the header's limits; Stage 1 then runs its
+    two-batch ring): the step runs with a clean error word, selects k channels
+    and equals Stage 2 on its own mask bit for bit.  No oracle at this size:
+    the properties hold at any size."""
+    d, f = 16384, 32768
+    k = (f * 30 + 50) // 100
+    g = torch.Generator(device="cuda")
+    g.manual_seed(123)
+    w = [(torch.randn(shape, generator=g, device="cuda") * 0.01).to(torch.bfloat16)
+         for shape in ((d, f), (d, f), (f, d))]
+    x = torch.randn(d, generator=g, device="cuda")
+    layer = prox.Layer(*w, tau=0.67, k=k, max_batch=1)
+    del w
+    torch.cuda.empty_cache()
+    taps = layer.debug_stage1(x)
+    idx = taps["idx_s"]
+    y = layer.forward(x)
+    y_m = layer.forward_with_mask(x, idx)
+    torch.cuda.synchronize()
+    sel = idx.cpu().numpy()
+    assert sel.size == k and np.all(np.diff(sel) > 0)
+    assert torch.isfinite(y).all()
+    assert torch.equal(y_m, y.reshape(-1))
+    assert layer.error_word() == 0
+    layer.close()
