@@ -71,12 +71,19 @@ def test_traffic_record_roundtrip(bench, tmp_path, monkeypatch):
     assert bench.profiled_traffic(wl) is None
 
 
-def test_kernel_source_hash_covers_every_source(bench, tmp_path, monkeypatch):
+def test_kernel_source_hash_covers_every_token_kernel_source(bench, tmp_path, monkeypatch):
+    # the traffic record is tied to the token kernel's sources: editing any of
+    # them changes the hash, editing another source does not
     src = tmp_path / "csrc"
     src.mkdir()
-    (src / "a.cu").write_text("int a;")
-    (src / "b.cuh").write_text("int b;")
+    for name in bench.TOKEN_KERNEL_SOURCES + ("batch.cu",):
+        (src / name).write_text("// " + name)
     monkeypatch.setattr(bench, "CSRC", str(src))
     h0 = bench.kernel_source_hash()
-    (src / "b.cuh").write_text("int b; // edited")
-    assert bench.kernel_source_hash() != h0
+    for name in bench.TOKEN_KERNEL_SOURCES:
+        (src / name).write_text("// edited " + name)
+        h1 = bench.kernel_source_hash()
+        assert h1 != h0
+        h0 = h1
+    (src / "batch.cu").write_text("// edited")
+    assert bench.kernel_source_hash() == h0
