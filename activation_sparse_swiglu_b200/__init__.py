@@ -346,8 +346,8 @@ class Layer:
         return rows.value, chans.value
 
     def debug_batch_masks(self, B: int, stream=None) -> torch.Tensor:
-        """uint8 [B, d_ff] per-token masks of the last forward_batch (CUDA)."""
-        m = torch.empty((B, self.d_ff), dtype=torch.uint8, device="cuda")
+        """int32 [B, d_ff] per-token masks of the last forward_batch (CUDA)."""
+        m = torch.empty((B, self.d_ff), dtype=torch.int32, device="cuda")
         check(lib.prox_debug_batch_masks(self.handle, _ptr(m), B, _stream(stream)))
         return m
 

@@ -112,7 +112,7 @@ __device__ __forceinline__ void split_bf16(float v, __nv_bfloat16* hi, __nv_bflo
 // (token, row) pairs and the tokens to the layer's statistics.
 __global__ void __launch_bounds__(256) batch_prepare_count_kernel(const float* __restrict__ X, int B, int d,
                                                                   float tau, BatchWs w,
-                                                                  unsigned long long* stats) {
+                                                                  unsigned long long* stats, int count_kept) {
   __shared__ int s_red[8];
   const int r = blockIdx.x * 256 + threadIdx.x;
   bool any = false;
@@ -139,7 +139,7 @@ __global__ void __launch_bounds__(256) batch_prepare_count_kernel(const float* _
     int kt = 0;
     for (int i = 0; i < 8; ++i) kt += s_red[i];
     if (stats) {
-      atomicAdd(stats, (unsigned long long)kt);
+      if (count_kept) atomicAdd(stats, (unsigned long long)kt);
       if (blockIdx.x == 0) atomicAdd(stats + 1, (unsigned long long)B);
     }
   }
@@ -219,6 +219,13 @@ struct S1Smem {
   int ntiles;
 };
 
+// The half slice's output held at stored position m of the decoded tile
+// (each word's outputs are stored 0 4 1 5 2 6 3 7).
+__device__ __forceinline__ int s1_output(int m) {
+  const int j = m & 7;
+  return (m & ~7) | (j >> 1) | ((j & 1) << 2);
+}
+
 // Grid (2 C, S1 splits): CTA (hs, s) takes the outputs of half slice hs and
 // the quantisation groups [G s / S1, G (s + 1) / S1); writes
 // part1[s][token][gate|up][channel] (the group-scaled sums of its groups).
@@ -281,7 +288,7 @@ __global__ void __launch_bounds__(S1_THREADS, 2) batch_stage1_kernel(const uint8
     for (int i = 0; i < 2; ++i)
 #pragma unroll
       for (int r = 0; r < 2; ++r) {
-        const int m = warp * 32 + i * 16 + g + 8 * r;
+        const int m = s1_output(warp * 32 + i * 16 + g + 8 * r);
         const int blk = (slice * 512 + half * 256) / 32 + (m >> 6);  // < F / 32 for real channels
         sc[i][r] = blk < F / 32 ? __half2float(__ldg(ps + ((size_t)grp * (F / 32) + blk) * 64 + (m & 63))) : 0.f;
       }
@@ -312,7 +319,10 @@ __global__ void __launch_bounds__(S1_THREADS, 2) batch_stage1_kernel(const uint8
     sm.blo[tid >> 5][tid & 31] = xl;
     fetch_x(t + 1, xh, xl);
     // decode: 32 rows x 64 words, 4 words per thread; word wd of row k holds
-    // outputs 8 wd .. 8 wd + 7 (nibble p is output 8 wd + p); the code is q + 8
+    // outputs 8 wd .. 8 wd + 7 (nibble p is output 8 wd + p; the code is
+    // q + 8).  Nibbles p and p + 4 sit 16 bits apart, so one mask-and-or puts
+    // both into a bf16 pair 128 + code; the stored order of the word's
+    // outputs is therefore 0 4 1 5 2 6 3 7 (s1_output maps it back).
     for (int j = tid; j < S1_KT * 64; j += S1_THREADS) {
       const int k = j >> 6, wd = j & 63;
       if (k < len) {
@@ -320,8 +330,7 @@ __global__ void __launch_bounds__(S1_THREADS, 2) batch_stage1_kernel(const uint8
         uint32_t o[4];
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
-          const uint32_t b = v >> (8 * p);  // nibbles 2p (low) and 2p + 1
-          const uint32_t pair = (b & 0xFu) | ((b & 0xF0u) << 12) | 0x43004300u;  // bf16 128 + code
+          const uint32_t pair = ((v >> (4 * p)) & 0x000F000Fu) | 0x43004300u;  // bf16 128 + code
           __nv_bfloat162 q = *reinterpret_cast<const __nv_bfloat162*>(&pair);
           q = __hsub2(q, __floats2bfloat162_rn(136.f, 136.f));  // exact: q in [-8, 7]
           o[p] = *reinterpret_cast<const uint32_t*>(&q);
@@ -368,7 +377,7 @@ __global__ void __launch_bounds__(S1_THREADS, 2) batch_stage1_kernel(const uint8
   for (int i = 0; i < 2; ++i)
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
-      const int m = warp * 32 + i * 16 + g + 8 * r;
+      const int m = s1_output(warp * 32 + i * 16 + g + 8 * r);
       const int kind = (m & 63) >> 5;
       const int ch = slice * 512 + half * 256 + (m >> 6) * 32 + (m & 31);
       if (ch < F)
@@ -803,7 +812,7 @@ size_t batch_ws_bytes(int d, int F, int s1, int s5, int ks) {
   const size_t Fp = (size_t)((F + 63) & ~63), G = (size_t)d / kGroup;
   return 4 * al256((size_t)NB * d * 2) + al256((size_t)d * 4) + 2 * al256(G * 4) + al256(16) +
          al256((size_t)(d + 255) / 256 * 4) + al256((size_t)(F + 255) / 256 * 4) +
-         al256((size_t)s1 * NB * 2 * F * 4) + al256((size_t)NB * F * 4) + al256((size_t)NB * F) +
+         al256((size_t)s1 * NB * 2 * F * 4) + al256((size_t)NB * F * 4) + al256((size_t)NB * F * 4) +
          2 * al256((size_t)F * 4) + al256(Fp / GU_M * ks * GU_M * NB * 2 * 4) +
          2 * al256((size_t)NB * Fp * 2) + al256((size_t)s5 * NB * d * 4);
 }
@@ -828,7 +837,7 @@ void carve_batch_ws(void* base, int d, int F, int s1, int s5, int ks, BatchWs* w
   w->ccount = reinterpret_cast<int*>(take((size_t)(F + 255) / 256 * 4));
   w->part1 = reinterpret_cast<float*>(take((size_t)s1 * NB * 2 * F * 4));
   w->scores = reinterpret_cast<float*>(take((size_t)NB * F * 4));
-  w->smask = reinterpret_cast<uint8_t*>(take((size_t)NB * F));
+  w->smask = reinterpret_cast<int32_t*>(take((size_t)NB * F * 4));
   w->ulist = reinterpret_cast<int*>(take((size_t)F * 4));
   w->utok = reinterpret_cast<uint32_t*>(take((size_t)F * 4));
   w->gup = reinterpret_cast<float*>(take(Fp / GU_M * ks * GU_M * NB * 2 * 4));  // Fp / 16 tiles
@@ -859,9 +868,29 @@ cudaError_t launch_batch(const prox_layer* L, const float* X, float* Y, int B, b
   const __nv_bfloat16* wgu = reinterpret_cast<const __nv_bfloat16*>(L->wgu);
   const __nv_bfloat16* wd = reinterpret_cast<const __nv_bfloat16*>(L->wd);
   const int rb = (d + 255) / 256, cb = (F + 255) / 256;
-  batch_prepare_count_kernel<<<rb, 256, 0, s>>>(X, B, d, L->tau, w, dense ? nullptr : L->ws.stats);
+  const bool per_token = !dense && B <= kBatchPerTokenStage1;
+  // (per token, Stage 1 itself counts the kept rows)
+  batch_prepare_count_kernel<<<rb, 256, 0, s>>>(X, B, d, L->tau, w, dense ? nullptr : L->ws.stats,
+                                                per_token ? 0 : 1);
   batch_prepare_place_kernel<<<rb, 256, 0, s>>>(X, B, d, L->tau, w);
-  if (!dense) {
+  if (per_token) {
+    // each token's Stage 1, scores and mask from the per-token kernel, which
+    // reads only that token's kept rows; then the union of the masks
+    for (int b = 0; b < B; ++b) {
+      TokenLaunch m;
+      m.x = X + (size_t)b * d;
+      m.stage1 = true;
+      m.mode = L->mask_mode == PROX_MASK_THRESHOLD ? 3 : 1;
+      m.k = L->k;
+      m.tau_s = L->tau_s;
+      m.select_only = true;
+      m.sel_mask = w.smask + (size_t)b * F;
+      cudaError_t e = launch_token(L, m, s, false);
+      if (e != cudaSuccess) return e;
+    }
+    batch_union_count_kernel<<<cb, 256, 0, s>>>(w, F, B, L->ws.stats);
+    batch_union_place_kernel<<<cb, 256, 0, s>>>(w, F, B);
+  } else if (!dense) {
     batch_stage1_kernel<<<dim3(2 * ((F + 511) / 512), L->b_s1), S1_THREADS, sizeof(S1Smem), s>>>(
         L->pq, reinterpret_cast<const __half*>(L->ps), d, F, w);
     const bool thr = L->mask_mode == PROX_MASK_THRESHOLD;

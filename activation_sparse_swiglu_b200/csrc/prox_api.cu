@@ -683,12 +683,12 @@ prox_status prox_batch_union_sizes(const prox_layer* L, int32_t* rows_host, int3
   return PROX_OK;
 }
 
-prox_status prox_debug_batch_masks(const prox_layer* L, uint8_t* masks, int B, void* stream) {
+prox_status prox_debug_batch_masks(const prox_layer* L, int32_t* masks, int B, void* stream) {
   prox_status st = check_layer(L);
   if (st != PROX_OK) return st;
   if (!L->bws_base) return fail(PROX_EINVAL, "the layer has no batched step (max_batch == 1)");
   if (!masks || B < 1 || B > prox::kBatchMax) return fail(PROX_EINVAL, "masks NULL or B out of [1, 16]");
-  PROX_CUDA(cudaMemcpyAsync(masks, L->bws.smask, (size_t)B * L->F, cudaMemcpyDeviceToDevice,
+  PROX_CUDA(cudaMemcpyAsync(masks, L->bws.smask, (size_t)B * L->F * 4, cudaMemcpyDeviceToDevice,
                             as_stream(stream)),
             "copy batch masks");
   return PROX_OK;

@@ -76,7 +76,7 @@ struct BatchWs {
   int* ccount = nullptr;           // [d_ff / 256] union channels per block of 256
   float* part1 = nullptr;          // [S1][16][2][F] Stage-1 sums per row split
   float* scores = nullptr;         // [16][F]
-  uint8_t* smask = nullptr;        // [16][F] per-token channel masks
+  int32_t* smask = nullptr;        // [16][F] per-token channel masks (1 = selected)
   int* ulist = nullptr;            // [F] the union channels, ascending
   uint32_t* utok = nullptr;        // [F] the tokens that selected each
   float* gup = nullptr;            // [Fp / 64 * KS][64][16][2] gate / up sums per work item
@@ -152,6 +152,9 @@ size_t batch_ws_bytes(int d, int F, int s1, int s5, int ks);
 void carve_batch_ws(void* base, int d, int F, int s1, int s5, int ks, BatchWs* w);
 cudaError_t launch_batch(const prox_layer* L, const float* X, float* Y, int B, bool dense,
                          cudaStream_t s);
+// Batches up to this size take each token's Stage 1 and mask from the
+// per-token kernel (select only) instead of the union Stage 1.
+constexpr int kBatchPerTokenStage1 = PROX_BATCH_PER_TOKEN_STAGE1;
 cudaError_t launch_barrier_probe(const prox_layer* L, cudaStream_t s);
 cudaError_t launch_token(const prox_layer* L, const TokenLaunch& m, cudaStream_t s, bool pdl);
 

@@ -56,6 +56,7 @@ import numpy as np  # noqa: E402
 METRIC = "batch-1 sparse-FFN tokens/s"
 UNIT = "tokens/s"
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "token_traffic.json")
+PER_TOKEN_STAGE1 = 4  # include/prox.h PROX_BATCH_PER_TOKEN_STAGE1
 CSRC = os.path.join(ROOT, "activation_sparse_swiglu_b200", "csrc")
 SPEC_HBM_GBS = 8000.0  # B200 HBM3e spec bandwidth (DGX figure), for the spec fraction
 ALL_LEGS = ("dense", "sweep", "threshold", "variants", "operating_points", "alpha", "e2e",
@@ -918,6 +919,9 @@ class Bench:
                 n_rows.append(r_)
                 n_ch.append(c_)
             mean_rows, mean_ch = float(np.mean(n_rows)), float(np.mean(n_ch))
+            if B <= PER_TOKEN_STAGE1:  # each token reads its own kept rows
+                xk = np.abs(lay.x_eval[:nb * B]) >= np.float32(tau)
+                mean_rows = float(xk.sum()) / nb
             union_bytes = mean_rows * C * 512 + mean_ch * 6 * d + 8 * B * d
             dense_bytes = 6.0 * d * f + 8 * B * d
             tok_c, _ = self.timer.tokens_per_s(chain, nb * B, steps)
@@ -930,7 +934,7 @@ class Bench:
                 "dense_tokens_per_s": round(tok_d, 1),
                 "speedup_vs_dense": round(tok_u / tok_d, 3),
                 "chain_speedup_vs_dense": round(tok_c / tok_d, 3),
-                "union_rows_frac": round(mean_rows / d, 4),
+                "stage1_rows_frac": round(mean_rows / d, 4),
                 "union_channels_frac": round(mean_ch / f, 4),
                 "union_bytes_per_batch": int(union_bytes),
                 "union_hbm_gbs": round(union_bytes * tok_u / B / 1e9, 1),
@@ -941,7 +945,8 @@ class Bench:
         self.result["llama3_70b"] = {
             "workload": f"llama3_70b ffn layer d_model={d} d_ff={f} s1=50% s2=70% k={k}, "
                         "per-token masks",
-            "paths": "union = prox_ffn_forward_batch (one batched step, union loads); chain = "
+            "paths": "union = prox_ffn_forward_batch (one batched step, union loads of the "
+                     "bf16 weights; Stage 1 per token for B <= 4, over the union rows above); chain = "
                      "prox_ffn_forward (B batch-1 launches); dense = prox_dense_ffn_batch (every "
                      "weight read once); bytes: union rows x proxy row + union channels x 6 d "
                      "(gate/up record + W_down row) + x/out; dense 6 d d_ff + x/out",

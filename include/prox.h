@@ -284,6 +284,10 @@ PROX_API prox_status prox_ffn_forward(const prox_layer* layer, const float* x, f
 PROX_API prox_status prox_dense_ffn(const prox_layer* layer, const float* x, float* out, int B,
                            void* stream);
 
+/* The largest batch whose tokens take their Stage 1 from the batch-1 kernel
+ * in prox_ffn_forward_batch (see there). */
+#define PROX_BATCH_PER_TOKEN_STAGE1 4
+
 /* The same step for B tokens at once, reading every weight byte the batch
  * needs once (the pages' kernels are batch 1 only, Prox §5.3 "Discussion";
  * the masks are still per token, Prox §4.1 and App. A.6):
@@ -292,6 +296,10 @@ PROX_API prox_status prox_dense_ffn(const prox_layer* layer, const float* x, flo
  *   takes its own top-k (or threshold) channel mask; the union of the
  *   selected channels' gate/up records and W_down rows is read once, each
  *   token contributing only through the channels it selected.
+ * Batches of at most PROX_BATCH_PER_TOKEN_STAGE1 tokens take each token's
+ * Stage 1 and mask from the batch-1 kernel instead (reading each token's own
+ * kept rows: fewer bytes and less decoding than the union at small B; their
+ * masks are then exactly the batch-1 masks).
  * The products run on the tensor cores (bf16 operands, fp32 accumulation,
  * x and the intermediate values split into two bf16 parts so that they carry
  * 16 significant bits); the sums are taken in another order than
@@ -378,10 +386,10 @@ PROX_API prox_status prox_forward_with_mask(prox_layer* layer, const float* x, c
                                    int k, float* out, float* s_sp, void* stream);
 
 /* Test-only: the per-token channel masks of the layer's last
- * prox_ffn_forward_batch, uint8 [B][d_ff] (1 = selected) into the device
+ * prox_ffn_forward_batch, int32 [B][d_ff] (1 = selected) into the device
  * buffer masks (caller-owned).  Stream-ordered; PROX_EINVAL on a layer
  * without the batched step, NULL masks or B outside [1, 16]. */
-PROX_API prox_status prox_debug_batch_masks(const prox_layer* layer, uint8_t* masks, int B, void* stream);
+PROX_API prox_status prox_debug_batch_masks(const prox_layer* layer, int32_t* masks, int B, void* stream);
 
 /* Test-only fault injection on the host: the nth device allocation that
  * prox_layer_create makes from now on (1 = the next one; a create makes nine:
