@@ -412,27 +412,38 @@ __device__ void run(const TokenArgs& a, unsigned char* smem, unsigned long long 
   const int nsl = span > first ? 2 : 1;  // slices the CTA's pair range touches
   const uint32_t tag = launch_tag(counter);  // (the counter was loaded at the kernel's start)
   // Element e = j*32 + 2*blk + h of the sums is the gate (h = 0) or up
-  // (h = 1) sum of channel m = blk*32 + j of the slice; it is stored at
-  // 2m + h, so the scoring threads (one per channel, consecutive channels)
-  // read consecutive 16-byte pairs, and each warp's stores cover whole
-  // sectors.
-  for (int pos = tid; pos < PART; pos += blockDim.x) {
-    const int m = pos >> 1;
-    const int ep = (m & 31) * 33 + 2 * (m >> 5) + (pos & 1);  // e in the padded layout
-    float p0 = 0.f, p1 = 0.f;
+  // (h = 1) sum of channel m = blk*32 + j of the slice; channel m's pair is
+  // stored at 2m, 2m + 1, so the scoring threads (one per channel,
+  // consecutive channels) read consecutive 16-byte pairs.  One thread per
+  // channel, one 16-byte store per touched slice: each warp's stores cover
+  // whole sectors.
+  for (int m = tid; m < PART / 2; m += blockDim.x) {
+    const int ep = (m & 31) * 33 + 2 * (m >> 5);  // the gate sum in the padded layout; up at + 1
+    float g0 = 0.f, u0 = 0.f, g1 = 0.f, u1 = 0.f;
 #pragma unroll
     for (int w = 0; w < NW; ++w) {
       const int kind = s_src[w];
-      const float v = s_tot[w * PARTP + ep];
-      if (kind == 1) p0 += v;
-      if (kind == 2) p1 += v;
+      const float vg = s_tot[w * PARTP + ep], vu = s_tot[w * PARTP + ep + 1];
+      if (kind == 1) {
+        g0 += vg;
+        u0 += vu;
+      }
+      if (kind == 2) {
+        g1 += vg;
+        u1 += vu;
+      }
       if (kind == 3) {
-        p0 += s_stash[ep];
-        p1 += v;
+        g0 += s_stash[ep];
+        u0 += s_stash[ep + 1];
+        g1 += vg;
+        u1 += vu;
       }
     }
-    st_tag(a.part + ((size_t)cta * 2) * PART + pos, tag_word(__float_as_uint(p0), tag));
-    if (nsl == 2) st_tag(a.part + ((size_t)cta * 2 + 1) * PART + pos, tag_word(__float_as_uint(p1), tag));
+    st_tag2(a.part + ((size_t)cta * 2) * PART + 2 * m, tag_word(__float_as_uint(g0), tag),
+            tag_word(__float_as_uint(u0), tag));
+    if (nsl == 2)
+      st_tag2(a.part + ((size_t)cta * 2 + 1) * PART + 2 * m, tag_word(__float_as_uint(g1), tag),
+              tag_word(__float_as_uint(u1), tag));
   }
 }
 
