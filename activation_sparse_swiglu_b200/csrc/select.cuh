@@ -36,6 +36,7 @@ constexpr int kOwnMax = 512;         // channels a CTA scores, at most
 // Shared scratch of the selection.
 struct alignas(16) SelectScratch {
   uint32_t own[kOwnMax];           // the keys of the CTA's own channels
+  float sg[kOwnMax], su[kOwnMax];  // their g~ and u~ while scoring
   uint32_t coarse[kCoarseBins];    // the CTA's coarse counts while scoring
   uint32_t ck[kBucketCap];         // candidate keys
   int32_t ci[kBucketCap];          // candidate channels

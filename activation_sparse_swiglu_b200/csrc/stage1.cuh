@@ -99,11 +99,13 @@ __device__ __forceinline__ int cta_of(int t, int T, int P) {
   return (int)(((unsigned)(t + 1) * (unsigned)P + (unsigned)T - 1u) / (unsigned)T) - 1;
 }
 
-// Scores the channels [F c / P, F (c + 1) / P) of CTA c (at most kOwnMax,
-// so one per thread): thread t adds the gate and up partials of channel
-// c0 + t over the CTAs whose pair ranges cover its slice, in CTA order,
-// polling each tagged partial until this launch's has arrived.  It writes the
-// score, keeps its key (the score's bits) in shared memory and publishes the
+// Scores the channels [F c / P, F (c + 1) / P) of CTA c (at most kOwnMax):
+// a group of threads per channel adds its gate and up partials over the CTAs
+// whose pair ranges cover its slice (the group's threads take interleaved CTA
+// subsets, then a fixed shuffle tree: deterministic), polling each tagged
+// partial until this launch's has arrived.  Thread t then takes channel
+// c0 + t: it writes the score, keeps its key (the score's bits) in shared
+// memory and publishes the
 // signed act(g~) u~ as a tagged word.  For the top-k rule the CTA first counts
 // its keys in shared-memory histograms; one thread per non-empty fine bin then
 // adds the CTA's count to the global bin, whose old value places the CTA's
@@ -122,48 +124,72 @@ __device__ void score_channels(const TokenArgs& a, bool histogram, SelectScratch
     for (int i = tid; i < kScoreBins; i += blockDim.x) fine[i] = 0u;
     __syncthreads();
   }
+  {
+    // g~ and u~ of the CTA's channels: tpc threads per channel (a power of two
+    // <= 32, as many as the CTA has threads for), thread `part` of a channel
+    // adding the partials of the CTAs i_lo + part, i_lo + part + tpc, ... in
+    // order, then the group's sums by a fixed shuffle tree (deterministic).
+    // Each tagged partial is polled until it carries this launch's tag.
+    const int nch = c1 - c0;
+    int tpc = 32;
+    while (tpc > 1 && tpc * nch > (int)blockDim.x) tpc >>= 1;
+    const int cl = tid / tpc, part = tid % tpc;
+    float g = 0.f, u = 0.f;
+    if (cl < nch) {
+      const int chl = c0 + cl;
+      const int c = chl / SLICE, m = chl % SLICE;
+      const int e = 2 * m;  // channel m's gate and up sums in a CTA's partial row
+      const int i_lo = cta_of(c * a.d, T, P);
+      const int i_hi = cta_of((c + 1) * a.d - 1, T, P);
+      for (int i0 = i_lo + part; i0 <= i_hi; i0 += 8 * tpc) {
+        ulonglong2 v[8];
+        int off[8];  // element offset of CTA i0 + q tpc's partial pair, or -1
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const int i = i0 + q * tpc;
+          off[q] = -1;
+          v[q] = make_ulonglong2(tag_word(0u, tag), tag_word(0u, tag));
+          if (i <= i_hi) {
+            const unsigned tlo = (unsigned)T * (unsigned)i / (unsigned)P;
+            const unsigned thi = (unsigned)T * (unsigned)(i + 1) / (unsigned)P;
+            if (thi > tlo) {  // CTA i holds pairs; slice c is its first or second
+              off[q] = (i * 2 + (c - (int)(tlo / (unsigned)a.d))) * PART + e;
+              v[q] = ld_tag2(a.part + off[q]);
+            }
+          }
+        }
+        const long long t0 = clock64();
+        for (;;) {
+          bool all = true;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) all = all && tag_ok(v[q].x, tag) && tag_ok(v[q].y, tag);
+          if (all || !wait_more(t0, a.err)) break;
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            if (off[q] >= 0 && !(tag_ok(v[q].x, tag) && tag_ok(v[q].y, tag))) v[q] = ld_tag2(a.part + off[q]);
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          g += __uint_as_float((uint32_t)v[q].x);
+          u += __uint_as_float((uint32_t)v[q].y);
+        }
+      }
+    }
+    for (int o = tpc >> 1; o > 0; o >>= 1) {
+      g += __shfl_xor_sync(0xffffffffu, g, o);
+      u += __shfl_xor_sync(0xffffffffu, u, o);
+    }
+    if (cl < nch && part == 0) {
+      sel.sg[cl] = g;
+      sel.su[cl] = u;
+    }
+    __syncthreads();
+  }
   const int ch = c0 + tid;
   const bool mine = ch < c1;
   uint32_t key = 0u, fb = 0u, rank = 0u;
   if (mine) {
-    const int c = ch / SLICE, m = ch % SLICE;
-    const int e = 2 * m;  // channel m's gate and up sums in a CTA's partial row
-    const int i_lo = cta_of(c * a.d, T, P);
-    const int i_hi = cta_of((c + 1) * a.d - 1, T, P);
-    float g = 0.f, u = 0.f;
-    for (int i0 = i_lo; i0 <= i_hi; i0 += 8) {
-      ulonglong2 v[8];
-      int off[8];  // element offset of CTA i0 + q's partial pair, or -1
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const int i = i0 + q;
-        off[q] = -1;
-        v[q] = make_ulonglong2(tag_word(0u, tag), tag_word(0u, tag));
-        if (i <= i_hi) {
-          const unsigned tlo = (unsigned)T * (unsigned)i / (unsigned)P;
-          const unsigned thi = (unsigned)T * (unsigned)(i + 1) / (unsigned)P;
-          if (thi > tlo) {  // CTA i holds pairs; slice c is its first or second
-            off[q] = (i * 2 + (c - (int)(tlo / (unsigned)a.d))) * PART + e;
-            v[q] = ld_tag2(a.part + off[q]);
-          }
-        }
-      }
-      const long long t0 = clock64();
-      for (;;) {
-        bool all = true;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) all = all && tag_ok(v[q].x, tag) && tag_ok(v[q].y, tag);
-        if (all || !wait_more(t0, a.err)) break;
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-          if (off[q] >= 0 && !(tag_ok(v[q].x, tag) && tag_ok(v[q].y, tag))) v[q] = ld_tag2(a.part + off[q]);
-      }
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        g += __uint_as_float((uint32_t)v[q].x);
-        u += __uint_as_float((uint32_t)v[q].y);
-      }
-    }
+    const float g = sel.sg[tid], u = sel.su[tid];
     stamp(a.ts, 3);
     const float sv = act_f32(g, a.act) * u;
     const float sc = fabsf(sv);
