@@ -383,10 +383,16 @@ prox_status prox_layer_create(const uint16_t* W_gate, const uint16_t* W_up, cons
     return fail(PROX_EUNSUPPORTED, "d_ff=%d over %d SMs exceeds 512 channels per CTA", d_ff, sms);
   }
   L->P = sms;
-  prox::choose_stage1_grid(L->d, L->F, sms, &L->C, &L->s1_lmax, &L->s1_nb);
+  prox::choose_stage1_grid(L->d, L->F, sms, &L->C, &L->s1_lmax, &L->s1_depth);
+  if (L->s1_depth < 2) {
+    delete L;
+    return fail(PROX_EUNSUPPORTED,
+                "d_model=%d, d_ff=%d over %d SMs: Stage 1's row tables leave no room for two k-tiles per warp",
+                d_model, d_ff, sms);
+  }
   size_t s2_smem = 0;
   prox::choose_stage2(L->d, L->F, sms, &L->ring_slots, &L->stage2_groups, &s2_smem);
-  const size_t s1_smem = prox::stage1_smem_bytes(L->s1_lmax, L->s1_nb);
+  const size_t s1_smem = prox::stage1_smem_bytes(L->s1_lmax, L->s1_depth, L->d);
   L->token_smem = s1_smem > s2_smem ? s1_smem : s2_smem;
   if (L->token_smem > (size_t)prox::kMaxSmemPerBlock) {
     const size_t need = L->token_smem;

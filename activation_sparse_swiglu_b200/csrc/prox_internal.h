@@ -98,9 +98,9 @@ struct prox_layer {
   // Per-token kernel: P CTAs (one per SM), token_smem bytes of shared memory.
   int P = 0;
   size_t token_smem = 0;
-  // Stage-1 geometry: C column slices, at most s1_lmax rows per CTA, s1_nb
-  // row batches in flight per warp
-  int C = 0, s1_lmax = 0, s1_nb = 4;
+  // Stage-1 geometry: C column slices, at most s1_lmax rows per CTA, s1_depth
+  // k-tiles in flight per Stage-1 warp
+  int C = 0, s1_lmax = 0, s1_depth = 0;
   // Stage-2 geometry
   int ring_slots = 0, stage2_groups = 1;
   // library-owned weights
@@ -182,8 +182,8 @@ cudaError_t launch_mask_to_list(const int32_t* mask, int n, int32_t* list, int32
 
 // Stage-1 column slices, per-CTA row capacity and ring depth for a shape on
 // `num_sms` SMs (one CTA each).
-void choose_stage1_grid(int d, int F, int num_sms, int* C, int* lmax, int* nb);
-size_t stage1_smem_bytes(int lmax, int nb);
+void choose_stage1_grid(int d, int F, int num_sms, int* C, int* lmax, int* depth);
+size_t stage1_smem_bytes(int lmax, int depth, int d);
 size_t stage1_part_floats(int P);
 // Stage-2 ring depth, consumer groups and shared memory for d_model = d.
 void choose_stage2(int d, int F, int num_sms, int* slots, int* groups, size_t* smem);

@@ -8,28 +8,42 @@
 // proxies; the proxy is stored slice-major, so a slice's kept rows are read in
 // ascending address order.  The C * d_model (slice, row) pairs, slice-major,
 // are split into equal contiguous ranges, one per CTA (a static split: a CTA's
-// range lies in at most two adjacent slices); each CTA thresholds the rows of
-// its range (|x_i| >= tau), compacts its kept pairs in order and splits them
-// into equal contiguous ranges, one per warp, so every warp streams the same
-// number of 512-byte row slices whatever the mask looks like.
+// range lies in at most two adjacent slices).  Each CTA thresholds the rows of
+// its range (|x_i| >= tau) and compacts its kept rows in order, grouped into
+// segments of one slice and one quantisation group, each segment padded to a
+// multiple of 8 rows (a k-tile).
 //
-// A warp streams its rows through a shared-memory ring with asynchronous
-// 16-byte copies (cp.async, L2 only; each lane copies and later reads back its
-// own chunk, so no barrier is needed), NB batches of four rows in flight, and
-// dequantises the INT4 codes in registers with fp32 (packed f32x2)
-// arithmetic, accumulating per quantisation group and scaling once per group
-// by the fp16 group scale.  A batch whose rows share one slice and one group
-// takes a path without any boundary checks.
+// The product runs on the integer tensor pipe, exactly.  Each kept x_i is
+// written as a fixed-point integer V_i = x_i 2^(29 - E) (E the exponent of
+// the CTA's largest kept |x|, so |V_i| < 2^30; exact for every x_i within a
+// factor 128 of that maximum, rounded to an integer below it) and V_i as four
+// signed 8-bit digits, V_i = sum_p v_ip 256^(3 - p).  A code c = q + 8 of the
+// offset-binary INT4 format becomes the signed byte 16 q with one LOP3 (the
+// nibble moved to the byte's top bits and its top bit flipped).  One
+// mma.sync m16n8k32 (s8 x s8 -> s32) then takes 8 kept rows x 8 code words
+// of one nibble parity: B holds the rows' bytes (k = 4 t + j is row t,
+// nibble pair j of the word), A the digits laid out so that output row
+// m = j + 4 p sees only the k with that j, times digit p.  The 32-bit integer
+// sums are exact; per segment they are combined over the digits, converted
+// to fp32, scaled by the fp16 group scale and added up in segment order.
+// Rows padded onto a segment have zero digits and contribute exactly zero.
 //
-// The warps' partial sums are combined in warp order into one partial vector
-// per touched slice and written to global memory (run).  After a grid
-// barrier, every CTA takes an even share of the channels and, for each, adds
-// the partials of the CTAs that hold its slice in CTA order (deterministic),
-// scores it, score_j = |act(g~_j) u~_j| (act the layer's gate activation:
-// SiLU, or GELU for a GeGLU FFN; the signed value is kept too when Stage 2
-// runs the A3 ablation), keeps its key in shared memory for the selection
-// and, for the top-k rule, counts it in the histograms and buckets of
-// select.cuh (score_channels).
+// The 16 warps form 4 groups; group q takes a quarter of the CTA's k-tiles
+// and warp v of a group the blocks 4v .. 4v+3 (128 bytes) of each of their
+// rows, streamed with 16-byte cp.async copies into the warp's own ring of
+// k-tile slots (no synchronisation between warps; the chunks of a row are
+// placed XOR-swizzled so the tensor-pipe operand reads are conflict-free),
+// together with the fp16 scales of each new segment.  Each warp's sums per
+// slice are combined over the 4 groups in shared memory, in group order, and
+// written channel-major as tagged words.
+
+// After the partials are written, every CTA takes an even share of the
+// channels and, for each, adds the partials of the CTAs that hold its slice
+// in CTA order (deterministic), scores it, score_j = |act(g~_j) u~_j| (act
+// the layer's gate activation: SiLU, or GELU for a GeGLU FFN; the signed
+// value is kept too when Stage 2 runs the A3 ablation), keeps its key in
+// shared memory for the selection and, for the top-k rule, counts it in the
+// histograms and buckets of select.cuh (score_channels).
 #pragma once
 #include "select.cuh"
 #include "token_args.cuh"
@@ -37,60 +51,45 @@
 namespace prox {
 namespace s1 {
 
-constexpr int NW = kStage1Warps;   // warps that stream rows
-constexpr int NT = NW * 32;
-static_assert(kMaxDModel % NT == 0, "rows per thread");
-constexpr int SLICE = 512;   // bytes (= channels of both proxies) per column slice
-constexpr int PART = 1024;   // partial values per slice: 32 chunks x 32 channels
-constexpr int PARTP = 32 * 33;  // the same in shared memory, rows of 32 padded to 33
-constexpr int U = 4;         // rows per batch
-constexpr int BATCH = U * SLICE;
+constexpr int NW = kStage1Warps;  // consumer warps: one 32-channel block each
+static_assert(NW == 16, "a 512-byte slice is 16 blocks of 32 channels");
+static_assert(kTokenThreads >= (NW + 1) * 32, "the producer warp");
+constexpr int SLICE = 512;        // bytes (= channels of both proxies) per column slice
+constexpr int PART = 1024;        // partial values per slice: (gate, up) per channel
+constexpr int KT = 8;             // rows per k-tile
+constexpr int NGRP = 4;           // warp groups: group q takes a quarter of the CTA's k-tiles
+constexpr int WPG = NW / NGRP;    // warps per group: warp v of a group takes blocks BPW v ...
+constexpr int BPW = 16 / WPG;     // blocks per warp
+constexpr int WROW = BPW * 32;    // bytes of a row slice one warp streams
+constexpr int WSLOT = KT * WROW + BPW * 128;  // a warp's ring slot: 8 rows, then 4 blocks' scales
+constexpr int kMaxDepth = 8;      // k-tiles in flight per warp, at most
+static_assert(WSLOT % 128 == 0, "slots keep 128-byte alignment");
 static_assert(kOwnMax <= kTokenThreads, "scoring takes one channel per thread");
 
-// (w & M) | e in one instruction; e is a register (the exponents come from
-// kernel parameters, so they are not folded into a second immediate).
-template <uint32_t M>
-__device__ __forceinline__ float andor(uint32_t w, uint32_t e) {
+// D += A B on the integer tensor pipe (m16n8k32, s8 x s8 -> s32).
+__device__ __forceinline__ void mma_s8(int* d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                       uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// The high nibbles of a code word (bytes' bits 4..7, codes c = q + 8) as
+// signed bytes 16 q: keep the top nibble of each byte and flip its top bit.
+__device__ __forceinline__ uint32_t codes_hi_s8(uint32_t w) {
   uint32_t r;
-  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(w), "n"(M), "r"(e));
-  return __uint_as_float(r);
+  asm("lop3.b32 %0, %1, 0xF0F0F0F0, 0x80808080, 0x6A;" : "=r"(r) : "r"(w));  // (w & b) ^ c
+  return r;
+}
+// The low nibbles the same way, after moving them up by 4 bits.
+__device__ __forceinline__ uint32_t codes_lo_s8(uint32_t w) { return codes_hi_s8(w << 4); }
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, 0, %2;" : "=r"(r) : "r"(a), "r"(sel));
+  return r;
 }
 
-// Eight INT4 codes of one 32-bit word (nibble p is channel 8w+p of the lane's
-// chunk, stored as q+8) into four float2 accumulators.  Each nibble is OR-ed
-// into the mantissa of a float whose exponent makes the nibble's lowest bit
-// worth exactly 1, so subtracting (2^e + 8) leaves q exactly; nibbles 5..7
-// are first shifted down by 12 bits.  This is the exponent-field construction
-// of an integer as a float (the "magic number" conversion, e.g. Hacker's
-// Delight, 2nd ed., §17-2, applied per nibble), with the offset of the
-// codes folded into the subtracted constant.
-__device__ __forceinline__ void acc_word(float2* a, uint32_t w, float2 x2, const Magic& mg) {
-  const uint32_t h = w >> 12;
-  const float2 v0 = __fadd2_rn(make_float2(andor<0x0000000Fu>(w, mg.e23), andor<0x000000F0u>(w, mg.e19)),
-                               make_float2(-8388616.0f, -524296.0f));
-  const float2 v1 = __fadd2_rn(make_float2(andor<0x00000F00u>(w, mg.e15), andor<0x0000F000u>(w, mg.e11)),
-                               make_float2(-32776.0f, -2056.0f));
-  const float2 v2 = __fadd2_rn(make_float2(andor<0x000F0000u>(w, mg.e7), andor<0x00000F00u>(h, mg.e15)),
-                               make_float2(-136.0f, -32776.0f));
-  const float2 v3 = __fadd2_rn(make_float2(andor<0x0000F000u>(h, mg.e11), andor<0x000F0000u>(h, mg.e7)),
-                               make_float2(-2056.0f, -136.0f));
-  a[0] = __ffma2_rn(v0, x2, a[0]);
-  a[1] = __ffma2_rn(v1, x2, a[1]);
-  a[2] = __ffma2_rn(v2, x2, a[2]);
-  a[3] = __ffma2_rn(v3, x2, a[3]);
-}
-
-__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
 
 // CTA holding pair t of T pairs split over P CTAs (CTA i holds
 // [floor(T i / P), floor(T (i + 1) / P))); never an empty CTA.  T * P < 2^31
@@ -220,88 +219,218 @@ __device__ void score_channels(const TokenArgs& a, bool histogram, SelectScratch
   }
 }
 
-// Shared memory: per-warp rings of NB batches, per-warp group-scaled sums,
-// the CTA's kept rows, the stash of the warp that crosses a slice boundary.
-template <int NB>
-constexpr size_t smem_bytes(int lmax) {
-  return (size_t)NW * NB * BATCH + (size_t)NW * PARTP * 4 + (size_t)lmax * 12 +
-         (size_t)PARTP * 4 + (37 + kTokenThreads) * 4;
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+// Waits until at most n of this thread's copy groups are pending (n < kMaxDepth).
+__device__ __forceinline__ void cp_async_wait_n(int n) {
+  switch (n) {
+    case 7: cp_async_wait<7>(); break;
+    case 6: cp_async_wait<6>(); break;
+    case 5: cp_async_wait<5>(); break;
+    case 4: cp_async_wait<4>(); break;
+    case 3: cp_async_wait<3>(); break;
+    case 2: cp_async_wait<2>(); break;
+    case 1: cp_async_wait<1>(); break;
+    default: cp_async_wait<0>(); break;
+  }
+}
+static_assert(kMaxDepth <= 8, "cp_async_wait_n covers depths up to 8");
+
+// Shared memory of Stage 1 (byte offsets from the start of the dynamic
+// block): the warps' rings [NW][depth][WSLOT], the groups' sums per slice
+// [2][NGRP][512][2] (float), then per padded row its byte offset in the
+// proxy (-1 for padding) and its digit word (byte p = digit p; stored k-tile
+// interleaved so rows t and t + 4 of a k-tile are adjacent), the segment of
+// each k-tile, per segment its kept rows and the kept / padded rows before
+// it, and block-scan scratch.  Segment s = sl * G + group (sl = 0, 1 the
+// CTA's first or second slice; G = d_model / 128).
+struct Layout {
+  size_t red, off, dig, ktseg, segn, rawb, padb, scan, misc, total;
+};
+// Rows of a CTA after padding: each of at most 2G segments adds at most 7.
+__host__ __device__ inline int padded_rows(int lmax, int d) {
+  return (lmax + 14 * (d >> 7) + KT - 1) & ~(KT - 1);
+}
+__host__ __device__ inline Layout layout(int depth, int lmax, int d) {
+  const int lp = padded_rows(lmax, d), nseg = 2 * (d >> 7);
+  Layout L;
+  size_t o = (size_t)NW * depth * WSLOT;
+  L.red = o;
+  o += 4 * (size_t)(2 * NGRP * PART);
+  L.off = o;
+  o += 4 * (size_t)lp;
+  L.dig = o;
+  o += 4 * (size_t)lp;
+  L.ktseg = o;
+  o += 4 * (size_t)(lp / KT);
+  L.segn = o;
+  o += 4 * (size_t)(nseg + 1);
+  L.rawb = o;
+  o += 4 * (size_t)(nseg + 1);
+  L.padb = o;
+  o += 4 * (size_t)(nseg + 1);
+  L.scan = o;
+  o += 4 * 33;
+  L.misc = o;
+  o += 4 * 4;
+  L.total = o;
+  return L;
+}
+// Where padded row `pos` keeps its digit word: rows t and t + 4 of a k-tile
+// side by side.
+__device__ __forceinline__ int dig_index(int pos) {
+  return (pos & ~7) | ((pos & 3) << 1) | ((pos >> 2) & 1);
+}
+// The balanced base-256 digits of the integer nearest to v (|v| < 2^30):
+// v = d0 256^3 + d1 256^2 + d2 256 + d3, each d in [-128, 127], byte p = d_p.
+__device__ __forceinline__ uint32_t digits_of(float v) {
+  int r = __float2int_rn(v);
+  const int d3 = (int)((unsigned)r << 24) >> 24;
+  r = (r - d3) >> 8;
+  const int d2 = (int)((unsigned)r << 24) >> 24;
+  r = (r - d2) >> 8;
+  const int d1 = (int)((unsigned)r << 24) >> 24;
+  const int d0 = (r - d1) >> 8;
+  return ((uint32_t)d0 & 255u) | (((uint32_t)d1 & 255u) << 8) | (((uint32_t)d2 & 255u) << 16) |
+         ((uint32_t)d3 << 24);
 }
 
-// The row loop of Stage 1: the CTA's partial sums of the slices its pair
-// range touches go to a.part as tagged words (the tag from the launch
-// counter read at the kernel's start).  Every thread of the CTA calls it;
-// warps NW and above take no rows.
-template <int NB>
+// Stage 1 of one token: the CTA's partial sums g~, u~ of the slices its pair
+// range touches go to a.part as tagged words (the tag from the launch counter
+// read at the kernel's start).  Every thread of the CTA calls it: warps
+// 0..NW-1 stream and multiply, the rest take part in the prologue and the
+// final combine.
 __device__ void run(const TokenArgs& a, unsigned char* smem, unsigned long long counter) {
-  constexpr int RING = NB * BATCH;  // ring bytes per warp
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int P = gridDim.x, cta = blockIdx.x;
-  const int n16 = a.F >> 4, nblk = a.F >> 5;
-  const Magic mg = a.mg;
-
-  unsigned char* ring = smem;                                        // [NW][RING]
-  float* s_tot = reinterpret_cast<float*>(smem + NW * RING);         // [NW][PARTP]
-  int2* s_rx = reinterpret_cast<int2*>(s_tot + NW * PARTP);          // [lmax] (offset, x)
-  int* s_key = reinterpret_cast<int*>(s_rx + a.lmax);                // [lmax] segment key
-  float* s_stash = reinterpret_cast<float*>(s_key + a.lmax);         // [PARTP]
-  int* s_scan = reinterpret_cast<int*>(s_stash + PARTP);             // [33]
-  int* s_m = s_scan + 33;                                            // [4]
-  int* s_src = s_m + 4;                                              // [kTokenThreads]
+  const int d = a.d, G = d >> 7, nseg = 2 * G, depth = a.s1_depth;
+  const Layout Ly = layout(depth, a.lmax, d);
+  float* s_red = reinterpret_cast<float*>(smem + Ly.red);
+  int* s_off = reinterpret_cast<int*>(smem + Ly.off);
+  uint32_t* s_dig = reinterpret_cast<uint32_t*>(smem + Ly.dig);
+  int* s_ktseg = reinterpret_cast<int*>(smem + Ly.ktseg);
+  int* s_segn = reinterpret_cast<int*>(smem + Ly.segn);
+  int* s_rawb = reinterpret_cast<int*>(smem + Ly.rawb);
+  int* s_padb = reinterpret_cast<int*>(smem + Ly.padb);
+  unsigned* s_scan = reinterpret_cast<unsigned*>(smem + Ly.scan);
+  unsigned* s_misc = reinterpret_cast<unsigned*>(smem + Ly.misc);  // [0] max |x| bits, [1] k-tiles
 
   // ---- this CTA's pairs: [tlo, thi) of the C * d (slice, row) pairs,
   // slice-major; pair p of the range is slice cA + (rA + p >= d), row
   // (rA + p) mod d.  The split is static: it does not depend on the token. ----
-  const int d = a.d;
   const unsigned T = (unsigned)a.C * (unsigned)d;  // T * P < 2^31
   const unsigned tlo = T * (unsigned)cta / (unsigned)P, thi = T * (unsigned)(cta + 1) / (unsigned)P;
   const int span = (int)(thi - tlo);               // <= d, since C < P
   const int cA = (int)(tlo / (unsigned)d), rA = (int)(tlo % (unsigned)d);
   const int first = min(span, d - rA);             // pairs of the range in slice cA
-  // ---- its kept pairs (|x_row| >= tau), in pair order: thread t owns pairs
-  // [t*per, (t+1)*per); the two slices' counts are packed in one word ----
+  const int nsl = span > first ? 2 : 1;            // slices the range touches
+  auto row_of = [&](int p) { return rA + p < d ? rA + p : rA + p - d; };
+  auto seg_of = [&](int p) { return (p < first ? 0 : G) + (row_of(p) >> 7); };
+  // thread t owns pairs [t*per, (t+1)*per); their x is loaded first
   const int per = (span + (int)blockDim.x - 1) / (int)blockDim.x;
   const int p0 = min(tid * per, span), p1 = min(p0 + per, span);
   float xv[4];
-  unsigned cnt = 0;
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {  // the first four pairs (all of them while span <= 4 * blockDim.x)
-    const int p = p0 + q;
-    xv[q] = 0.f;
-    if (p < p1) {
-      const int row = rA + p < d ? rA + p : rA + p - d;
-      xv[q] = __ldg(a.x + row);
-      if (fabsf(xv[q]) >= a.tau) cnt += p < first ? 1u : 0x10000u;
+  for (int q = 0; q < 4; ++q) xv[q] = p0 + q < p1 ? __ldg(a.x + row_of(p0 + q)) : 0.f;
+  for (int i = tid; i <= nseg; i += blockDim.x) s_segn[i] = 0;
+  for (int i = tid; i < 2 * NGRP * PART; i += blockDim.x) s_red[i] = 0.f;
+  if (tid == 0) s_misc[0] = 0u;
+  __syncthreads();
+  // ---- kept rows (|x| >= tau): count per thread and per segment, and the
+  // largest kept |x| ----
+  unsigned cnt = 0, mx = 0;
+  auto count = [&](int p, float v) {
+    if (fabsf(v) >= a.tau) {
+      ++cnt;
+      mx = max(mx, __float_as_uint(fabsf(v)));
+      atomicAdd(&s_segn[seg_of(p)], 1);
+    }
+  };
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    if (p0 + q < p1) count(p0 + q, xv[q]);
+  for (int p = p0 + 4; p < p1; ++p) count(p, __ldg(a.x + row_of(p)));  // d > 4 * blockDim.x
+  mx = __reduce_max_sync(0xffffffffu, mx);
+  if (lane == 0 && mx) atomicMax(&s_misc[0], mx);
+  unsigned len;
+  const unsigned pre = block_exclusive_scan(cnt, s_scan, &len);
+  // per segment: kept rows before it and padded rows before it (warp 0)
+  if (warp == 0) {
+    const int spl = (nseg + 31) / 32;
+    int raw = 0, pad = 0;
+    for (int i = 0; i < spl; ++i) {
+      const int s = lane * spl + i;
+      const int n = s < nseg ? s_segn[s] : 0;
+      raw += n;
+      pad += (n + KT - 1) & ~(KT - 1);
+    }
+    int ri = raw, pi = pad;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int rn = __shfl_up_sync(0xffffffffu, ri, o), pn = __shfl_up_sync(0xffffffffu, pi, o);
+      if (lane >= o) {
+        ri += rn;
+        pi += pn;
+      }
+    }
+    int rb = ri - raw, pb = pi - pad;
+    for (int i = 0; i < spl; ++i) {
+      const int s = lane * spl + i;
+      if (s < nseg) {
+        const int n = s_segn[s];
+        s_rawb[s] = rb;
+        s_padb[s] = pb;
+        rb += n;
+        pb += (n + KT - 1) & ~(KT - 1);
+      }
+    }
+    if (lane == 31) {
+      s_padb[nseg] = pi;
+      s_misc[1] = (unsigned)pi / KT;
     }
   }
-  for (int p = p0 + 4; p < p1; ++p) {  // longer ranges (d > 4 * blockDim.x)
-    const int row = rA + p < d ? rA + p : rA + p - d;
-    if (fabsf(__ldg(a.x + row)) >= a.tau) cnt += p < first ? 1u : 0x10000u;
-  }
-  unsigned tot;
-  const unsigned pre = block_exclusive_scan(cnt, reinterpret_cast<unsigned*>(s_scan), &tot);
-  const int l_split = (int)(tot & 0xFFFFu);        // kept pairs in slice cA
-  const int len = l_split + (int)(tot >> 16);      // kept pairs of the CTA
+  __syncthreads();
+  // E: the exponent of the largest kept |x| (clamped so every power of two
+  // below stays a normal float); V = x 2^(29 - E) has |V| < 2^30.
+  int E = (int)(s_misc[0] >> 23) - 127;
+  E = max(E, -93);
+  const float vscale = __int_as_float((127 + 29 - E) << 23);
   {
-    int l0 = (int)(pre & 0xFFFFu), l1 = l_split + (int)(pre >> 16);
-    // the row slice's byte offset in the proxy, and its segment key (slice,
-    // quantisation group), nondecreasing over the CTA's rows
+    // each kept row at its padded position: offset of its row slice, digits
+    int l = (int)pre;
     auto place = [&](int p, float v) {
       if (fabsf(v) >= a.tau) {
-        const int row = rA + p < d ? rA + p : rA + p - d;
-        const int sl = p < first ? 0 : 1;
-        const int l = sl ? l1++ : l0++;
-        s_rx[l] = make_int2(((cA + sl) * d + row) * SLICE, __float_as_int(v));
-        s_key[l] = sl * 128 + (row >> 7);
+        const int row = row_of(p), sl = p < first ? 0 : 1;
+        const int s = sl * G + (row >> 7);
+        const int pos = s_padb[s] + l - s_rawb[s];
+        ++l;
+        s_off[pos] = ((cA + sl) * d + row) * SLICE;
+        s_dig[dig_index(pos)] = digits_of(v * vscale);
+        if ((pos & (KT - 1)) == 0) s_ktseg[pos / KT] = s;
       }
     };
 #pragma unroll
     for (int q = 0; q < 4; ++q)
       if (p0 + q < p1) place(p0 + q, xv[q]);
-    for (int p = p0 + 4; p < p1; ++p) place(p, __ldg(a.x + (rA + p < d ? rA + p : rA + p - d)));
+    for (int p = p0 + 4; p < p1; ++p) place(p, __ldg(a.x + row_of(p)));
+    // padding rows: nothing to copy, zero digits
+    for (int s = tid; s < nseg; s += blockDim.x) {
+      const int n = s_segn[s];
+      for (int i = n; i < ((n + KT - 1) & ~(KT - 1)); ++i) {
+        const int pos = s_padb[s] + i;
+        s_off[pos] = -1;
+        s_dig[dig_index(pos)] = 0u;
+      }
+    }
   }
   // realised input sparsity: the kept rows counted once, in slice 0
-  if (tid == 0 && cA == 0 && l_split > 0) atomicAdd(a.stats, (unsigned long long)l_split);
+  if (tid == 0 && cA == 0 && s_rawb[G] > 0) atomicAdd(a.stats, (unsigned long long)s_rawb[G]);
   if (cta == 0 && (a.idx_x || a.n_x)) {
     // test taps: the token's kept rows, ascending, and their number
     const int rpt = (d + (int)blockDim.x - 1) / (int)blockDim.x;
@@ -309,167 +438,147 @@ __device__ void run(const TokenArgs& a, unsigned char* smem, unsigned long long 
     int c = 0;
     for (int row = q0; row < q1; ++row) c += fabsf(__ldg(a.x + row)) >= a.tau;
     int n_all;
-    int pos = block_exclusive_scan(c, s_scan, &n_all);
+    int pos = block_exclusive_scan(c, reinterpret_cast<int*>(s_scan), &n_all);
     for (int row = q0; row < q1; ++row)
       if (fabsf(__ldg(a.x + row)) >= a.tau && a.idx_x) a.idx_x[pos++] = row;
     if (tid == 0 && a.n_x) *a.n_x = n_all;
   }
   __syncthreads();
   stamp(a.ts, 8);
+  const int nkt = (int)s_misc[1];
+  const float fin = __int_as_float((127 + E - 33) << 23);  // 2^(E - 33): V, and q as 16 q
 
   if (warp < NW) {
-    // ---- this warp's local rows [wl0, wl1) ----
-    const int wl0 = (int)((long long)len * warp / NW);
-    const int wl1 = (int)((long long)len * (warp + 1) / NW);
-    const int nbw = (wl1 - wl0 + U - 1) / U;
-    unsigned char* wring = ring + warp * RING + lane * 16;
-    const uint8_t* pq_lane = a.pq + lane * 16;
-    float* wtot = s_tot + warp * PARTP + lane;  // element j*32 + lane (at j*33 + lane): channel j of the chunk
+    const int q = warp / WPG, v = warp % WPG;
+    const int k0 = (int)((long long)nkt * q / NGRP), n = (int)((long long)nkt * (q + 1) / NGRP) - k0;
+    unsigned char* wring = smem + (size_t)warp * depth * WSLOT;
+    const int nblk = a.F >> 5;
+    const uint32_t lastw = (uint32_t)(a.F - (a.C - 1) * SLICE);  // bytes of a row of the last slice
+    // ---- copies of local k-tile i into slot i % depth: lane 8 r + c copies
+    // chunk c of rows r and r + 4 (16 bytes at byte 128 v + 16 c of the row
+    // slice) to position c ^ 2 (r mod 4) of the row; at a segment's first
+    // k-tile, lane 8 b + c also copies chunk c of block b's scales. ----
+    const int cc = lane & 7, cr = lane >> 3;
+    const uint32_t wbyte = (uint32_t)(v * WROW + 16 * cc);
+    auto issue = [&](int i) {
+      if (i < n) {
+        const int kt = k0 + i;
+        unsigned char* slot = wring + (size_t)(i % depth) * WSLOT;
+        const int s = s_ktseg[kt];
+        const int sl = s >= G ? 1 : 0;
+        const uint32_t width = cA + sl == a.C - 1 ? lastw : (uint32_t)SLICE;
 #pragma unroll
-    for (int j = 0; j < 32; ++j) wtot[j * 33] = 0.f;
-    // Only the last slice can be narrower than 512 bytes; a warp with rows there
-    // checks each lane's chunk before copying it.
-    const bool checked = (a.F % SLICE) != 0 && wl1 > wl0 &&
-                         cA + (wl1 - 1 >= l_split ? 1 : 0) == a.C - 1;
-    auto issue = [&](int j) {
-      if (j < nbw) {
-        unsigned char* dst = wring + (j % NB) * BATCH;
-        const int l0 = wl0 + j * U;
-        if (!checked && l0 + U <= wl1) {
-#pragma unroll
-          for (int u = 0; u < U; ++u)
-            cp_async16(dst + u * SLICE, pq_lane + (uint32_t)s_rx[l0 + u].x);
-        } else {
-          for (int u = 0; u < U && l0 + u < wl1; ++u) {
-            const int l = l0 + u;
-            const int c16 = (cA + (l >= l_split ? 1 : 0)) * 32 + lane;
-            if (c16 < n16) cp_async16(dst + u * SLICE, pq_lane + (uint32_t)s_rx[l].x);
-          }
+        for (int h = 0; h < 2; ++h) {
+          const int r = cr + 4 * h;
+          const int off = s_off[kt * KT + r];
+          if (off >= 0 && wbyte < width) cp_async16(slot + r * WROW + 16 * (cc ^ (2 * cr)), a.pq + off + wbyte);
+        }
+        if (i == 0 || s != s_ktseg[kt - 1]) {
+          const int B = (cA + sl) * 16 + v * BPW + cr;
+          if (B < nblk)
+            cp_async16(slot + KT * WROW + cr * 128 + 16 * cc,
+                       a.ps + ((size_t)(s - sl * G) * nblk + B) * 64 + 8 * cc);
         }
       }
       cp_async_commit();
     };
-    float2 acc[16];
+    // ---- operands: lane (g, t) = (lane / 4, lane mod 4) ----
+    const int g = lane >> 2, t = lane & 3, j = g & 3, pg = g >> 2;
+    // A fragment: byte j of each register holds digit pg (a0, a2) or pg + 2
+    // (a1, a3) of row t (a0, a1) or t + 4 (a2, a3); the other bytes are 0
+    const uint32_t sel0 = 0x4444u ^ ((uint32_t)(pg ^ 4) << (4 * j));
+    const uint32_t sel1 = 0x4444u ^ ((uint32_t)((pg + 2) ^ 4) << (4 * j));
+    // weights of the digits this lane's accumulator rows carry
+    const float wA = pg ? 65536.f : 16777216.f, wB = pg ? 1.f : 256.f;
+    // B fragment: word g of block b in rows t and t + 4 (swizzled chunk)
+    auto boff = [&](int b) { return t * WROW + 16 * ((2 * b + (g >> 2)) ^ (2 * t)) + 4 * (g & 3); };
+    // scales of a lane's sums (nibbles 2j, 2j + 1 of words 2t and 2t + 1) in
+    // a slot's scale area: block b, proxy t / 2, channel 16 (t mod 2) + 2j
+    const int soff = KT * WROW + 64 * (t >> 1) + 32 * (t & 1) + 4 * j;
+    int dl[BPW][4], dh[BPW][4];
+    uint32_t sc[BPW][2];
 #pragma unroll
-    for (int h = 0; h < 16; ++h) acc[h] = make_float2(0.f, 0.f);
-    uint4 sc[4];            // fp16 scales of the current (slice, group) for this lane's chunk
-    int cur_key = -1, cur_g = -1;
-    float okf = 0.f;        // 1 when this lane's chunk exists in the current slice
-    // group end: tot += scale * acc (tot in shared memory), acc = 0
-    auto flush = [&]() {
+    for (int b = 0; b < BPW; ++b)
 #pragma unroll
-      for (int qd = 0; qd < 4; ++qd) {
-        const uint32_t sw[4] = {sc[qd].x, sc[qd].y, sc[qd].z, sc[qd].w};
+      for (int i = 0; i < 4; ++i) dl[b][i] = dh[b][i] = 0;
+    // segment end: combine the digits' rows (lanes g and g ^ 4), scale and
+    // add to the group's sums of the segment's slice, s_red[sl][q][m][proxy]
+    // (lanes g < 4; lanes g >= 4 hold the same values)
+    auto flush = [&](int sl) {
+      float* red = s_red + ((size_t)sl * NGRP + q) * 512 * 2 + (t >> 1);
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          const int h = qd * 4 + m;
-          const float2 s2 = __half22float2(*reinterpret_cast<const __half2*>(&sw[m]));
-          wtot[(2 * h) * 33] = fmaf(s2.x, acc[h].x, wtot[(2 * h) * 33]);
-          wtot[(2 * h + 1) * 33] = fmaf(s2.y, acc[h].y, wtot[(2 * h + 1) * 33]);
-          acc[h] = make_float2(0.f, 0.f);
+      for (int b = 0; b < BPW; ++b) {
+        float l0 = fmaf((float)dl[b][0], wA, (float)dl[b][2] * wB);  // word 2t,     nibble 2j
+        float l1 = fmaf((float)dl[b][1], wA, (float)dl[b][3] * wB);  // word 2t + 1, nibble 2j
+        float h0 = fmaf((float)dh[b][0], wA, (float)dh[b][2] * wB);  // word 2t,     nibble 2j + 1
+        float h1 = fmaf((float)dh[b][1], wA, (float)dh[b][3] * wB);  // word 2t + 1, nibble 2j + 1
+        l0 += __shfl_xor_sync(0xffffffffu, l0, 16);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, 16);
+        h0 += __shfl_xor_sync(0xffffffffu, h0, 16);
+        h1 += __shfl_xor_sync(0xffffffffu, h1, 16);
+        const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&sc[b][0]));
+        const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&sc[b][1]));
+        if (g < 4) {
+          // channel of (word 2t + k / 2, nibble 2j + k mod 2) in the slice
+          const int m0 = 32 * (BPW * v + b) + 16 * (t & 1) + 2 * j;
+          red[2 * m0] = fmaf(f0.x, l0, red[2 * m0]);
+          red[2 * (m0 + 1)] = fmaf(f0.y, h0, red[2 * (m0 + 1)]);
+          red[2 * (m0 + 8)] = fmaf(f1.x, l1, red[2 * (m0 + 8)]);
+          red[2 * (m0 + 9)] = fmaf(f1.y, h1, red[2 * (m0 + 9)]);
         }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) dl[b][i] = dh[b][i] = 0;
       }
     };
-    auto row_fma = [&](const unsigned char* src, float xv) {
-      const uint4 v = *reinterpret_cast<const uint4*>(src);
-      const float2 x2 = make_float2(xv * okf, xv * okf);
-      acc_word(acc + 0, v.x, x2, mg);
-      acc_word(acc + 4, v.y, x2, mg);
-      acc_word(acc + 8, v.z, x2, mg);
-      acc_word(acc + 12, v.w, x2, mg);
-    };
+    int cur = -1;
+    for (int i = 0; i < depth - 1; ++i) issue(i);
+    for (int i = 0; i < n; ++i) {
+      issue(i + depth - 1);
+      cp_async_wait_n(depth - 1);  // this lane's copies of k-tile i have landed
+      __syncwarp();                // and every lane's
+      const int kt = k0 + i;
+      const unsigned char* slot = wring + (size_t)(i % depth) * WSLOT;
+      const int s = s_ktseg[kt];
+      if (s != cur) {
+        if (cur >= 0) flush(cur >= G ? 1 : 0);
+        cur = s;
 #pragma unroll
-    for (int j = 0; j < NB - 1; ++j) issue(j);
-    for (int j = 0; j < nbw; ++j) {
-      issue(j + NB - 1);
-      cp_async_wait<NB - 1>();  // this lane's copies of batch j have landed
-      const unsigned char* src = wring + (j % NB) * BATCH;
-      const int first = wl0 + j * U;
-      const int last = min(first + U, wl1);
-      if (last - first == U && s_key[first] == cur_key && s_key[last - 1] == cur_key) {
-        // one segment: no boundary checks
-#pragma unroll
-        for (int u = 0; u < U; ++u)
-          row_fma(src + u * SLICE, __int_as_float(s_rx[first + u].y));
-      } else {
-        for (int l = first; l < last; ++l) {
-          const int key = s_key[l];
-          if (key != cur_key) {
-            if (cur_g >= 0) flush();
-            if (cur_key >= 0 && (key >> 7) != (cur_key >> 7)) {
-              // the warp crosses into the next slice: park the first slice's sums
-#pragma unroll
-              for (int j2 = 0; j2 < 32; ++j2) {
-                s_stash[j2 * 33 + lane] = wtot[j2 * 33];
-                wtot[j2 * 33] = 0.f;
-              }
-            }
-            cur_key = key;
-            cur_g = key & 127;
-            const int c16 = (cA + (key >> 7)) * 32 + lane;
-            okf = c16 < n16 ? 1.f : 0.f;
-#pragma unroll
-            for (int qd = 0; qd < 4; ++qd) sc[qd] = make_uint4(0u, 0u, 0u, 0u);
-            if (c16 < n16) {
-              const uint4* sp = reinterpret_cast<const uint4*>(
-                  a.ps + ((size_t)cur_g * nblk + (c16 >> 1)) * 64 + (c16 & 1) * 32);
-#pragma unroll
-              for (int qd = 0; qd < 4; ++qd) sc[qd] = __ldg(sp + qd);
-            }
-          }
-          row_fma(src + (l - first) * SLICE, __int_as_float(s_rx[l].y));
+        for (int b = 0; b < BPW; ++b) {
+          sc[b][0] = *reinterpret_cast<const uint32_t*>(slot + soff + 128 * b);
+          sc[b][1] = *reinterpret_cast<const uint32_t*>(slot + soff + 128 * b + 16);
         }
       }
+      const uint2 dg = *reinterpret_cast<const uint2*>(s_dig + kt * KT + 2 * t);
+      const uint32_t a0 = prmt(dg.x, sel0), a1 = prmt(dg.x, sel1);
+      const uint32_t a2 = prmt(dg.y, sel0), a3 = prmt(dg.y, sel1);
+#pragma unroll
+      for (int b = 0; b < BPW; ++b) {
+        const uint32_t w0 = *reinterpret_cast<const uint32_t*>(slot + boff(b));
+        const uint32_t w1 = *reinterpret_cast<const uint32_t*>(slot + boff(b) + 4 * WROW);
+        mma_s8(dl[b], a0, a1, a2, a3, codes_lo_s8(w0), codes_lo_s8(w1));
+        mma_s8(dh[b], a0, a1, a2, a3, codes_hi_s8(w0), codes_hi_s8(w1));
+      }
+      __syncwarp();  // every lane's reads of the slot come before its refill
     }
     cp_async_wait<0>();
-    if (cur_g >= 0) flush();
+    if (cur >= 0) flush(cur >= G ? 1 : 0);
   }
   __syncthreads();
   stamp(a.ts, 9);
-
-  // ---- the CTA's partials per touched slice (warp order), then report ----
-  // warp w's share: bit 0 -> its sums belong to the CTA's first slice, bit 1 ->
-  // to the second, both -> it crossed (first-slice sums in the stash)
-  if (tid < NW) {
-    const int l0 = (int)((long long)len * tid / NW), l1 = (int)((long long)len * (tid + 1) / NW);
-    s_src[tid] = l1 <= l0 ? 0 : (l1 <= l_split ? 1 : (l0 >= l_split ? 2 : 3));
-  }
-  __syncthreads();
-  const int nsl = span > first ? 2 : 1;  // slices the CTA's pair range touches
-  const uint32_t tag = launch_tag(counter);  // (the counter was loaded at the kernel's start)
-  // Element e = j*32 + 2*blk + h of the sums is the gate (h = 0) or up
-  // (h = 1) sum of channel m = blk*32 + j of the slice; channel m's pair is
-  // stored at 2m, 2m + 1, so the scoring threads (one per channel,
-  // consecutive channels) read consecutive 16-byte pairs.  One thread per
-  // channel, one 16-byte store per touched slice: each warp's stores cover
-  // whole sectors.
-  for (int m = tid; m < PART / 2; m += blockDim.x) {
-    const int ep = (m & 31) * 33 + 2 * (m >> 5);  // the gate sum in the padded layout; up at + 1
-    float g0 = 0.f, u0 = 0.f, g1 = 0.f, u1 = 0.f;
+  // ---- the CTA's partials: the groups' sums in group order, channel-major
+  // (channel m's gate and up sums at 2m, 2m + 1) ----
+  const uint32_t tag = launch_tag(counter);
+  for (int e = tid; e < nsl * 512; e += blockDim.x) {
+    const int sl = e >> 9, m = e & 511;
+    float gs = 0.f, us = 0.f;
 #pragma unroll
-    for (int w = 0; w < NW; ++w) {
-      const int kind = s_src[w];
-      const float vg = s_tot[w * PARTP + ep], vu = s_tot[w * PARTP + ep + 1];
-      if (kind == 1) {
-        g0 += vg;
-        u0 += vu;
-      }
-      if (kind == 2) {
-        g1 += vg;
-        u1 += vu;
-      }
-      if (kind == 3) {
-        g0 += s_stash[ep];
-        u0 += s_stash[ep + 1];
-        g1 += vg;
-        u1 += vu;
-      }
+    for (int qq = 0; qq < NGRP; ++qq) {
+      const float2 v2 = *reinterpret_cast<const float2*>(s_red + (((size_t)sl * NGRP + qq) * 512 + m) * 2);
+      gs += v2.x;
+      us += v2.y;
     }
-    st_tag2(a.part + ((size_t)cta * 2) * PART + 2 * m, tag_word(__float_as_uint(g0), tag),
-            tag_word(__float_as_uint(u0), tag));
-    if (nsl == 2)
-      st_tag2(a.part + ((size_t)cta * 2 + 1) * PART + 2 * m, tag_word(__float_as_uint(g1), tag),
-              tag_word(__float_as_uint(u1), tag));
+    st_tag2(a.part + ((size_t)cta * 2 + sl) * PART + 2 * m, tag_word(__float_as_uint(gs * fin), tag),
+            tag_word(__float_as_uint(us * fin), tag));
   }
 }
 

@@ -92,7 +92,7 @@ __device__ void reduce_output(const TokenArgs& a, uint32_t tag, unsigned char* s
   }
 }
 
-template <int NB, int MAXM>
+template <int MAXM>
 __global__ void __launch_bounds__(kTokenThreads, 1) token_kernel(TokenArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   stamp_timer(a.ts, 0, 22);
@@ -104,7 +104,7 @@ __global__ void __launch_bounds__(kTokenThreads, 1) token_kernel(TokenArgs a) {
   const unsigned long long gv = ld_relaxed_u64(a.gbar);
   stamp(a.ts, 1);
   const bool topk = a.mode == kModeTopK;
-  if (a.stage1) s1::run<NB>(a, smem, gv);
+  if (a.stage1) s1::run(a, smem, gv);
   // the launch index e: every earlier launch added kPhases * gridDim.x to the
   // counter, and fewer than that many of this launch's additions can be in it
   const unsigned long long e = gv / ((unsigned long long)kPhases * gridDim.x);
@@ -160,49 +160,35 @@ __global__ void barrier_probe_kernel(unsigned long long* gbar, int* err) {
   phase_wait(ph, 1);
 }
 
-template <int NB>
-size_t stage1_smem(int lmax) {
-  return s1::smem_bytes<NB>(lmax);
-}
-
-template <int NB, int MAXM>
+template <int MAXM>
 cudaError_t set_attr() {
-  return cudaFuncSetAttribute(token_kernel<NB, MAXM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  return cudaFuncSetAttribute(token_kernel<MAXM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               kMaxSmemPerBlock);
 }
 
-template <int NB>
-cudaError_t set_attrs_nb() {
-  cudaError_t e;
-  if ((e = set_attr<NB, 1>()) != cudaSuccess) return e;
-  if ((e = set_attr<NB, 2>()) != cudaSuccess) return e;
-  if ((e = set_attr<NB, 3>()) != cudaSuccess) return e;
-  return set_attr<NB, 4>();
-}
-
-template <int NB>
-cudaError_t launch_nb(const cudaLaunchConfig_t& cfg, int maxm, const TokenArgs& a) {
-  if (maxm <= 1) return cudaLaunchKernelEx(&cfg, token_kernel<NB, 1>, a);
-  if (maxm == 2) return cudaLaunchKernelEx(&cfg, token_kernel<NB, 2>, a);
-  if (maxm == 3) return cudaLaunchKernelEx(&cfg, token_kernel<NB, 3>, a);
-  return cudaLaunchKernelEx(&cfg, token_kernel<NB, 4>, a);
+cudaError_t launch_maxm(const cudaLaunchConfig_t& cfg, int maxm, const TokenArgs& a) {
+  if (maxm <= 1) return cudaLaunchKernelEx(&cfg, token_kernel<1>, a);
+  if (maxm == 2) return cudaLaunchKernelEx(&cfg, token_kernel<2>, a);
+  if (maxm == 3) return cudaLaunchKernelEx(&cfg, token_kernel<3>, a);
+  return cudaLaunchKernelEx(&cfg, token_kernel<4>, a);
 }
 
 }  // namespace
 
-void choose_stage1_grid(int d, int F, int num_sms, int* C, int* lmax, int* nb) {
+void choose_stage1_grid(int d, int F, int num_sms, int* C, int* lmax, int* depth) {
   *C = (F + s1::SLICE - 1) / s1::SLICE;
   // a CTA's share of the C * n_x pairs, n_x <= d
   *lmax = (int)(((long long)(*C) * d + num_sms - 1) / num_sms) + 1;
-  // four batches in flight per warp when they fit, else three, else two
-  *nb = 4;
-  if (s1::smem_bytes<4>(*lmax) > (size_t)kMaxSmemPerBlock) *nb = 3;
-  if (s1::smem_bytes<3>(*lmax) > (size_t)kMaxSmemPerBlock) *nb = 2;
+  // as many k-tiles in flight per warp as the shared memory left by the
+  // tables holds, at most kMaxDepth
+  const size_t tables = s1::layout(0, *lmax, d).total;
+  const long long room = (long long)kMaxSmemPerBlock - (long long)tables;
+  long long k = room > 0 ? room / ((long long)s1::NW * s1::WSLOT) : 0;
+  if (k > s1::kMaxDepth) k = s1::kMaxDepth;
+  *depth = (int)k;
 }
 
-size_t stage1_smem_bytes(int lmax, int nb) {
-  return nb == 4 ? stage1_smem<4>(lmax) : nb == 3 ? stage1_smem<3>(lmax) : stage1_smem<2>(lmax);
-}
+size_t stage1_smem_bytes(int lmax, int depth, int d) { return s1::layout(depth, lmax, d).total; }
 
 size_t stage1_part_floats(int P) { return (size_t)P * 2 * s1::PART; }
 
@@ -240,9 +226,10 @@ int stage2_maxm(int d, int groups) {
 
 cudaError_t setup_token_kernels() {
   cudaError_t e;
-  if ((e = set_attrs_nb<4>()) != cudaSuccess) return e;
-  if ((e = set_attrs_nb<3>()) != cudaSuccess) return e;
-  return set_attrs_nb<2>();
+  if ((e = set_attr<1>()) != cudaSuccess) return e;
+  if ((e = set_attr<2>()) != cudaSuccess) return e;
+  if ((e = set_attr<3>()) != cudaSuccess) return e;
+  return set_attr<4>();
 }
 
 cudaError_t launch_barrier_probe(const prox_layer* L, cudaStream_t s) {
@@ -262,6 +249,7 @@ cudaError_t launch_token(const prox_layer* L, const TokenLaunch& m, cudaStream_t
   a.F = L->F;
   a.C = L->C;
   a.lmax = L->s1_lmax;
+  a.s1_depth = L->s1_depth;
   a.tau = L->tau;
   a.slots = L->ring_slots;
   a.groups = L->stage2_groups;
@@ -294,7 +282,6 @@ cudaError_t launch_token(const prox_layer* L, const TokenLaunch& m, cudaStream_t
   a.sel_mask = m.sel_mask;
   a.s_sp = m.s_sp;
   a.ts = m.phase_ns;
-  a.mg = Magic{0x4B000000u, 0x49000000u, 0x47000000u, 0x45000000u, 0x43000000u};
 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(L->P, 1, 1);
@@ -309,9 +296,7 @@ cudaError_t launch_token(const prox_layer* L, const TokenLaunch& m, cudaStream_t
   cfg.attrs = attr;
   cfg.numAttrs = 2;
   const int maxm = stage2_maxm(L->d, L->stage2_groups);
-  if (L->s1_nb == 4) return launch_nb<4>(cfg, maxm, a);
-  if (L->s1_nb == 3) return launch_nb<3>(cfg, maxm, a);
-  return launch_nb<2>(cfg, maxm, a);
+  return launch_maxm(cfg, maxm, a);
 }
 
 }  // namespace prox

@@ -1,6 +1,5 @@
 // Arguments of the fused per-token kernel (token.cu) and the small device
-// primitives its phases share: the tagged exchange words and the exponent
-// words of the INT4 decode.
+// primitives its phases share: the tagged exchange words and the phase hints.
 #pragma once
 
 #include "prox_device.cuh"
@@ -17,11 +16,6 @@ enum TokenMode : int {
   kModeThreshold = 3,  // score >= tau_s (Prox §4.1)
 };
 
-// Exponent words for the nibble decode: 2^23, 2^19, 2^15, 2^11, 2^7.
-struct Magic {
-  uint32_t e23, e19, e15, e11, e7;
-};
-
 struct TokenArgs {
   const float* x;        // [d] this token's input
   float* out;            // [d] this token's output (Stage 2 modes)
@@ -34,6 +28,7 @@ struct TokenArgs {
   // Stage-1 geometry
   int C;                 // 512-byte column slices of a proxy row
   int lmax;              // kept-row capacity of a CTA
+  int s1_depth;          // Stage-1 k-tiles in flight per warp
   float tau;             // tau_x
   // Stage-2 geometry
   int slots, groups, max_rec;
@@ -69,7 +64,6 @@ struct TokenArgs {
   int32_t* sel_mask;     // 1/0 per channel (top-k / threshold)
   float* s_sp;           // act(g) u per selected channel
   unsigned long long* ts;  // optional phase stamps [P][kPhaseStamps]
-  Magic mg;
 };
 
 // Phase stamp i of this CTA (the SM's clock64 cycle count) when stamps were
@@ -77,12 +71,14 @@ struct TokenArgs {
 // only at entry, slot 22, and exit, slot 23, with the exit cycle count in
 // slot 21, to place the cycle counts on one ns time line):
 // 0 kernel entry, 1 previous kernel complete, 8 kept rows compacted, 9 Stage-1
-// row loop done, 2 Stage-1 partials written, 3 the partials of thread 0's
-// channel received, 10 the CTA's channels scored and counted, 14 the coarse
-// histogram complete, 15 the top-k cut found, 4 the CTA's Stage-2 channels
-// known, 11 Stage-2 ring set up, 12 gate/up phase done, 5 partial output row
-// written, 6 the partial rows of the CTA's columns received, 7 output
-// written; slot 13 holds the CTA's Stage-2 channel count, not a time.
+// row loop done (the CTA's partials stored), 2 phase 0 reported, 16 phase 0
+// complete, 3 the partials of thread 0's channel received, 10 the CTA's
+// channels scored and counted, 17 phase 1 complete, 14 the coarse histogram
+// complete, 15 the top-k cut found, 18 phase 2 complete, 4 the CTA's Stage-2
+// channels known, 11 Stage-2 ring set up, 12 gate/up phase done, 5 partial
+// output row written, 19 phase 3 complete, 6 the partial rows of the CTA's
+// columns received, 7 output written, 21 exit; slot 13 holds the CTA's
+// Stage-2 channel count, not a time.
 __device__ __forceinline__ void stamp(unsigned long long* ts, int i) {
   if (ts && threadIdx.x == 0) ts[(size_t)blockIdx.x * kPhaseStamps + i] = (unsigned long long)clock64();
 }
@@ -110,21 +106,6 @@ __device__ __forceinline__ void fence_acq_rel_gpu() {
   asm volatile("fence.acq_rel.gpu;" ::: "memory");
 }
 
-// Grid-wide barriers of one launch whose CTAs are all resident (cooperative
-// launch, one CTA per SM).  The layer's 64-bit arrival counter only grows:
-// thread 0 of every CTA reads it once when the launch starts; the previous
-// launch on the layer is complete by then and every barrier adds exactly
-// gridDim.x arrivals, so rounding the value read down to a multiple of
-// gridDim.x gives every CTA the same base even when faster CTAs have already
-// arrived at the first barrier.  Barrier i of the launch is complete once the
-// counter reaches base + i * expected.  A CTA's thread 0, after a bar.sync, releases the CTA's
-// writes (fence) and arrives with a reduction (no round trip); it then polls
-// the counter and acquires (fence) once the target is reached.  So every
-// write made before the barrier by any thread of any CTA is visible to every
-// thread after it.  The wait is bounded: when it runs out the CTA sets
-// PROX_DEVERR_WAIT_TIMEOUT, marks itself dead (later barriers do not wait)
-// and carries on, so a CTA that never arrives cannot hang the GPU; the host
-// resets the counter in prox_layer_error.
 // Tagged words.  Everything one CTA of a launch writes for others to read is
 // a 64-bit word holding a 32-bit payload and, in its high half, the launch's
 // tag, stored and loaded with single 64-bit relaxed accesses (single-copy

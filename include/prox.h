@@ -22,13 +22,13 @@
  *  - Shape rules (else PROX_EINVAL, checked before any launch):
  *    d_model > 0 and d_model % 128 == 0; d_ff > 0 and d_ff % 32 == 0;
  *    d_model <= 16384; d_ff <= 32768; 1 <= k <= d_ff; pointers 16-byte aligned.
- *    Stage 1 keeps its share of the kept input rows in shared memory beside a
- *    ring of at least two row batches, which bounds ceil(d_ff/512) * d_model
- *    <= 7730 * (number of SMs), and the scoring takes one channel per thread,
- *    which bounds d_ff <= 512 * (number of SMs): on a 148-SM B200 every shape
- *    the rules above admit (at most 64 * 16384 = 1.05 M <= 1.14 M).  On a
- *    device with fewer SMs prox_layer_create returns PROX_EUNSUPPORTED beyond
- *    them.
+ *    Stage 1 keeps a table entry per kept input row of its share in shared
+ *    memory beside its copy ring (at least two 8-row tiles per warp), which
+ *    bounds ceil(d_ff/512) * d_model <= 15535 * (number of SMs), and the
+ *    scoring takes one channel per thread, which bounds d_ff <= 512 * (number
+ *    of SMs): on a 148-SM B200 every shape the rules above admit (at most
+ *    64 * 16384 = 1.05 M <= 2.29 M).  On a device with fewer SMs
+ *    prox_layer_create returns PROX_EUNSUPPORTED beyond them.
  *  - Errors: every call returns a prox_status; prox_last_error() copies a
  *    message for the calling thread's last failure.  No C++ exception crosses
  *    this boundary.  Device-side checks (an index out of range in a caller's
