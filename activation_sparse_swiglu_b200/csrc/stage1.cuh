@@ -246,19 +246,22 @@ static_assert(kMaxDepth <= 8, "cp_async_wait_n covers depths up to 8");
 // block): the warps' rings [NW][depth][WSLOT], the groups' sums per slice
 // [2][NGRP][512][2] (float), then per padded row its byte offset in the
 // proxy (-1 for padding) and its digit word (byte p = digit p; stored k-tile
-// interleaved so rows t and t + 4 of a k-tile are adjacent), the segment of
-// each k-tile, per segment its kept rows and the kept / padded rows before
-// it, and block-scan scratch.  Segment s = sl * G + group (sl = 0, 1 the
+// interleaved so rows t and t + 4 of a k-tile are adjacent), the segment
+// code of each k-tile, each segment's kept rows, the warps' largest kept
+// |x|, block-scan scratch and two words.  A segment is an aligned 128-pair
+// chunk of the (slice, row) pair space: one slice and one quantisation group
+// (d_model is a multiple of 128); its code is sl * G + group (sl = 0, 1 the
 // CTA's first or second slice; G = d_model / 128).
 struct Layout {
-  size_t red, off, dig, ktseg, segn, rawb, padb, scan, misc, total;
+  size_t red, off, dig, ktseg, segn, wmax, scan, misc, total;
 };
-// Rows of a CTA after padding: each of at most 2G segments adds at most 7.
+// Rows of a CTA after padding: each of its at most d/128 + 2 segments adds
+// at most 7.
 __host__ __device__ inline int padded_rows(int lmax, int d) {
-  return (lmax + 14 * (d >> 7) + KT - 1) & ~(KT - 1);
+  return (lmax + 14 * (d >> 7) + 14 + KT - 1) & ~(KT - 1);
 }
 __host__ __device__ inline Layout layout(int depth, int lmax, int d) {
-  const int lp = padded_rows(lmax, d), nseg = 2 * (d >> 7);
+  const int lp = padded_rows(lmax, d), nseg = (d >> 7) + 2;
   Layout L;
   size_t o = (size_t)NW * depth * WSLOT;
   L.red = o;
@@ -270,11 +273,9 @@ __host__ __device__ inline Layout layout(int depth, int lmax, int d) {
   L.ktseg = o;
   o += 4 * (size_t)(lp / KT);
   L.segn = o;
-  o += 4 * (size_t)(nseg + 1);
-  L.rawb = o;
-  o += 4 * (size_t)(nseg + 1);
-  L.padb = o;
-  o += 4 * (size_t)(nseg + 1);
+  o += 4 * (size_t)nseg;
+  L.wmax = o;
+  o += 4 * 32;
   L.scan = o;
   o += 4 * 33;
   L.misc = o;
@@ -307,130 +308,122 @@ __device__ __forceinline__ uint32_t digits_of(float v) {
 // 0..NW-1 stream and multiply, the rest take part in the prologue and the
 // final combine.
 __device__ void run(const TokenArgs& a, unsigned char* smem, unsigned long long counter) {
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nwarps = blockDim.x >> 5;
   const int P = gridDim.x, cta = blockIdx.x;
-  const int d = a.d, G = d >> 7, nseg = 2 * G, depth = a.s1_depth;
+  const int d = a.d, G = d >> 7, depth = a.s1_depth;
   const Layout Ly = layout(depth, a.lmax, d);
   float* s_red = reinterpret_cast<float*>(smem + Ly.red);
   int* s_off = reinterpret_cast<int*>(smem + Ly.off);
   uint32_t* s_dig = reinterpret_cast<uint32_t*>(smem + Ly.dig);
   int* s_ktseg = reinterpret_cast<int*>(smem + Ly.ktseg);
   int* s_segn = reinterpret_cast<int*>(smem + Ly.segn);
-  int* s_rawb = reinterpret_cast<int*>(smem + Ly.rawb);
-  int* s_padb = reinterpret_cast<int*>(smem + Ly.padb);
+  unsigned* s_wmax = reinterpret_cast<unsigned*>(smem + Ly.wmax);
   unsigned* s_scan = reinterpret_cast<unsigned*>(smem + Ly.scan);
-  unsigned* s_misc = reinterpret_cast<unsigned*>(smem + Ly.misc);  // [0] max |x| bits, [1] k-tiles
+  unsigned* s_misc = reinterpret_cast<unsigned*>(smem + Ly.misc);  // [1] k-tiles
 
   // ---- this CTA's pairs: [tlo, thi) of the C * d (slice, row) pairs,
-  // slice-major; pair p of the range is slice cA + (rA + p >= d), row
-  // (rA + p) mod d.  The split is static: it does not depend on the token. ----
+  // slice-major (pair t is slice t / d, row t mod d).  The split is static:
+  // it does not depend on the token. ----
   const unsigned T = (unsigned)a.C * (unsigned)d;  // T * P < 2^31
   const unsigned tlo = T * (unsigned)cta / (unsigned)P, thi = T * (unsigned)(cta + 1) / (unsigned)P;
   const int span = (int)(thi - tlo);               // <= d, since C < P
-  const int cA = (int)(tlo / (unsigned)d), rA = (int)(tlo % (unsigned)d);
-  const int first = min(span, d - rA);             // pairs of the range in slice cA
-  const int nsl = span > first ? 2 : 1;            // slices the range touches
-  auto row_of = [&](int p) { return rA + p < d ? rA + p : rA + p - d; };
-  auto seg_of = [&](int p) { return (p < first ? 0 : G) + (row_of(p) >> 7); };
-  // thread t owns pairs [t*per, (t+1)*per); their x is loaded first
-  const int per = (span + (int)blockDim.x - 1) / (int)blockDim.x;
-  const int p0 = min(tid * per, span), p1 = min(p0 + per, span);
-  float xv[4];
+  const int cA = (int)(tlo / (unsigned)d);
+  const int nsl = span > 0 && (int)((thi - 1) / (unsigned)d) > cA ? 2 : 1;  // slices the range touches
+  // its segments: the aligned 128-pair chunks [128 (s0 + ls), + 128) it meets
+  const int s0 = (int)(tlo >> 7);
+  const int nls = span > 0 ? (int)((thi - 1) >> 7) - s0 + 1 : 0;
+  // Warp w takes the segments w, w + nwarps, ...; lane l the pairs 4l .. 4l+3
+  // of one: x_row for the 4 rows in one load, kept = inside the range and
+  // |x| >= tau, as a 4-bit mask.
+  auto seg_mask = [&](int ls, float4& xv, int& slice, int& row0) {
+    const unsigned base = (unsigned)(s0 + ls) << 7;
+    slice = (int)(base / (unsigned)d);
+    row0 = (int)(base - (unsigned)slice * (unsigned)d);
+    xv = __ldg(reinterpret_cast<const float4*>(a.x + row0) + lane);
+    const float v[4] = {xv.x, xv.y, xv.z, xv.w};
+    unsigned m = 0;
 #pragma unroll
-  for (int q = 0; q < 4; ++q) xv[q] = p0 + q < p1 ? __ldg(a.x + row_of(p0 + q)) : 0.f;
-  for (int i = tid; i <= nseg; i += blockDim.x) s_segn[i] = 0;
-  for (int i = tid; i < 2 * NGRP * PART; i += blockDim.x) s_red[i] = 0.f;
-  if (tid == 0) s_misc[0] = 0u;
-  __syncthreads();
-  // ---- kept rows (|x| >= tau): count per thread and per segment, and the
-  // largest kept |x| ----
-  unsigned cnt = 0, mx = 0;
-  auto count = [&](int p, float v) {
-    if (fabsf(v) >= a.tau) {
-      ++cnt;
-      mx = max(mx, __float_as_uint(fabsf(v)));
-      atomicAdd(&s_segn[seg_of(p)], 1);
+    for (int k = 0; k < 4; ++k) {
+      const unsigned gp = base + 4u * (unsigned)lane + (unsigned)k;
+      if (gp >= tlo && gp < thi && fabsf(v[k]) >= a.tau) m |= 1u << k;
     }
+    return m;
   };
+  // pass 1: kept rows per segment, the largest kept |x|
+  unsigned mx = 0;
+  for (int ls = warp; ls < nls; ls += nwarps) {
+    float4 xv;
+    int slice, row0;
+    const unsigned m = seg_mask(ls, xv, slice, row0);
+    const float v[4] = {xv.x, xv.y, xv.z, xv.w};
 #pragma unroll
-  for (int q = 0; q < 4; ++q)
-    if (p0 + q < p1) count(p0 + q, xv[q]);
-  for (int p = p0 + 4; p < p1; ++p) count(p, __ldg(a.x + row_of(p)));  // d > 4 * blockDim.x
+    for (int k = 0; k < 4; ++k)
+      if (m & (1u << k)) mx = max(mx, __float_as_uint(fabsf(v[k])));
+    const int n = __reduce_add_sync(0xffffffffu, (unsigned)__popc(m));
+    if (lane == 0) s_segn[ls] = n;
+  }
   mx = __reduce_max_sync(0xffffffffu, mx);
-  if (lane == 0 && mx) atomicMax(&s_misc[0], mx);
-  unsigned len;
-  const unsigned pre = block_exclusive_scan(cnt, s_scan, &len);
-  // per segment: kept rows before it and padded rows before it (warp 0)
-  if (warp == 0) {
-    const int spl = (nseg + 31) / 32;
-    int raw = 0, pad = 0;
-    for (int i = 0; i < spl; ++i) {
-      const int s = lane * spl + i;
-      const int n = s < nseg ? s_segn[s] : 0;
-      raw += n;
-      pad += (n + KT - 1) & ~(KT - 1);
-    }
-    int ri = raw, pi = pad;
+  if (lane == 0) s_wmax[warp] = mx;
+  // each warp zeroes its own entries of the groups' sums (warp v of group q:
+  // channels of blocks BPW v .. BPW v + 3, both slices, both proxies)
+  if (warp < NW) {
+    const int q = warp / WPG, v = warp % WPG;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int rn = __shfl_up_sync(0xffffffffu, ri, o), pn = __shfl_up_sync(0xffffffffu, pi, o);
-      if (lane >= o) {
-        ri += rn;
-        pi += pn;
-      }
-    }
-    int rb = ri - raw, pb = pi - pad;
-    for (int i = 0; i < spl; ++i) {
-      const int s = lane * spl + i;
-      if (s < nseg) {
-        const int n = s_segn[s];
-        s_rawb[s] = rb;
-        s_padb[s] = pb;
-        rb += n;
-        pb += (n + KT - 1) & ~(KT - 1);
-      }
-    }
-    if (lane == 31) {
-      s_padb[nseg] = pi;
-      s_misc[1] = (unsigned)pi / KT;
+    for (int i = 0; i < 2 * BPW * 32 * 2 / 32; ++i) {
+      const int e = i * 32 + lane;  // (slice, channel of the warp's blocks, proxy)
+      const int sl = e >> 8, m = BPW * 32 * v + ((e >> 1) & 127), pr = e & 1;
+      s_red[(((size_t)sl * NGRP + q) * 512 + m) * 2 + pr] = 0.f;
     }
   }
   __syncthreads();
   // E: the exponent of the largest kept |x| (clamped so every power of two
   // below stays a normal float); V = x 2^(29 - E) has |V| < 2^30.
-  int E = (int)(s_misc[0] >> 23) - 127;
-  E = max(E, -93);
+  unsigned mxb = 0;
+  for (int w = 0; w < nwarps; ++w) mxb = max(mxb, s_wmax[w]);
+  const int E = max((int)(mxb >> 23) - 127, -93);
   const float vscale = __int_as_float((127 + 29 - E) << 23);
-  {
-    // each kept row at its padded position: offset of its row slice, digits
-    int l = (int)pre;
-    auto place = [&](int p, float v) {
-      if (fabsf(v) >= a.tau) {
-        const int row = row_of(p), sl = p < first ? 0 : 1;
-        const int s = sl * G + (row >> 7);
-        const int pos = s_padb[s] + l - s_rawb[s];
-        ++l;
-        s_off[pos] = ((cA + sl) * d + row) * SLICE;
-        s_dig[dig_index(pos)] = digits_of(v * vscale);
-        if ((pos & (KT - 1)) == 0) s_ktseg[pos / KT] = s;
-      }
-    };
+  // pass 2: each kept row at its padded position (padded rows of the earlier
+  // segments + its rank in its segment), with its row slice's offset and its
+  // digits; the segment's padding rows (nothing to copy, zero digits) and
+  // the segment code of its k-tiles
+  for (int ls = warp; ls < nls; ls += nwarps) {
+    int pb = 0;
+    for (int i = lane; i < ls; i += 32) pb += (s_segn[i] + KT - 1) & ~(KT - 1);
+    pb = (int)__reduce_add_sync(0xffffffffu, (unsigned)pb);
+    float4 xv;
+    int slice, row0;
+    const unsigned m = seg_mask(ls, xv, slice, row0);
+    const float v[4] = {xv.x, xv.y, xv.z, xv.w};
+    int incl = __popc(m);
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-      if (p0 + q < p1) place(p0 + q, xv[q]);
-    for (int p = p0 + 4; p < p1; ++p) place(p, __ldg(a.x + row_of(p)));
-    // padding rows: nothing to copy, zero digits
-    for (int s = tid; s < nseg; s += blockDim.x) {
-      const int n = s_segn[s];
-      for (int i = n; i < ((n + KT - 1) & ~(KT - 1)); ++i) {
-        const int pos = s_padb[s] + i;
-        s_off[pos] = -1;
-        s_dig[dig_index(pos)] = 0u;
-      }
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
     }
+    int pos = pb + incl - __popc(m);
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      if (m & (1u << k)) {
+        s_off[pos] = (slice * d + row0 + 4 * lane + k) * SLICE;
+        s_dig[dig_index(pos)] = digits_of(v[k] * vscale);
+        ++pos;
+      }
+    const int n = s_segn[ls], padded = (n + KT - 1) & ~(KT - 1);
+    for (int i = n + lane; i < padded; i += 32) {
+      s_off[pb + i] = -1;
+      s_dig[dig_index(pb + i)] = 0u;
+    }
+    const int code = (slice - cA) * G + (row0 >> 7);
+    for (int i = lane; i < padded / KT; i += 32) s_ktseg[pb / KT + i] = code;
+    // realised input sparsity: the kept rows counted once, in slice 0
+    if (lane == 0 && slice == 0 && n > 0) atomicAdd(a.stats, (unsigned long long)n);
   }
-  // realised input sparsity: the kept rows counted once, in slice 0
-  if (tid == 0 && cA == 0 && s_rawb[G] > 0) atomicAdd(a.stats, (unsigned long long)s_rawb[G]);
+  if (warp == 0) {
+    int tot = 0;
+    for (int i = lane; i < nls; i += 32) tot += (s_segn[i] + KT - 1) & ~(KT - 1);
+    tot = (int)__reduce_add_sync(0xffffffffu, (unsigned)tot);
+    if (lane == 0) s_misc[1] = (unsigned)tot / KT;
+  }
   if (cta == 0 && (a.idx_x || a.n_x)) {
     // test taps: the token's kept rows, ascending, and their number
     const int rpt = (d + (int)blockDim.x - 1) / (int)blockDim.x;
