@@ -148,9 +148,9 @@ PROX_API prox_status prox_calibrate_thresholds(const float* X_cal, int n_tok, in
  * of 2056 uint32 (8 KB) per device, which every device that loads the
  * library holds until the process exits.  Set-up: the first call made on a
  * device (with that device current) looks up the array's device address with
- * cudaGetSymbolAddress and caches it per device and CUDA context; make that
- * first call before any stream capture.  A device reset (cudaDeviceReset) or
- * a new primary context makes the next call look the address up again.
+ * cudaGetSymbolAddress and caches it per device and CUDA context.  A device
+ * reset (cudaDeviceReset) or a new primary context makes the next call look
+ * the address up again.
  * Every call zeroes the histogram it needs before counting, so nothing has to
  * start at zero.  Calls that overlap on one device (other streams, other
  * threads) share that scratch and race: serialise them.  X_cal: fp32

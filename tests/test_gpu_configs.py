@@ -244,8 +244,9 @@ def test_stack_threshold_rule_small(prox):
 # ---------------------------------------------------------------------------
 
 def test_largest_shape_runs(prox):
-    """d_model 16384, d_ff 32768 (the header's limits; Stage 1 then runs its
-    two-batch ring): the step runs with a clean error word, selects k channels
+    """d_model 16384, d_ff 32768 (the header's limits; Stage 1 then holds the
+    most kept rows per CTA and its shallowest copy rings): the step runs with a
+    clean error word, selects k channels
     and equals Stage 2 on its own mask bit for bit.  No oracle at this size:
     the properties hold at any size."""
     d, f = 16384, 32768
