@@ -118,10 +118,9 @@ __device__ void score_channels(const TokenArgs& a, bool histogram, SelectScratch
   const int c1 = (int)(((long long)a.F * (cta + 1)) / P);
   const int T = a.C * a.d;
   uint32_t* fine = select_keys(sel);  // [kScoreBins]: the CTA's counts, then its bucket offsets
-  if (histogram) {
+  if (histogram) {  // (ordered before the counting by the barrier after the partial sums)
     for (int i = tid; i < kCoarseBins; i += blockDim.x) sel.coarse[i] = 0u;
     for (int i = tid; i < kScoreBins; i += blockDim.x) fine[i] = 0u;
-    __syncthreads();
   }
   {
     // g~ and u~ of the CTA's channels: tpc threads per channel (a power of two
@@ -306,8 +305,8 @@ __device__ __forceinline__ uint32_t digits_of(float v) {
 // range touches go to a.part as tagged words (the tag from the launch counter
 // read at the kernel's start).  Every thread of the CTA calls it: warps
 // 0..NW-1 stream and multiply, the rest take part in the prologue and the
-// final combine.
-__device__ void run(const TokenArgs& a, unsigned char* smem, unsigned long long counter) {
+// final combine.  Returns the launch index (launch_index(counter)).
+__device__ unsigned long long run(const TokenArgs& a, unsigned char* smem, unsigned long long counter) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nwarps = blockDim.x >> 5;
   const int P = gridDim.x, cta = blockIdx.x;
   const int d = a.d, G = d >> 7, depth = a.s1_depth;
@@ -560,7 +559,8 @@ __device__ void run(const TokenArgs& a, unsigned char* smem, unsigned long long 
   stamp(a.ts, 9);
   // ---- the CTA's partials: the groups' sums in group order, channel-major
   // (channel m's gate and up sums at 2m, 2m + 1) ----
-  const uint32_t tag = launch_tag(counter);
+  const unsigned long long index = launch_index(counter);
+  const uint32_t tag = launch_tag(index);
   for (int e = tid; e < nsl * 512; e += blockDim.x) {
     const int sl = e >> 9, m = e & 511;
     float gs = 0.f, us = 0.f;
@@ -573,6 +573,7 @@ __device__ void run(const TokenArgs& a, unsigned char* smem, unsigned long long 
     st_tag2(a.part + ((size_t)cta * 2 + sl) * PART + 2 * m, tag_word(__float_as_uint(gs * fin), tag),
             tag_word(__float_as_uint(us * fin), tag));
   }
+  return index;
 }
 
 }  // namespace s1

@@ -104,11 +104,9 @@ __global__ void __launch_bounds__(kTokenThreads, 1) token_kernel(TokenArgs a) {
   const unsigned long long gv = ld_relaxed_u64(a.gbar);
   stamp(a.ts, 1);
   const bool topk = a.mode == kModeTopK;
-  if (a.stage1) s1::run(a, smem, gv);
-  // the launch index e: every earlier launch added kPhases * gridDim.x to the
-  // counter, and fewer than that many of this launch's additions can be in it
-  const unsigned long long e = gv / ((unsigned long long)kPhases * gridDim.x);
-  const uint32_t tag = launch_tag(gv);
+  // the launch index (Stage 1 works it out when it first needs the tag)
+  const unsigned long long e = a.stage1 ? s1::run(a, smem, gv) : launch_index(gv);
+  const uint32_t tag = launch_tag(e);
   const int par = (int)(e & 1ull);
   const Phases ph{a.gbar, e * kPhases * gridDim.x, a.err};
   {

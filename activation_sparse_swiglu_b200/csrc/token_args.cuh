@@ -170,9 +170,14 @@ __device__ __forceinline__ bool wait_more(long long t0, int* err) {
 // the writes it follows costs a re-poll, never a wrong value.  No fence.
 constexpr int kPhases = 4;
 
-// The launch's tag from the launch counter read at its start.
-__device__ __forceinline__ uint32_t launch_tag(unsigned long long counter) {
-  return (uint32_t)(counter / ((unsigned long long)kPhases * gridDim.x)) | 0x80000000u;
+// The launch's index from the launch counter read at its start: every
+// earlier launch added kPhases * gridDim.x to it, and fewer than that many of
+// this launch's additions can be in it.  Its tag: the index, top bit set.
+__device__ __forceinline__ unsigned long long launch_index(unsigned long long counter) {
+  return counter / ((unsigned long long)kPhases * gridDim.x);
+}
+__device__ __forceinline__ uint32_t launch_tag(unsigned long long index) {
+  return (uint32_t)index | 0x80000000u;
 }
 
 struct Phases {
