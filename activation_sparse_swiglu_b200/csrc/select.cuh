@@ -162,27 +162,56 @@ __device__ int radix_tie(Items items, uint32_t T, int want, SelectScratch& sc) {
   return (int)ip;
 }
 
-// Among bins read in descending bin order (thread t holds the count of the
-// t-th largest bin, 0 past the last), the one holding the krem-th largest
-// key: writes its position t and the rank wanted inside it to misc[0],
-// misc[1] and its count to misc[2] (position 0, rank 1, count 0 when the
-// counts hold fewer than krem keys).  Returns the sum of the counts.  Every
-// thread calls it.
-__device__ __forceinline__ int find_bin_desc(int count, int krem, SelectScratch& sc) {
-  if (threadIdx.x == 0) {
-    sc.misc[0] = 0;
-    sc.misc[1] = 1;
-    sc.misc[2] = 0;
+// Warp 0's share of the cut: among nb bins (a multiple of 32, at most 128)
+// read from the top (bins[nb - 1] first), the one holding the krem-th largest
+// key, once the counts add up to `want` (polled: counts only grow; bounded).
+// Writes its position from the top, the rank wanted inside it and its count
+// to misc[m0 .. m0 + 2] (0, 1, 0 when no bin holds it); the CTA reads them
+// after a barrier.
+__device__ __forceinline__ void warp_find_bin_desc(const uint32_t* bins, int nb, int krem, int want,
+                                                   SelectScratch& sc, int m0, int* err) {
+  const int lane = threadIdx.x & 31, bpl = nb >> 5;
+  const long long t0 = clock64();
+  int c[4] = {0, 0, 0, 0}, sum = 0, incl = 0;
+  for (;;) {
+    sum = 0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (q < bpl) {
+        c[q] = (int)ld_relaxed_u32(bins + (nb - 1 - (lane * bpl + q)));
+        sum += c[q];
+      }
+    incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    int stop = __shfl_sync(0xffffffffu, incl, 31) == want;
+    if (!stop && lane == 0) stop = !wait_more(t0, err);
+    if (__shfl_sync(0xffffffffu, stop, 0)) break;
   }
-  int total;
-  const int above = block_exclusive_scan(count, sc.scan, &total);
-  if (count > 0 && above < krem && above + count >= krem) {
-    sc.misc[0] = (int)threadIdx.x;
-    sc.misc[1] = krem - above;
-    sc.misc[2] = count;
+  if (lane == 0) {
+    sc.misc[m0] = 0;
+    sc.misc[m0 + 1] = 1;
+    sc.misc[m0 + 2] = 0;
   }
-  __syncthreads();
-  return total;
+  __syncwarp();
+  const int above = incl - sum;
+  if (sum > 0 && above < krem && incl >= krem) {
+    int acc = above;
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (q < bpl) {
+        if (acc + c[q] >= krem) {
+          sc.misc[m0] = lane * bpl + q;
+          sc.misc[m0 + 1] = krem - acc;
+          sc.misc[m0 + 2] = c[q];
+          break;
+        }
+        acc += c[q];
+      }
+  }
 }
 
 // The exact cut of the launch; every CTA calls it once it has added its own
@@ -196,28 +225,21 @@ __device__ inline TopkCut select_cut(const uint32_t* hist, const uint32_t* chist
                               int k, SelectScratch& sc, uint32_t tag, int* err,
                               unsigned long long* ts) {
   const int tid = threadIdx.x;
-  // 1. the coarse bin (bins read from the top)
-  long long t0 = clock64();
-  for (;;) {
-    const int cnt = tid < kCoarseBins ? (int)ld_relaxed_u32(chist + (kCoarseBins - 1 - tid)) : 0;
-    if (find_bin_desc(cnt, k, sc) == F || !wait_more(t0, err)) break;
-  }
+  long long t0;
+  // 1. the coarse bin (bins read from the top; warp 0 polls and scans them)
+  if (tid < 32) warp_find_bin_desc(chist, kCoarseBins, k, F, sc, 0, err);
+  __syncthreads();
   stamp(ts, 14);
   const int cb = kCoarseBins - 1 - sc.misc[0];
   const int k1 = sc.misc[1];
   const int ncb = sc.misc[2];
-  __syncthreads();
   // 2. its fine bins
   const int fb0 = cb * kFinePerCoarse;
-  t0 = clock64();
-  for (;;) {
-    const int cnt = tid < kFinePerCoarse ? (int)ld_relaxed_u32(hist + fb0 + (kFinePerCoarse - 1 - tid)) : 0;
-    if (find_bin_desc(cnt, k1, sc) == ncb || !wait_more(t0, err)) break;
-  }
-  const uint32_t b1 = (uint32_t)(fb0 + kFinePerCoarse - 1 - sc.misc[0]);
-  const int krem = sc.misc[1];
-  const int n1 = sc.misc[2];
+  if (tid < 32) warp_find_bin_desc(hist + fb0, kFinePerCoarse, k1, ncb, sc, 3, err);
   __syncthreads();
+  const uint32_t b1 = (uint32_t)(fb0 + kFinePerCoarse - 1 - sc.misc[3]);
+  const int krem = sc.misc[4];
+  const int n1 = sc.misc[5];
   TopkCut cut;
   if (n1 <= kBucketCap) {
     // 3. the candidates, ranked: the one with krem - 1 larger (key, ~channel)
