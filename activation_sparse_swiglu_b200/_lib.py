@@ -85,6 +85,7 @@ SIGNATURES = {
     "prox_forward_with_mask": (_I, [_P, _P, _P, _I, _P, _P, _P]),
     "prox_debug_fail_alloc": (_I, [_I]),
     "prox_debug_wait_timeout": (_I, [_P, _P]),
+    "prox_debug_token_geometry": (_I, [_I, _I, _I, _P]),
     "prox_rmsnorm": (_I, [_P, _P, _I, _I, _F, _P]),
     "prox_copy": (_I, [_P, _P, _S, _P]),
     "prox_last_error": (_S, [ctypes.c_char_p, _S]),

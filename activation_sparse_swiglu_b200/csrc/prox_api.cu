@@ -347,6 +347,30 @@ prox_status prox_calibrate_thresholds_noalloc(const float* X_cal, int n_tok, int
   return PROX_OK;
 }
 
+// The per-token kernel's geometry for L->d x L->F over L->P SMs (one CTA
+// per SM): Stage 1's slices, kept-row capacity and copy depth, Stage 2's
+// ring, and the shared memory of the launch; PROX_EUNSUPPORTED when the
+// device has too few or too many SMs for the shape.  Host only.
+static prox_status plan_token_kernel(prox_layer* L) {
+  const int sms = L->P;
+  if (sms < 1 || sms > prox::kMaxCtas)
+    return fail(PROX_EUNSUPPORTED, "%d SMs: the per-token kernel supports 1 to %d CTAs", sms, prox::kMaxCtas);
+  if ((L->F + sms - 1) / sms > 512)
+    return fail(PROX_EUNSUPPORTED, "d_ff=%d over %d SMs exceeds 512 channels per CTA", L->F, sms);
+  prox::choose_stage1_grid(L->d, L->F, sms, &L->C, &L->s1_lmax, &L->s1_depth);
+  if (L->s1_depth < 2)
+    return fail(PROX_EUNSUPPORTED,
+                "d_model=%d, d_ff=%d over %d SMs: Stage 1's row tables leave no room for two k-tiles per warp",
+                L->d, L->F, sms);
+  size_t s2_smem = 0;
+  prox::choose_stage2(L->d, L->F, sms, &L->ring_slots, &L->stage2_groups, &s2_smem);
+  const size_t s1_smem = prox::stage1_smem_bytes(L->s1_lmax, L->s1_depth, L->d);
+  L->token_smem = s1_smem > s2_smem ? s1_smem : s2_smem;
+  if (L->token_smem > (size_t)prox::kMaxSmemPerBlock)
+    return fail(PROX_EUNSUPPORTED, "per-token kernel shared memory %zu exceeds the per-CTA limit", L->token_smem);
+  return PROX_OK;
+}
+
 prox_status prox_layer_create(const uint16_t* W_gate, const uint16_t* W_up, const uint16_t* W_down,
                               int d_model, int d_ff, float tau_x, int k, int max_batch,
                               void* stream, prox_layer** out_host) {
@@ -373,31 +397,10 @@ prox_status prox_layer_create(const uint16_t* W_gate, const uint16_t* W_up, cons
   L->tau = tau_x;
   L->device = dev;
   L->num_sms = sms;
-  if (sms > prox::kMaxCtas) {
-    delete L;
-    return fail(PROX_EUNSUPPORTED, "%d SMs exceed the %d CTAs the per-token kernel supports", sms,
-                prox::kMaxCtas);
-  }
-  if ((d_ff + sms - 1) / sms > 512) {
-    delete L;
-    return fail(PROX_EUNSUPPORTED, "d_ff=%d over %d SMs exceeds 512 channels per CTA", d_ff, sms);
-  }
   L->P = sms;
-  prox::choose_stage1_grid(L->d, L->F, sms, &L->C, &L->s1_lmax, &L->s1_depth);
-  if (L->s1_depth < 2) {
+  if ((st = plan_token_kernel(L)) != PROX_OK) {
     delete L;
-    return fail(PROX_EUNSUPPORTED,
-                "d_model=%d, d_ff=%d over %d SMs: Stage 1's row tables leave no room for two k-tiles per warp",
-                d_model, d_ff, sms);
-  }
-  size_t s2_smem = 0;
-  prox::choose_stage2(L->d, L->F, sms, &L->ring_slots, &L->stage2_groups, &s2_smem);
-  const size_t s1_smem = prox::stage1_smem_bytes(L->s1_lmax, L->s1_depth, L->d);
-  L->token_smem = s1_smem > s2_smem ? s1_smem : s2_smem;
-  if (L->token_smem > (size_t)prox::kMaxSmemPerBlock) {
-    const size_t need = L->token_smem;
-    delete L;
-    return fail(PROX_EUNSUPPORTED, "per-token kernel shared memory %zu exceeds the per-CTA limit", need);
+    return st;
   }
 
   cudaStream_t s = as_stream(stream);
@@ -441,6 +444,25 @@ prox_status prox_layer_create(const uint16_t* W_gate, const uint16_t* W_up, cons
     return st;
   }
   *out_host = L;
+  return PROX_OK;
+}
+
+prox_status prox_debug_token_geometry(int d_model, int d_ff, int num_sms, int32_t* out_host) {
+  if (!out_host) return fail(PROX_EINVAL, "out_host is NULL");
+  prox_status st = check_shape(d_model, d_ff);
+  if (st != PROX_OK) return st;
+  prox_layer L;
+  L.d = d_model;
+  L.F = d_ff;
+  L.G = d_model / prox::kGroup;
+  L.P = num_sms;
+  if ((st = plan_token_kernel(&L)) != PROX_OK) return st;
+  out_host[0] = L.C;
+  out_host[1] = L.s1_lmax;
+  out_host[2] = L.s1_depth;
+  out_host[3] = L.ring_slots;
+  out_host[4] = L.stage2_groups;
+  out_host[5] = (int32_t)L.token_smem;
   return PROX_OK;
 }
 

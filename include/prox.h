@@ -399,6 +399,17 @@ PROX_API prox_status prox_debug_batch_masks(const prox_layer* layer, int32_t* ma
  * Process-wide; nothing fails on the device.  nth < 0 gives PROX_EINVAL. */
 PROX_API prox_status prox_debug_fail_alloc(int nth);
 
+/* Host-only plan of the per-token kernel for d_model x d_ff over num_sms
+ * SMs, as prox_layer_create would make it on such a device (no GPU needed):
+ * out_host (host, int32 [6]) receives the Stage-1 column slices, the kept-row
+ * capacity per CTA, the Stage-1 copy depth (8-row tiles in flight per warp),
+ * the Stage-2 ring slots, the Stage-2 consumer groups and the launch's
+ * dynamic shared memory in bytes.  Errors as prox_layer_create:
+ * PROX_EINVAL for a shape outside the rules, PROX_EUNSUPPORTED when the shape
+ * needs more shared memory per CTA, or more channels per CTA, than
+ * num_sms SMs give.  For tests of the shape rules. */
+PROX_API prox_status prox_debug_token_geometry(int d_model, int d_ff, int num_sms, int32_t* out_host);
+
 /* Test-only exercise of the bounded device waits, with no fault: launches one
  * CTA that adds one to the layer's launch counter and waits for a second
  * addition that never comes.  The wait runs out after its bound (2e8 SM
