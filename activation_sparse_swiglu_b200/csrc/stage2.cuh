@@ -7,17 +7,16 @@
 // Every CTA finds the token's exact top-k cut (select.cuh: key T and the tie
 // cut) or applies the score threshold, lists the channels of its own range
 // [F c / P, F (c + 1) / P) -- the channels it scored -- past it, ascending, at
-// the range's start in a.sel_list and writes their count; after a grid
-// barrier CTA c takes the ranks
-// [S c / P, S (c + 1) / P) of the whole selection (S channels, ascending), so
-// every CTA streams the same number of channels (to one) whatever the mask
-// looks like; a given list is split the same way by list position, and the
-// dense baseline splits all channels.  A given list is
-// split by list position the same way, and the dense baseline splits all
-// channels.  Producer lanes stream, with 1-D bulk async copies (TMA engine)
-// into a ring of slots, first the gate/up channel records of the CTA's
-// channels (gate column then up column, d_model bf16 each: one copy per
-// channel), then their W_down rows (two rows per slot).  The consumer warps
+// the range's start in a.sel_list and writes their count; once every CTA's
+// count is in (a phase of the launch counter, token_args.cuh), CTA c takes
+// the ranks [S c / P, S (c + 1) / P) of the whole selection (S channels,
+// ascending), so every CTA streams the same number of channels (to one)
+// whatever the mask looks like; a given list is split the same way by list
+// position, and the dense baseline splits all channels.  Producer lanes
+// stream, with 1-D bulk async copies (TMA engine) into a ring of slots, first
+// the gate/up channel records of the CTA's channels (gate column then up
+// column, d_model bf16 each: one copy per channel), then their W_down rows
+// (two rows per slot).  The consumer warps
 // take every ring item in order (so each mbarrier wait is for the phase right
 // after one the waiting thread has already seen complete):
 //   phase A: for each channel every warp of the owning group forms partial
@@ -29,8 +28,8 @@
 //            gate/up records and takes s_j = s~_j from Stage 1);
 //   phase B: the warps accumulate y_part += s_j W_down[j, :] for the CTA's
 //            channels, each thread owning 8-column groups of the output.
-// The CTA's fp32 partial row goes to global memory; the kernel adds the
-// partial rows in a fixed order after a grid barrier.
+// The CTA's fp32 partial row goes to global memory as tagged words; the
+// kernel adds the partial rows in a fixed order (token.cu).
 #pragma once
 #include "select.cuh"
 #include "token_args.cuh"

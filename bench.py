@@ -40,6 +40,7 @@ import json
 import math
 import os
 import platform
+import re
 import statistics
 import subprocess
 import sys
@@ -201,14 +202,25 @@ TOKEN_KERNEL_SOURCES = ("token.cu", "token_args.cuh", "stage1.cuh", "stage2.cuh"
                         "prox_device.cuh")
 
 
+_COMMENT = re.compile(r"//[^\n]*|/\*.*?\*/", re.S)
+
+
+def _code_only(text: str) -> str:
+    """A C++/CUDA source without its comments and blank lines (the kernel
+    sources hold no comment markers inside string literals)."""
+    return "\n".join(line.rstrip() for line in _COMMENT.sub("", text).splitlines() if line.strip())
+
+
 def kernel_source_hash() -> str:
-    """Hash of the per-token kernel's source files; a traffic record counts
-    only while they hash the same as when it was taken."""
+    """Hash of the per-token kernel's code (its source files, comments
+    stripped); a traffic record counts only while the code hashes the same as
+    when it was taken, so any change to the code voids it and a comment edit
+    does not."""
     h = hashlib.sha256()
     for name in TOKEN_KERNEL_SOURCES:
-        with open(os.path.join(CSRC, name), "rb") as fh:
+        with open(os.path.join(CSRC, name), encoding="utf-8") as fh:
             h.update(name.encode())
-            h.update(fh.read())
+            h.update(_code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

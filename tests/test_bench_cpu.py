@@ -72,18 +72,21 @@ def test_traffic_record_roundtrip(bench, tmp_path, monkeypatch):
 
 
 def test_kernel_source_hash_covers_every_token_kernel_source(bench, tmp_path, monkeypatch):
-    # the traffic record is tied to the token kernel's sources: editing any of
-    # them changes the hash, editing another source does not
+    # the traffic record is tied to the token kernel's code: editing the code
+    # of any of its sources changes the hash; editing only comments, or
+    # another source, does not
     src = tmp_path / "csrc"
     src.mkdir()
     for name in bench.TOKEN_KERNEL_SOURCES + ("batch.cu",):
-        (src / name).write_text("// " + name)
+        (src / name).write_text("// " + name + "\nint v = 0;\n")
     monkeypatch.setattr(bench, "CSRC", str(src))
     h0 = bench.kernel_source_hash()
     for name in bench.TOKEN_KERNEL_SOURCES:
-        (src / name).write_text("// edited " + name)
+        (src / name).write_text("/* reworded\n comment */ // " + name + "\n\nint v = 0;  // same code\n")
+        assert bench.kernel_source_hash() == h0
+        (src / name).write_text("// " + name + "\nint v = 1;\n")
         h1 = bench.kernel_source_hash()
         assert h1 != h0
         h0 = h1
-    (src / "batch.cu").write_text("// edited")
+    (src / "batch.cu").write_text("int w = 2;\n")
     assert bench.kernel_source_hash() == h0
